@@ -1,0 +1,397 @@
+"""Benchmark of the GDN layer on B200: prefill tokens/s and decode GB/s.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Workloads (synthetic, seeded; see linear_attention_12_b200/inputs.py):
+  * prefill: B=1, L=32768, 16 QK / 48 V heads, d=128, bf16 q/k/v, fp32 gates,
+    S0 = 0, chunk 64 -- the headline ``value`` (tokens/s, whole job);
+  * decode: 256 sequences x 48 V heads (16 QK heads), fp32 states updated in
+    place (805 MB) -- reported in the ``decode`` object (GB/s).
+Each rank runs its own replica (the layer shards by sequence and head with no
+exchange step; nothing is communicated), so scaling is weak.  Timing: W
+untimed warm-up steps, then K steps bracketed by a barrier and
+torch.cuda.synchronize(); CUDA events on the launching stream; the max over
+ranks is reported.  Inputs (1.09 GB per prefill step, 1.6 GB per decode step)
+are larger than L2, so no flush is needed between iterations.
+
+``--impl reference`` times the fp64 CPU oracle (the only reference
+implementation there is) on rank 0, on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "GDN prefill tokens/s (L=32K, 48 V heads) and decode GB/s vs roofline, 1 B200"
+L = 32768
+H_QK, H_V, D = 16, 48, 128
+DEC_B = 256
+# Algorithmic bytes: q, k (H_qk*d bf16 each), v and o (H_v*d bf16 each), two fp32 gates
+# per V head; plus the final state (H_v * d * d fp32) once per sequence.
+BYTES_PER_TOKEN = 2 * H_QK * D * 2 + 2 * H_V * D * 2 + 2 * H_V * 4          # 33,152
+STATE_BYTES = H_V * D * D * 4                                                 # 3,145,728
+# Algorithmic FLOPs per token per V head: 6 d^2 (W S, Q S, K^T Delta) + 3 C d
+# (three triangular C x C x d products at half) + 2 C d / 3 (grams at half,
+# shared by the 3 V heads of a QK head), C = 64.
+FLOP_PER_TOKEN = H_V * (6 * D * D + 3 * 64 * D + (2 * 64 * D) // 3)
+DEC_BYTES = 2 * DEC_B * H_V * D * D * 4 + DEC_B * (2 * H_QK * D * 2 + 2 * H_V * D * 2 + 2 * H_V * 4)
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d["hbm_gbs"], d["bf16_tflops"], d.get("bf16_tflops_sustained"), "measured"
+    return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clocks / throttle reasons sampled during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [x.strip() for x in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for nm, val in zip(names, parts[5:9]):
+                if val.lower() == "active":
+                    reasons.add(nm)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["not recorded"]}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def dist_setup(n_gpus):
+    import torch
+    import torch.distributed as dist
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        torch.cuda.set_device(local)
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    return rank, world, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x, world):
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def run_ours(args):
+    import torch
+    from linear_attention_12_b200 import gdn, inputs
+
+    rank, world, local = dist_setup(args.gpus)
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    hbm_peak, tf_peak, tf_sust, peak_src = load_peaks()
+    stream = torch.cuda.current_stream()
+
+    # ---------------- prefill workload, inputs resident in HBM
+    case = inputs.qwen_prefill_32k(L)
+    q, k, v = case.q.to(dev), case.k.to(dev), case.v.to(dev)
+    la, be = case.log_alpha.to(dev), case.beta.to(dev)
+    cu = case.cu_seqlens.to(dev)
+    o = torch.empty((L, H_V, D), dtype=torch.bfloat16, device=dev)
+    Sf = torch.empty((1, H_V, D, D), dtype=torch.float32, device=dev)
+
+    def prefill_step():
+        gdn.prefill(q, k, v, la, be, None, cu, o=o, S_final=Sf)
+
+    for _ in range(args.warmup):
+        prefill_step()
+    torch.cuda.synchronize()
+    assert gdn.last_device_error() == gdn.GDN_OK
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+    barrier(world)
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clocks:
+        t0 = torch.cuda.Event(enable_timing=True)
+        t1 = torch.cuda.Event(enable_timing=True)
+        t0.record(stream)
+        for i in range(args.steps):
+            ev[i][0].record(stream)
+            prefill_step()
+            ev[i][1].record(stream)
+        t1.record(stream)
+        torch.cuda.synchronize()
+        barrier(world)
+    total_ms = max_over_ranks(t0.elapsed_time(t1), world)
+    kern_ms = [a.elapsed_time(b) for a, b in ev]
+    kern_avg_ms = statistics.mean(kern_ms)
+    assert gdn.last_device_error() == gdn.GDN_OK
+    ms_per_step = total_ms / args.steps
+    value = world * L * args.steps / (total_ms / 1e3)
+
+    bytes_per_launch = BYTES_PER_TOKEN * L + STATE_BYTES
+    flops_per_launch = FLOP_PER_TOKEN * L
+    achieved_gbs = bytes_per_launch / (kern_avg_ms / 1e3) / 1e9
+    t_hbm = bytes_per_launch / (hbm_peak * 1e9)
+    t_tc = flops_per_launch / (tf_peak * 1e12)
+
+    # ---------------- decode workload (states in place)
+    dc = inputs.batched_decode_256()
+    S = dc.S0.to(dev)
+    dq, dk_, dv_, dla, dbe = (x.to(dev) for x in dc.step(0))
+    do = torch.empty((DEC_B, H_V, D), dtype=torch.bfloat16, device=dev)
+    dec_steps = max(args.steps, 20)
+    for _ in range(max(args.warmup, 3)):
+        gdn.decode_step(dq, dk_, dv_, dla, dbe, S, o=do)
+    torch.cuda.synchronize()
+    barrier(world)
+    d0 = torch.cuda.Event(enable_timing=True)
+    d1 = torch.cuda.Event(enable_timing=True)
+    d0.record(stream)
+    for _ in range(dec_steps):
+        gdn.decode_step(dq, dk_, dv_, dla, dbe, S, o=do)
+    d1.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    dec_ms = max_over_ranks(d0.elapsed_time(d1), world) / dec_steps
+    assert gdn.last_device_error() == gdn.GDN_OK
+    dec_gbs = DEC_BYTES / (dec_ms / 1e3) / 1e9
+    del S, dq, dk_, dv_, dla, dbe, do
+
+    # ---------------- end to end through the public API, host buffers
+    hq, hk, hv = (x.pin_memory() for x in (case.q, case.k, case.v))
+    hla, hbe = case.log_alpha.pin_memory(), case.beta.pin_memory()
+    ho = torch.empty((L, H_V, D), dtype=torch.bfloat16).pin_memory()
+    hS = torch.empty((1, H_V, D, D), dtype=torch.float32).pin_memory()
+    h2d = sum(x.numel() * x.element_size() for x in (hq, hk, hv, hla, hbe))
+    d2h = ho.numel() * ho.element_size() + hS.numel() * hS.element_size()
+
+    def e2e_step():
+        q.copy_(hq, non_blocking=True)
+        k.copy_(hk, non_blocking=True)
+        v.copy_(hv, non_blocking=True)
+        la.copy_(hla, non_blocking=True)
+        be.copy_(hbe, non_blocking=True)
+        prefill_step()
+        ho.copy_(o, non_blocking=True)
+        hS.copy_(Sf, non_blocking=True)
+
+    e2e_steps = max(3, min(args.steps, 10))
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize()
+    barrier(world)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world) / e2e_steps
+    e2e_value = world * L / (e2e_ms / 1e3)
+
+    # ---------------- CPU baseline (the oracle as it stands), rank 0 at N=1 only
+    cpu = None
+    if world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(case, args.cpu_tokens)
+
+    if rank == 0:
+        line = {
+            "metric": METRIC,
+            "value": value,
+            "unit": "tokens/s",
+            "n_gpus": world,
+            "steps": args.steps,
+            "warmup": args.warmup,
+            "ms_per_step": ms_per_step,
+            "higher_is_better": True,
+            "scaling": "weak",
+            "vs_baseline": None,
+            "dtype": "bf16",
+            "data": "synthetic",
+            "config": {
+                "workload": f"prefill B=1 L={L} H_qk={H_QK} H_v={H_V} d={D} bf16 q/k/v, "
+                            "fp32 gates/state, chunk 64, S0=0",
+                "global_batch": world,
+                "seq_len": L,
+                "parallelism": f"replicas x{world}",
+                "l2": "inputs larger than L2 (1.09 GB per step); no flush",
+            },
+            "roofline": {
+                "bound": "hbm",
+                "achieved": achieved_gbs,
+                "peak": hbm_peak,
+                "unit": "GB/s",
+                "frac": achieved_gbs / hbm_peak,
+                "traffic": args.traffic,
+                "peak_source": peak_src,
+                "kernel_us": kern_avg_ms * 1e3,
+                "roofline_us": max(t_hbm, t_tc) * 1e6,
+                "hbm_term_us": t_hbm * 1e6,
+                "tensor_term_us": t_tc * 1e6,
+                "frac_of_roofline_time": max(t_hbm, t_tc) / (kern_avg_ms / 1e3),
+                "tflops": flops_per_launch / (kern_avg_ms / 1e3) / 1e12,
+            },
+            "decode": {
+                "value": dec_gbs,
+                "unit": "GB/s",
+                "us_per_step": dec_ms * 1e3,
+                "bytes_per_step": DEC_BYTES,
+                "peak": hbm_peak,
+                "frac": dec_gbs / hbm_peak,
+                "workload": f"decode B={DEC_B} H_qk={H_QK} H_v={H_V} d={D}, fp32 state in place",
+                "steps": dec_steps,
+            },
+            "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+            "gpu_launches": args.steps,
+            "clocks": clocks.summary(),
+        }
+        if cpu is not None:
+            line["cpu_baseline"] = cpu
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+def cpu_baseline(case, tokens):
+    """The fp64 oracle on all 48 V heads of the first ``tokens`` tokens."""
+    import oracle
+    T = min(tokens, case.T)
+    n_threads = oracle.default_threads()
+    args = (case.q[:T], case.k[:T], case.v[:T], case.log_alpha[:T], case.beta[:T])
+    t0 = time.perf_counter()
+    oracle.prefill(*args, want_o=True, n_threads=n_threads)
+    dt = time.perf_counter() - t0
+    return {"value": T / dt, "unit": "tokens/s", "cores": min(n_threads, H_V),
+            "kind": "oracle",
+            "sample": f"first {T} of {case.T} tokens, all {H_V} V heads, fp64, {dt:.1f} s"}
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    from linear_attention_12_b200 import inputs
+    case = inputs.qwen_prefill_32k(L)
+    import oracle
+    oracle.build()
+    T = min(args.cpu_tokens, L)
+    for _ in range(args.warmup):
+        cpu_baseline(case, min(T, 256))
+    times = []
+    for _ in range(args.steps):
+        r = cpu_baseline(case, T)
+        times.append(T / r["value"])
+    value = args.steps * T / sum(times)
+    line = {
+        "impl": "reference",
+        "metric": METRIC,
+        "value": value,
+        "unit": "tokens/s",
+        "n_gpus": 1,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": 1e3 * sum(times) / args.steps,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "f64",
+        "data": "synthetic",
+        "config": {
+            "workload": f"prefill B=1 L={L} H_qk={H_QK} H_v={H_V} d={D} (oracle on a "
+                        f"{T}-token sample per step)",
+            "global_batch": 1, "seq_len": L, "parallelism": "cpu threads",
+        },
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": r["cores"],
+                         "kind": "oracle", "sample": r["sample"]},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__.split("\n\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--cpu-tokens", type=int, default=2048,
+                    help="tokens of the CPU-oracle sample (all 48 heads)")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--traffic", type=float, default=None,
+                    help="DRAM bytes per prefill launch from an ncu capture, if known")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,138 @@
+/*
+ * gdn.h -- C ABI of libgdn.so, a B200 (sm_100a) implementation of the Gated
+ * DeltaNet (GDN) token mixer.
+ *
+ * The operation (bjdmk.com.cn article "为什么 Qwen3.8-Flash-Next 值得单独跑一遍",
+ * section 2.1 "Gated DeltaNet 负责廉价压缩历史", state-update formula):
+ *
+ *     S_t = alpha_t (I - beta_t k_t k_t^T) S_{t-1} + beta_t k_t v_t^T
+ *     o_t = S_t^T q_t            (post-update state, no scale factor)
+ *
+ * S_t is a d_k x d_v fp32 matrix per (sequence, value head); alpha_t =
+ * exp(log_alpha[t,h]) is the forget gate and beta_t = beta[t,h] the write
+ * strength, one scalar each per (token, value head).  H_v value heads share
+ * H_qk query/key heads: value head h reads q/k head h / (H_v / H_qk)
+ * (section 2.1 of the same article and the jianying88.com article
+ * "Qwen3.8-Flash-Next混合注意力深度解析", section 三: 48 V heads, 16 QK heads,
+ * head dim 128).  The readout is not printed on the pages; o_t = S_t^T q_t
+ * is the reading this library implements.
+ *
+ * Conventions shared by every call
+ *   - All tensor pointers are DEVICE pointers owned by the caller; the library
+ *     allocates no device memory and keeps no per-call state.  The only
+ *     library-global state is a per-device status word in a static
+ *     __device__ variable (see gdn_get_last_device_error).
+ *   - Layouts are dense, row-major, packed token-major ("varlen" packing):
+ *       q, k      [T, H_qk, dk]      io_dtype
+ *       v, o      [T, H_v,  dv]      io_dtype
+ *       log_alpha [T, H_v]           fp32  (log of the forget gate, <= 0 in normal use)
+ *       beta      [T, H_v]           fp32
+ *       S0/S_final/S_inout [N, H_v, dk, dv] fp32 (row i = key dim, column j = value dim)
+ *   - dk = dv = 128 is the only supported head size; H_v % H_qk == 0.
+ *   - q, k, v, o and the state pointers must be 16-byte aligned; log_alpha,
+ *     beta and cu_seqlens 4-byte aligned; the workspace 256-byte aligned.
+ *   - Calls are asynchronous on `stream` (a cudaStream_t passed as void*;
+ *     NULL = the legacy default stream) and return GDN_OK once the work is
+ *     enqueued.  Argument errors are detected on the host before anything is
+ *     launched and leave every output untouched.
+ *   - Inputs are used as given: no normalisation of q/k, no gate activation,
+ *     no scaling.
+ */
+#ifndef GDN_H_
+#define GDN_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define GDN_API __attribute__((visibility("default")))
+#else
+#define GDN_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    GDN_OK = 0,
+    GDN_ERR_INVALID_ARG = 1,  /* null/misaligned pointer, bad size, H_v % H_qk != 0, ... */
+    GDN_ERR_UNSUPPORTED = 2,  /* dk/dv != 128, or the device is not compute capability 10.0 */
+    GDN_ERR_CUDA = 3,         /* a CUDA runtime/driver call or a kernel launch failed */
+    GDN_ERR_TIMEOUT = 4,      /* a device-side bounded wait gave up (see gdn_get_last_device_error) */
+    GDN_ERR_WORKSPACE = 5     /* workspace pointer/size too small for this call */
+} gdn_status;
+
+typedef enum {
+    GDN_BF16 = 1,  /* q, k, v and o are bfloat16 */
+    GDN_F32 = 2    /* q, k, v and o are float32 (computed through bf16 tensor-core operands) */
+} gdn_dtype;
+
+/*
+ * gdn_prefill -- run the recurrence over N packed sequences (chunked prefill).
+ *
+ *   q, k, v, log_alpha, beta : inputs, layouts above, T tokens in total.
+ *   S0        : initial state per (sequence, value head), or NULL for zeros.
+ *   cu_seqlens: device int32 [N+1], cu[0] = 0, non-decreasing, cu[N] = T;
+ *               sequence n is tokens [cu[n], cu[n+1]).  Its contents are not
+ *               read on the host; malformed contents are undefined behaviour.
+ *               Zero-length sequences are allowed (their S_final = S0).
+ *   o         : output [T, H_v, dv] in io_dtype (every row is written).
+ *   S_final   : final state per (sequence, value head), or NULL to skip it.
+ *               May alias S0 exactly (in-place state update); no other overlap
+ *               between outputs and inputs is allowed.
+ *   workspace : device scratch of at least gdn_prefill_workspace_size(...)
+ *               bytes (may be NULL when that size is 0), owned by the caller
+ *               and not used after the work on `stream` completes.
+ *
+ * Returns GDN_OK, GDN_ERR_INVALID_ARG, GDN_ERR_UNSUPPORTED, GDN_ERR_WORKSPACE
+ * or GDN_ERR_CUDA.
+ */
+GDN_API gdn_status gdn_prefill(const void *q, const void *k, const void *v,
+                       const float *log_alpha, const float *beta,
+                       const float *S0, const int32_t *cu_seqlens,
+                       int32_t N, int32_t T, int32_t H_qk, int32_t H_v,
+                       int32_t dk, int32_t dv, gdn_dtype io_dtype,
+                       void *o, float *S_final,
+                       void *workspace, size_t workspace_bytes, void *stream);
+
+/* Bytes of device workspace gdn_prefill needs for these sizes (0 when none). */
+GDN_API size_t gdn_prefill_workspace_size(int32_t N, int32_t T, int32_t H_qk, int32_t H_v,
+                                  int32_t dk, int32_t dv, gdn_dtype io_dtype);
+
+/*
+ * gdn_decode_step -- advance B independent sequences by one token each.
+ *
+ *   q, k [B, H_qk, dk], v [B, H_v, dv] (io_dtype); log_alpha, beta [B, H_v] fp32.
+ *   S_inout [B, H_v, dk, dv] fp32: read, then overwritten in place with S_t.
+ *   o [B, H_v, dv] (io_dtype): o = S_t^T q_t.
+ *
+ * One pass over the state: the kernel reads each 64 KiB state once, forms
+ * S^T k and S^T q, and writes the updated state once.
+ * Returns GDN_OK, GDN_ERR_INVALID_ARG, GDN_ERR_UNSUPPORTED or GDN_ERR_CUDA.
+ */
+GDN_API gdn_status gdn_decode_step(const void *q, const void *k, const void *v,
+                           const float *log_alpha, const float *beta,
+                           float *S_inout, int32_t B, int32_t H_qk, int32_t H_v,
+                           int32_t dk, int32_t dv, gdn_dtype io_dtype,
+                           void *o, void *stream);
+
+/*
+ * gdn_get_last_device_error -- synchronise `stream`, then read and clear the
+ * current device's status word.  Returns GDN_ERR_TIMEOUT if a kernel gave up
+ * on a bounded wait since the last call, GDN_ERR_CUDA if the synchronisation
+ * failed, GDN_OK otherwise.
+ */
+GDN_API gdn_status gdn_get_last_device_error(void *stream);
+
+/* Static, human-readable name of a status code. */
+GDN_API const char *gdn_status_string(gdn_status status);
+
+/* Library version as MAJOR*10000 + MINOR*100 + PATCH. */
+GDN_API int32_t gdn_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GDN_H_ */

@@ -1,0 +1,140 @@
+// gdn_api.cu -- the C ABI of libgdn.so (declared in include/gdn.h).
+//
+// Host-side argument validation, capability check, dispatch to the kernel
+// launchers, and the device status word.  Every argument error is detected
+// here, before any CUDA call, so invalid calls neither launch nor touch
+// outputs (and can be tested on a machine without a GPU).
+#include <cuda_runtime.h>
+
+#include "../../include/gdn.h"
+#include "gdn_common.cuh"
+#include "gdn_internal.h"
+
+namespace gdn {
+
+__device__ unsigned int g_status = 0u;
+
+cudaError_t read_and_clear_status(unsigned int* status, cudaStream_t stream) {
+    cudaError_t e = cudaStreamSynchronize(stream);
+    if (e != cudaSuccess) return e;
+    e = cudaMemcpyFromSymbolAsync(status, g_status, sizeof(unsigned int), 0,
+                                  cudaMemcpyDeviceToHost, stream);
+    if (e != cudaSuccess) return e;
+    const unsigned int zero = 0u;
+    e = cudaMemcpyToSymbolAsync(g_status, &zero, sizeof(unsigned int), 0,
+                                cudaMemcpyHostToDevice, stream);
+    if (e != cudaSuccess) return e;
+    return cudaStreamSynchronize(stream);
+}
+
+}  // namespace gdn
+
+namespace {
+
+constexpr int kHeadDim = 128;
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+// 0 = OK, otherwise a gdn_status.
+gdn_status check_device() {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return GDN_ERR_CUDA;
+    int major = 0, minor = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
+        return GDN_ERR_CUDA;
+    if (major != 10 || minor != 0) return GDN_ERR_UNSUPPORTED;
+    return GDN_OK;
+}
+
+gdn_status check_heads(int32_t H_qk, int32_t H_v, int32_t dk, int32_t dv, gdn_dtype dt) {
+    if (H_qk <= 0 || H_v <= 0 || H_v % H_qk != 0) return GDN_ERR_INVALID_ARG;
+    if (dt != GDN_BF16 && dt != GDN_F32) return GDN_ERR_INVALID_ARG;
+    if (dk != kHeadDim || dv != kHeadDim) return GDN_ERR_UNSUPPORTED;
+    return GDN_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* gdn_status_string(gdn_status s) {
+    switch (s) {
+        case GDN_OK: return "GDN_OK";
+        case GDN_ERR_INVALID_ARG: return "GDN_ERR_INVALID_ARG";
+        case GDN_ERR_UNSUPPORTED: return "GDN_ERR_UNSUPPORTED";
+        case GDN_ERR_CUDA: return "GDN_ERR_CUDA";
+        case GDN_ERR_TIMEOUT: return "GDN_ERR_TIMEOUT";
+        case GDN_ERR_WORKSPACE: return "GDN_ERR_WORKSPACE";
+    }
+    return "GDN_ERR_UNKNOWN";
+}
+
+int32_t gdn_version(void) { return 100; }
+
+size_t gdn_prefill_workspace_size(int32_t N, int32_t T, int32_t H_qk, int32_t H_v, int32_t dk,
+                                  int32_t dv, gdn_dtype io_dtype) {
+    if (N <= 0 || T < 0 || check_heads(H_qk, H_v, dk, dv, io_dtype) != GDN_OK) return 0;
+    return gdn::prefill_workspace_bytes(N, T, H_qk, H_v, io_dtype == GDN_BF16);
+}
+
+gdn_status gdn_prefill(const void* q, const void* k, const void* v, const float* log_alpha,
+                       const float* beta, const float* S0, const int32_t* cu_seqlens, int32_t N,
+                       int32_t T, int32_t H_qk, int32_t H_v, int32_t dk, int32_t dv,
+                       gdn_dtype io_dtype, void* o, float* S_final, void* workspace,
+                       size_t workspace_bytes, void* stream) {
+    gdn_status st = check_heads(H_qk, H_v, dk, dv, io_dtype);
+    if (st != GDN_OK) return st;
+    if (N <= 0 || T < 0) return GDN_ERR_INVALID_ARG;
+    // Every element index must fit in 64-bit arithmetic and every token
+    // coordinate in the int32 coordinates of the tensor maps.
+    if ((long long)T * H_v * kHeadDim >= (1ll << 40)) return GDN_ERR_INVALID_ARG;
+    if (!cu_seqlens || !aligned(cu_seqlens, 4)) return GDN_ERR_INVALID_ARG;
+    if (T > 0) {
+        if (!q || !k || !v || !log_alpha || !beta || !o) return GDN_ERR_INVALID_ARG;
+        if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) ||
+            !aligned(log_alpha, 4) || !aligned(beta, 4))
+            return GDN_ERR_INVALID_ARG;
+    }
+    if ((S0 && !aligned(S0, 16)) || (S_final && !aligned(S_final, 16))) return GDN_ERR_INVALID_ARG;
+    const bool bf16 = io_dtype == GDN_BF16;
+    const size_t need = gdn::prefill_workspace_bytes(N, T, H_qk, H_v, bf16);
+    if (need > 0 && (!workspace || workspace_bytes < need || !aligned(workspace, 256)))
+        return GDN_ERR_WORKSPACE;
+    st = check_device();
+    if (st != GDN_OK) return st;
+    cudaError_t e = gdn::launch_prefill(q, k, v, log_alpha, beta, S0, cu_seqlens, N, T, H_qk,
+                                        H_v, bf16, o, S_final, workspace,
+                                        static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+}
+
+gdn_status gdn_decode_step(const void* q, const void* k, const void* v, const float* log_alpha,
+                           const float* beta, float* S_inout, int32_t B, int32_t H_qk,
+                           int32_t H_v, int32_t dk, int32_t dv, gdn_dtype io_dtype, void* o,
+                           void* stream) {
+    gdn_status st = check_heads(H_qk, H_v, dk, dv, io_dtype);
+    if (st != GDN_OK) return st;
+    if (B < 0) return GDN_ERR_INVALID_ARG;
+    if ((long long)B * H_v >= (1ll << 31)) return GDN_ERR_INVALID_ARG;
+    if (B == 0) return GDN_OK;
+    if (!q || !k || !v || !log_alpha || !beta || !S_inout || !o) return GDN_ERR_INVALID_ARG;
+    if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) ||
+        !aligned(S_inout, 16) || !aligned(log_alpha, 4) || !aligned(beta, 4))
+        return GDN_ERR_INVALID_ARG;
+    st = check_device();
+    if (st != GDN_OK) return st;
+    cudaError_t e = gdn::launch_decode_step(q, k, v, log_alpha, beta, S_inout, B, H_qk, H_v,
+                                            io_dtype == GDN_BF16, o,
+                                            static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+}
+
+gdn_status gdn_get_last_device_error(void* stream) {
+    unsigned int status = 0u;
+    if (gdn::read_and_clear_status(&status, static_cast<cudaStream_t>(stream)) != cudaSuccess)
+        return GDN_ERR_CUDA;
+    return status == GDN_DEV_OK ? GDN_OK : GDN_ERR_TIMEOUT;
+}
+
+}  // extern "C"

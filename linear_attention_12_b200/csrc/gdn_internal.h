@@ -1,0 +1,24 @@
+// gdn_internal.h -- launchers behind the C ABI (not part of the public header).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace gdn {
+
+cudaError_t launch_decode_step(const void* q, const void* k, const void* v,
+                               const float* log_alpha, const float* beta, float* S, int B,
+                               int H_qk, int H_v, bool bf16, void* o, cudaStream_t stream);
+
+// Workspace bytes the prefill needs (fp32 I/O stages bf16 copies of q, k, v).
+size_t prefill_workspace_bytes(int N, int T, int H_qk, int H_v, bool bf16);
+
+cudaError_t launch_prefill(const void* q, const void* k, const void* v, const float* log_alpha,
+                           const float* beta, const float* S0, const int32_t* cu_seqlens, int N,
+                           int T, int H_qk, int H_v, bool bf16, void* o, float* S_final,
+                           void* workspace, cudaStream_t stream);
+
+cudaError_t read_and_clear_status(unsigned int* status, cudaStream_t stream);
+
+}  // namespace gdn

@@ -1,0 +1,168 @@
+"""ctypes binding of ``libgdn.so`` (C ABI in ``include/gdn.h``).
+
+Argument marshalling only: every step of the computation runs in the CUDA
+library.  PyTorch provides device memory and the current stream.  There is no
+fallback: if the library is missing, or a call fails, an exception is raised.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libgdn.so")
+
+GDN_OK = 0
+GDN_ERR_INVALID_ARG = 1
+GDN_ERR_UNSUPPORTED = 2
+GDN_ERR_CUDA = 3
+GDN_ERR_TIMEOUT = 4
+GDN_ERR_WORKSPACE = 5
+GDN_BF16 = 1
+GDN_F32 = 2
+
+# Every exported symbol of include/gdn.h with its ctypes signature.
+_c = ctypes
+SIGNATURES = {
+    "gdn_prefill": (_c.c_int, [_c.c_void_p, _c.c_void_p, _c.c_void_p, _c.c_void_p, _c.c_void_p,
+                               _c.c_void_p, _c.c_void_p, _c.c_int32, _c.c_int32, _c.c_int32,
+                               _c.c_int32, _c.c_int32, _c.c_int32, _c.c_int, _c.c_void_p,
+                               _c.c_void_p, _c.c_void_p, _c.c_size_t, _c.c_void_p]),
+    "gdn_prefill_workspace_size": (_c.c_size_t, [_c.c_int32] * 6 + [_c.c_int]),
+    "gdn_decode_step": (_c.c_int, [_c.c_void_p, _c.c_void_p, _c.c_void_p, _c.c_void_p,
+                                   _c.c_void_p, _c.c_void_p, _c.c_int32, _c.c_int32, _c.c_int32,
+                                   _c.c_int32, _c.c_int32, _c.c_int, _c.c_void_p, _c.c_void_p]),
+    "gdn_get_last_device_error": (_c.c_int, [_c.c_void_p]),
+    "gdn_status_string": (_c.c_char_p, [_c.c_int]),
+    "gdn_version": (_c.c_int32, []),
+}
+
+_lock = threading.Lock()
+_lib = None
+
+
+class GDNError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where} failed: {status_string(status)}")
+
+
+def lib() -> ctypes.CDLL:
+    """Load ``libgdn.so`` (once).  Raises if it has not been built."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            if not os.path.exists(LIB_PATH):
+                raise RuntimeError(
+                    f"{LIB_PATH} is missing: build it with "
+                    "`python -m linear_attention_12_b200.build`")
+            L = ctypes.CDLL(LIB_PATH)
+            for name, (res, args) in SIGNATURES.items():
+                fn = getattr(L, name)
+                fn.restype = res
+                fn.argtypes = args
+            _lib = L
+    return _lib
+
+
+def status_string(status: int) -> str:
+    return lib().gdn_status_string(int(status)).decode()
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream_handle(stream=None):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _io_dtype(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return GDN_BF16
+    if t.dtype == torch.float32:
+        return GDN_F32
+    raise TypeError(f"q/k/v must be bfloat16 or float32, got {t.dtype}")
+
+
+def _check(t, name, dtype=None, shape=None):
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TypeError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+
+
+def workspace_size(N, T, H_qk, H_v, d=128, io_dtype=GDN_BF16) -> int:
+    return int(lib().gdn_prefill_workspace_size(N, T, H_qk, H_v, d, d, io_dtype))
+
+
+def prefill(q, k, v, log_alpha, beta, S0=None, cu_seqlens=None, *, o=None, S_final=None,
+            want_state=True, workspace=None, stream=None):
+    """Chunked prefill.  Returns ``(o, S_final)`` (``S_final`` None if not wanted)."""
+    T, H_qk, dk = q.shape
+    H_v, dv = v.shape[1], v.shape[2]
+    dt = q.dtype
+    _check(q, "q", dt)
+    _check(k, "k", dt, q.shape)
+    _check(v, "v", dt, (T, H_v, dv))
+    _check(log_alpha, "log_alpha", torch.float32, (T, H_v))
+    _check(beta, "beta", torch.float32, (T, H_v))
+    if cu_seqlens is None:
+        cu_seqlens = torch.tensor([0, T], dtype=torch.int32, device=q.device)
+    _check(cu_seqlens, "cu_seqlens", torch.int32)
+    N = cu_seqlens.numel() - 1
+    if S0 is not None:
+        _check(S0, "S0", torch.float32, (N, H_v, dk, dv))
+    if o is None:
+        o = torch.empty((T, H_v, dv), dtype=dt, device=q.device)
+    _check(o, "o", dt, (T, H_v, dv))
+    if S_final is None and want_state:
+        S_final = torch.empty((N, H_v, dk, dv), dtype=torch.float32, device=q.device)
+    if S_final is not None:
+        _check(S_final, "S_final", torch.float32, (N, H_v, dk, dv))
+    io = _io_dtype(q)
+    need = workspace_size(N, T, H_qk, H_v, dk, io)
+    if need and workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    wbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    st = lib().gdn_prefill(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _ptr(S0),
+                           _ptr(cu_seqlens), N, T, H_qk, H_v, dk, dv, io, _ptr(o), _ptr(S_final),
+                           _ptr(workspace), wbytes, _stream_handle(stream))
+    if st != GDN_OK:
+        raise GDNError(st, "gdn_prefill")
+    return o, S_final
+
+
+def decode_step(q, k, v, log_alpha, beta, S, *, o=None, stream=None):
+    """One decode step; ``S`` [B, H_v, dk, dv] fp32 is updated in place.  Returns ``o``."""
+    B, H_qk, dk = q.shape
+    H_v, dv = v.shape[1], v.shape[2]
+    dt = q.dtype
+    _check(q, "q", dt)
+    _check(k, "k", dt, q.shape)
+    _check(v, "v", dt, (B, H_v, dv))
+    _check(log_alpha, "log_alpha", torch.float32, (B, H_v))
+    _check(beta, "beta", torch.float32, (B, H_v))
+    _check(S, "S", torch.float32, (B, H_v, dk, dv))
+    if o is None:
+        o = torch.empty((B, H_v, dv), dtype=dt, device=q.device)
+    _check(o, "o", dt, (B, H_v, dv))
+    st = lib().gdn_decode_step(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _ptr(S),
+                               B, H_qk, H_v, dk, dv, _io_dtype(q), _ptr(o),
+                               _stream_handle(stream))
+    if st != GDN_OK:
+        raise GDNError(st, "gdn_decode_step")
+    return o
+
+
+def last_device_error(stream=None) -> int:
+    """Synchronise the stream and return (and clear) the device status."""
+    return int(lib().gdn_get_last_device_error(_stream_handle(stream)))

@@ -181,17 +181,22 @@ def prefill(q, k, v, log_alpha, beta, S0=None, cu_seqlens=None, heads=None,
 def decode_step(q, k, v, log_alpha, beta, S, units_bh=None, n_threads=None):
     """One decode step for a batch: q, k ``[B, H_qk, dk]``, v ``[B, H_v, dv]``,
     gates ``[B, H_v]``, S ``[B, H_v, dk, dv]``.  Returns ``(o [B,H_v,dv], S_new)``
-    in fp64.  ``units_bh`` optionally limits the work to a list of (b, h)
-    pairs; the returned arrays then hold one row per pair, in that order.
+    in fp64.  With ``units_bh`` (a list of (b, h) pairs) only those units are
+    advanced: S is then ``[len(units_bh), dk, dv]`` (one state per pair) and the
+    returned arrays hold one row per pair, in that order.
     """
     qn = _as_np(q)
     B = qn.shape[0]
     vn = _as_np(v)
     H_v, dv = vn.shape[1], vn.shape[2]
     Sn = np.asarray(_as_np(S), dtype=np.float64)
-    pairs = [(b, h) for b in range(B) for h in range(H_v)] if units_bh is None else list(units_bh)
+    if units_bh is None:
+        pairs = [(b, h) for b in range(B) for h in range(H_v)]
+        S_init = Sn.reshape(B * H_v, *Sn.shape[2:])
+    else:
+        pairs = [(int(b), int(h)) for (b, h) in units_bh]
+        S_init = Sn
     units = [(b, b + 1, h) for (b, h) in pairs]
-    S_init = np.stack([Sn[b, h] for (b, h) in pairs])
     S_out, o_list = run_units(qn, _as_np(k), vn, log_alpha, beta, units, S_init, True, n_threads)
     o = np.stack([x[0] for x in o_list])
     if units_bh is None:

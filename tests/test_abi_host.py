@@ -1,0 +1,118 @@
+"""Host-side tests of the C ABI (no GPU needed): the library loads, exports
+every symbol the header declares, and rejects invalid arguments on the host
+before any CUDA call."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from linear_attention_12_b200 import build as gdn_build
+from linear_attention_12_b200 import gdn
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    gdn_build.build()
+    return gdn.lib()
+
+
+def _declared_symbols():
+    text = open(os.path.join(ROOT, "include", "gdn.h")).read()
+    return set(re.findall(r"GDN_API\s+[\w\s\*]+?\b(gdn_\w+)\s*\(", text))
+
+
+def test_header_declares_expected_entry_points():
+    assert {"gdn_prefill", "gdn_prefill_workspace_size", "gdn_decode_step",
+            "gdn_get_last_device_error", "gdn_status_string", "gdn_version"} <= _declared_symbols()
+
+
+def test_library_exports_every_declared_symbol(L):
+    for name in _declared_symbols():
+        assert hasattr(L, name), name
+    assert set(gdn.SIGNATURES) == _declared_symbols()
+
+
+def test_status_strings(L):
+    for code, name in [(0, "GDN_OK"), (1, "GDN_ERR_INVALID_ARG"), (2, "GDN_ERR_UNSUPPORTED"),
+                       (3, "GDN_ERR_CUDA"), (4, "GDN_ERR_TIMEOUT"), (5, "GDN_ERR_WORKSPACE")]:
+        assert gdn.status_string(code) == name
+    assert L.gdn_version() == 100
+
+
+def test_workspace_size(L):
+    assert gdn.workspace_size(1, 32768, 16, 48, 128, gdn.GDN_BF16) == 0
+    ws = gdn.workspace_size(1, 256, 1, 1, 128, gdn.GDN_F32)
+    assert ws >= 3 * 256 * 128 * 2
+    assert gdn.workspace_size(0, 256, 1, 1, 128, gdn.GDN_F32) == 0  # invalid -> 0
+
+
+# Fake, never dereferenced device addresses: validation fails before any use.
+P = 0x10000
+BAD = 0x10001  # misaligned
+
+
+def _prefill(L, **kw):
+    a = dict(q=P, k=P, v=P, la=P, be=P, S0=None, cu=P, N=1, T=64, H_qk=1, H_v=1, dk=128,
+             dv=128, dt=gdn.GDN_BF16, o=P, Sf=None, ws=None, wsb=0, stream=None)
+    a.update(kw)
+    return L.gdn_prefill(a["q"], a["k"], a["v"], a["la"], a["be"], a["S0"], a["cu"], a["N"],
+                         a["T"], a["H_qk"], a["H_v"], a["dk"], a["dv"], a["dt"], a["o"], a["Sf"],
+                         a["ws"], a["wsb"], a["stream"])
+
+
+@pytest.mark.parametrize("kw,expect", [
+    (dict(q=None), gdn.GDN_ERR_INVALID_ARG),
+    (dict(o=None), gdn.GDN_ERR_INVALID_ARG),
+    (dict(cu=None), gdn.GDN_ERR_INVALID_ARG),
+    (dict(v=BAD), gdn.GDN_ERR_INVALID_ARG),
+    (dict(S0=BAD), gdn.GDN_ERR_INVALID_ARG),
+    (dict(H_qk=3, H_v=4), gdn.GDN_ERR_INVALID_ARG),
+    (dict(H_qk=0), gdn.GDN_ERR_INVALID_ARG),
+    (dict(N=0), gdn.GDN_ERR_INVALID_ARG),
+    (dict(T=-1), gdn.GDN_ERR_INVALID_ARG),
+    (dict(dt=7), gdn.GDN_ERR_INVALID_ARG),
+    (dict(dk=64, dv=64), gdn.GDN_ERR_UNSUPPORTED),
+    (dict(dv=256), gdn.GDN_ERR_UNSUPPORTED),
+    (dict(dt=gdn.GDN_F32), gdn.GDN_ERR_WORKSPACE),
+    (dict(dt=gdn.GDN_F32, ws=P, wsb=16), gdn.GDN_ERR_WORKSPACE),
+])
+def test_prefill_rejects_bad_arguments_on_host(L, kw, expect):
+    assert _prefill(L, **kw) == expect
+
+
+def _decode(L, **kw):
+    a = dict(q=P, k=P, v=P, la=P, be=P, S=P, B=4, H_qk=1, H_v=3, dk=128, dv=128,
+             dt=gdn.GDN_BF16, o=P, stream=None)
+    a.update(kw)
+    return L.gdn_decode_step(a["q"], a["k"], a["v"], a["la"], a["be"], a["S"], a["B"], a["H_qk"],
+                             a["H_v"], a["dk"], a["dv"], a["dt"], a["o"], a["stream"])
+
+
+@pytest.mark.parametrize("kw,expect", [
+    (dict(S=None), gdn.GDN_ERR_INVALID_ARG),
+    (dict(S=BAD), gdn.GDN_ERR_INVALID_ARG),
+    (dict(q=P + 8), gdn.GDN_ERR_INVALID_ARG),
+    (dict(B=-1), gdn.GDN_ERR_INVALID_ARG),
+    (dict(H_qk=2, H_v=3), gdn.GDN_ERR_INVALID_ARG),
+    (dict(dk=96), gdn.GDN_ERR_UNSUPPORTED),
+    (dict(B=0, q=None, S=None), gdn.GDN_OK),  # nothing to do, nothing touched
+])
+def test_decode_rejects_bad_arguments_on_host(L, kw, expect):
+    assert _decode(L, **kw) == expect
+
+
+def test_binding_refuses_cpu_tensors(L):
+    import torch
+    x = torch.zeros(4, 1, 128, dtype=torch.bfloat16)
+    with pytest.raises(TypeError):
+        gdn.decode_step(x, x, x, torch.zeros(4, 1), torch.zeros(4, 1), torch.zeros(4, 1, 128, 128))
+
+
+def test_binding_has_no_cpu_fallback():
+    """The product binding must not reach the oracle or any CPU path."""
+    src = open(os.path.join(ROOT, "linear_attention_12_b200", "gdn.py")).read()
+    assert "oracle" not in src
+    assert "import numpy" not in src
