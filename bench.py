@@ -32,7 +32,7 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "GDN prefill tokens/s (L=32K, 48 V heads) and decode GB/s vs roofline, 1 B200"
-L = 32768
+L = 32768  # the benchmarked sequence length (--seq-len overrides it for profiling captures)
 H_QK, H_V, D = 16, 48, 128
 DEC_B = 256
 # Algorithmic bytes: q, k (H_qk*d bf16 each), v and o (H_v*d bf16 each), two fp32 gates
@@ -141,6 +141,85 @@ def max_over_ranks(x, world):
     return float(t.item())
 
 
+def run_decode(args, dev, stream, world):
+    """Time decode steps on the 256-sequence workload; returns (ms per step, GB/s)."""
+    import torch
+    from linear_attention_12_b200 import gdn, inputs
+    dc = inputs.batched_decode_256()
+    S = dc.S0.to(dev)
+    dq, dk_, dv_, dla, dbe = (x.to(dev) for x in dc.step(0))
+    do = torch.empty((DEC_B, H_V, D), dtype=torch.bfloat16, device=dev)
+    dec_steps = max(args.steps, 20)
+    for _ in range(max(args.warmup, 3)):
+        gdn.decode_step(dq, dk_, dv_, dla, dbe, S, o=do)
+    torch.cuda.synchronize()
+    barrier(world)
+    d0 = torch.cuda.Event(enable_timing=True)
+    d1 = torch.cuda.Event(enable_timing=True)
+    d0.record(stream)
+    for _ in range(dec_steps):
+        gdn.decode_step(dq, dk_, dv_, dla, dbe, S, o=do)
+    d1.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    dec_ms = max_over_ranks(d0.elapsed_time(d1), world) / dec_steps
+    assert gdn.last_device_error() == gdn.GDN_OK
+    return dec_ms, DEC_BYTES / (dec_ms / 1e3) / 1e9
+
+
+def run_e2e(args, case, q, k, v, la, be, o, Sf, prefill_step, stream, world, L):
+    """Prefill through the public API with the inputs in pinned host memory:
+    each step copies q, k, v and the gates in and o and S_final out."""
+    import torch
+    hq, hk, hv = (x.pin_memory() for x in (case.q, case.k, case.v))
+    hla, hbe = case.log_alpha.pin_memory(), case.beta.pin_memory()
+    ho = torch.empty((L, H_V, D), dtype=torch.bfloat16).pin_memory()
+    hS = torch.empty((1, H_V, D, D), dtype=torch.float32).pin_memory()
+    h2d = sum(x.numel() * x.element_size() for x in (hq, hk, hv, hla, hbe))
+    d2h = ho.numel() * ho.element_size() + hS.numel() * hS.element_size()
+
+    def e2e_step():
+        q.copy_(hq, non_blocking=True)
+        k.copy_(hk, non_blocking=True)
+        v.copy_(hv, non_blocking=True)
+        la.copy_(hla, non_blocking=True)
+        be.copy_(hbe, non_blocking=True)
+        prefill_step()
+        ho.copy_(o, non_blocking=True)
+        hS.copy_(Sf, non_blocking=True)
+
+    e2e_steps = max(3, min(args.steps, 10))
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize()
+    barrier(world)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world) / e2e_steps
+    return world * L / (e2e_ms / 1e3), e2e_ms, h2d, d2h
+
+
+def traffic_from_profile(L):
+    """DRAM bytes per prefill launch from the committed ncu summary, if it was
+    taken on the current kernel source; else None."""
+    import hashlib
+    p = os.path.join(ROOT, "profiles", "prefill_traffic.json")
+    src = os.path.join(ROOT, "linear_attention_12_b200", "csrc", "gdn_prefill.cu")
+    if not os.path.exists(p):
+        return None
+    d = json.load(open(p))
+    sha = hashlib.sha256(open(src, "rb").read()).hexdigest()
+    if d.get("kernel_source_sha256") != sha:
+        return None
+    return d["dram_bytes_per_token"] * L + d.get("dram_bytes_fixed", 0)
+
+
 def run_ours(args):
     import torch
     from linear_attention_12_b200 import gdn, inputs
@@ -152,7 +231,8 @@ def run_ours(args):
     stream = torch.cuda.current_stream()
 
     # ---------------- prefill workload, inputs resident in HBM
-    case = inputs.qwen_prefill_32k(L)
+    case = inputs.qwen_prefill_32k(args.seq_len)
+    L = args.seq_len
     q, k, v = case.q.to(dev), case.k.to(dev), case.v.to(dev)
     la, be = case.log_alpha.to(dev), case.beta.to(dev)
     cu = case.cu_seqlens.to(dev)
@@ -195,67 +275,21 @@ def run_ours(args):
     t_tc = flops_per_launch / (tf_peak * 1e12)
 
     # ---------------- decode workload (states in place)
-    dc = inputs.batched_decode_256()
-    S = dc.S0.to(dev)
-    dq, dk_, dv_, dla, dbe = (x.to(dev) for x in dc.step(0))
-    do = torch.empty((DEC_B, H_V, D), dtype=torch.bfloat16, device=dev)
-    dec_steps = max(args.steps, 20)
-    for _ in range(max(args.warmup, 3)):
-        gdn.decode_step(dq, dk_, dv_, dla, dbe, S, o=do)
-    torch.cuda.synchronize()
-    barrier(world)
-    d0 = torch.cuda.Event(enable_timing=True)
-    d1 = torch.cuda.Event(enable_timing=True)
-    d0.record(stream)
-    for _ in range(dec_steps):
-        gdn.decode_step(dq, dk_, dv_, dla, dbe, S, o=do)
-    d1.record(stream)
-    torch.cuda.synchronize()
-    barrier(world)
-    dec_ms = max_over_ranks(d0.elapsed_time(d1), world) / dec_steps
-    assert gdn.last_device_error() == gdn.GDN_OK
-    dec_gbs = DEC_BYTES / (dec_ms / 1e3) / 1e9
-    del S, dq, dk_, dv_, dla, dbe, do
+    dec_ms = dec_gbs = None
+    if not args.no_decode:
+        dec_ms, dec_gbs = run_decode(args, dev, stream, world)
 
     # ---------------- end to end through the public API, host buffers
-    hq, hk, hv = (x.pin_memory() for x in (case.q, case.k, case.v))
-    hla, hbe = case.log_alpha.pin_memory(), case.beta.pin_memory()
-    ho = torch.empty((L, H_V, D), dtype=torch.bfloat16).pin_memory()
-    hS = torch.empty((1, H_V, D, D), dtype=torch.float32).pin_memory()
-    h2d = sum(x.numel() * x.element_size() for x in (hq, hk, hv, hla, hbe))
-    d2h = ho.numel() * ho.element_size() + hS.numel() * hS.element_size()
-
-    def e2e_step():
-        q.copy_(hq, non_blocking=True)
-        k.copy_(hk, non_blocking=True)
-        v.copy_(hv, non_blocking=True)
-        la.copy_(hla, non_blocking=True)
-        be.copy_(hbe, non_blocking=True)
-        prefill_step()
-        ho.copy_(o, non_blocking=True)
-        hS.copy_(Sf, non_blocking=True)
-
-    e2e_steps = max(3, min(args.steps, 10))
-    for _ in range(2):
-        e2e_step()
-    torch.cuda.synchronize()
-    barrier(world)
-    e0 = torch.cuda.Event(enable_timing=True)
-    e1 = torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(e2e_steps):
-        e2e_step()
-    e1.record(stream)
-    torch.cuda.synchronize()
-    barrier(world)
-    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world) / e2e_steps
-    e2e_value = world * L / (e2e_ms / 1e3)
+    e2e_value = e2e_ms = None
+    h2d = d2h = 0
+    if not args.no_e2e:
+        e2e_value, e2e_ms, h2d, d2h = run_e2e(args, case, q, k, v, la, be, o, Sf, prefill_step,
+                                              stream, world, L)
 
     # ---------------- CPU baseline (the oracle as it stands), rank 0 at N=1 only
     cpu = None
     if world == 1 and not args.no_cpu_baseline:
-        cpu = cpu_baseline(case, args.cpu_tokens)
-
+        cpu = cpu_baseline(case, args.cpu_baseline_tokens)
     if rank == 0:
         line = {
             "metric": METRIC,
@@ -284,7 +318,7 @@ def run_ours(args):
                 "peak": hbm_peak,
                 "unit": "GB/s",
                 "frac": achieved_gbs / hbm_peak,
-                "traffic": args.traffic,
+                "traffic": traffic_from_profile(L),
                 "peak_source": peak_src,
                 "kernel_us": kern_avg_ms * 1e3,
                 "roofline_us": max(t_hbm, t_tc) * 1e6,
@@ -293,7 +327,7 @@ def run_ours(args):
                 "frac_of_roofline_time": max(t_hbm, t_tc) / (kern_avg_ms / 1e3),
                 "tflops": flops_per_launch / (kern_avg_ms / 1e3) / 1e12,
             },
-            "decode": {
+            "decode": None if dec_gbs is None else {
                 "value": dec_gbs,
                 "unit": "GB/s",
                 "us_per_step": dec_ms * 1e3,
@@ -301,10 +335,11 @@ def run_ours(args):
                 "peak": hbm_peak,
                 "frac": dec_gbs / hbm_peak,
                 "workload": f"decode B={DEC_B} H_qk={H_QK} H_v={H_V} d={D}, fp32 state in place",
-                "steps": dec_steps,
+                "steps": max(args.steps, 20),
             },
-            "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
-                    "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+            "e2e": None if e2e_value is None else {
+                "value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
             "gpu_launches": args.steps,
             "clocks": clocks.summary(),
         }
@@ -380,10 +415,14 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--cpu-tokens", type=int, default=2048,
-                    help="tokens of the CPU-oracle sample (all 48 heads)")
+                    help="tokens per step of the reference arm's oracle sample (all 48 heads)")
+    ap.add_argument("--cpu-baseline-tokens", type=int, default=8192,
+                    help="tokens of the cpu_baseline oracle sample (all 48 heads)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--traffic", type=float, default=None,
-                    help="DRAM bytes per prefill launch from an ncu capture, if known")
+    ap.add_argument("--seq-len", type=int, default=L,
+                    help="prefill length (the benchmark is L=32768; smaller only for profiling)")
+    ap.add_argument("--no-decode", action="store_true", help="skip the decode measurement")
+    ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer measurement")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

@@ -664,13 +664,18 @@ cudaError_t launch_prefill(const void* q, const void* k, const void* v, const fl
         !make_map(&mv, vb, T, (uint64_t)H_v * D))
         return cudaErrorInvalidValue;
     PrefillParams prm{log_alpha, beta, S0, cu_seqlens, o, S_final, H_qk, H_v, N, T};
-    // Slice width: narrow slices (more CTAs) when there are few (sequence, head) units.
-    const long long units = (long long)N * H_v;
+    // Slice width: one CTA per SM at most (each holds ~190 KB of shared memory), so
+    // split the head into four 32-column slices only when that still fits in one
+    // wave; otherwise two 64-column slices (half the redundant per-chunk work).
+    int num_sms = 148, dev = 0;
+    if (cudaGetDevice(&dev) == cudaSuccess)
+        cudaDeviceGetAttribute(&num_sms, cudaDevAttrMultiProcessorCount, dev);
+    const bool narrow = (long long)N * H_v * 4 <= num_sms;
     if (bf16) {
-        if (units * 2 >= 148) return launch_ns<64, __nv_bfloat16>(mq, mk, mv, prm, N, stream);
+        if (!narrow) return launch_ns<64, __nv_bfloat16>(mq, mk, mv, prm, N, stream);
         return launch_ns<32, __nv_bfloat16>(mq, mk, mv, prm, N, stream);
     }
-    if (units * 2 >= 148) return launch_ns<64, float>(mq, mk, mv, prm, N, stream);
+    if (!narrow) return launch_ns<64, float>(mq, mk, mv, prm, N, stream);
     return launch_ns<32, float>(mq, mk, mv, prm, N, stream);
 }
 
