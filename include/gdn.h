@@ -101,6 +101,39 @@ GDN_API size_t gdn_prefill_workspace_size(int32_t N, int32_t T, int32_t H_qk, in
                                   int32_t dk, int32_t dv, gdn_dtype io_dtype);
 
 /*
+ * gdn_prefill_noalloc -- gdn_prefill for callers that cannot allocate device
+ * memory.  (No counterpart in the paper: this is an interface convenience.)
+ *
+ * Some callers can't call cudaMalloc: plug-ins run inside a server or framework
+ * that owns all device memory through its own pool and hands each operator only
+ * its input and output tensors, or latency-critical loops where an allocation
+ * (which may synchronise the device or fail on a fragmented heap) is not
+ * allowed.  This entry point takes the same arguments as gdn_prefill minus the
+ * workspace and allocates nothing: the scratch it needs (bf16 copies of q, k, v
+ * when io_dtype is GDN_F32; none for GDN_BF16) lives in a fixed device array
+ * inside the library, of gdn_prefill_noalloc_max_scratch_bytes() bytes
+ * (16 MiB), which every GPU that loads the library holds until the process
+ * exits.  Calls whose scratch would exceed it return GDN_ERR_WORKSPACE and
+ * launch nothing; use gdn_prefill with a caller-owned workspace instead.
+ *
+ * The first call on each device looks up the array's device address
+ * (cudaGetSymbolAddress, with that device current); make that first call
+ * before any stream capture.  All calls share the one array, which keeps the
+ * last call's contents: calls that may overlap on the GPU (different streams
+ * without ordering between them) race on it.  Results and errors are otherwise
+ * those of gdn_prefill.
+ */
+GDN_API gdn_status gdn_prefill_noalloc(const void *q, const void *k, const void *v,
+                               const float *log_alpha, const float *beta,
+                               const float *S0, const int32_t *cu_seqlens,
+                               int32_t N, int32_t T, int32_t H_qk, int32_t H_v,
+                               int32_t dk, int32_t dv, gdn_dtype io_dtype,
+                               void *o, float *S_final, void *stream);
+
+/* Size in bytes of the fixed scratch array behind gdn_prefill_noalloc. */
+GDN_API size_t gdn_prefill_noalloc_max_scratch_bytes(void);
+
+/*
  * gdn_decode_step -- advance B independent sequences by one token each.
  *
  *   q, k [B, H_qk, dk], v [B, H_v, dv] (io_dtype); log_alpha, beta [B, H_v] fp32.

@@ -109,6 +109,24 @@ gdn_status gdn_prefill(const void* q, const void* k, const void* v, const float*
     return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
 }
 
+gdn_status gdn_prefill_noalloc(const void* q, const void* k, const void* v,
+                               const float* log_alpha, const float* beta, const float* S0,
+                               const int32_t* cu_seqlens, int32_t N, int32_t T, int32_t H_qk,
+                               int32_t H_v, int32_t dk, int32_t dv, gdn_dtype io_dtype, void* o,
+                               float* S_final, void* stream) {
+    // The scratch this call needs is the workspace gdn_prefill would take; it
+    // comes from the library's fixed device array instead of the caller.
+    const size_t need = gdn_prefill_workspace_size(N, T, H_qk, H_v, dk, dv, io_dtype);
+    if (need > gdn::noalloc_scratch_bytes()) return GDN_ERR_WORKSPACE;
+    void* scratch = nullptr;
+    if (need > 0 && gdn::noalloc_scratch_address(&scratch) != cudaSuccess) return GDN_ERR_CUDA;
+    return gdn_prefill(q, k, v, log_alpha, beta, S0, cu_seqlens, N, T, H_qk, H_v, dk, dv,
+                       io_dtype, o, S_final, scratch, need > 0 ? gdn::noalloc_scratch_bytes() : 0,
+                       stream);
+}
+
+size_t gdn_prefill_noalloc_max_scratch_bytes(void) { return gdn::noalloc_scratch_bytes(); }
+
 gdn_status gdn_decode_step(const void* q, const void* k, const void* v, const float* log_alpha,
                            const float* beta, float* S_inout, int32_t B, int32_t H_qk,
                            int32_t H_v, int32_t dk, int32_t dv, gdn_dtype io_dtype, void* o,

@@ -21,4 +21,9 @@ cudaError_t launch_prefill(const void* q, const void* k, const void* v, const fl
 
 cudaError_t read_and_clear_status(unsigned int* status, cudaStream_t stream);
 
+// Fixed-size device scratch used by gdn_prefill_noalloc (bytes, and its address
+// on the current device; the address is looked up once per device).
+size_t noalloc_scratch_bytes();
+cudaError_t noalloc_scratch_address(void** out);
+
 }  // namespace gdn

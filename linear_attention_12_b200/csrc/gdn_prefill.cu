@@ -626,6 +626,35 @@ cudaError_t launch_ns(const CUtensorMap& mq, const CUtensorMap& mk, const CUtens
 
 }  // namespace
 
+// ---- scratch for gdn_prefill_noalloc -------------------------------------
+// A file-scope device array that stands in for the caller's workspace (the bf16
+// copies of fp32 q, k, v).  Every GPU that loads the library holds it until the
+// process exits.  Its host-side name is not a device address: the address is
+// obtained once per device with cudaGetSymbolAddress, with that device current.
+constexpr size_t kNoAllocScratchBytes = size_t(16) << 20;  // 16 MiB
+static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];
+
+size_t noalloc_scratch_bytes() { return kNoAllocScratchBytes; }
+
+cudaError_t noalloc_scratch_address(void** out) {
+    constexpr int kMaxDevices = 64;
+    static std::mutex mu;
+    static void* addr[kMaxDevices] = {};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lock(mu);
+    if (!addr[dev]) {
+        void* p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+        if (e != cudaSuccess) return e;
+        addr[dev] = p;
+    }
+    *out = addr[dev];
+    return cudaSuccess;
+}
+
 size_t prefill_workspace_bytes(int N, int T, int H_qk, int H_v, bool bf16) {
     (void)N;
     if (bf16) return 0;

@@ -32,6 +32,12 @@ SIGNATURES = {
                                _c.c_int32, _c.c_int32, _c.c_int32, _c.c_int, _c.c_void_p,
                                _c.c_void_p, _c.c_void_p, _c.c_size_t, _c.c_void_p]),
     "gdn_prefill_workspace_size": (_c.c_size_t, [_c.c_int32] * 6 + [_c.c_int]),
+    "gdn_prefill_noalloc": (_c.c_int, [_c.c_void_p, _c.c_void_p, _c.c_void_p, _c.c_void_p,
+                                       _c.c_void_p, _c.c_void_p, _c.c_void_p, _c.c_int32,
+                                       _c.c_int32, _c.c_int32, _c.c_int32, _c.c_int32,
+                                       _c.c_int32, _c.c_int, _c.c_void_p, _c.c_void_p,
+                                       _c.c_void_p]),
+    "gdn_prefill_noalloc_max_scratch_bytes": (_c.c_size_t, []),
     "gdn_decode_step": (_c.c_int, [_c.c_void_p, _c.c_void_p, _c.c_void_p, _c.c_void_p,
                                    _c.c_void_p, _c.c_void_p, _c.c_int32, _c.c_int32, _c.c_int32,
                                    _c.c_int32, _c.c_int32, _c.c_int, _c.c_void_p, _c.c_void_p]),

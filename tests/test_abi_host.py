@@ -116,3 +116,18 @@ def test_binding_has_no_cpu_fallback():
     src = open(os.path.join(ROOT, "linear_attention_12_b200", "gdn.py")).read()
     assert "oracle" not in src
     assert "import numpy" not in src
+
+
+def test_noalloc_rejects_scratch_beyond_its_maximum_on_host(L):
+    """The no-allocation prefill refuses, before any CUDA call, a call whose
+    scratch would exceed its fixed array."""
+    cap = L.gdn_prefill_noalloc_max_scratch_bytes()
+    assert cap == 16 << 20
+    T = cap // ((2 * 16 + 48) * 128 * 2) + 64
+    st = L.gdn_prefill_noalloc(P, P, P, P, P, None, P, 1, T, 16, 48, 128, 128, gdn.GDN_F32,
+                               P, None, None)
+    assert st == gdn.GDN_ERR_WORKSPACE
+    # invalid arguments are still rejected by the prefill's own checks
+    st = L.gdn_prefill_noalloc(None, P, P, P, P, None, P, 1, 64, 1, 1, 128, 128, gdn.GDN_BF16,
+                               P, None, None)
+    assert st == gdn.GDN_ERR_INVALID_ARG
