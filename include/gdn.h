@@ -83,7 +83,12 @@ typedef enum {
  *               between outputs and inputs is allowed.
  *   workspace : device scratch of at least gdn_prefill_workspace_size(...)
  *               bytes (may be NULL when that size is 0), owned by the caller
- *               and not used after the work on `stream` completes.
+ *               and not used after the work on `stream` completes.  It holds
+ *               one 16,912-byte "chunk operator" record per (chunk slot, value
+ *               head) -- N + ceil(T / 64) slots; about 416 MB for T = 32,768
+ *               and 48 value heads -- written by the first of the two passes
+ *               of the prefill and read by the second, plus bf16 copies of
+ *               q, k, v when io_dtype is GDN_F32.
  *
  * Returns GDN_OK, GDN_ERR_INVALID_ARG, GDN_ERR_UNSUPPORTED, GDN_ERR_WORKSPACE
  * or GDN_ERR_CUDA.
@@ -96,7 +101,8 @@ GDN_API gdn_status gdn_prefill(const void *q, const void *k, const void *v,
                        void *o, float *S_final,
                        void *workspace, size_t workspace_bytes, void *stream);
 
-/* Bytes of device workspace gdn_prefill needs for these sizes (0 when none). */
+/* Bytes of device workspace gdn_prefill needs for these sizes (0 when T == 0
+ * or the arguments are invalid). */
 GDN_API size_t gdn_prefill_workspace_size(int32_t N, int32_t T, int32_t H_qk, int32_t H_v,
                                   int32_t dk, int32_t dv, gdn_dtype io_dtype);
 
@@ -109,8 +115,8 @@ GDN_API size_t gdn_prefill_workspace_size(int32_t N, int32_t T, int32_t H_qk, in
  * its input and output tensors, or latency-critical loops where an allocation
  * (which may synchronise the device or fail on a fragmented heap) is not
  * allowed.  This entry point takes the same arguments as gdn_prefill minus the
- * workspace and allocates nothing: the scratch it needs (bf16 copies of q, k, v
- * when io_dtype is GDN_F32; none for GDN_BF16) lives in a fixed device array
+ * workspace and allocates nothing: the scratch it needs (what
+ * gdn_prefill_workspace_size reports for the same sizes) lives in a fixed device array
  * inside the library, of gdn_prefill_noalloc_max_scratch_bytes() bytes
  * (16 MiB), which every GPU that loads the library holds until the process
  * exits.  Calls whose scratch would exceed it return GDN_ERR_WORKSPACE and

@@ -78,11 +78,16 @@ size_t gdn_prefill_workspace_size(int32_t N, int32_t T, int32_t H_qk, int32_t H_
     return gdn::prefill_workspace_bytes(N, T, H_qk, H_v, io_dtype == GDN_BF16);
 }
 
-gdn_status gdn_prefill(const void* q, const void* k, const void* v, const float* log_alpha,
-                       const float* beta, const float* S0, const int32_t* cu_seqlens, int32_t N,
-                       int32_t T, int32_t H_qk, int32_t H_v, int32_t dk, int32_t dv,
-                       gdn_dtype io_dtype, void* o, float* S_final, void* workspace,
-                       size_t workspace_bytes, void* stream) {
+}  // extern "C"
+
+namespace {
+
+// Every host-side check of a prefill call except the workspace.
+gdn_status check_prefill_args(const void* q, const void* k, const void* v, const float* log_alpha,
+                              const float* beta, const float* S0, const int32_t* cu_seqlens,
+                              int32_t N, int32_t T, int32_t H_qk, int32_t H_v, int32_t dk,
+                              int32_t dv, gdn_dtype io_dtype, const void* o,
+                              const float* S_final) {
     gdn_status st = check_heads(H_qk, H_v, dk, dv, io_dtype);
     if (st != GDN_OK) return st;
     if (N <= 0 || T < 0) return GDN_ERR_INVALID_ARG;
@@ -97,6 +102,21 @@ gdn_status gdn_prefill(const void* q, const void* k, const void* v, const float*
             return GDN_ERR_INVALID_ARG;
     }
     if ((S0 && !aligned(S0, 16)) || (S_final && !aligned(S_final, 16))) return GDN_ERR_INVALID_ARG;
+    return GDN_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+gdn_status gdn_prefill(const void* q, const void* k, const void* v, const float* log_alpha,
+                       const float* beta, const float* S0, const int32_t* cu_seqlens, int32_t N,
+                       int32_t T, int32_t H_qk, int32_t H_v, int32_t dk, int32_t dv,
+                       gdn_dtype io_dtype, void* o, float* S_final, void* workspace,
+                       size_t workspace_bytes, void* stream) {
+    gdn_status st = check_prefill_args(q, k, v, log_alpha, beta, S0, cu_seqlens, N, T, H_qk, H_v,
+                                       dk, dv, io_dtype, o, S_final);
+    if (st != GDN_OK) return st;
     const bool bf16 = io_dtype == GDN_BF16;
     const size_t need = gdn::prefill_workspace_bytes(N, T, H_qk, H_v, bf16);
     if (need > 0 && (!workspace || workspace_bytes < need || !aligned(workspace, 256)))
@@ -114,6 +134,9 @@ gdn_status gdn_prefill_noalloc(const void* q, const void* k, const void* v,
                                const int32_t* cu_seqlens, int32_t N, int32_t T, int32_t H_qk,
                                int32_t H_v, int32_t dk, int32_t dv, gdn_dtype io_dtype, void* o,
                                float* S_final, void* stream) {
+    gdn_status st = check_prefill_args(q, k, v, log_alpha, beta, S0, cu_seqlens, N, T, H_qk, H_v,
+                                       dk, dv, io_dtype, o, S_final);
+    if (st != GDN_OK) return st;
     // The scratch this call needs is the workspace gdn_prefill would take; it
     // comes from the library's fixed device array instead of the caller.
     const size_t need = gdn_prefill_workspace_size(N, T, H_qk, H_v, dk, dv, io_dtype);

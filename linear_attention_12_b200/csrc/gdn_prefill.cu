@@ -1,6 +1,10 @@
-// gdn_prefill.cu -- chunked GDN prefill (sm_100a): TMA tile loads, warp-level
-// bf16 tensor-core products (ldmatrix + mma.sync m16n8k16, fp32 accumulate),
-// fp32 triangular solve on CUDA cores, state resident in registers.
+// gdn_prefill.cu -- chunked GDN prefill (sm_100a) in two kernels: a fully
+// parallel pass over all chunks that computes each chunk's state-independent
+// operators, and a sequential pass that carries the state through the chunks.
+// Both use TMA / bulk copies into 128-byte-swizzled shared-memory tiles and
+// warp-level bf16 tensor-core products (ldmatrix + mma.sync m16n8k16, fp32
+// accumulate); the triangular solve runs in fp32 (tf32 tensor-core block
+// products); the state stays in registers for the whole sequence.
 //
 // Operation: the gated delta rule of the bjdmk.com.cn article (section 2.1,
 // state-update formula) over packed sequences, with readout o_t = S_t^T q_t.
@@ -8,28 +12,36 @@
 // representation but prints no formulas; the chunk algebra used here is
 // derived from the recurrence itself.  For a chunk of C = 64 tokens with entry
 // state S (d_k x d_v), cumulative log-gates g_r = sum_{i<=r} log alpha_i,
-// gamma_r = exp(g_r):
+// gamma_r = exp(g_r), d_r = exp(g_C - g_r) (zero past the sequence end):
 //
-//   A_rj  = beta_r exp(g_r - g_j) (k_r . k_j)  for j < r     (strictly lower)
-//   T     = (I + A)^{-1}                                      (unit lower)
-//   W     = T diag(beta gamma) K,   U = T diag(beta) V
-//   Delta = U - W S                                           (true write vectors)
-//   O     = diag(gamma) Q S + (M o Q K^T) Delta,  M_rj = exp(g_r - g_j), j <= r
-//   S    <- gamma_C S + K^T diag(exp(g_C - g_j)) Delta
+//   A     = strict_lower( diag(beta) (M o K K^T) ),  M_rj = exp(g_r - g_j)
+//   T     = (I + A)^{-1},   T_b = T diag(beta)                 (unit lower / lower)
+//   X     = V - diag(gamma) K S
+//   Delta = T_b X                                              (true write vectors)
+//   O     = diag(gamma) Q S + (M o Q K^T) Delta
+//   S    <- gamma_C S + K^T diag(d) Delta
 //
-// Work split: one CTA per (sequence, value head, d_v slice of NS columns);
-// the columns of S evolve independently, so slices need no communication.
-// Each math warp keeps 16 rows x NS columns of S as fp32 mma accumulators for
-// the whole sequence.
+// (Delta equals U - W S of the WY form with U = T_b V and W = T_b diag(gamma) K.)
 //
-// Roles (288 threads): warps 0-7 are the math warps; warp 8 is the TMA
-// producer, which streams K, Q (64 x 128 bf16 each) and the V slice (64 x 64
-// bf16) of every chunk into a 2-stage ring of 128-byte-swizzled tiles.  Every
-// operand tile in shared memory uses that swizzle (16-byte chunk c of row r
-// stored at chunk c ^ (r % 8)), so ldmatrix reads are bank-conflict free.
+// Pass 1, chunk_ops_kernel: one CTA per (chunk, query/key head).  Both grams
+// K K^T and Q K^T (lower 16x16 blocks only) are computed once and shared by
+// the value heads of that query/key head; per value head the CTA builds the
+// masks, solves for T and writes one "chunk operator" record to the
+// workspace: T_b and M o Q K^T as 128-byte-swizzled bf16 tiles plus gamma, d
+// and gamma_C.  A record is written by one bulk copy and read by one.
 //
-// Every mbarrier wait is bounded (gdn_common.cuh); on a timeout the CTA
-// records the error in the device status word, lets its copies land and exits.
+// Pass 2, state_pass_kernel: one CTA per (sequence, value head, d_v slice of
+// NS columns); the columns of S evolve independently, so slices need no
+// communication.  Eight warps each own 16 rows of S as fp32 mma accumulators;
+// warps 0-3 compute K S and Q S (one pass over S) and the output rows; all
+// eight compute Delta and update the state.  One thread streams each chunk's K, Q, V tiles and
+// operator record into a 3-stage ring, refilling a stage as soon as the chain
+// releases it.
+//
+// Every mbarrier wait is bounded (gdn_common.cuh); every named barrier inside
+// the chunk loop also votes on whether all of its threads are still healthy,
+// so a timeout makes the CTA leave the loop together, drain its in-flight
+// copies (bounded) and exit.
 #include <cudaTypedefs.h>
 
 #include <mutex>
@@ -41,55 +53,65 @@ namespace gdn {
 
 namespace {
 
-constexpr int C = 64;           // chunk length
-constexpr int D = 128;          // head dim (d_k = d_v)
-constexpr int NSTAGE = 2;       // TMA ring depth
-constexpr int kMathWarps = 8;
-constexpr int kMathThreads = kMathWarps * 32;
-constexpr int kThreads = kMathThreads + 32;
+constexpr int C = 64;            // chunk length
+constexpr int D = 128;           // head dim (d_k = d_v)
+constexpr uint32_t HALF = 8192;  // one 64 x 64 bf16 tile: 64 rows x 128 B
+constexpr float LOG2E = 1.4426950408889634f;
 
-// ---- shared memory layout (byte offsets from a 1024-aligned base) ----
-// ring stage: K (two 64-column halves, 8 KB each), Q (same), V slice (8 KB)
-constexpr uint32_t HALF = 8192;                        // 64 rows x 128 B
-constexpr uint32_t ST_K = 0, ST_Q = 2 * HALF, ST_V = 4 * HALF;
-constexpr uint32_t STAGE_BYTES = 5 * HALF;
-constexpr uint32_t OFF_RING = 0;
-constexpr uint32_t OFF_TBG = OFF_RING + NSTAGE * STAGE_BYTES;  // T diag(beta gamma), 64x64
-constexpr uint32_t OFF_TB = OFF_TBG + HALF;                    // T diag(beta), 64x64
-constexpr uint32_t OFF_MQ = OFF_TB + HALF;                     // (M o Q K^T), 64x64
-constexpr uint32_t OFF_W = OFF_MQ + HALF;                      // -W, 64x128 (two halves)
-constexpr uint32_t OFF_SB = OFF_W + 2 * HALF;                  // S in bf16, 128 x 64
-constexpr uint32_t OFF_DU = OFF_SB + 2 * HALF;                 // Delta, 64 x 64
-constexpr uint32_t OFF_DD = OFF_DU + HALF;                     // d o Delta, 64 x 64
-constexpr uint32_t OFF_AF = OFF_DD + HALF;                     // A in fp32, 64 x 68
-constexpr int AF_LD = 68;
-constexpr uint32_t OFF_TF = OFF_AF + 64 * AF_LD * 4;           // T in fp32, 64 x 68
-constexpr uint32_t OFF_XS = OFF_TF + 64 * AF_LD * 4;           // 3 x 16 x 16 fp32 scratch
-constexpr uint32_t OFF_VEC = OFF_XS + 3 * 256 * 4;             // g, beta, gamma, dscale, carry
-constexpr uint32_t OFF_BAR = OFF_VEC + 5 * 64 * 4;
-constexpr int NBAR = 2 * NSTAGE;                               // full[2], empty[2]
-constexpr uint32_t OFF_MISC = OFF_BAR + NBAR * 8;              // abort flag
-constexpr uint32_t SMEM_USED = OFF_MISC + 16;
-constexpr uint32_t SMEM_ALLOC = SMEM_USED + 1024;              // slack for 1024-byte alignment
-static_assert(SMEM_ALLOC <= 232448, "shared memory budget");
+// ---- chunk operator record (workspace), also its image in shared memory ----
+constexpr uint32_t REC_TB = 0;                 // T diag(beta), 64 x 64 bf16, swizzled
+constexpr uint32_t REC_MQ = HALF;              // M o Q K^T,    64 x 64 bf16, swizzled
+constexpr uint32_t REC_VEC = 2 * HALF;         // gamma[64], d[64], gamma_C, pad -> 132 floats
+constexpr uint32_t REC_VEC_FLOATS = 132;
+constexpr uint32_t REC_BYTES = REC_VEC + REC_VEC_FLOATS * 4;  // 16,912
+static_assert(REC_BYTES % 16 == 0, "bulk copies move multiples of 16 bytes");
 
-enum Bar { B_FULL = 0, B_EMPTY = NSTAGE };
-
-#ifdef GDN_DEBUG_TRACE
-__device__ volatile int* g_trace = nullptr;
-__device__ __forceinline__ void trace_mark(int role, int phase, int c) {
-    volatile int* t = g_trace;
-    if (t) {
-        const int cta = blockIdx.x + gridDim.x * (blockIdx.y + gridDim.y * blockIdx.z);
-        if (cta < 1024) t[cta * 4 + role] = (phase << 20) | (c & 0xFFFFF);
-        __threadfence_system();
-    }
+// Record slot of chunk c of sequence n (first token t0 = cu[n] + 64 c):
+// j = n + floor(t0 / 64).  Distinct chunks get distinct slots, all below
+// N + ceil(T / 64), without reading cu_seqlens on the host.
+__host__ __device__ __forceinline__ long long record_slot(int n, int t0) {
+    return (long long)n + t0 / C;
 }
-#define TRACE_T(tid, role, phase, c) \
-    do { if (threadIdx.x == (tid)) trace_mark(role, phase, c); } while (0)
-#else
-#define TRACE_T(tid, role, phase, c) ((void)0)
-#endif
+
+// ---- pass 1 shared memory ----
+constexpr int P1_THREADS = 256;
+constexpr int AF_LD = 68;                                      // fp32 row stride of A and T
+constexpr int XS_LD16 = 24, XS_LD32 = 40;                      // solve scratch strides
+constexpr uint32_t P1_K = 0;                                   // K, 64 x 128 (two halves)
+constexpr uint32_t P1_Q = 2 * HALF;                            // Q
+constexpr uint32_t P1_REC = 4 * HALF;                          // two record buffers
+constexpr uint32_t P1_REC_STRIDE = 17408;                      // REC_BYTES rounded to 1 KB
+constexpr uint32_t P1_AF = P1_REC + 2 * P1_REC_STRIDE;         // A, fp32 64 x 68
+constexpr uint32_t P1_TF = P1_AF + 64 * AF_LD * 4;             // T, fp32 64 x 68
+constexpr uint32_t P1_XS = P1_TF + 64 * AF_LD * 4;             // 1280 floats
+constexpr uint32_t P1_VEC = P1_XS + 32 * XS_LD32 * 4;          // per value head: g[64], beta[64]
+constexpr int P1_MAX_GROUP = 4;                                // value heads per query/key head
+constexpr uint32_t P1_BAR = P1_VEC + P1_MAX_GROUP * 128 * 4;
+constexpr uint32_t P1_MISC = P1_BAR + 8;
+constexpr uint32_t P1_SMEM = P1_MISC + 16 + 1024;
+static_assert(P1_REC_STRIDE >= REC_BYTES && P1_AF % 16 == 0, "pass 1 layout");
+static_assert(2 * P1_SMEM + 2048 <= 233472, "two pass-1 CTAs per SM");
+
+// ---- pass 2 shared memory ----
+constexpr int NSTAGE = 3;
+constexpr int P2_CHAIN_WARPS = 8;
+constexpr int P2_CHAIN_THREADS = P2_CHAIN_WARPS * 32;
+constexpr int P2_THREADS = P2_CHAIN_THREADS;
+constexpr int P2_LOADER = 128;                                 // thread that issues the copies
+constexpr int BAR_CHAIN = 1;
+// ring stage: K and Q (two 64-column halves each), V slice, operator record
+constexpr uint32_t ST_K = 0, ST_Q = 2 * HALF, ST_V = 4 * HALF, ST_REC = 5 * HALF;
+constexpr uint32_t STAGE_BYTES = ((ST_REC + REC_BYTES + 1023) / 1024) * 1024;
+constexpr uint32_t STAGE_TX = 5 * HALF + REC_BYTES;           // bytes landing per stage
+constexpr uint32_t P2_SB = NSTAGE * STAGE_BYTES;               // S in bf16, 128 x 64
+constexpr uint32_t P2_X = P2_SB + 2 * HALF;                    // X, 64 x 64
+constexpr uint32_t P2_DU = P2_X + HALF;                        // Delta
+constexpr uint32_t P2_DD = P2_DU + HALF;                       // d o Delta
+constexpr uint32_t P2_BAR = P2_DD + HALF;
+enum Bar2 { B2_FULL = 0, NBAR2 = NSTAGE };
+constexpr uint32_t P2_MISC = P2_BAR + NBAR2 * 8;
+constexpr uint32_t P2_SMEM = P2_MISC + 16 + 1024;
+static_assert(P2_SMEM <= 232448, "pass 2 shared memory budget");
 
 __device__ __forceinline__ float ex2(float x) {
     float y;
@@ -97,8 +119,35 @@ __device__ __forceinline__ float ex2(float x) {
     return y;
 }
 
-__device__ __forceinline__ void math_bar() {
-    asm volatile("bar.sync 1, %0;" ::"n"(kMathThreads) : "memory");
+template <int ID, int N>
+__device__ __forceinline__ void bar_sync() {
+    asm volatile("bar.sync %0, %1;" ::"n"(ID), "n"(N) : "memory");
+}
+// Named barrier that also returns the AND of every participant's `ok`.
+template <int ID, int N>
+__device__ __forceinline__ bool bar_and(bool ok) {
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred pi, po;\n\t"
+        "setp.ne.u32 pi, %1, 0;\n\t"
+        "bar.red.and.pred po, %2, %3, pi;\n\t"
+        "selp.u32 %0, 1, 0, po;\n\t}"
+        : "=r"(r)
+        : "r"((uint32_t)ok), "n"(ID), "n"(N)
+        : "memory");
+    return r != 0;
+}
+
+// Wait bounded in time only (used to drain in-flight copies after an abort).
+__device__ __forceinline__ void mbar_wait_drain(uint64_t* bar, uint32_t parity) {
+    const uint32_t addr = smem_u32(bar);
+    const unsigned long long t0 = globaltimer();
+    while (!mbar_try_wait(addr, parity)) {
+        if (globaltimer() - t0 > kWaitLimitNs) {
+            atomicOr(&g_status, GDN_DEV_TIMEOUT);
+            return;
+        }
+    }
 }
 
 // Address of element (row, col) of a 128B-swizzled tile whose 64-column
@@ -153,35 +202,30 @@ __device__ __forceinline__ void ldb_mn(uint32_t base, uint32_t half, int n0, int
     ldsm_x4_t(taddr(base, k0 + (lane & 7) + ((j & 1) << 3), n0 + ((j >> 1) << 3), half), b);
 }
 
-// acc[NT][4] += A(16 x 16*KS) * B(16*KS x 8*NT)
-template <int NT, int KS, bool A_MN, bool B_MN>
-__device__ __forceinline__ void warp_gemm(float (*acc)[4], uint32_t a_base, uint32_t a_half,
-                                          int m0, uint32_t b_base, uint32_t b_half, int lane) {
-    static_assert(NT % 2 == 0, "n-tiles come in pairs");
-#pragma unroll
-    for (int ks = 0; ks < KS; ++ks) {
-        uint32_t a[4];
-        if (A_MN)
-            lda_mn(a_base, a_half, m0, 16 * ks, lane, a);
-        else
-            lda_k(a_base, a_half, m0, 16 * ks, lane, a);
-#pragma unroll
-        for (int np = 0; np < NT / 2; ++np) {
-            uint32_t b[4];
-            if (B_MN)
-                ldb_mn(b_base, b_half, 16 * np, 16 * ks, lane, b);
-            else
-                ldb_k(b_base, b_half, 16 * np, 16 * ks, lane, b);
-            mma16816(acc[2 * np], a, b[0], b[1]);
-            mma16816(acc[2 * np + 1], a, b[2], b[3]);
-        }
-    }
-}
-
 __device__ __forceinline__ uint32_t pack2(float lo, float hi) { return pack_bf16x2(lo, hi); }
 
-// Store an accumulator tile (rows m0.., NT n-tiles) as bf16 into a swizzled tile
-// (rows = accumulator rows), scaled per row by rs_lo (row g) and rs_hi (row g+8).
+__device__ __forceinline__ uint32_t to_tf32(float x) {
+    uint32_t r;
+    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+    return r;
+}
+// D += A (16 x 8, fp32 rows of stride lda) * B (8 x 8, fp32 rows of stride ldb), both
+// rounded to tf32, fp32 accumulate (m16n8k8).
+__device__ __forceinline__ void mma_tf32(float* d, const float* A, int lda, const float* B,
+                                         int ldb, int lane) {
+    const int g = lane >> 2, t = lane & 3;
+    const uint32_t a0 = to_tf32(A[g * lda + t]), a1 = to_tf32(A[(g + 8) * lda + t]);
+    const uint32_t a2 = to_tf32(A[g * lda + t + 4]), a3 = to_tf32(A[(g + 8) * lda + t + 4]);
+    const uint32_t b0 = to_tf32(B[t * ldb + g]), b1 = to_tf32(B[(t + 4) * ldb + g]);
+    asm volatile(
+        "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 "
+        "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// Store an accumulator tile (rows m0.., NT n-tiles from column 0) as bf16 into a
+// swizzled tile, scaled per row by rs_lo (row g) and rs_hi (row g+8).
 template <int NT>
 __device__ __forceinline__ void store_acc_bf16(uint8_t* smem, uint32_t base_off, uint32_t half,
                                                int m0, const float (*acc)[4], int lane,
@@ -197,17 +241,6 @@ __device__ __forceinline__ void store_acc_bf16(uint8_t* smem, uint32_t base_off,
     }
 }
 
-struct PrefillParams {
-    const float* log_alpha;
-    const float* beta;
-    const float* S0;
-    const int32_t* cu_seqlens;
-    void* o;
-    float* S_final;
-    int H_qk, H_v;
-    int N, T;
-};
-
 template <typename IO>
 __device__ __forceinline__ void store2(IO* p, float a, float b);
 template <>
@@ -219,82 +252,416 @@ __device__ __forceinline__ void store2<__nv_bfloat16>(__nv_bfloat16* p, float a,
     *reinterpret_cast<uint32_t*>(p) = pack2(a, b);
 }
 
-template <int NS, typename IO>
-__global__ void __launch_bounds__(kThreads, 1)
-    prefill_kernel(const __grid_constant__ CUtensorMap map_q,
-                   const __grid_constant__ CUtensorMap map_k,
-                   const __grid_constant__ CUtensorMap map_v, const PrefillParams p) {
-    static_assert(NS == 32 || NS == 64, "slice width");
-    constexpr int NT = NS / 8;  // n-tiles of a slice
+struct PrefillParams {
+    const float* log_alpha;
+    const float* beta;
+    const float* S0;
+    const int32_t* cu_seqlens;
+    void* o;
+    float* S_final;
+    uint8_t* records;  // chunk operator records, REC_BYTES each
+    int H_qk, H_v;
+    int N, T;
+};
+
+// Sequence n and chunk c of record slot j, or n = -1 if no chunk maps to j.
+// The first slot of sequence n, n + floor(cu[n] / 64), increases strictly with
+// n, so the owner of j is the last sequence whose first slot is <= j.
+__device__ __forceinline__ void slot_owner(const int32_t* cu, int N, int j, int& n, int& c) {
+    int lo = 0, hi = N - 1;
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (record_slot(mid, cu[mid]) <= j) lo = mid; else hi = mid - 1;
+    }
+    n = lo;
+    c = j - (int)record_slot(lo, cu[lo]);
+    const int nch = (cu[lo + 1] - cu[lo] + C - 1) / C;
+    if (c < 0 || c >= nch) n = -1;
+}
+
+// ============================================================================
+// Pass 1: chunk operators.  Grid (record slots, H_qk, value-head batches of 4).
+// ============================================================================
+__global__ void __launch_bounds__(P1_THREADS, 2)
+    chunk_ops_kernel(const __grid_constant__ CUtensorMap map_q,
+                     const __grid_constant__ CUtensorMap map_k, const PrefillParams p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
     const uint32_t sb = smem_u32(sm);
-    uint64_t* bars = reinterpret_cast<uint64_t*>(sm + OFF_BAR);
-    volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + OFF_MISC);
-    float* s_g = reinterpret_cast<float*>(sm + OFF_VEC);  // g_r * log2(e)
-    float* s_b = s_g + 64;                                // beta_r (0 past the end)
-    float* s_gam = s_g + 128;                             // gamma_r
-    float* s_ds = s_g + 192;                              // exp(g_C - g_r)
-    float* s_carry = s_g + 256;
+    uint64_t* bar = reinterpret_cast<uint64_t*>(sm + P1_BAR);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + P1_MISC);
+    float* Af = reinterpret_cast<float*>(sm + P1_AF);
+    float* Tf = reinterpret_cast<float*>(sm + P1_TF);
+    float* Xs = reinterpret_cast<float*>(sm + P1_XS);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int g = lane >> 2, t4 = lane & 3;
+    const int pt = threadIdx.x;
+    int n, c;
+    slot_owner(p.cu_seqlens, p.N, blockIdx.x, n, c);
+    if (n < 0) return;  // uniform across the CTA
+    const int hq = blockIdx.y;
+    const int group = p.H_v / p.H_qk;
+    const int hv0 = hq * group + blockIdx.z * P1_MAX_GROUP;
+    const int nheads = min(P1_MAX_GROUP, group - blockIdx.z * P1_MAX_GROUP);
+    const int t_end = p.cu_seqlens[n + 1];
+    const int t0 = p.cu_seqlens[n] + c * C;
+    const int valid = min(C, t_end - t0);
+    const long long slot = record_slot(n, t0);
+
+    if (pt == 0) {
+        mbar_init(bar, 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    __syncthreads();
+    if (pt == 0) {
+        mbar_arrive_expect_tx(bar, 4 * HALF);
+        tma_load_2d(sm + P1_K, &map_k, hq * D, t0, bar);
+        tma_load_2d(sm + P1_K + HALF, &map_k, hq * D + 64, t0, bar);
+        tma_load_2d(sm + P1_Q, &map_q, hq * D, t0, bar);
+        tma_load_2d(sm + P1_Q + HALF, &map_q, hq * D + 64, t0, bar);
+    }
+    // decay scan per value head: warp w < nheads handles head hv0 + w
+    // (lane l: tokens 2l, 2l+1); T's upper blocks are zeroed meanwhile
+    if (warp < nheads) {
+        const int h = hv0 + warp;
+        float la[2] = {0.f, 0.f}, be[2] = {0.f, 0.f};
+#pragma unroll
+        for (int e = 0; e < 2; ++e)
+            if (2 * lane + e < valid) {
+                la[e] = p.log_alpha[(size_t)(t0 + 2 * lane + e) * p.H_v + h];
+                be[e] = p.beta[(size_t)(t0 + 2 * lane + e) * p.H_v + h];
+            }
+        const float x0 = la[0] * LOG2E, x1 = la[1] * LOG2E;
+        float incl = x0 + x1;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const float y = __shfl_up_sync(0xffffffffu, incl, off);
+            if (lane >= off) incl += y;
+        }
+        float* v = reinterpret_cast<float*>(sm + P1_VEC) + warp * 128;
+        *reinterpret_cast<float2*>(v + 2 * lane) = make_float2(incl - x1, incl);
+        *reinterpret_cast<float2*>(v + 64 + 2 * lane) = make_float2(be[0], be[1]);
+    }
+    for (int i = pt; i < 64 * AF_LD / 4; i += P1_THREADS)
+        reinterpret_cast<float4*>(Tf)[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+    const bool ok = mbar_wait(bar, 0, abort_flag);
+    __syncwarp();
+    if (!__syncthreads_and(ok)) {
+        // the copy may still land: wait for it (bounded) before the CTA exits
+        if (pt == 0) mbar_wait_drain(bar, 0);
+        __syncthreads();
+        return;
+    }
+    if (valid < C) {  // zero K and Q rows past the end of the sequence
+        for (int i = pt; i < 4 * 64 * 8; i += P1_THREADS) {
+            const int tile = i / 512, row = (i >> 3) & 63, ch = i & 7;
+            if (row >= valid)
+                *reinterpret_cast<uint4*>(sm + tile * HALF + row * 128 + ch * 16) =
+                    make_uint4(0, 0, 0, 0);
+        }
+        __syncthreads();
+    }
+
+    // ---- grams, lower 16x16 blocks only.  Warp: type (0: K K^T, 1: Q K^T) and
+    // up to three blocks (bi, bj), sorted by bi.
+    const int gtype = warp & 1;
+    int nblk, bi0, bj0, bi1, bj1, bi2, bj2;
+    switch (warp >> 1) {
+        case 0: nblk = 2; bi0 = 3; bj0 = 0; bi1 = 3; bj1 = 1; bi2 = 3; bj2 = 1; break;
+        case 1: nblk = 2; bi0 = 3; bj0 = 2; bi1 = 3; bj1 = 3; bi2 = 3; bj2 = 3; break;
+        case 2: nblk = 3; bi0 = 2; bj0 = 0; bi1 = 2; bj1 = 1; bi2 = 2; bj2 = 2; break;
+        default: nblk = 3; bi0 = 1; bj0 = 0; bi1 = 1; bj1 = 1; bi2 = 0; bj2 = 0; break;
+    }
+    const int gbi[3] = {bi0, bi1, bi2};
+    const int gbj[3] = {bj0, bj1, bj2};
+    float acc[3][2][4];
+#pragma unroll
+    for (int b = 0; b < 3; ++b)
+#pragma unroll
+        for (int i = 0; i < 2; ++i)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) acc[b][i][e] = 0.f;
+    {
+        const uint32_t abase = sb + (gtype ? P1_Q : P1_K);
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks) {
+            uint32_t a[4];
+#pragma unroll
+            for (int b = 0; b < 3; ++b) {
+                if (b < nblk) {
+                    if (b == 0 || gbi[b] != gbi[b - 1])
+                        lda_k(abase, HALF, 16 * gbi[b], 16 * ks, lane, a);
+                    uint32_t bb[4];
+                    ldb_k(sb + P1_K, HALF, 16 * gbj[b], 16 * ks, lane, bb);
+                    mma16816(acc[b][0], a, bb[0], bb[1]);
+                    mma16816(acc[b][1], a, bb[2], bb[3]);
+                }
+            }
+        }
+    }
+
+    for (int vh = 0; vh < nheads; ++vh) {
+        const int h = hv0 + vh;
+        const float* s_g = reinterpret_cast<const float*>(sm + P1_VEC) + vh * 128;
+        const float* s_b = s_g + 64;
+        uint8_t* rec = sm + P1_REC + (vh & 1) * P1_REC_STRIDE;
+        if (vh >= 2) {  // the record buffer's previous bulk store must have read it
+            if (pt == 0) bulk_wait_read<1>();
+            __syncthreads();
+        }
+        // ---- masks: A -> Af (fp32), M o Q K^T -> the record (bf16)
+#pragma unroll
+        for (int b = 0; b < 3; ++b) {
+            if (b < nblk) {
+#pragma unroll
+                for (int hl = 0; hl < 2; ++hl) {
+                    const int r = 16 * gbi[b] + g + 8 * hl;
+                    const float gr = s_g[r], br = s_b[r];
+#pragma unroll
+                    for (int nt = 0; nt < 2; ++nt) {
+                        const int j = 16 * gbj[b] + 8 * nt + 2 * t4;
+                        const float2 gj = *reinterpret_cast<const float2*>(s_g + j);
+                        const float x0 = acc[b][nt][2 * hl], x1 = acc[b][nt][2 * hl + 1];
+                        const float e0 = (j <= r) ? ex2(gr - gj.x) : 0.f;
+                        const float e1 = (j + 1 <= r) ? ex2(gr - gj.y) : 0.f;
+                        if (gtype == 0) {
+                            const float a0 = (j < r) ? br * e0 * x0 : 0.f;
+                            const float a1 = (j + 1 < r) ? br * e1 * x1 : 0.f;
+                            *reinterpret_cast<float2*>(Af + r * AF_LD + j) = make_float2(a0, a1);
+                        } else {
+                            *reinterpret_cast<uint32_t*>(rec + REC_MQ + taddr_e(0, r, j, 0)) =
+                                pack2(e0 * x0, e1 * x1);
+                        }
+                    }
+                }
+            }
+        }
+        __syncthreads();
+
+        // ---- T = (I + A)^{-1}, fp32.  Diagonal 16x16 blocks by forward substitution
+        // (thread = column cc of block b), then the off-diagonal blocks from tf32
+        // tensor-core block products:
+        //   T_10 = -T_11 (A_10 T_00),  T_32 = -T_33 (A_32 T_22),
+        //   T_ba = -T_bb (A_ba T_aa)   (a = rows/columns 0..31, b = 32..63)
+        if (pt < C) {
+            const int b = pt >> 4, cc = pt & 15;
+            const float* Ab = Af + (16 * b) * AF_LD + 16 * b;
+            float x[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) x[i] = (i == cc) ? 1.f : 0.f;
+#pragma unroll
+            for (int jj = 0; jj < 15; ++jj) {
+                const float xj = x[jj];
+#pragma unroll
+                for (int i = jj + 1; i < 16; ++i) x[i] = fmaf(-Ab[i * AF_LD + jj], xj, x[i]);
+            }
+#pragma unroll
+            for (int i = 0; i < 16; ++i) Tf[(16 * b + i) * AF_LD + 16 * b + cc] = x[i];
+        }
+        __syncthreads();
+        if (warp < 4) {  // X = A_10 T_00 (warps 0,1) and A_32 T_22 (warps 2,3), one n-tile each
+            const int blk = warp >> 1, nt = warp & 1, bi = 1 + 2 * blk, bj = 2 * blk;
+            float d[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int ks = 0; ks < 2; ++ks)
+                mma_tf32(d, Af + (16 * bi) * AF_LD + 16 * bj + 8 * ks, AF_LD,
+                         Tf + (16 * bj + 8 * ks) * AF_LD + 16 * bj + 8 * nt, AF_LD, lane);
+            float* xo = Xs + blk * 16 * XS_LD16 + 8 * nt + 2 * t4;
+            *reinterpret_cast<float2*>(xo + g * XS_LD16) = make_float2(d[0], d[1]);
+            *reinterpret_cast<float2*>(xo + (g + 8) * XS_LD16) = make_float2(d[2], d[3]);
+        }
+        __syncthreads();
+        if (warp < 4) {  // T_10 = -T_11 X, T_32 = -T_33 X
+            const int blk = warp >> 1, nt = warp & 1, bi = 1 + 2 * blk, bj = 2 * blk;
+            float d[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int ks = 0; ks < 2; ++ks)
+                mma_tf32(d, Tf + (16 * bi) * AF_LD + 16 * bi + 8 * ks, AF_LD,
+                         Xs + blk * 16 * XS_LD16 + 8 * ks * XS_LD16 + 8 * nt, XS_LD16, lane);
+            float* to = Tf + (16 * bi) * AF_LD + 16 * bj + 8 * nt + 2 * t4;
+            *reinterpret_cast<float2*>(to + g * AF_LD) = make_float2(-d[0], -d[1]);
+            *reinterpret_cast<float2*>(to + (g + 8) * AF_LD) = make_float2(-d[2], -d[3]);
+        }
+        __syncthreads();
+        const int qm = warp >> 2, qn = warp & 3;  // 32x32 products: m-tile qm, n-tile qn
+        {  // X = A_ba T_aa  (T_aa's upper-right 16x16 block is zero)
+            float d[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks)
+                if (qn < 2 || ks >= 2)
+                    mma_tf32(d, Af + (32 + 16 * qm) * AF_LD + 8 * ks, AF_LD,
+                             Tf + (8 * ks) * AF_LD + 8 * qn, AF_LD, lane);
+            float* xo = Xs + (16 * qm) * XS_LD32 + 8 * qn + 2 * t4;
+            *reinterpret_cast<float2*>(xo + g * XS_LD32) = make_float2(d[0], d[1]);
+            *reinterpret_cast<float2*>(xo + (g + 8) * XS_LD32) = make_float2(d[2], d[3]);
+        }
+        __syncthreads();
+        {  // T_ba = -T_bb X  (T_bb's upper-right 16x16 block is zero)
+            float d[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks)
+                if (qm == 1 || ks < 2)
+                    mma_tf32(d, Tf + (32 + 16 * qm) * AF_LD + 32 + 8 * ks, AF_LD,
+                             Xs + (8 * ks) * XS_LD32 + 8 * qn, XS_LD32, lane);
+            float* to = Tf + (32 + 16 * qm) * AF_LD + 8 * qn + 2 * t4;
+            *reinterpret_cast<float2*>(to + g * AF_LD) = make_float2(-d[0], -d[1]);
+            *reinterpret_cast<float2*>(to + (g + 8) * AF_LD) = make_float2(-d[2], -d[3]);
+        }
+        __syncthreads();
+        // ---- T diag(beta) as a bf16 tile (lower blocks; the upper ones are never read)
+        for (int idx = pt; idx < 64 * 8; idx += P1_THREADS) {
+            const int r = idx >> 3, ch = idx & 7;
+            if ((ch >> 1) <= (r >> 4)) {
+                const float4 t0v = *reinterpret_cast<const float4*>(Tf + r * AF_LD + 8 * ch);
+                const float4 t1v = *reinterpret_cast<const float4*>(Tf + r * AF_LD + 8 * ch + 4);
+                const float4 b0 = *reinterpret_cast<const float4*>(s_b + 8 * ch);
+                const float4 b1 = *reinterpret_cast<const float4*>(s_b + 8 * ch + 4);
+                *reinterpret_cast<uint4*>(rec + REC_TB + taddr(0, r, 8 * ch, 0)) = make_uint4(
+                    pack2(t0v.x * b0.x, t0v.y * b0.y), pack2(t0v.z * b0.z, t0v.w * b0.w),
+                    pack2(t1v.x * b1.x, t1v.y * b1.y), pack2(t1v.z * b1.z, t1v.w * b1.w));
+            }
+        }
+        // gamma_r, d_r (zero past the sequence end) and gamma_C
+        if (pt < C) {
+            float* rv = reinterpret_cast<float*>(rec + REC_VEC);
+            const float gr = s_g[pt], gC = s_g[C - 1];
+            rv[pt] = ex2(gr);
+            rv[64 + pt] = (pt < valid) ? ex2(gC - gr) : 0.f;
+            if (pt == 0) rv[128] = ex2(gC);
+        }
+        fence_proxy_async_smem();  // generic writes, read next by the bulk copy
+        __syncthreads();
+        if (pt == 0) {
+            bulk_store(p.records + (size_t)(slot * p.H_v + h) * REC_BYTES, rec, REC_BYTES);
+            bulk_commit();
+        }
+    }
+    if (pt == 0) bulk_wait_all();
+}
+
+__device__ __forceinline__ void ldsm_x2_t(uint32_t a, uint32_t* r) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x2.trans.shared.b16 {%0,%1}, [%2];"
+                 : "=r"(r[0]), "=r"(r[1])
+                 : "r"(a));
+}
+// B fragment of one n-tile (n0) x (k0..k0+15) from an MN-major tile (stored rows k, cols n).
+__device__ __forceinline__ void ldb_mn1(uint32_t base, int n0, int k0, int lane, uint32_t* b) {
+    ldsm_x2_t(taddr(base, k0 + (lane & 7) + (((lane >> 3) & 1) << 3), n0, 0), b);
+}
+
+// Delta = T_b X for row block rb (rows 16 rb .. +15) and n-tiles of column half H
+// of an NT-tile slice, stored as bf16 Delta and d o Delta.
+template <int NT, int H>
+__device__ __forceinline__ void delta_half(uint8_t* sm, uint32_t tb, uint32_t xt, int rb,
+                                           int lane, float d_lo, float d_hi) {
+    constexpr int N0 = H * (NT / 2), N1 = (H + 1) * (NT / 2);
+    float acc[N1 - N0][4];
+#pragma unroll
+    for (int i = 0; i < N1 - N0; ++i)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) acc[i][e] = 0.f;
+#pragma unroll
+    for (int ks = 0; ks < 4; ++ks) {
+        if (ks <= rb) {
+            uint32_t a[4];
+            lda_k(tb, 0, 16 * rb, 16 * ks, lane, a);
+#pragma unroll
+            for (int nt = N0; nt < N1; nt += 2) {
+                if (nt + 1 < N1) {
+                    uint32_t b[4];
+                    ldb_mn(xt, 0, 8 * nt, 16 * ks, lane, b);
+                    mma16816(acc[nt - N0], a, b[0], b[1]);
+                    mma16816(acc[nt - N0 + 1], a, b[2], b[3]);
+                } else {
+                    uint32_t b[2];
+                    ldb_mn1(xt, 8 * nt, 16 * ks, lane, b);
+                    mma16816(acc[nt - N0], a, b[0], b[1]);
+                }
+            }
+        }
+    }
+    const int g = lane >> 2, t = lane & 3, r = 16 * rb + g;
+#pragma unroll
+    for (int i = 0; i < N1 - N0; ++i) {
+        const int col = 8 * (N0 + i) + 2 * t;
+        *reinterpret_cast<uint32_t*>(sm + taddr_e(P2_DU, r, col, 0)) = pack2(acc[i][0], acc[i][1]);
+        *reinterpret_cast<uint32_t*>(sm + taddr_e(P2_DU, r + 8, col, 0)) =
+            pack2(acc[i][2], acc[i][3]);
+        *reinterpret_cast<uint32_t*>(sm + taddr_e(P2_DD, r, col, 0)) =
+            pack2(acc[i][0] * d_lo, acc[i][1] * d_lo);
+        *reinterpret_cast<uint32_t*>(sm + taddr_e(P2_DD, r + 8, col, 0)) =
+            pack2(acc[i][2] * d_hi, acc[i][3] * d_hi);
+    }
+}
+
+// ============================================================================
+// Pass 2: state pass.  Grid (d_v slices, H_v, N).
+// ============================================================================
+template <int NS, typename IO>
+__global__ void __launch_bounds__(P2_THREADS, 1)
+    state_pass_kernel(const __grid_constant__ CUtensorMap map_q,
+                      const __grid_constant__ CUtensorMap map_k,
+                      const __grid_constant__ CUtensorMap map_v, const PrefillParams p) {
+    static_assert(NS == 32 || NS == 48 || NS == 64, "slice width");
+    constexpr int NT = NS / 8;  // n-tiles of a slice
+    constexpr int NP = NT / 2;  // n-tile pairs
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+    const uint32_t sb = smem_u32(sm);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(sm + P2_BAR);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + P2_MISC);
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
+    const int g = lane >> 2, t4 = lane & 3;
     const int h = blockIdx.y;
     const int n = blockIdx.z;
     const int hq = h / (p.H_v / p.H_qk);
     const int col0 = blockIdx.x * NS;
+    const int ncols = min(NS, D - col0);
     const int t_beg = p.cu_seqlens[n];
     const int t_end = p.cu_seqlens[n + 1];
     const int nchunks = (t_end - t_beg + C - 1) / C;
 
     if (threadIdx.x == 0) {
-        for (int i = 0; i < NBAR; ++i) mbar_init(&bars[i], 1);
+        for (int i = 0; i < NBAR2; ++i) mbar_init(&bars[i], 1);
         *abort_flag = 0;
         fence_mbar_init();
     }
     __syncthreads();
 
-    if (warp == kMathWarps) {
-        // ------------------------------------------------------------ TMA producer
-        int issued = 0;
-        for (int c = 0; c < nchunks; ++c) {
-            const int s = c % NSTAGE;
-            if (c >= NSTAGE) {
-                const bool ok = mbar_wait(&bars[B_EMPTY + s], ((c / NSTAGE) - 1) & 1, abort_flag);
-                if (!__all_sync(0xffffffffu, ok)) break;
-            }
-            if (lane == 0) {
-                uint8_t* st = sm + OFF_RING + s * STAGE_BYTES;
-                const int y = t_beg + c * C;
-                mbar_arrive_expect_tx(&bars[B_FULL + s], STAGE_BYTES);
-                tma_load_2d(st + ST_K, &map_k, hq * D, y, &bars[B_FULL + s]);
-                tma_load_2d(st + ST_K + HALF, &map_k, hq * D + 64, y, &bars[B_FULL + s]);
-                tma_load_2d(st + ST_Q, &map_q, hq * D, y, &bars[B_FULL + s]);
-                tma_load_2d(st + ST_Q + HALF, &map_q, hq * D + 64, y, &bars[B_FULL + s]);
-                tma_load_2d(st + ST_V, &map_v, h * D + col0, y, &bars[B_FULL + s]);
-            }
-            __syncwarp();
-            issued = c + 1;
-        }
-        // Drain: no copy may still be landing in shared memory when the CTA exits.
-        for (int c = max(0, issued - NSTAGE); c < issued; ++c)
-            mbar_wait(&bars[B_FULL + (c % NSTAGE)], (c / NSTAGE) & 1, abort_flag);
-        __syncwarp();
-        TRACE_T(kMathThreads, 0, 4, issued);
-    } else {
-        // ------------------------------------------------------------ math warps
+    // Copies of chunk c into ring stage c % NSTAGE: K, Q (both halves), the V slice
+    // and the chunk's operator record.  Issued by one thread; a stage is refilled
+    // only after every chain warp has finished with it.
+    auto issue_chunk = [&](int c) {
+        const int s = c % NSTAGE;
+        uint8_t* st = sm + s * STAGE_BYTES;
+        const int y = t_beg + c * C;
+        uint64_t* full = &bars[B2_FULL + s];
+        mbar_arrive_expect_tx(full, STAGE_TX);
+        tma_load_2d(st + ST_K, &map_k, hq * D, y, full);
+        tma_load_2d(st + ST_K + HALF, &map_k, hq * D + 64, y, full);
+        tma_load_2d(st + ST_Q, &map_q, hq * D, y, full);
+        tma_load_2d(st + ST_Q + HALF, &map_q, hq * D + 64, y, full);
+        tma_load_2d(st + ST_V, &map_v, h * D + col0, y, full);
+        bulk_load(st + ST_REC, p.records + (size_t)(record_slot(n, y) * p.H_v + h) * REC_BYTES,
+                  REC_BYTES, full);
+    };
+    int issued = 0;
+    if (threadIdx.x == P2_LOADER)
+        for (; issued < min(NSTAGE, nchunks); ++issued) issue_chunk(issued);
+    {
+        // ------------------------------------------------------------ chain warps
         const int tid = threadIdx.x;
-        const int g = lane >> 2, t4 = lane & 3;
-        const int m0 = 16 * (warp & 3);       // this warp's 16-row block of 64-row products
-        const bool upper = warp < 4;          // warps 0-3 vs 4-7
-        float* Af = reinterpret_cast<float*>(sm + OFF_AF);
-        float* Tf = reinterpret_cast<float*>(sm + OFF_TF);
-        float* Xs = reinterpret_cast<float*>(sm + OFF_XS);
-        const float LOG2E = 1.4426950408889634f;
-        const int ncols = min(NS, D - col0);
+        const bool mw = warp < 4;        // warps 0-3 also compute K S, Q S and the output
+        const int m0 = 16 * (warp & 3);  // this warp's 16 rows of the 64-row products
+        const int r0 = 16 * warp;        // this warp's 16 rows of S
 
-        // S rows 16*warp + {g, g+8}, columns 8*nt + 2*t4 + {0,1}, as fp32 accumulators
+        // S rows r0 + {g, g+8}, columns 8 nt + 2 t4 + {0, 1}
         float Sacc[NT][4];
         {
             const float* s0 = p.S0 ? p.S0 + ((size_t)n * p.H_v + h) * D * D : nullptr;
@@ -302,214 +669,118 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
-                    const int row = 16 * warp + g + ((e >> 1) << 3);
+                    const int row = r0 + g + ((e >> 1) << 3);
                     const int col = 8 * nt + 2 * t4 + (e & 1);
                     Sacc[nt][e] = (s0 && col < ncols) ? s0[(size_t)row * D + col0 + col] : 0.f;
                 }
-            store_acc_bf16<NT>(sm, OFF_SB, HALF, 16 * warp, Sacc, lane, 1.f, 1.f);
+            store_acc_bf16<NT>(sm, P2_SB, 0, r0, Sacc, lane, 1.f, 1.f);
         }
-
-        float keep[NT][4];  // warps 0-3: U then Delta; warps 4-7: gamma o (Q S), then O
+        bar_sync<BAR_CHAIN, P2_CHAIN_THREADS>();
 
         for (int c = 0; c < nchunks; ++c) {
             const int s = c % NSTAGE;
+            const uint32_t st = sb + s * STAGE_BYTES;
+            const uint8_t* stp = sm + s * STAGE_BYTES;
+            const float* rv = reinterpret_cast<const float*>(stp + ST_REC + REC_VEC);
             const int tc0 = t_beg + c * C;
             const int valid = min(C, t_end - tc0);
-            const uint32_t st = sb + OFF_RING + s * STAGE_BYTES;
-            uint8_t* stp = sm + OFF_RING + s * STAGE_BYTES;
-            TRACE_T(0, 2, 20, c);
+            const bool ok = mbar_wait(&bars[B2_FULL + s], (c / NSTAGE) & 1, abort_flag);
+            __syncwarp();
 
-            // gates of this chunk (rows past the sequence end: log alpha = 0, beta = 0)
-            float la = 0.f, be = 0.f;
-            if (tid < C && tid < valid) {
-                la = p.log_alpha[(size_t)(tc0 + tid) * p.H_v + h];
-                be = p.beta[(size_t)(tc0 + tid) * p.H_v + h];
-            }
-            const bool ok = mbar_wait(&bars[B_FULL + s], (c / NSTAGE) & 1, abort_flag);
-            if (!__all_sync(0xffffffffu, ok)) break;
-            if (valid < C) {  // zero K, Q, V rows past the end of the sequence
-                for (int i = tid; i < 5 * 64 * 8; i += kMathThreads) {
-                    const int tile = i / 512, row = (i >> 3) & 63, ch = i & 7;
-                    if (row >= valid)
-                        *reinterpret_cast<uint4*>(stp + tile * HALF + row * 128 + ch * 16) =
-                            make_uint4(0, 0, 0, 0);
-                }
-            }
-            // inclusive scan of log alpha (rows 0..63 live in warps 0 and 1)
-            float gsum = la * LOG2E;
-            if (tid < C) {
+            // ---- warps 0-3: K S and Q S for rows m0 .. m0+15 (one pass over S)
+            float accK[NT][4], accQ[NT][4];
+            if (mw) {
 #pragma unroll
-                for (int off = 1; off < 32; off <<= 1) {
-                    const float y = __shfl_up_sync(0xffffffffu, gsum, off);
-                    if (lane >= off) gsum += y;
-                }
-                if (tid == 31) s_carry[0] = gsum;
-            }
-            math_bar();
-            if (tid >= 32 && tid < C) gsum += s_carry[0];
-            if (tid < C) {
-                s_g[tid] = gsum;
-                s_b[tid] = be;
-            }
-            math_bar();
-            const float gC = s_g[C - 1];
-            if (tid < C) {
-                s_gam[tid] = ex2(gsum);
-                s_ds[tid] = (tid < valid) ? ex2(gC - gsum) : 0.f;
-            }
-
-            // ---- grams: warps 0-3 rows of K K^T (-> A), warps 4-7 rows of Q K^T (-> M_Q)
-            {
-                float acc[8][4];
+                for (int i = 0; i < NT; ++i)
 #pragma unroll
-                for (int i = 0; i < 8; ++i) acc[i][0] = acc[i][1] = acc[i][2] = acc[i][3] = 0.f;
-                warp_gemm<8, 8, false, false>(acc, st + (upper ? ST_K : ST_Q), HALF, m0,
-                                              st + ST_K, HALF, lane);
-                const int r_lo = m0 + g, r_hi = m0 + g + 8;
-                const float g_lo = s_g[r_lo], g_hi = s_g[r_hi];
-                if (upper) {
-                    const float b_lo = s_b[r_lo], b_hi = s_b[r_hi];
+                    for (int e = 0; e < 4; ++e) accK[i][e] = accQ[i][e] = 0.f;
 #pragma unroll
-                    for (int nt = 0; nt < 8; ++nt) {
-                        const int j = 8 * nt + 2 * t4;
-                        float2 lo, hi;
-                        lo.x = (j < r_lo) ? b_lo * ex2(g_lo - s_g[j]) * acc[nt][0] : 0.f;
-                        lo.y = (j + 1 < r_lo) ? b_lo * ex2(g_lo - s_g[j + 1]) * acc[nt][1] : 0.f;
-                        hi.x = (j < r_hi) ? b_hi * ex2(g_hi - s_g[j]) * acc[nt][2] : 0.f;
-                        hi.y = (j + 1 < r_hi) ? b_hi * ex2(g_hi - s_g[j + 1]) * acc[nt][3] : 0.f;
-                        *reinterpret_cast<float2*>(Af + r_lo * AF_LD + j) = lo;
-                        *reinterpret_cast<float2*>(Af + r_hi * AF_LD + j) = hi;
-                    }
-                } else {
-                    const bool v_lo = r_lo < valid, v_hi = r_hi < valid;
+                for (int ks = 0; ks < 8; ++ks) {
+                    uint32_t ak[4], aq[4];
+                    lda_k(st + ST_K, HALF, m0, 16 * ks, lane, ak);
+                    lda_k(st + ST_Q, HALF, m0, 16 * ks, lane, aq);
 #pragma unroll
-                    for (int nt = 0; nt < 8; ++nt) {
-                        const int j = 8 * nt + 2 * t4;
-                        const float m00 = (v_lo && j <= r_lo) ? ex2(g_lo - s_g[j]) * acc[nt][0] : 0.f;
-                        const float m01 = (v_lo && j + 1 <= r_lo) ? ex2(g_lo - s_g[j + 1]) * acc[nt][1] : 0.f;
-                        const float m10 = (v_hi && j <= r_hi) ? ex2(g_hi - s_g[j]) * acc[nt][2] : 0.f;
-                        const float m11 = (v_hi && j + 1 <= r_hi) ? ex2(g_hi - s_g[j + 1]) * acc[nt][3] : 0.f;
-                        *reinterpret_cast<uint32_t*>(sm + taddr_e(OFF_MQ, r_lo, j, HALF)) = pack2(m00, m01);
-                        *reinterpret_cast<uint32_t*>(sm + taddr_e(OFF_MQ, r_hi, j, HALF)) = pack2(m10, m11);
+                    for (int np = 0; np < NP; ++np) {
+                        uint32_t b[4];
+                        ldb_mn(sb + P2_SB, 0, 16 * np, 16 * ks, lane, b);
+                        mma16816(accK[2 * np], ak, b[0], b[1]);
+                        mma16816(accK[2 * np + 1], ak, b[2], b[3]);
+                        mma16816(accQ[2 * np], aq, b[0], b[1]);
+                        mma16816(accQ[2 * np + 1], aq, b[2], b[3]);
                     }
                 }
-            }
-            for (int i = tid; i < 64 * AF_LD / 4; i += kMathThreads)
-                reinterpret_cast<float4*>(Tf)[i] = make_float4(0.f, 0.f, 0.f, 0.f);
-            math_bar();
-            TRACE_T(0, 2, 22, c);
-
-            // ---- T = (I + A)^{-1}: diagonal 16x16 blocks by forward substitution
-            if (tid < C) {
-                const int b = tid >> 4, cc = tid & 15;
-                const float* Ab = Af + (16 * b) * AF_LD + 16 * b;
-                float x[16];
-#pragma unroll
-                for (int i = 0; i < 16; ++i) {
-                    float sacc = 0.f;
-#pragma unroll
-                    for (int j = 0; j < i; ++j) sacc = fmaf(-Ab[i * AF_LD + j], x[j], sacc);
-                    x[i] = (i == cc) ? 1.f : ((i > cc) ? sacc : 0.f);
-                }
-#pragma unroll
-                for (int i = 0; i < 16; ++i) Tf[(16 * b + i) * AF_LD + 16 * b + cc] = x[i];
-            }
-            math_bar();
-            // off-diagonal blocks by distance l = i - j:  X = sum_{k=j}^{i-1} A_ik T_kj ; T_ij = -T_ii X
-#pragma unroll 1
-            for (int l = 1; l < 4; ++l) {
-                const int nb = 4 - l;
-                for (int e = tid; e < nb * 256; e += kMathThreads) {
-                    const int blk = e >> 8, a = (e >> 4) & 15, bc = e & 15;
-                    const int bi = blk + l, bj = blk;
-                    float x = 0.f;
-                    for (int kb = bj; kb < bi; ++kb) {
-                        const float* ar = Af + (16 * bi + a) * AF_LD + 16 * kb;
-                        const float* tcol = Tf + (16 * kb) * AF_LD + 16 * bj + bc;
-#pragma unroll
-                        for (int m = 0; m < 16; ++m) x = fmaf(ar[m], tcol[m * AF_LD], x);
-                    }
-                    Xs[e] = x;
-                }
-                math_bar();
-                for (int e = tid; e < nb * 256; e += kMathThreads) {
-                    const int blk = e >> 8, a = (e >> 4) & 15, bc = e & 15;
-                    const int bi = blk + l, bj = blk;
-                    const float* tr = Tf + (16 * bi + a) * AF_LD + 16 * bi;
-                    const float* xc = Xs + blk * 256 + bc;
-                    float y = 0.f;
-#pragma unroll
-                    for (int m = 0; m < 16; ++m) y = fmaf(tr[m], xc[m * 16], y);
-                    Tf[(16 * bi + a) * AF_LD + 16 * bj + bc] = -y;
-                }
-                math_bar();
-            }
-            // T_bg = T diag(beta gamma), T_b = T diag(beta) -> bf16 K-major tiles;
-            // thread (row, part): parts 0-1 fill T_bg, parts 2-3 fill T_b, 32 columns each
-            {
-                const int row = tid & 63, part = tid >> 6;
-                const bool with_gamma = part < 2;
-                const int cb = 32 * (part & 1);
-                const uint32_t dst = with_gamma ? OFF_TBG : OFF_TB;
-                const float* trow = Tf + row * AF_LD;
-#pragma unroll
-                for (int ch = 0; ch < 4; ++ch) {
-                    float m[8];
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) {
-                        const int j = cb + 8 * ch + e;
-                        m[e] = trow[j] * (with_gamma ? s_b[j] * s_gam[j] : s_b[j]);
-                    }
-                    uint4 u;
-                    u.x = pack2(m[0], m[1]);
-                    u.y = pack2(m[2], m[3]);
-                    u.z = pack2(m[4], m[5]);
-                    u.w = pack2(m[6], m[7]);
-                    *reinterpret_cast<uint4*>(sm + taddr(dst, row, cb + 8 * ch, HALF)) = u;
-                }
-            }
-            math_bar();
-            TRACE_T(0, 2, 23, c);
-
-            // ---- warps 4-7: W = T_bg K (-> -W tile);  warps 0-3: U = T_b V (registers)
-            if (!upper) {
-                float acc[16][4];
-#pragma unroll
-                for (int i = 0; i < 16; ++i) acc[i][0] = acc[i][1] = acc[i][2] = acc[i][3] = 0.f;
-                warp_gemm<16, 4, false, true>(acc, sb + OFF_TBG, HALF, m0, st + ST_K, HALF, lane);
-                store_acc_bf16<16>(sm, OFF_W, HALF, m0, acc, lane, -1.f, -1.f);
-            } else {
-#pragma unroll
-                for (int i = 0; i < NT; ++i) keep[i][0] = keep[i][1] = keep[i][2] = keep[i][3] = 0.f;
-                warp_gemm<NT, 4, false, true>(keep, sb + OFF_TB, HALF, m0, st + ST_V, HALF, lane);
-            }
-            math_bar();
-
-            // ---- warps 0-3: Delta = U + (-W) S;  warps 4-7: Q S
-            if (upper) {
-                warp_gemm<NT, 8, false, true>(keep, sb + OFF_W, HALF, m0, sb + OFF_SB, HALF, lane);
-                const float d_lo = s_ds[m0 + g], d_hi = s_ds[m0 + g + 8];
-                store_acc_bf16<NT>(sm, OFF_DU, HALF, m0, keep, lane, 1.f, 1.f);
-                store_acc_bf16<NT>(sm, OFF_DD, HALF, m0, keep, lane, d_lo, d_hi);
-            } else {
-#pragma unroll
-                for (int i = 0; i < NT; ++i) keep[i][0] = keep[i][1] = keep[i][2] = keep[i][3] = 0.f;
-                warp_gemm<NT, 8, false, true>(keep, st + ST_Q, HALF, m0, sb + OFF_SB, HALF, lane);
-                const float gm_lo = s_gam[m0 + g], gm_hi = s_gam[m0 + g + 8];
+                // X = V - gamma o (K S)   (rows past the sequence end are zero: V and K are);
+                // gamma o (Q S) is kept for the output
+                const float gm_lo = rv[m0 + g], gm_hi = rv[m0 + g + 8];
+                const uint8_t* vt = stp + ST_V;
 #pragma unroll
                 for (int nt = 0; nt < NT; ++nt) {
-                    keep[nt][0] *= gm_lo;
-                    keep[nt][1] *= gm_lo;
-                    keep[nt][2] *= gm_hi;
-                    keep[nt][3] *= gm_hi;
+                    const int col = 8 * nt + 2 * t4;
+                    const float2 v_lo = __bfloat1622float2(
+                        *reinterpret_cast<const __nv_bfloat162*>(vt + taddr_e(0, m0 + g, col, 0)));
+                    const float2 v_hi = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(
+                        vt + taddr_e(0, m0 + g + 8, col, 0)));
+                    accK[nt][0] = v_lo.x - gm_lo * accK[nt][0];
+                    accK[nt][1] = v_lo.y - gm_lo * accK[nt][1];
+                    accK[nt][2] = v_hi.x - gm_hi * accK[nt][2];
+                    accK[nt][3] = v_hi.y - gm_hi * accK[nt][3];
+                    accQ[nt][0] *= gm_lo;
+                    accQ[nt][1] *= gm_lo;
+                    accQ[nt][2] *= gm_hi;
+                    accQ[nt][3] *= gm_hi;
+                }
+                store_acc_bf16<NT>(sm, P2_X, 0, m0, accK, lane, 1.f, 1.f);
+            }
+            if (!bar_and<BAR_CHAIN, P2_CHAIN_THREADS>(ok)) break;
+
+            // ---- Delta = T_b X: all eight warps, warp = (row block m0 / 16, column half);
+            // T_b is lower triangular, so row block rb needs key blocks 0..rb only
+            {
+                const int rb = warp & 3;
+                const float d_lo = rv[64 + m0 + g], d_hi = rv[64 + m0 + g + 8];
+                if (warp < 4)
+                    delta_half<NT, 0>(sm, st + ST_REC + REC_TB, sb + P2_X, rb, lane, d_lo, d_hi);
+                else
+                    delta_half<NT, 1>(sm, st + ST_REC + REC_TB, sb + P2_X, rb, lane, d_lo, d_hi);
+            }
+            if (!bar_and<BAR_CHAIN, P2_CHAIN_THREADS>(ok)) break;
+
+            // ---- S <- gamma_C S + K^T (d o Delta)   (rows r0 .. r0+15)
+            {
+                const float gamC = rv[128];
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) Sacc[nt][e] *= gamC;
+#pragma unroll
+                for (int ks = 0; ks < 4; ++ks) {
+                    uint32_t a[4];
+                    lda_mn(st + ST_K, HALF, r0, 16 * ks, lane, a);
+#pragma unroll
+                    for (int np = 0; np < NP; ++np) {
+                        uint32_t b[4];
+                        ldb_mn(sb + P2_DD, 0, 16 * np, 16 * ks, lane, b);
+                        mma16816(Sacc[2 * np], a, b[0], b[1]);
+                        mma16816(Sacc[2 * np + 1], a, b[2], b[3]);
+                    }
                 }
             }
-            math_bar();
-            TRACE_T(0, 2, 25, c);
-
-            // ---- warps 4-7: O = gamma (Q S) + (M o Q K^T) Delta, stored
-            if (!upper) {
-                warp_gemm<NT, 4, false, true>(keep, sb + OFF_MQ, HALF, m0, sb + OFF_DU, HALF, lane);
+            // ---- O = gamma o (Q S) + (M o Q K^T) Delta   (warps 0-3), stored
+            if (mw) {
+#pragma unroll
+                for (int ks = 0; ks < 4; ++ks) {
+                    if (ks <= warp) {
+                        uint32_t a[4];
+                        lda_k(st + ST_REC + REC_MQ, 0, m0, 16 * ks, lane, a);
+#pragma unroll
+                        for (int np = 0; np < NP; ++np) {
+                            uint32_t b[4];
+                            ldb_mn(sb + P2_DU, 0, 16 * np, 16 * ks, lane, b);
+                            mma16816(accQ[2 * np], a, b[0], b[1]);
+                            mma16816(accQ[2 * np + 1], a, b[2], b[3]);
+                        }
+                    }
+                }
                 IO* ob = static_cast<IO*>(p.o);
 #pragma unroll
                 for (int hl = 0; hl < 2; ++hl) {
@@ -520,28 +791,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                         for (int nt = 0; nt < NT; ++nt) {
                             const int col = 8 * nt + 2 * t4;
                             if (col < ncols)
-                                store2<IO>(orow + col, keep[nt][2 * hl], keep[nt][2 * hl + 1]);
+                                store2<IO>(orow + col, accQ[nt][2 * hl], accQ[nt][2 * hl + 1]);
                         }
                     }
                 }
             }
-            // ---- all warps: S <- gamma_C S + K^T (d o Delta)  (rows 16*warp .. +15)
-            {
-                const float gamC = ex2(gC);
-#pragma unroll
-                for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) Sacc[nt][e] *= gamC;
-                warp_gemm<NT, 4, true, true>(Sacc, st + ST_K, HALF, 16 * warp, sb + OFF_DD, HALF,
-                                            lane);
-            }
-            // Every read of this chunk's ring stage is done; generic writes to it (the
-            // zeroed padding rows) are ordered before the next TMA refill.
-            fence_proxy_async_smem();
-            math_bar();
-            if (tid == 0) mbar_arrive(&bars[B_EMPTY + s]);
-            store_acc_bf16<NT>(sm, OFF_SB, HALF, 16 * warp, Sacc, lane, 1.f, 1.f);
-            TRACE_T(0, 2, 27, c);
+            store_acc_bf16<NT>(sm, P2_SB, 0, r0, Sacc, lane, 1.f, 1.f);
+            if (!bar_and<BAR_CHAIN, P2_CHAIN_THREADS>(ok)) break;
+            // this ring stage is free again: refill it with the chunk NSTAGE ahead
+            if (tid == P2_LOADER && c + NSTAGE < nchunks) issue_chunk(issued++);
         }
         if (p.S_final && !*abort_flag) {
             float* sf = p.S_final + ((size_t)n * p.H_v + h) * D * D;
@@ -549,15 +807,18 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
                 for (int hl = 0; hl < 2; ++hl) {
-                    const int row = 16 * warp + g + 8 * hl;
+                    const int row = r0 + g + 8 * hl;
                     const int col = 8 * nt + 2 * t4;
                     if (col < ncols)
                         *reinterpret_cast<float2*>(sf + (size_t)row * D + col0 + col) =
                             make_float2(Sacc[nt][2 * hl], Sacc[nt][2 * hl + 1]);
                 }
         }
-        TRACE_T(0, 2, 30, nchunks);
     }
+    // Drain: no copy may still be landing in shared memory when the CTA exits.
+    if (threadIdx.x == P2_LOADER)
+        for (int c = max(0, issued - NSTAGE); c < issued; ++c)
+            mbar_wait_drain(&bars[B2_FULL + (c % NSTAGE)], (c / NSTAGE) & 1);
     __syncthreads();
 }
 
@@ -613,15 +874,27 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols) {
 }
 
 template <int NS, typename IO>
-cudaError_t launch_ns(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
-                      const PrefillParams& prm, int N, cudaStream_t stream) {
-    auto kern = prefill_kernel<NS, IO>;
+cudaError_t launch_pass2(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+                         const PrefillParams& prm, int N, cudaStream_t stream) {
+    auto kern = state_pass_kernel<NS, IO>;
     cudaError_t e =
-        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_ALLOC);
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, P2_SMEM);
     if (e != cudaSuccess) return e;
-    dim3 grid(D / NS, prm.H_v, N);
-    kern<<<grid, kThreads, SMEM_ALLOC, stream>>>(mq, mk, mv, prm);
+    dim3 grid((D + NS - 1) / NS, prm.H_v, N);
+    kern<<<grid, P2_THREADS, P2_SMEM, stream>>>(mq, mk, mv, prm);
     return cudaGetLastError();
+}
+
+size_t up256(size_t b) { return (b + 255) & ~size_t(255); }
+
+size_t staging_bytes(int T, int H_qk, int H_v, bool bf16) {
+    if (bf16) return 0;
+    return up256((size_t)T * H_qk * D * 2) * 2 + up256((size_t)T * H_v * D * 2);
+}
+
+size_t record_bytes(int N, int T, int H_v) {
+    const size_t slots = (size_t)N + ((size_t)T + C - 1) / C;
+    return up256(slots * H_v * REC_BYTES);
 }
 
 }  // namespace
@@ -656,10 +929,8 @@ cudaError_t noalloc_scratch_address(void** out) {
 }
 
 size_t prefill_workspace_bytes(int N, int T, int H_qk, int H_v, bool bf16) {
-    (void)N;
-    if (bf16) return 0;
-    auto up = [](size_t b) { return (b + 255) & ~size_t(255); };
-    return up((size_t)T * H_qk * D * 2) * 2 + up((size_t)T * H_v * D * 2);
+    if (T == 0) return 0;
+    return staging_bytes(T, H_qk, H_v, bf16) + record_bytes(N, T, H_v);
 }
 
 cudaError_t launch_prefill(const void* q, const void* k, const void* v, const float* log_alpha,
@@ -671,14 +942,13 @@ cudaError_t launch_prefill(const void* q, const void* k, const void* v, const fl
         copy_state_kernel<<<592, 256, 0, stream>>>(S0, S_final, (size_t)N * H_v * D * D / 4);
         return cudaGetLastError();
     }
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
     const void *qb = q, *kb = k, *vb = v;
     if (!bf16) {
-        auto up = [](size_t b) { return (b + 255) & ~size_t(255); };
-        uint8_t* ws = static_cast<uint8_t*>(workspace);
         const size_t nqk = (size_t)T * H_qk * D, nv = (size_t)T * H_v * D;
         __nv_bfloat16* q16 = reinterpret_cast<__nv_bfloat16*>(ws);
-        __nv_bfloat16* k16 = reinterpret_cast<__nv_bfloat16*>(ws + up(nqk * 2));
-        __nv_bfloat16* v16 = reinterpret_cast<__nv_bfloat16*>(ws + 2 * up(nqk * 2));
+        __nv_bfloat16* k16 = reinterpret_cast<__nv_bfloat16*>(ws + up256(nqk * 2));
+        __nv_bfloat16* v16 = reinterpret_cast<__nv_bfloat16*>(ws + 2 * up256(nqk * 2));
         f32_to_bf16_kernel<<<592, 256, 0, stream>>>(static_cast<const float*>(q), q16, nqk / 4);
         f32_to_bf16_kernel<<<592, 256, 0, stream>>>(static_cast<const float*>(k), k16, nqk / 4);
         f32_to_bf16_kernel<<<592, 256, 0, stream>>>(static_cast<const float*>(v), v16, nv / 4);
@@ -688,31 +958,42 @@ cudaError_t launch_prefill(const void* q, const void* k, const void* v, const fl
         kb = k16;
         vb = v16;
     }
+    uint8_t* records = ws + staging_bytes(T, H_qk, H_v, bf16);
     CUtensorMap mq, mk, mv;
     if (!make_map(&mq, qb, T, (uint64_t)H_qk * D) || !make_map(&mk, kb, T, (uint64_t)H_qk * D) ||
         !make_map(&mv, vb, T, (uint64_t)H_v * D))
         return cudaErrorInvalidValue;
-    PrefillParams prm{log_alpha, beta, S0, cu_seqlens, o, S_final, H_qk, H_v, N, T};
-    // Slice width: one CTA per SM at most (each holds ~190 KB of shared memory), so
-    // split the head into four 32-column slices only when that still fits in one
-    // wave; otherwise two 64-column slices (half the redundant per-chunk work).
+    PrefillParams prm{log_alpha, beta, S0, cu_seqlens, o, S_final, records, H_qk, H_v, N, T};
+
+    // pass 1: every chunk's operators, all chunks at once
+    {
+        cudaError_t e = cudaFuncSetAttribute(chunk_ops_kernel,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, P1_SMEM);
+        if (e != cudaSuccess) return e;
+        const int group = H_v / H_qk;
+        const long long slots = (long long)N + ((long long)T + C - 1) / C;
+        dim3 grid((unsigned)slots, H_qk, (group + P1_MAX_GROUP - 1) / P1_MAX_GROUP);
+        chunk_ops_kernel<<<grid, P1_THREADS, P1_SMEM, stream>>>(mq, mk, prm);
+        e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+    }
+    // pass 2: the state through the chunks.  One CTA per SM at most (each holds
+    // ~212 KB of shared memory): split every value head into as many d_v slices
+    // (4 x 32, 3 x 48 or 2 x 64 columns) as still fit in one wave, so few long
+    // sequences still cover the SMs.
     int num_sms = 148, dev = 0;
     if (cudaGetDevice(&dev) == cudaSuccess)
         cudaDeviceGetAttribute(&num_sms, cudaDevAttrMultiProcessorCount, dev);
-    const bool narrow = (long long)N * H_v * 4 <= num_sms;
+    const long long units = (long long)N * H_v;
+    const int ns = units * 4 <= num_sms ? 32 : (units * 3 <= num_sms ? 48 : 64);
     if (bf16) {
-        if (!narrow) return launch_ns<64, __nv_bfloat16>(mq, mk, mv, prm, N, stream);
-        return launch_ns<32, __nv_bfloat16>(mq, mk, mv, prm, N, stream);
+        if (ns == 64) return launch_pass2<64, __nv_bfloat16>(mq, mk, mv, prm, N, stream);
+        if (ns == 48) return launch_pass2<48, __nv_bfloat16>(mq, mk, mv, prm, N, stream);
+        return launch_pass2<32, __nv_bfloat16>(mq, mk, mv, prm, N, stream);
     }
-    if (!narrow) return launch_ns<64, float>(mq, mk, mv, prm, N, stream);
-    return launch_ns<32, float>(mq, mk, mv, prm, N, stream);
+    if (ns == 64) return launch_pass2<64, float>(mq, mk, mv, prm, N, stream);
+    if (ns == 48) return launch_pass2<48, float>(mq, mk, mv, prm, N, stream);
+    return launch_pass2<32, float>(mq, mk, mv, prm, N, stream);
 }
 
 }  // namespace gdn
-
-#ifdef GDN_DEBUG_TRACE
-extern "C" __attribute__((visibility("default"))) int gdn_debug_set_trace(void* host_mapped) {
-    volatile int* p = static_cast<volatile int*>(host_mapped);
-    return (int)cudaMemcpyToSymbol(gdn::g_trace, &p, sizeof(p));
-}
-#endif

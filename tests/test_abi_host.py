@@ -42,10 +42,17 @@ def test_status_strings(L):
     assert L.gdn_version() == 100
 
 
+REC_BYTES = 2 * 64 * 64 * 2 + 132 * 4  # per (chunk slot, value head): two bf16 tiles + vectors
+
+
 def test_workspace_size(L):
-    assert gdn.workspace_size(1, 32768, 16, 48, 128, gdn.GDN_BF16) == 0
-    ws = gdn.workspace_size(1, 256, 1, 1, 128, gdn.GDN_F32)
-    assert ws >= 3 * 256 * 128 * 2
+    # one chunk-operator record per (chunk slot, value head); slots = N + ceil(T / 64)
+    ws = gdn.workspace_size(1, 32768, 16, 48, 128, gdn.GDN_BF16)
+    assert ws >= (1 + 512) * 48 * REC_BYTES
+    assert ws < (1 + 512) * 48 * REC_BYTES + 256
+    ws32 = gdn.workspace_size(1, 256, 1, 1, 128, gdn.GDN_F32)
+    assert ws32 >= 3 * 256 * 128 * 2 + (1 + 4) * REC_BYTES  # + bf16 copies of q, k, v
+    assert gdn.workspace_size(3, 0, 1, 1, 128, gdn.GDN_BF16) == 0  # nothing to do
     assert gdn.workspace_size(0, 256, 1, 1, 128, gdn.GDN_F32) == 0  # invalid -> 0
 
 
