@@ -44,6 +44,7 @@
 // copies (bounded) and exit.
 #include <cudaTypedefs.h>
 
+#include <algorithm>
 #include <mutex>
 
 #include "gdn_common.cuh"
@@ -75,22 +76,21 @@ __host__ __device__ __forceinline__ long long record_slot(int n, int t0) {
 
 // ---- pass 1 shared memory ----
 constexpr int P1_THREADS = 256;
+constexpr int P1_MAX_GROUP = 4;                                // value heads per work item
 constexpr int AF_LD = 68;                                      // fp32 row stride of A and T
-constexpr int XS_LD16 = 24, XS_LD32 = 40;                      // solve scratch strides
 constexpr uint32_t P1_K = 0;                                   // K, 64 x 128 (two halves)
 constexpr uint32_t P1_Q = 2 * HALF;                            // Q
-constexpr uint32_t P1_REC = 4 * HALF;                          // two record buffers
+constexpr uint32_t P1_AF = 0;                                  // after the grams: A, fp32 64 x 68
+constexpr uint32_t P1_TF = 64 * AF_LD * 4;                     //                  T, fp32 64 x 68
+constexpr uint32_t P1_REC = ((2 * 64 * AF_LD * 4 + 1023) / 1024) * 1024;  // one record
 constexpr uint32_t P1_REC_STRIDE = 17408;                      // REC_BYTES rounded to 1 KB
-constexpr uint32_t P1_AF = P1_REC + 2 * P1_REC_STRIDE;         // A, fp32 64 x 68
-constexpr uint32_t P1_TF = P1_AF + 64 * AF_LD * 4;             // T, fp32 64 x 68
-constexpr uint32_t P1_XS = P1_TF + 64 * AF_LD * 4;             // 1280 floats
-constexpr uint32_t P1_VEC = P1_XS + 32 * XS_LD32 * 4;          // per value head: g[64], beta[64]
-constexpr int P1_MAX_GROUP = 4;                                // value heads per query/key head
+constexpr uint32_t P1_XS = P1_REC + P1_REC_STRIDE;             // 256 floats per warp (warps 0-3)
+constexpr uint32_t P1_VEC = P1_XS + 4 * 256 * 4;               // per value head: g[64], beta[64]
 constexpr uint32_t P1_BAR = P1_VEC + P1_MAX_GROUP * 128 * 4;
 constexpr uint32_t P1_MISC = P1_BAR + 8;
 constexpr uint32_t P1_SMEM = P1_MISC + 16 + 1024;
-static_assert(P1_REC_STRIDE >= REC_BYTES && P1_AF % 16 == 0, "pass 1 layout");
-static_assert(2 * P1_SMEM + 2048 <= 233472, "two pass-1 CTAs per SM");
+static_assert(P1_REC_STRIDE >= REC_BYTES && P1_REC >= 4 * HALF, "pass 1 layout");
+static_assert(3 * (P1_SMEM + 1024) <= 233472, "three pass-1 CTAs per SM");
 
 // ---- pass 2 shared memory ----
 constexpr int NSTAGE = 3;
@@ -280,9 +280,11 @@ __device__ __forceinline__ void slot_owner(const int32_t* cu, int N, int j, int&
 }
 
 // ============================================================================
-// Pass 1: chunk operators.  Grid (record slots, H_qk, value-head batches of 4).
+// Pass 1: chunk operators.  Grid (record slots, H_qk, batches of up to 4 value
+// heads of that head); three CTAs per SM.  A and T reuse the K and Q tiles'
+// shared memory once the grams are in registers.
 // ============================================================================
-__global__ void __launch_bounds__(P1_THREADS, 2)
+__global__ void __launch_bounds__(P1_THREADS, 3)
     chunk_ops_kernel(const __grid_constant__ CUtensorMap map_q,
                      const __grid_constant__ CUtensorMap map_k, const PrefillParams p) {
     extern __shared__ uint8_t smem_raw[];
@@ -345,8 +347,6 @@ __global__ void __launch_bounds__(P1_THREADS, 2)
         *reinterpret_cast<float2*>(v + 2 * lane) = make_float2(incl - x1, incl);
         *reinterpret_cast<float2*>(v + 64 + 2 * lane) = make_float2(be[0], be[1]);
     }
-    for (int i = pt; i < 64 * AF_LD / 4; i += P1_THREADS)
-        reinterpret_cast<float4*>(Tf)[i] = make_float4(0.f, 0.f, 0.f, 0.f);
     const bool ok = mbar_wait(bar, 0, abort_flag);
     __syncwarp();
     if (!__syncthreads_and(ok)) {
@@ -402,16 +402,17 @@ __global__ void __launch_bounds__(P1_THREADS, 2)
             }
         }
     }
+    // K and Q are dead: their space now holds A and T.  T's blocks above the
+    // diagonal are read as zeros by the solve and never written.
+    __syncthreads();
+    for (int i = pt; i < 64 * AF_LD / 4; i += P1_THREADS)
+        reinterpret_cast<float4*>(Tf)[i] = make_float4(0.f, 0.f, 0.f, 0.f);
 
     for (int vh = 0; vh < nheads; ++vh) {
         const int h = hv0 + vh;
         const float* s_g = reinterpret_cast<const float*>(sm + P1_VEC) + vh * 128;
         const float* s_b = s_g + 64;
-        uint8_t* rec = sm + P1_REC + (vh & 1) * P1_REC_STRIDE;
-        if (vh >= 2) {  // the record buffer's previous bulk store must have read it
-            if (pt == 0) bulk_wait_read<1>();
-            __syncthreads();
-        }
+        uint8_t* rec = sm + P1_REC;  // refilled per value head (see the store below)
         // ---- masks: A -> Af (fp32), M o Q K^T -> the record (bf16)
 #pragma unroll
         for (int b = 0; b < 3; ++b) {
@@ -462,53 +463,60 @@ __global__ void __launch_bounds__(P1_THREADS, 2)
             for (int i = 0; i < 16; ++i) Tf[(16 * b + i) * AF_LD + 16 * b + cc] = x[i];
         }
         __syncthreads();
-        if (warp < 4) {  // X = A_10 T_00 (warps 0,1) and A_32 T_22 (warps 2,3), one n-tile each
+        // Off-diagonal blocks from tf32 tensor-core block products (warps 0-3; the
+        // intermediate goes through a per-warp scratch to become an operand):
+        //   T_10 = -T_11 (A_10 T_00),  T_32 = -T_33 (A_32 T_22)   (one n-tile per warp)
+        float* xw = Xs + warp * 256;
+        if (warp < 4) {
             const int blk = warp >> 1, nt = warp & 1, bi = 1 + 2 * blk, bj = 2 * blk;
             float d[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
             for (int ks = 0; ks < 2; ++ks)
                 mma_tf32(d, Af + (16 * bi) * AF_LD + 16 * bj + 8 * ks, AF_LD,
                          Tf + (16 * bj + 8 * ks) * AF_LD + 16 * bj + 8 * nt, AF_LD, lane);
-            float* xo = Xs + blk * 16 * XS_LD16 + 8 * nt + 2 * t4;
-            *reinterpret_cast<float2*>(xo + g * XS_LD16) = make_float2(d[0], d[1]);
-            *reinterpret_cast<float2*>(xo + (g + 8) * XS_LD16) = make_float2(d[2], d[3]);
-        }
-        __syncthreads();
-        if (warp < 4) {  // T_10 = -T_11 X, T_32 = -T_33 X
-            const int blk = warp >> 1, nt = warp & 1, bi = 1 + 2 * blk, bj = 2 * blk;
-            float d[4] = {0.f, 0.f, 0.f, 0.f};
+            *reinterpret_cast<float2*>(xw + g * 8 + 2 * t4) = make_float2(d[0], d[1]);
+            *reinterpret_cast<float2*>(xw + (g + 8) * 8 + 2 * t4) = make_float2(d[2], d[3]);
+            __syncwarp();
+            float e[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
             for (int ks = 0; ks < 2; ++ks)
-                mma_tf32(d, Tf + (16 * bi) * AF_LD + 16 * bi + 8 * ks, AF_LD,
-                         Xs + blk * 16 * XS_LD16 + 8 * ks * XS_LD16 + 8 * nt, XS_LD16, lane);
+                mma_tf32(e, Tf + (16 * bi) * AF_LD + 16 * bi + 8 * ks, AF_LD, xw + 8 * ks * 8, 8,
+                         lane);
             float* to = Tf + (16 * bi) * AF_LD + 16 * bj + 8 * nt + 2 * t4;
-            *reinterpret_cast<float2*>(to + g * AF_LD) = make_float2(-d[0], -d[1]);
-            *reinterpret_cast<float2*>(to + (g + 8) * AF_LD) = make_float2(-d[2], -d[3]);
+            *reinterpret_cast<float2*>(to + g * AF_LD) = make_float2(-e[0], -e[1]);
+            *reinterpret_cast<float2*>(to + (g + 8) * AF_LD) = make_float2(-e[2], -e[3]);
         }
         __syncthreads();
-        const int qm = warp >> 2, qn = warp & 3;  // 32x32 products: m-tile qm, n-tile qn
-        {  // X = A_ba T_aa  (T_aa's upper-right 16x16 block is zero)
-            float d[4] = {0.f, 0.f, 0.f, 0.f};
+        //   T_ba = -T_bb (A_ba T_aa)  (a = rows/columns 0..31, b = 32..63): warp qn owns
+        //   n-tile qn of both m-tiles; T_aa's and T_bb's upper-right blocks are zero
+        if (warp < 4) {
+            const int qn = warp;
+            float x0[4] = {0.f, 0.f, 0.f, 0.f}, x1[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
             for (int ks = 0; ks < 4; ++ks)
-                if (qn < 2 || ks >= 2)
-                    mma_tf32(d, Af + (32 + 16 * qm) * AF_LD + 8 * ks, AF_LD,
-                             Tf + (8 * ks) * AF_LD + 8 * qn, AF_LD, lane);
-            float* xo = Xs + (16 * qm) * XS_LD32 + 8 * qn + 2 * t4;
-            *reinterpret_cast<float2*>(xo + g * XS_LD32) = make_float2(d[0], d[1]);
-            *reinterpret_cast<float2*>(xo + (g + 8) * XS_LD32) = make_float2(d[2], d[3]);
-        }
-        __syncthreads();
-        {  // T_ba = -T_bb X  (T_bb's upper-right 16x16 block is zero)
-            float d[4] = {0.f, 0.f, 0.f, 0.f};
+                if (qn < 2 || ks >= 2) {
+                    mma_tf32(x0, Af + 32 * AF_LD + 8 * ks, AF_LD, Tf + (8 * ks) * AF_LD + 8 * qn,
+                             AF_LD, lane);
+                    mma_tf32(x1, Af + 48 * AF_LD + 8 * ks, AF_LD, Tf + (8 * ks) * AF_LD + 8 * qn,
+                             AF_LD, lane);
+                }
+            *reinterpret_cast<float2*>(xw + g * 8 + 2 * t4) = make_float2(x0[0], x0[1]);
+            *reinterpret_cast<float2*>(xw + (g + 8) * 8 + 2 * t4) = make_float2(x0[2], x0[3]);
+            *reinterpret_cast<float2*>(xw + (g + 16) * 8 + 2 * t4) = make_float2(x1[0], x1[1]);
+            *reinterpret_cast<float2*>(xw + (g + 24) * 8 + 2 * t4) = make_float2(x1[2], x1[3]);
+            __syncwarp();
+            float y0[4] = {0.f, 0.f, 0.f, 0.f}, y1[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-            for (int ks = 0; ks < 4; ++ks)
-                if (qm == 1 || ks < 2)
-                    mma_tf32(d, Tf + (32 + 16 * qm) * AF_LD + 32 + 8 * ks, AF_LD,
-                             Xs + (8 * ks) * XS_LD32 + 8 * qn, XS_LD32, lane);
-            float* to = Tf + (32 + 16 * qm) * AF_LD + 8 * qn + 2 * t4;
-            *reinterpret_cast<float2*>(to + g * AF_LD) = make_float2(-d[0], -d[1]);
-            *reinterpret_cast<float2*>(to + (g + 8) * AF_LD) = make_float2(-d[2], -d[3]);
+            for (int ks = 0; ks < 4; ++ks) {
+                if (ks < 2)
+                    mma_tf32(y0, Tf + 32 * AF_LD + 32 + 8 * ks, AF_LD, xw + 8 * ks * 8, 8, lane);
+                mma_tf32(y1, Tf + 48 * AF_LD + 32 + 8 * ks, AF_LD, xw + 8 * ks * 8, 8, lane);
+            }
+            float* to = Tf + 32 * AF_LD + 8 * qn + 2 * t4;
+            *reinterpret_cast<float2*>(to + g * AF_LD) = make_float2(-y0[0], -y0[1]);
+            *reinterpret_cast<float2*>(to + (g + 8) * AF_LD) = make_float2(-y0[2], -y0[3]);
+            *reinterpret_cast<float2*>(to + (g + 16) * AF_LD) = make_float2(-y1[0], -y1[1]);
+            *reinterpret_cast<float2*>(to + (g + 24) * AF_LD) = make_float2(-y1[2], -y1[3]);
         }
         __syncthreads();
         // ---- T diag(beta) as a bf16 tile (lower blocks; the upper ones are never read)
@@ -537,10 +545,14 @@ __global__ void __launch_bounds__(P1_THREADS, 2)
         if (pt == 0) {
             bulk_store(p.records + (size_t)(slot * p.H_v + h) * REC_BYTES, rec, REC_BYTES);
             bulk_commit();
+            bulk_wait_read<0>();  // the record buffer is refilled by the next value head
         }
+        __syncthreads();
     }
     if (pt == 0) bulk_wait_all();
 }
+
+
 
 __device__ __forceinline__ void ldsm_x2_t(uint32_t a, uint32_t* r) {
     asm volatile("ldmatrix.sync.aligned.m8n8.x2.trans.shared.b16 {%0,%1}, [%2];"
@@ -966,6 +978,9 @@ cudaError_t launch_prefill(const void* q, const void* k, const void* v, const fl
     PrefillParams prm{log_alpha, beta, S0, cu_seqlens, o, S_final, records, H_qk, H_v, N, T};
 
     // pass 1: every chunk's operators, all chunks at once
+    int num_sms = 148, dev = 0;
+    if (cudaGetDevice(&dev) == cudaSuccess)
+        cudaDeviceGetAttribute(&num_sms, cudaDevAttrMultiProcessorCount, dev);
     {
         cudaError_t e = cudaFuncSetAttribute(chunk_ops_kernel,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize, P1_SMEM);
@@ -981,9 +996,6 @@ cudaError_t launch_prefill(const void* q, const void* k, const void* v, const fl
     // ~212 KB of shared memory): split every value head into as many d_v slices
     // (4 x 32, 3 x 48 or 2 x 64 columns) as still fit in one wave, so few long
     // sequences still cover the SMs.
-    int num_sms = 148, dev = 0;
-    if (cudaGetDevice(&dev) == cudaSuccess)
-        cudaDeviceGetAttribute(&num_sms, cudaDevAttrMultiProcessorCount, dev);
     const long long units = (long long)N * H_v;
     const int ns = units * 4 <= num_sms ? 32 : (units * 3 <= num_sms ? 48 : 64);
     if (bf16) {
