@@ -164,6 +164,22 @@ GDN_API gdn_status gdn_decode_step(const void *q, const void *k, const void *v,
  */
 GDN_API gdn_status gdn_get_last_device_error(void *stream);
 
+/*
+ * gdn_selftest_bounded_wait -- exercise the library's failure detection on
+ * the device.  (No counterpart in the paper: a test hook for the bounded
+ * waits every kernel of the library uses.)
+ *
+ * Enqueues on `stream` one small kernel whose threads wait, through the same
+ * bounded mbarrier wait the prefill kernels use, on a barrier that nothing
+ * ever arrives at.  The wait gives up after its time limit (about 2 s),
+ * records GDN_ERR_TIMEOUT in the device status word and the kernel returns
+ * normally: no fault, no trap, and the context stays usable.  The next
+ * gdn_get_last_device_error(stream) returns GDN_ERR_TIMEOUT (and clears it).
+ * Returns GDN_OK once enqueued, GDN_ERR_UNSUPPORTED on a device other than
+ * compute capability 10.0, GDN_ERR_CUDA if the launch failed.
+ */
+GDN_API gdn_status gdn_selftest_bounded_wait(void *stream);
+
 /* Static, human-readable name of a status code. */
 GDN_API const char *gdn_status_string(gdn_status status);
 

@@ -27,6 +27,21 @@ cudaError_t read_and_clear_status(unsigned int* status, cudaStream_t stream) {
     return cudaStreamSynchronize(stream);
 }
 
+// Waits (bounded) on an mbarrier that nothing arrives at: the wait gives up,
+// records the timeout in the status word, and every thread returns.
+__global__ void selftest_bounded_wait_kernel() {
+    __shared__ uint64_t bar;
+    __shared__ int abort_flag;
+    if (threadIdx.x == 0) {
+        mbar_init(&bar, 1);
+        abort_flag = 0;
+        fence_mbar_init();
+    }
+    __syncthreads();
+    mbar_wait(&bar, 0, &abort_flag);
+    __syncthreads();
+}
+
 }  // namespace gdn
 
 namespace {
@@ -169,6 +184,13 @@ gdn_status gdn_decode_step(const void* q, const void* k, const void* v, const fl
                                             io_dtype == GDN_BF16, o,
                                             static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+}
+
+gdn_status gdn_selftest_bounded_wait(void* stream) {
+    gdn_status st = check_device();
+    if (st != GDN_OK) return st;
+    gdn::selftest_bounded_wait_kernel<<<1, 64, 0, static_cast<cudaStream_t>(stream)>>>();
+    return cudaGetLastError() == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
 }
 
 gdn_status gdn_get_last_device_error(void* stream) {

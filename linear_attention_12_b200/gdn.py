@@ -42,6 +42,7 @@ SIGNATURES = {
                                    _c.c_void_p, _c.c_void_p, _c.c_int32, _c.c_int32, _c.c_int32,
                                    _c.c_int32, _c.c_int32, _c.c_int, _c.c_void_p, _c.c_void_p]),
     "gdn_get_last_device_error": (_c.c_int, [_c.c_void_p]),
+    "gdn_selftest_bounded_wait": (_c.c_int, [_c.c_void_p]),
     "gdn_status_string": (_c.c_char_p, [_c.c_int]),
     "gdn_version": (_c.c_int32, []),
 }
@@ -167,6 +168,13 @@ def decode_step(q, k, v, log_alpha, beta, S, *, o=None, stream=None):
     if st != GDN_OK:
         raise GDNError(st, "gdn_decode_step")
     return o
+
+
+def selftest_bounded_wait(stream=None) -> None:
+    """Enqueue the library's bounded-wait self-test (a wait that runs out)."""
+    st = lib().gdn_selftest_bounded_wait(_stream_handle(stream))
+    if st != GDN_OK:
+        raise GDNError(st, "gdn_selftest_bounded_wait")
 
 
 def last_device_error(stream=None) -> int:
