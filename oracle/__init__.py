@@ -18,6 +18,9 @@ Two independent formulations live here:
   with numpy.  Slow (O(d^3) per token); for tiny cases only.  It exists to pin
   the C oracle against a differently-written evaluation of the page's formula.
 
+``oracle.frontend`` holds the front end (short causal convolution, L2
+normalisation of q and k, gate activations) in fp64 numpy; see its header.
+
 Inputs are numpy arrays (or CPU torch tensors) in the library's layouts:
 q, k ``[T, H_qk, dk]``; v ``[T, H_v, dv]`` (bf16 as uint16 bits, or float32);
 log_alpha, beta ``[T, H_v]`` float32; S0 ``[N, H_v, dk, dv]`` float32 or None;
