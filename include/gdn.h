@@ -68,6 +68,11 @@ typedef enum {
     GDN_F32 = 2    /* q, k, v and o are float32 (computed through bf16 tensor-core operands) */
 } gdn_dtype;
 
+typedef enum {
+    GDN_ACT_NONE = 0,  /* no activation after the short convolution */
+    GDN_ACT_SILU = 1   /* y * sigmoid(y) after the short convolution */
+} gdn_activation;
+
 /*
  * gdn_prefill -- run the recurrence over N packed sequences (chunked prefill).
  *
@@ -179,6 +184,57 @@ GDN_API gdn_status gdn_get_last_device_error(void *stream);
  * compute capability 10.0, GDN_ERR_CUDA if the launch failed.
  */
 GDN_API gdn_status gdn_selftest_bounded_wait(void *stream);
+
+/*
+ * gdn_frontend -- the step before the recurrence: turn a layer's raw q, k, v
+ * projections and gate pre-activations into gdn_prefill's inputs.
+ *
+ * The jianying88.com article "Qwen3.8-Flash-Next混合注意力深度解析…",
+ * section 三, gives the GDN layer a short convolution of kernel width 4
+ * (config linear_conv_kernel_dim 4) and prints no formula.  This library
+ * reads it as a causal depthwise convolution of every q, k and v channel
+ * within its sequence, followed by an optional activation (the pages name
+ * none), then normalises q and k per (token, head) and activates the gates as
+ * the workloads' recipes do:
+ *
+ *     y[t, c]   = sum_{i=0..3} conv_w[c, i] x[t - 3 + i, c]   (x = 0 before the sequence start)
+ *     y         = act(y)                                      (GDN_ACT_NONE or GDN_ACT_SILU)
+ *     q, k      = y / sqrt(sum over the head's d channels of y^2 + eps)
+ *     v         = y
+ *     log_alpha = -softplus(a),  beta = sigmoid(b)
+ *
+ *   q_raw, k_raw [T, H_qk, dk], v_raw [T, H_v, dv] : io_dtype; a, b [T, H_v] fp32.
+ *   conv_w    : fp32 [(2 H_qk + H_v) * 128, 4]: the q channels (head-major),
+ *               then k, then v; tap 3 weighs the current token.
+ *   cu_seqlens: as for gdn_prefill (the convolution restarts at each sequence).
+ *   q, k, v   : outputs, shapes and dtype of the raw inputs (must not overlap them).
+ *   log_alpha, beta : outputs [T, H_v] fp32.
+ *   All tensor pointers 16-byte aligned; a, b, log_alpha, beta 4-byte aligned.
+ *
+ * Returns GDN_OK, GDN_ERR_INVALID_ARG, GDN_ERR_UNSUPPORTED or GDN_ERR_CUDA.
+ */
+GDN_API gdn_status gdn_frontend(const void *q_raw, const void *k_raw, const void *v_raw,
+                        const float *conv_w, const float *a, const float *b,
+                        const int32_t *cu_seqlens, int32_t N, int32_t T,
+                        int32_t H_qk, int32_t H_v, int32_t dk, int32_t dv,
+                        gdn_dtype io_dtype, gdn_activation act, float eps,
+                        void *q, void *k, void *v, float *log_alpha, float *beta,
+                        void *stream);
+
+/*
+ * gdn_frontend_decode_step -- gdn_frontend for one new token of each of B
+ * sequences.  conv_state [B, 3, (2 H_qk + H_v) * 128] (io_dtype) holds each
+ * sequence's last three raw input rows, oldest first (zeros at a sequence's
+ * start); it is read, then shifted in place to end with this token's raw row.
+ * Other arguments as for gdn_frontend with T = B rows and no cu_seqlens.
+ */
+GDN_API gdn_status gdn_frontend_decode_step(const void *q_raw, const void *k_raw,
+                                    const void *v_raw, const float *conv_w,
+                                    const float *a, const float *b, void *conv_state,
+                                    int32_t B, int32_t H_qk, int32_t H_v, int32_t dk,
+                                    int32_t dv, gdn_dtype io_dtype, gdn_activation act,
+                                    float eps, void *q, void *k, void *v,
+                                    float *log_alpha, float *beta, void *stream);
 
 /* Static, human-readable name of a status code. */
 GDN_API const char *gdn_status_string(gdn_status status);

@@ -186,6 +186,61 @@ gdn_status gdn_decode_step(const void* q, const void* k, const void* v, const fl
     return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
 }
 
+gdn_status gdn_frontend(const void* q_raw, const void* k_raw, const void* v_raw,
+                        const float* conv_w, const float* a, const float* b,
+                        const int32_t* cu_seqlens, int32_t N, int32_t T, int32_t H_qk,
+                        int32_t H_v, int32_t dk, int32_t dv, gdn_dtype io_dtype,
+                        gdn_activation act, float eps, void* q, void* k, void* v,
+                        float* log_alpha, float* beta, void* stream) {
+    gdn_status st = check_heads(H_qk, H_v, dk, dv, io_dtype);
+    if (st != GDN_OK) return st;
+    if (N <= 0 || T < 0 || (act != GDN_ACT_NONE && act != GDN_ACT_SILU) || !(eps >= 0.f))
+        return GDN_ERR_INVALID_ARG;
+    if ((long long)T * H_v * kHeadDim >= (1ll << 40)) return GDN_ERR_INVALID_ARG;
+    if (!cu_seqlens || !aligned(cu_seqlens, 4)) return GDN_ERR_INVALID_ARG;
+    if (T > 0) {
+        const void* p16[] = {q_raw, k_raw, v_raw, conv_w, q, k, v};
+        for (const void* ptr : p16)
+            if (!ptr || !aligned(ptr, 16)) return GDN_ERR_INVALID_ARG;
+        const void* p4[] = {a, b, log_alpha, beta};
+        for (const void* ptr : p4)
+            if (!ptr || !aligned(ptr, 4)) return GDN_ERR_INVALID_ARG;
+    }
+    st = check_device();
+    if (st != GDN_OK) return st;
+    cudaError_t e = gdn::launch_frontend(q_raw, k_raw, v_raw, conv_w, a, b, cu_seqlens, N, T, H_qk,
+                                         H_v, io_dtype == GDN_BF16, (int)act, eps, q, k, v,
+                                         log_alpha, beta, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+}
+
+gdn_status gdn_frontend_decode_step(const void* q_raw, const void* k_raw, const void* v_raw,
+                                    const float* conv_w, const float* a, const float* b,
+                                    void* conv_state, int32_t B, int32_t H_qk, int32_t H_v,
+                                    int32_t dk, int32_t dv, gdn_dtype io_dtype,
+                                    gdn_activation act, float eps, void* q, void* k, void* v,
+                                    float* log_alpha, float* beta, void* stream) {
+    gdn_status st = check_heads(H_qk, H_v, dk, dv, io_dtype);
+    if (st != GDN_OK) return st;
+    if (B < 0 || (act != GDN_ACT_NONE && act != GDN_ACT_SILU) || !(eps >= 0.f))
+        return GDN_ERR_INVALID_ARG;
+    if ((long long)B * (2 * H_qk + H_v) >= (1ll << 31)) return GDN_ERR_INVALID_ARG;
+    if (B == 0) return GDN_OK;
+    const void* p16[] = {q_raw, k_raw, v_raw, conv_w, conv_state, q, k, v};
+    for (const void* ptr : p16)
+        if (!ptr || !aligned(ptr, 16)) return GDN_ERR_INVALID_ARG;
+    const void* p4[] = {a, b, log_alpha, beta};
+    for (const void* ptr : p4)
+        if (!ptr || !aligned(ptr, 4)) return GDN_ERR_INVALID_ARG;
+    st = check_device();
+    if (st != GDN_OK) return st;
+    cudaError_t e = gdn::launch_frontend_decode(q_raw, k_raw, v_raw, conv_w, a, b, conv_state, B,
+                                                H_qk, H_v, io_dtype == GDN_BF16, (int)act, eps,
+                                                q, k, v, log_alpha, beta,
+                                                static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+}
+
 gdn_status gdn_selftest_bounded_wait(void* stream) {
     gdn_status st = check_device();
     if (st != GDN_OK) return st;

@@ -19,6 +19,18 @@ cudaError_t launch_prefill(const void* q, const void* k, const void* v, const fl
                            int T, int H_qk, int H_v, bool bf16, void* o, float* S_final,
                            void* workspace, cudaStream_t stream);
 
+cudaError_t launch_frontend(const void* q_raw, const void* k_raw, const void* v_raw,
+                            const float* conv_w, const float* a, const float* b,
+                            const int32_t* cu_seqlens, int N, int T, int H_qk, int H_v,
+                            bool bf16, int act, float eps, void* q, void* k, void* v,
+                            float* log_alpha, float* beta, cudaStream_t stream);
+
+cudaError_t launch_frontend_decode(const void* q_raw, const void* k_raw, const void* v_raw,
+                                   const float* conv_w, const float* a, const float* b,
+                                   void* conv_state, int B, int H_qk, int H_v, bool bf16, int act,
+                                   float eps, void* q, void* k, void* v, float* log_alpha,
+                                   float* beta, cudaStream_t stream);
+
 cudaError_t read_and_clear_status(unsigned int* status, cudaStream_t stream);
 
 // Fixed-size device scratch used by gdn_prefill_noalloc (bytes, and its address

@@ -23,6 +23,9 @@ GDN_ERR_TIMEOUT = 4
 GDN_ERR_WORKSPACE = 5
 GDN_BF16 = 1
 GDN_F32 = 2
+GDN_ACT_NONE = 0
+GDN_ACT_SILU = 1
+_ACTS = {"none": GDN_ACT_NONE, "silu": GDN_ACT_SILU}
 
 # Every exported symbol of include/gdn.h with its ctypes signature.
 _c = ctypes
@@ -41,6 +44,11 @@ SIGNATURES = {
     "gdn_decode_step": (_c.c_int, [_c.c_void_p, _c.c_void_p, _c.c_void_p, _c.c_void_p,
                                    _c.c_void_p, _c.c_void_p, _c.c_int32, _c.c_int32, _c.c_int32,
                                    _c.c_int32, _c.c_int32, _c.c_int, _c.c_void_p, _c.c_void_p]),
+    "gdn_frontend": (_c.c_int, [_c.c_void_p] * 7 + [_c.c_int32] * 6 + [_c.c_int, _c.c_int,
+                                                                         _c.c_float] +
+                     [_c.c_void_p] * 6),
+    "gdn_frontend_decode_step": (_c.c_int, [_c.c_void_p] * 7 + [_c.c_int32] * 5 +
+                                 [_c.c_int, _c.c_int, _c.c_float] + [_c.c_void_p] * 6),
     "gdn_get_last_device_error": (_c.c_int, [_c.c_void_p]),
     "gdn_selftest_bounded_wait": (_c.c_int, [_c.c_void_p]),
     "gdn_status_string": (_c.c_char_p, [_c.c_int]),
@@ -168,6 +176,68 @@ def decode_step(q, k, v, log_alpha, beta, S, *, o=None, stream=None):
     if st != GDN_OK:
         raise GDNError(st, "gdn_decode_step")
     return o
+
+
+def frontend(q_raw, k_raw, v_raw, conv_w, a, b, cu_seqlens=None, *, act="none", eps=1e-6,
+             out=None, stream=None):
+    """Short causal convolution, q/k L2 normalisation and gate activations.
+
+    Returns ``(q, k, v, log_alpha, beta)`` -- gdn_prefill's inputs.  ``out``
+    may supply those five tensors."""
+    T, H_qk, dk = q_raw.shape
+    H_v, dv = v_raw.shape[1], v_raw.shape[2]
+    dt = q_raw.dtype
+    _check(q_raw, "q_raw", dt)
+    _check(k_raw, "k_raw", dt, q_raw.shape)
+    _check(v_raw, "v_raw", dt, (T, H_v, dv))
+    _check(conv_w, "conv_w", torch.float32, ((2 * H_qk + H_v) * dk, 4))
+    _check(a, "a", torch.float32, (T, H_v))
+    _check(b, "b", torch.float32, (T, H_v))
+    if cu_seqlens is None:
+        cu_seqlens = torch.tensor([0, T], dtype=torch.int32, device=q_raw.device)
+    _check(cu_seqlens, "cu_seqlens", torch.int32)
+    N = cu_seqlens.numel() - 1
+    if out is None:
+        out = (torch.empty_like(q_raw), torch.empty_like(k_raw), torch.empty_like(v_raw),
+               torch.empty_like(a), torch.empty_like(b))
+    q, k, v, la, be = out
+    for t, ref, name in ((q, q_raw, "q"), (k, k_raw, "k"), (v, v_raw, "v")):
+        _check(t, name, dt, ref.shape)
+    _check(la, "log_alpha", torch.float32, (T, H_v))
+    _check(be, "beta", torch.float32, (T, H_v))
+    st = lib().gdn_frontend(_ptr(q_raw), _ptr(k_raw), _ptr(v_raw), _ptr(conv_w), _ptr(a), _ptr(b),
+                            _ptr(cu_seqlens), N, T, H_qk, H_v, dk, dv, _io_dtype(q_raw),
+                            _ACTS[act], float(eps), _ptr(q), _ptr(k), _ptr(v), _ptr(la), _ptr(be),
+                            _stream_handle(stream))
+    if st != GDN_OK:
+        raise GDNError(st, "gdn_frontend")
+    return q, k, v, la, be
+
+
+def frontend_decode_step(q_raw, k_raw, v_raw, conv_w, a, b, conv_state, *, act="none", eps=1e-6,
+                         stream=None):
+    """One decode step of the front end; ``conv_state`` [B, 3, C] is shifted in
+    place.  Returns ``(q, k, v, log_alpha, beta)``."""
+    B, H_qk, dk = q_raw.shape
+    H_v, dv = v_raw.shape[1], v_raw.shape[2]
+    dt = q_raw.dtype
+    _check(q_raw, "q_raw", dt)
+    _check(k_raw, "k_raw", dt, q_raw.shape)
+    _check(v_raw, "v_raw", dt, (B, H_v, dv))
+    _check(conv_w, "conv_w", torch.float32, ((2 * H_qk + H_v) * dk, 4))
+    _check(a, "a", torch.float32, (B, H_v))
+    _check(b, "b", torch.float32, (B, H_v))
+    _check(conv_state, "conv_state", dt, (B, 3, (2 * H_qk + H_v) * dk))
+    q, k, v = torch.empty_like(q_raw), torch.empty_like(k_raw), torch.empty_like(v_raw)
+    la, be = torch.empty_like(a), torch.empty_like(b)
+    st = lib().gdn_frontend_decode_step(_ptr(q_raw), _ptr(k_raw), _ptr(v_raw), _ptr(conv_w),
+                                        _ptr(a), _ptr(b), _ptr(conv_state), B, H_qk, H_v, dk, dv,
+                                        _io_dtype(q_raw), _ACTS[act], float(eps), _ptr(q),
+                                        _ptr(k), _ptr(v), _ptr(la), _ptr(be),
+                                        _stream_handle(stream))
+    if st != GDN_OK:
+        raise GDNError(st, "gdn_frontend_decode_step")
+    return q, k, v, la, be
 
 
 def selftest_bounded_wait(stream=None) -> None:

@@ -15,6 +15,11 @@ of Qwen3.8-Flash-Next: 16 QK heads shared by 48 V heads, head dim 128):
 * S0 = 0.02 * N(0, 1), fp32, or absent (zeros);
 * packed variable-length batches draw their lengths first, uniformly in
   [lo, hi], from the same generator; cu_seqlens is their prefix sum.
+
+Front-end inputs (the raw projections before the short convolution): q_raw,
+k_raw, v_raw ~ N(0, 1) in the I/O dtype, gate pre-activations a, b ~ N(0, 1)
+fp32, convolution weights 0.5 * N(0, 1) fp32 ``[(2 H_qk + H_v) d, 4]``; drawn in
+the order q_raw, k_raw, v_raw, a, b, conv_w.
 """
 from __future__ import annotations
 
@@ -153,3 +158,37 @@ def make_decode(B=256, H_qk=16, H_v=48, d=128, seed=4) -> DecodeCase:
 def batched_decode_256():
     """256 sequences x 48 V heads (16 QK heads), d=128, 512 steps from seed 4."""
     return make_decode(256, 16, 48, 128, seed=4)
+
+
+@dataclasses.dataclass
+class FrontendCase:
+    name: str
+    q_raw: torch.Tensor
+    k_raw: torch.Tensor
+    v_raw: torch.Tensor
+    a: torch.Tensor
+    b: torch.Tensor
+    conv_w: torch.Tensor
+    cu_seqlens: torch.Tensor
+    H_qk: int
+    H_v: int
+    d: int
+
+    @property
+    def T(self) -> int:
+        return self.q_raw.shape[0]
+
+
+def make_frontend(name, seqlens, H_qk, H_v, d=128, dtype=torch.bfloat16, seed=0) -> FrontendCase:
+    """Draw the raw inputs of the front end for packed sequences of ``seqlens``."""
+    gen = torch.Generator().manual_seed(seed)
+    cu = torch.zeros(len(seqlens) + 1, dtype=torch.int32)
+    cu[1:] = torch.cumsum(torch.tensor(seqlens, dtype=torch.int64), 0).to(torch.int32)
+    T = int(cu[-1])
+    q = _draw_rows(gen, T, (H_qk, d), dtype, False)
+    k = _draw_rows(gen, T, (H_qk, d), dtype, False)
+    v = _draw_rows(gen, T, (H_v, d), dtype, False)
+    a = _draw_rows(gen, T, (H_v,), torch.float32, False)
+    b = _draw_rows(gen, T, (H_v,), torch.float32, False)
+    w = 0.5 * _normal(gen, ((2 * H_qk + H_v) * d, 4))
+    return FrontendCase(name, q, k, v, a, b, w, cu, H_qk, H_v, d)

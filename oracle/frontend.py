@@ -80,15 +80,19 @@ def frontend(q_raw, k_raw, v_raw, conv_w, a, b, cu_seqlens=None, act="none", eps
     with the shapes of the inputs.
 
     ``rows`` (optional token indices) restricts the computation to those
-    tokens; the other rows of the returned arrays are NaN.  Each output row
+    tokens and returns only their rows, in that order.  Each output row
     depends on its own token and the three before it, so sampled rows of a
     large input are exact.
     """
-    qr, kr, vr = _widen(q_raw), _widen(k_raw), _widen(v_raw)
-    T, H_qk, d = qr.shape
-    H_v = vr.shape[1]
+    T, H_qk, d = tuple(q_raw.shape)
+    H_v = v_raw.shape[1]
     w = _as_np(conv_w).astype(np.float64).reshape((2 * H_qk + H_v) * d, 4)
-    x = np.concatenate([qr.reshape(T, -1), kr.reshape(T, -1), vr.reshape(T, -1)], axis=1)
+
+    def rows_of(idx):  # raw rows [len(idx), C] in fp64, the q, k, v channels side by side
+        return np.concatenate([_widen(q_raw[idx]).reshape(len(idx), -1),
+                               _widen(k_raw[idx]).reshape(len(idx), -1),
+                               _widen(v_raw[idx]).reshape(len(idx), -1)], axis=1)
+
     if cu_seqlens is None:
         cu = np.array([0, T])
     elif isinstance(cu_seqlens, (list, tuple)):
@@ -96,36 +100,27 @@ def frontend(q_raw, k_raw, v_raw, conv_w, a, b, cu_seqlens=None, act="none", eps
     else:
         cu = _as_np(cu_seqlens).astype(np.int64)
     if rows is None:
-        y = causal_conv(x, w, cu)
         sel = np.arange(T)
+        y = causal_conv(rows_of(sel), w, cu)
     else:
+        # only the sampled rows and the three before each are widened
         sel = np.asarray(rows, dtype=np.int64)
-        y = np.full_like(x, np.nan)
+        y = np.zeros((len(sel), w.shape[0]))
         starts = cu[np.searchsorted(cu, sel, side="right") - 1]
-        for t, t0 in zip(sel, starts):
-            acc = np.zeros(x.shape[1])
-            for i in range(4):
-                tt = t - 3 + i
-                if tt >= t0:
-                    acc = acc + w[:, i] * x[tt]
-            y[t] = acc
+        for r, (t, t0) in enumerate(zip(sel, starts)):
+            taps = [t - 3 + i for i in range(4) if t - 3 + i >= t0]
+            xs = rows_of(np.array(taps, dtype=np.int64))
+            for j, tt in enumerate(taps):
+                y[r] = y[r] + w[:, tt - t + 3] * xs[j]
+    R = len(sel)
     y = _act(y, act)
     nq = H_qk * d
-    q = _l2norm(y[:, :nq].reshape(T, H_qk, d), eps)
-    k = _l2norm(y[:, nq:2 * nq].reshape(T, H_qk, d), eps)
-    v = y[:, 2 * nq:].reshape(T, H_v, d)
-    ad = _as_np(a).astype(np.float64)
-    bd = _as_np(b).astype(np.float64)
-    log_alpha = -softplus(ad)
-    beta = sigmoid(bd)
-    if rows is not None:
-        mask = np.ones(T, dtype=bool)
-        mask[sel] = False
-        log_alpha = log_alpha.copy()
-        beta = beta.copy()
-        log_alpha[mask] = np.nan
-        beta[mask] = np.nan
-    return q, k, v, log_alpha, beta
+    q = _l2norm(y[:, :nq].reshape(R, H_qk, d), eps)
+    k = _l2norm(y[:, nq:2 * nq].reshape(R, H_qk, d), eps)
+    v = y[:, 2 * nq:].reshape(R, H_v, d)
+    ad = _as_np(a).astype(np.float64)[sel]
+    bd = _as_np(b).astype(np.float64)[sel]
+    return q, k, v, -softplus(ad), sigmoid(bd)
 
 
 def frontend_decode_step(q_raw, k_raw, v_raw, conv_w, a, b, conv_state, act="none", eps=1e-6):

@@ -138,3 +138,45 @@ def test_noalloc_rejects_scratch_beyond_its_maximum_on_host(L):
     st = L.gdn_prefill_noalloc(None, P, P, P, P, None, P, 1, 64, 1, 1, 128, 128, gdn.GDN_BF16,
                                P, None, None)
     assert st == gdn.GDN_ERR_INVALID_ARG
+
+
+def _frontend(L, **kw):
+    a = dict(q=P, k=P, v=P, w=P, a=P, b=P, cu=P, N=1, T=64, H_qk=1, H_v=3, dk=128, dv=128,
+             dt=gdn.GDN_BF16, act=gdn.GDN_ACT_NONE, eps=1e-6, oq=P, ok=P, ov=P, la=P, be=P,
+             stream=None)
+    a.update(kw)
+    return L.gdn_frontend(a["q"], a["k"], a["v"], a["w"], a["a"], a["b"], a["cu"], a["N"],
+                          a["T"], a["H_qk"], a["H_v"], a["dk"], a["dv"], a["dt"], a["act"],
+                          a["eps"], a["oq"], a["ok"], a["ov"], a["la"], a["be"], a["stream"])
+
+
+@pytest.mark.parametrize("kw,expect", [
+    (dict(q=None), gdn.GDN_ERR_INVALID_ARG),
+    (dict(w=P + 4), gdn.GDN_ERR_INVALID_ARG),   # the weight is read as float4
+    (dict(ov=BAD), gdn.GDN_ERR_INVALID_ARG),
+    (dict(la=None), gdn.GDN_ERR_INVALID_ARG),
+    (dict(act=2), gdn.GDN_ERR_INVALID_ARG),
+    (dict(eps=-1.0), gdn.GDN_ERR_INVALID_ARG),
+    (dict(eps=float("nan")), gdn.GDN_ERR_INVALID_ARG),
+    (dict(N=0), gdn.GDN_ERR_INVALID_ARG),
+    (dict(H_qk=2, H_v=3), gdn.GDN_ERR_INVALID_ARG),
+    (dict(dk=64, dv=64), gdn.GDN_ERR_UNSUPPORTED),
+])
+def test_frontend_rejects_bad_arguments_on_host(L, kw, expect):
+    assert _frontend(L, **kw) == expect
+
+
+def test_frontend_decode_rejects_bad_arguments_on_host(L):
+    def call(**kw):
+        a = dict(q=P, k=P, v=P, w=P, a=P, b=P, st=P, B=2, H_qk=1, H_v=3, dk=128, dv=128,
+                 dt=gdn.GDN_BF16, act=gdn.GDN_ACT_SILU, eps=0.0, oq=P, ok=P, ov=P, la=P, be=P)
+        a.update(kw)
+        return L.gdn_frontend_decode_step(a["q"], a["k"], a["v"], a["w"], a["a"], a["b"],
+                                          a["st"], a["B"], a["H_qk"], a["H_v"], a["dk"], a["dv"],
+                                          a["dt"], a["act"], a["eps"], a["oq"], a["ok"], a["ov"],
+                                          a["la"], a["be"], None)
+    assert call(st=None) == gdn.GDN_ERR_INVALID_ARG
+    assert call(st=BAD) == gdn.GDN_ERR_INVALID_ARG
+    assert call(B=-1) == gdn.GDN_ERR_INVALID_ARG
+    assert call(act=7) == gdn.GDN_ERR_INVALID_ARG
+    assert call(B=0, q=None, st=None) == gdn.GDN_OK  # nothing to do, nothing touched
