@@ -6,7 +6,10 @@ Workloads (synthetic, seeded; see linear_attention_12_b200/inputs.py):
   * prefill: B=1, L=32768, 16 QK / 48 V heads, d=128, bf16 q/k/v, fp32 gates,
     S0 = 0, chunk 64 -- the headline ``value`` (tokens/s, whole job);
   * decode: 256 sequences x 48 V heads (16 QK heads), fp32 states updated in
-    place (805 MB) -- reported in the ``decode`` object (GB/s).
+    place (805 MB) -- reported in the ``decode`` object (GB/s);
+  * front end: the short convolution, q/k normalisation and gate activations
+    over the raw inputs of the L=32768 prefill (1.37 GB moved) -- reported in
+    the ``frontend`` object (GB/s).
 Each rank runs its own replica (the layer shards by sequence and head with no
 exchange step; nothing is communicated), so scaling is weak.  Timing: W
 untimed warm-up steps, then K steps bracketed by a barrier and
@@ -44,6 +47,10 @@ STATE_BYTES = H_V * D * D * 4                                                 # 
 # shared by the 3 V heads of a QK head), C = 64.
 FLOP_PER_TOKEN = H_V * (6 * D * D + 3 * 64 * D + (2 * 64 * D) // 3)
 DEC_BYTES = 2 * DEC_B * H_V * D * D * 4 + DEC_B * (2 * H_QK * D * 2 + 2 * H_V * D * 2 + 2 * H_V * 4)
+# front end, per token: raw q, k, v read and normalised q, k, v written (bf16),
+# a, b read and log_alpha, beta written (fp32); plus the conv weight once
+FE_BYTES_PER_TOKEN = 2 * (2 * H_QK + H_V) * D * 2 + 4 * H_V * 4                # 41,728
+FE_WEIGHT_BYTES = (2 * H_QK + H_V) * D * 4 * 4                                  # 163,840
 
 
 def load_peaks():
@@ -55,45 +62,107 @@ def load_peaks():
 
 
 class ClockSampler:
-    """nvidia-smi clocks / throttle reasons sampled during the timed region."""
+    """SM clock and clock-event (throttle) reasons sampled during the timed region.
 
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    Reads NVML every ~2 ms from a thread (nvidia-smi's 200 ms loop would see
+    at most one sample of a region that lasts tens of milliseconds); only
+    samples taken between __enter__ and __exit__ count.  Falls back to
+    ``nvidia-smi -lms 200`` when NVML cannot be opened.  Only reads settings.
+    """
+
+    # NVML clock-event reason bits -> names used in the output
+    REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown"}
+    SMI_FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+                  "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+                  "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
     def __init__(self, gpu_index: int):
         self.gpu = gpu_index
+        self.samples = []       # (time, sm_mhz, reason bits)
+        self.max_mhz = None
+        self.source = None
         self.proc = None
-        self.lines = []
+        self.smi_lines = []
+        self._stop = threading.Event()
+        self.t_start = self.t_stop = None
+
+    def _nvml_handle(self):
+        import pynvml
+        import torch
+        pynvml.nvmlInit()
+        props = torch.cuda.get_device_properties(self.gpu)
+        try:
+            bus = f"{props.pci_domain_id:08X}:{props.pci_bus_id:02X}:{props.pci_device_id:02X}.0"
+            return pynvml, pynvml.nvmlDeviceGetHandleByPciBusId(bus)
+        except Exception:
+            return pynvml, pynvml.nvmlDeviceGetHandleByIndex(self.gpu)
+
+    def _poll(self, nv, h):
+        while not self._stop.is_set():
+            try:
+                mhz = nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)
+                bits = nv.nvmlDeviceGetCurrentClocksEventReasons(h)
+                self.samples.append((time.monotonic(), float(mhz), int(bits)))
+            except Exception:
+                pass
+            time.sleep(0.002)
 
     def __enter__(self):
         try:
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "200"],
-                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-            self.t = threading.Thread(target=self._read, daemon=True)
-            self.t.start()
-        except (OSError, FileNotFoundError):
-            self.proc = None
+            nv, h = self._nvml_handle()
+            self.max_mhz = float(nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM))
+            self.source = "nvml"
+            self.thread = threading.Thread(target=self._poll, args=(nv, h), daemon=True)
+            self.thread.start()
+            t_wait = time.monotonic() + 2.0
+            while not self.samples and time.monotonic() < t_wait:
+                time.sleep(0.001)
+        except Exception:
+            self.source = None
+            try:
+                self.proc = subprocess.Popen(
+                    ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.SMI_FIELDS}",
+                     "--format=csv,noheader,nounits", "-lms", "200"],
+                    stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+                self.source = "nvidia-smi"
+                self.thread = threading.Thread(target=self._read_smi, daemon=True)
+                self.thread.start()
+                time.sleep(0.5)  # let nvidia-smi start before the region
+            except (OSError, FileNotFoundError):
+                self.proc = None
+        self.t_start = time.monotonic()
         return self
 
-    def _read(self):
+    def _read_smi(self):
         for line in self.proc.stdout:
-            self.lines.append(line.strip())
+            self.smi_lines.append(line.strip())
 
     def __exit__(self, *a):
+        self.t_stop = time.monotonic()
+        self._stop.set()
         if self.proc is not None:
+            time.sleep(0.3)  # one more nvidia-smi sample
             self.proc.terminate()
             try:
                 self.proc.wait(timeout=5)
             except subprocess.TimeoutExpired:
                 self.proc.kill()
+        elif self.source == "nvml":
+            self.thread.join(timeout=1.0)
 
     def summary(self):
+        if self.source == "nvml":
+            inside = [(m, b) for t, m, b in self.samples if self.t_start <= t <= self.t_stop]
+            if not inside:
+                return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["not recorded"],
+                        "source": "nvml"}
+            reasons = sorted({nm for _, b in inside for bit, nm in self.REASONS.items() if b & bit})
+            return {"sm_mhz": statistics.median(m for m, _ in inside), "sm_max_mhz": self.max_mhz,
+                    "reasons": reasons, "samples": len(inside), "source": "nvml"}
         sm, mx, reasons = [], None, set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in self.lines:
+        for ln in self.smi_lines:
             parts = [x.strip() for x in ln.split(",")]
             if len(parts) < 9:
                 continue
@@ -108,7 +177,7 @@ class ClockSampler:
         if not sm:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["not recorded"]}
         return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
-                "samples": len(sm)}
+                "samples": len(sm), "source": "nvidia-smi"}
 
 
 def dist_setup(n_gpus):
@@ -136,7 +205,8 @@ def max_over_ranks(x, world):
         return x
     import torch
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
 
@@ -165,6 +235,36 @@ def run_decode(args, dev, stream, world):
     dec_ms = max_over_ranks(d0.elapsed_time(d1), world) / dec_steps
     assert gdn.last_device_error() == gdn.GDN_OK
     return dec_ms, DEC_BYTES / (dec_ms / 1e3) / 1e9
+
+
+def run_frontend(args, dev, stream, world, L):
+    """Time the front end on raw inputs of the prefill's shape; returns
+    (ms per call, GB/s)."""
+    import torch
+    from linear_attention_12_b200 import gdn, inputs
+    fc = inputs.make_frontend(f"frontend_L{L}", [L], H_QK, H_V, d=D, seed=5)
+    qr, kr, vr, a, b, w = (x.to(dev) for x in (fc.q_raw, fc.k_raw, fc.v_raw, fc.a, fc.b,
+                                                fc.conv_w))
+    del fc
+    cu = torch.tensor([0, L], dtype=torch.int32, device=dev)
+    out = (torch.empty_like(qr), torch.empty_like(kr), torch.empty_like(vr),
+           torch.empty_like(a), torch.empty_like(b))
+    fe_steps = max(args.steps, 20)
+    for _ in range(max(args.warmup, 3)):
+        gdn.frontend(qr, kr, vr, w, a, b, cu, out=out)
+    torch.cuda.synchronize()
+    barrier(world)
+    f0 = torch.cuda.Event(enable_timing=True)
+    f1 = torch.cuda.Event(enable_timing=True)
+    f0.record(stream)
+    for _ in range(fe_steps):
+        gdn.frontend(qr, kr, vr, w, a, b, cu, out=out)
+    f1.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    fe_ms = max_over_ranks(f0.elapsed_time(f1), world) / fe_steps
+    assert gdn.last_device_error() == gdn.GDN_OK
+    return fe_ms, (FE_BYTES_PER_TOKEN * L + FE_WEIGHT_BYTES) / (fe_ms / 1e3) / 1e9
 
 
 def run_e2e(args, case, q, k, v, la, be, o, Sf, prefill_step, stream, world, L):
@@ -283,6 +383,11 @@ def run_ours(args):
     if not args.no_decode:
         dec_ms, dec_gbs = run_decode(args, dev, stream, world)
 
+    # ---------------- front end on raw inputs of the same shape
+    fe_ms = fe_gbs = None
+    if not args.no_frontend:
+        fe_ms, fe_gbs = run_frontend(args, dev, stream, world, L)
+
     # ---------------- end to end through the public API, host buffers
     e2e_value = e2e_ms = None
     h2d = d2h = 0
@@ -340,6 +445,17 @@ def run_ours(args):
                 "peak": hbm_peak,
                 "frac": dec_gbs / hbm_peak,
                 "workload": f"decode B={DEC_B} H_qk={H_QK} H_v={H_V} d={D}, fp32 state in place",
+                "steps": max(args.steps, 20),
+            },
+            "frontend": None if fe_gbs is None else {
+                "value": fe_gbs,
+                "unit": "GB/s",
+                "us_per_call": fe_ms * 1e3,
+                "bytes_per_call": FE_BYTES_PER_TOKEN * L + FE_WEIGHT_BYTES,
+                "peak": hbm_peak,
+                "frac": fe_gbs / hbm_peak,
+                "workload": f"front end L={L} H_qk={H_QK} H_v={H_V} d={D} bf16, width-4 conv, "
+                            "no activation, eps 1e-6",
                 "steps": max(args.steps, 20),
             },
             "e2e": None if e2e_value is None else {
@@ -422,13 +538,14 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--cpu-tokens", type=int, default=2048,
                     help="tokens per step of the reference arm's oracle sample (all 48 heads)")
-    ap.add_argument("--cpu-baseline-tokens", type=int, default=8192,
+    ap.add_argument("--cpu-baseline-tokens", type=int, default=L,
                     help="tokens of the cpu_baseline oracle sample (all 48 heads)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--seq-len", type=int, default=L,
                     help="prefill length (the benchmark is L=32768; smaller only for profiling)")
     ap.add_argument("--no-decode", action="store_true", help="skip the decode measurement")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer measurement")
+    ap.add_argument("--no-frontend", action="store_true", help="skip the front-end measurement")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
