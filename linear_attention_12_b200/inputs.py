@@ -144,6 +144,13 @@ class DecodeCase:
         la, be = _draw_gates(gen, self.B, self.H_v, 0.0)
         return q, k, v, la, be
 
+    def window(self, s: int, M: int, dtype=torch.bfloat16):
+        """Inputs of steps ``s .. s+M-1`` stacked on a token axis (a verify window
+        of M drafted tokens): q, k ``[B, M, H_qk, d]``, v ``[B, M, H_v, d]``,
+        gates ``[B, M, H_v]`` -- the same values ``step`` draws one by one."""
+        steps = [self.step(s + j, dtype) for j in range(M)]
+        return tuple(torch.stack([st[i] for st in steps], dim=1) for i in range(5))
+
 
 def make_decode(B=256, H_qk=16, H_v=48, d=128, seed=4) -> DecodeCase:
     """Batched decode: B sequences, persistent fp32 states from 0.02 * N(0, 1)."""

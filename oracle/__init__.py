@@ -6,7 +6,7 @@ library (``linear_attention_12_b200``) and never imports it.
 
 Two independent formulations live here:
 
-* :func:`prefill` / :func:`decode_step` -- the sequential recurrence of the
+* :func:`prefill` / :func:`decode_step` / :func:`decode_multi` -- the sequential recurrence of the
   bjdmk.com.cn article "为什么 Qwen3.8-Flash-Next 值得单独跑一遍", section 2.1
   "Gated DeltaNet 负责廉价压缩历史" (state-update formula), evaluated token by
   token in plain C (``gdn_oracle.c``) in fp64, in its expanded "new value
@@ -205,6 +205,30 @@ def decode_step(q, k, v, log_alpha, beta, S, units_bh=None, n_threads=None):
     if units_bh is None:
         return o.reshape(B, H_v, dv), S_out.reshape(B, H_v, *S_out.shape[1:])
     return o, S_out
+
+
+def decode_multi(q, k, v, log_alpha, beta, S, n_threads=None):
+    """M decode steps per sequence, taken in order (speculative verification of
+    1 + k drafted tokens): q, k ``[B, M, H_qk, dk]``, v ``[B, M, H_v, dv]``,
+    gates ``[B, M, H_v]``, S ``[B, H_v, dk, dv]``.
+
+    Token j of every sequence is one application of the state-update formula
+    to the state left by token j - 1, i.e. :func:`decode_step` called M times.
+    Returns ``(o [B, M, H_v, dv], S_steps [B, M, H_v, dk, dv])`` in fp64, where
+    ``S_steps[:, j]`` is the state after token j (the state to keep when the
+    first j + 1 tokens are accepted).
+    """
+    qn, kn, vn = _as_np(q), _as_np(k), _as_np(v)
+    la, be = _as_np(log_alpha), _as_np(beta)
+    M = qn.shape[1]
+    state = S
+    outs, states = [], []
+    for j in range(M):
+        o_j, state = decode_step(qn[:, j], kn[:, j], vn[:, j], la[:, j], be[:, j], state,
+                                 n_threads=n_threads)
+        outs.append(o_j)
+        states.append(state)
+    return np.stack(outs, axis=1), np.stack(states, axis=1)
 
 
 def _widen(x) -> np.ndarray:
