@@ -7,6 +7,8 @@ Workloads (synthetic, seeded; see linear_attention_12_b200/inputs.py):
     S0 = 0, chunk 64 -- the headline ``value`` (tokens/s, whole job);
   * decode: 256 sequences x 48 V heads (16 QK heads), fp32 states updated in
     place (805 MB) -- reported in the ``decode`` object (GB/s);
+  * multi-token decode: 4 tokens per sequence for the same 256 x 48 heads, a
+    state checkpoint after each (4.0 GB moved) -- the ``decode_multi`` object;
   * front end: the short convolution, q/k normalisation and gate activations
     over the raw inputs of the L=32768 prefill (1.37 GB moved) -- reported in
     the ``frontend`` object (GB/s).
@@ -47,6 +49,11 @@ STATE_BYTES = H_V * D * D * 4                                                 # 
 # shared by the 3 V heads of a QK head), C = 64.
 FLOP_PER_TOKEN = H_V * (6 * D * D + 3 * 64 * D + (2 * 64 * D) // 3)
 DEC_BYTES = 2 * DEC_B * H_V * D * D * 4 + DEC_B * (2 * H_QK * D * 2 + 2 * H_V * D * 2 + 2 * H_V * 4)
+# multi-token decode (speculative verification, M = 4 tokens: 3 drafted + 1):
+# the state read once and written after each token, plus the tokens' inputs/outputs
+DM_M = 4
+DM_BYTES = ((1 + DM_M) * DEC_B * H_V * D * D * 4
+            + DEC_B * DM_M * (2 * H_QK * D * 2 + 2 * H_V * D * 2 + 2 * H_V * 4))
 # front end, per token: raw q, k, v read and normalised q, k, v written (bf16),
 # a, b read and log_alpha, beta written (fp32); plus the conv weight once
 FE_BYTES_PER_TOKEN = 2 * (2 * H_QK + H_V) * D * 2 + 4 * H_V * 4                # 41,728
@@ -237,6 +244,34 @@ def run_decode(args, dev, stream, world):
     return dec_ms, DEC_BYTES / (dec_ms / 1e3) / 1e9
 
 
+def run_decode_multi(args, dev, stream, world):
+    """Time M = 4 token verification steps on the 256-sequence workload;
+    returns (ms per call, GB/s)."""
+    import torch
+    from linear_attention_12_b200 import gdn, inputs
+    dc = inputs.batched_decode_256()
+    S_in = dc.S0.to(dev)
+    win = [x.to(dev) for x in dc.window(0, DM_M)]
+    o = torch.empty((DEC_B, DM_M, H_V, D), dtype=torch.bfloat16, device=dev)
+    S_steps = torch.empty((DEC_B, DM_M, H_V, D, D), dtype=torch.float32, device=dev)
+    n = max(args.steps, 10)
+    for _ in range(max(args.warmup, 3)):
+        gdn.decode_multi(*win, S_in, o=o, S_steps=S_steps)
+    torch.cuda.synchronize()
+    barrier(world)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(n):
+        gdn.decode_multi(*win, S_in, o=o, S_steps=S_steps)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    ms = max_over_ranks(e0.elapsed_time(e1), world) / n
+    assert gdn.last_device_error() == gdn.GDN_OK
+    return ms, DM_BYTES / (ms / 1e3) / 1e9
+
+
 def run_frontend(args, dev, stream, world, L):
     """Time the front end on raw inputs of the prefill's shape; returns
     (ms per call, GB/s)."""
@@ -383,6 +418,11 @@ def run_ours(args):
     if not args.no_decode:
         dec_ms, dec_gbs = run_decode(args, dev, stream, world)
 
+    # ---------------- multi-token decode (verification of 3 drafted tokens)
+    dm_ms = dm_gbs = None
+    if not args.no_decode:
+        dm_ms, dm_gbs = run_decode_multi(args, dev, stream, world)
+
     # ---------------- front end on raw inputs of the same shape
     fe_ms = fe_gbs = None
     if not args.no_frontend:
@@ -446,6 +486,18 @@ def run_ours(args):
                 "frac": dec_gbs / hbm_peak,
                 "workload": f"decode B={DEC_B} H_qk={H_QK} H_v={H_V} d={D}, fp32 state in place",
                 "steps": max(args.steps, 20),
+            },
+            "decode_multi": None if dm_gbs is None else {
+                "value": dm_gbs,
+                "unit": "GB/s",
+                "us_per_call": dm_ms * 1e3,
+                "tokens_per_s": DEC_B * DM_M / (dm_ms / 1e3),
+                "bytes_per_call": DM_BYTES,
+                "peak": hbm_peak,
+                "frac": dm_gbs / hbm_peak,
+                "workload": f"decode of M={DM_M} tokens per sequence, B={DEC_B} H_qk={H_QK} "
+                            f"H_v={H_V} d={D}, fp32 state read once, a checkpoint per token",
+                "steps": max(args.steps, 10),
             },
             "frontend": None if fe_gbs is None else {
                 "value": fe_gbs,

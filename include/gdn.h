@@ -161,6 +161,38 @@ GDN_API gdn_status gdn_decode_step(const void *q, const void *k, const void *v,
                            int32_t dk, int32_t dv, gdn_dtype io_dtype,
                            void *o, void *stream);
 
+/* Most tokens per sequence that one gdn_decode_multi call takes. */
+#define GDN_MAX_DECODE_TOKENS 8
+
+/*
+ * gdn_decode_multi -- advance B independent sequences by M tokens each, keeping
+ * the state after every token (speculative verification of drafted tokens).
+ *
+ * Defined by the same state-update formula as gdn_decode_step (bjdmk.com.cn
+ * article "为什么 Qwen3.8-Flash-Next 值得单独跑一遍", section 2.1), applied to the
+ * M tokens of each sequence in order; the pages' multi-token prediction runs
+ * with num_speculative_tokens = 3, i.e. M = 4 tokens per verification step.
+ *
+ *   q, k [B, M, H_qk, dk], v [B, M, H_v, dv] (io_dtype), token-major within a
+ *     sequence; log_alpha, beta [B, M, H_v] fp32.
+ *   S_in [B, H_v, dk, dv] fp32: the state before the first token (read only).
+ *   o [B, M, H_v, dv] (io_dtype): o[b, j] = S_{b,j}^T q[b, j].
+ *   S_steps [B, M, H_v, dk, dv] fp32 (written): S_steps[b, j] is the state after
+ *     token j -- the state to continue from when the first j + 1 tokens are
+ *     accepted.
+ *
+ * 1 <= M <= GDN_MAX_DECODE_TOKENS.  S_steps must not overlap S_in, except that
+ * M == 1 with S_steps == S_in updates the state in place (gdn_decode_step).
+ * One pass over the state: each 64 KiB state is read once and written M times.
+ * The caller owns every buffer.
+ * Returns GDN_OK, GDN_ERR_INVALID_ARG, GDN_ERR_UNSUPPORTED or GDN_ERR_CUDA.
+ */
+GDN_API gdn_status gdn_decode_multi(const void *q, const void *k, const void *v,
+                            const float *log_alpha, const float *beta,
+                            const float *S_in, int32_t B, int32_t M, int32_t H_qk,
+                            int32_t H_v, int32_t dk, int32_t dv, gdn_dtype io_dtype,
+                            void *o, float *S_steps, void *stream);
+
 /*
  * gdn_get_last_device_error -- synchronise `stream`, then read and clear the
  * current device's status word.  Returns GDN_ERR_TIMEOUT if a kernel gave up

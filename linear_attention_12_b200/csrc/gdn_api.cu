@@ -186,6 +186,36 @@ gdn_status gdn_decode_step(const void* q, const void* k, const void* v, const fl
     return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
 }
 
+gdn_status gdn_decode_multi(const void* q, const void* k, const void* v, const float* log_alpha,
+                            const float* beta, const float* S_in, int32_t B, int32_t M,
+                            int32_t H_qk, int32_t H_v, int32_t dk, int32_t dv,
+                            gdn_dtype io_dtype, void* o, float* S_steps, void* stream) {
+    gdn_status st = check_heads(H_qk, H_v, dk, dv, io_dtype);
+    if (st != GDN_OK) return st;
+    if (B < 0 || M < 1 || M > GDN_MAX_DECODE_TOKENS) return GDN_ERR_INVALID_ARG;
+    if ((long long)B * M * H_v >= (1ll << 31)) return GDN_ERR_INVALID_ARG;
+    if (B == 0) return GDN_OK;
+    if (!q || !k || !v || !log_alpha || !beta || !S_in || !o || !S_steps)
+        return GDN_ERR_INVALID_ARG;
+    if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) ||
+        !aligned(S_in, 16) || !aligned(S_steps, 16) || !aligned(log_alpha, 4) ||
+        !aligned(beta, 4))
+        return GDN_ERR_INVALID_ARG;
+    // the kernel reads S_in while other blocks write S_steps: no overlap, except
+    // the in-place single step
+    const uintptr_t in0 = reinterpret_cast<uintptr_t>(S_in);
+    const uintptr_t in1 = in0 + (uintptr_t)B * H_v * dk * dv * sizeof(float);
+    const uintptr_t out0 = reinterpret_cast<uintptr_t>(S_steps);
+    const uintptr_t out1 = out0 + (uintptr_t)B * M * H_v * dk * dv * sizeof(float);
+    if (in0 < out1 && out0 < in1 && !(M == 1 && in0 == out0)) return GDN_ERR_INVALID_ARG;
+    st = check_device();
+    if (st != GDN_OK) return st;
+    cudaError_t e = gdn::launch_decode_multi(q, k, v, log_alpha, beta, S_in, S_steps, B, M, H_qk,
+                                             H_v, io_dtype == GDN_BF16, o,
+                                             static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+}
+
 gdn_status gdn_frontend(const void* q_raw, const void* k_raw, const void* v_raw,
                         const float* conv_w, const float* a, const float* b,
                         const int32_t* cu_seqlens, int32_t N, int32_t T, int32_t H_qk,

@@ -10,6 +10,10 @@ namespace gdn {
 cudaError_t launch_decode_step(const void* q, const void* k, const void* v,
                                const float* log_alpha, const float* beta, float* S, int B,
                                int H_qk, int H_v, bool bf16, void* o, cudaStream_t stream);
+cudaError_t launch_decode_multi(const void* q, const void* k, const void* v,
+                                const float* log_alpha, const float* beta, const float* S_in,
+                                float* S_steps, int B, int M, int H_qk, int H_v, bool bf16,
+                                void* o, cudaStream_t stream);
 
 // Workspace bytes the prefill needs (fp32 I/O stages bf16 copies of q, k, v).
 size_t prefill_workspace_bytes(int N, int T, int H_qk, int H_v, bool bf16);

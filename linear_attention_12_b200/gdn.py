@@ -44,6 +44,8 @@ SIGNATURES = {
     "gdn_decode_step": (_c.c_int, [_c.c_void_p, _c.c_void_p, _c.c_void_p, _c.c_void_p,
                                    _c.c_void_p, _c.c_void_p, _c.c_int32, _c.c_int32, _c.c_int32,
                                    _c.c_int32, _c.c_int32, _c.c_int, _c.c_void_p, _c.c_void_p]),
+    "gdn_decode_multi": (_c.c_int, [_c.c_void_p] * 6 + [_c.c_int32] * 6 + [_c.c_int, _c.c_void_p,
+                                                                          _c.c_void_p, _c.c_void_p]),
     "gdn_frontend": (_c.c_int, [_c.c_void_p] * 7 + [_c.c_int32] * 6 + [_c.c_int, _c.c_int,
                                                                          _c.c_float] +
                      [_c.c_void_p] * 6),
@@ -176,6 +178,39 @@ def decode_step(q, k, v, log_alpha, beta, S, *, o=None, stream=None):
     if st != GDN_OK:
         raise GDNError(st, "gdn_decode_step")
     return o
+
+
+MAX_DECODE_TOKENS = 8  # GDN_MAX_DECODE_TOKENS
+
+
+def decode_multi(q, k, v, log_alpha, beta, S_in, *, o=None, S_steps=None, stream=None):
+    """M tokens per sequence in one pass over the state (speculative verification).
+
+    q, k [B, M, H_qk, dk], v [B, M, H_v, dv], gates [B, M, H_v], S_in
+    [B, H_v, dk, dv] fp32 (read only).  Returns ``(o [B, M, H_v, dv],
+    S_steps [B, M, H_v, dk, dv])`` where ``S_steps[:, j]`` is the state after
+    token j."""
+    B, M, H_qk, dk = q.shape
+    H_v, dv = v.shape[2], v.shape[3]
+    dt = q.dtype
+    _check(q, "q", dt)
+    _check(k, "k", dt, q.shape)
+    _check(v, "v", dt, (B, M, H_v, dv))
+    _check(log_alpha, "log_alpha", torch.float32, (B, M, H_v))
+    _check(beta, "beta", torch.float32, (B, M, H_v))
+    _check(S_in, "S_in", torch.float32, (B, H_v, dk, dv))
+    if o is None:
+        o = torch.empty((B, M, H_v, dv), dtype=dt, device=q.device)
+    if S_steps is None:
+        S_steps = torch.empty((B, M, H_v, dk, dv), dtype=torch.float32, device=q.device)
+    _check(o, "o", dt, (B, M, H_v, dv))
+    _check(S_steps, "S_steps", torch.float32, (B, M, H_v, dk, dv))
+    st = lib().gdn_decode_multi(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta),
+                                _ptr(S_in), B, M, H_qk, H_v, dk, dv, _io_dtype(q), _ptr(o),
+                                _ptr(S_steps), _stream_handle(stream))
+    if st != GDN_OK:
+        raise GDNError(st, "gdn_decode_multi")
+    return o, S_steps
 
 
 def frontend(q_raw, k_raw, v_raw, conv_w, a, b, cu_seqlens=None, *, act="none", eps=1e-6,

@@ -111,6 +111,36 @@ def test_decode_rejects_bad_arguments_on_host(L, kw, expect):
     assert _decode(L, **kw) == expect
 
 
+def _decode_multi(L, **kw):
+    a = dict(q=P, k=P, v=P, la=P, be=P, S=P, B=4, M=4, H_qk=1, H_v=3, dk=128, dv=128,
+             dt=gdn.GDN_BF16, o=P, Ss=P + (1 << 30), stream=None)
+    a.update(kw)
+    return L.gdn_decode_multi(a["q"], a["k"], a["v"], a["la"], a["be"], a["S"], a["B"], a["M"],
+                              a["H_qk"], a["H_v"], a["dk"], a["dv"], a["dt"], a["o"], a["Ss"],
+                              a["stream"])
+
+
+_STATE = 3 * 128 * 128 * 4  # bytes of one sequence's states at H_v = 3
+
+
+@pytest.mark.parametrize("kw,expect", [
+    (dict(M=0), gdn.GDN_ERR_INVALID_ARG),
+    (dict(M=9), gdn.GDN_ERR_INVALID_ARG),   # above GDN_MAX_DECODE_TOKENS
+    (dict(Ss=None), gdn.GDN_ERR_INVALID_ARG),
+    (dict(Ss=P + 8), gdn.GDN_ERR_INVALID_ARG),
+    (dict(S=BAD), gdn.GDN_ERR_INVALID_ARG),
+    (dict(B=-1), gdn.GDN_ERR_INVALID_ARG),
+    (dict(Ss=P), gdn.GDN_ERR_INVALID_ARG),                      # checkpoints over the input
+    (dict(Ss=P + 4 * _STATE - 16 * 1024), gdn.GDN_ERR_INVALID_ARG),  # partial overlap
+    (dict(M=1, Ss=P + _STATE), gdn.GDN_ERR_INVALID_ARG),        # M = 1, shifted: overlap
+    (dict(H_qk=2, H_v=3), gdn.GDN_ERR_INVALID_ARG),
+    (dict(dv=64), gdn.GDN_ERR_UNSUPPORTED),
+    (dict(B=0, q=None, S=None, Ss=None), gdn.GDN_OK),  # nothing to do, nothing touched
+])
+def test_decode_multi_rejects_bad_arguments_on_host(L, kw, expect):
+    assert _decode_multi(L, **kw) == expect
+
+
 def test_binding_refuses_cpu_tensors(L):
     import torch
     x = torch.zeros(4, 1, 128, dtype=torch.bfloat16)
