@@ -93,7 +93,10 @@ typedef enum {
  *               head) -- N + ceil(T / 64) slots; about 416 MB for T = 32,768
  *               and 48 value heads -- written by the first of the two passes
  *               of the prefill and read by the second, plus bf16 copies of
- *               q, k, v when io_dtype is GDN_F32.
+ *               q, k, v when io_dtype is GDN_F32.  When few sequences x value
+ *               heads would leave SMs idle, gdn_prefill splits the sequences
+ *               (gdn_prefill_segmented with segments = 0) and the workspace
+ *               also holds that split's states.
  *
  * Returns GDN_OK, GDN_ERR_INVALID_ARG, GDN_ERR_UNSUPPORTED, GDN_ERR_WORKSPACE
  * or GDN_ERR_CUDA.
@@ -107,9 +110,65 @@ GDN_API gdn_status gdn_prefill(const void *q, const void *k, const void *v,
                        void *workspace, size_t workspace_bytes, void *stream);
 
 /* Bytes of device workspace gdn_prefill needs for these sizes (0 when T == 0
- * or the arguments are invalid). */
+ * or the arguments are invalid).  Includes what the automatic sequence split
+ * (gdn_prefill_segmented) needs on the current device. */
 GDN_API size_t gdn_prefill_workspace_size(int32_t N, int32_t T, int32_t H_qk, int32_t H_v,
                                   int32_t dk, int32_t dv, gdn_dtype io_dtype);
+
+/* Most segments per sequence gdn_prefill_segmented takes. */
+#define GDN_MAX_PREFILL_SEGMENTS 64
+
+/*
+ * gdn_prefill_segmented -- gdn_prefill with each sequence split into `segments`
+ * pieces that run side by side on one GPU (sequence parallelism within the
+ * card, for inputs with too few sequences x value heads to fill the SMs: long
+ * contexts, or the few heads a tensor-parallel shard holds).
+ *
+ * The Qwen3.8-Flash-Next article of alwayszhang ("GDN+QSA、门控残差与 N-gram
+ * Embedding…", section 九) names intra-card context parallelism among the
+ * FlashQLA kernel techniques and gives no formulas.  The split done here is
+ * exact, not a truncation of the decay:
+ *   1. The state after a segment is affine in the state before it,
+ *      S_end = P_s S_start + R_s.
+ *   2. Every segment runs twice side by side: from S = 0, which gives R_s, and
+ *      from S = I with v = 0, which gives the d_k x d_k propagator P_s.
+ *   3. A scan over the segments gives each entering state.
+ *   4. Every segment then runs again from that state and writes its outputs.
+ * Segments are whole 64-token chunks: sequence n is cut into `segments`
+ * pieces of ceil(ceil(len_n / 64) / segments) chunks, and trailing pieces may
+ * be empty.  The cost is about 2.5 times the state-carrying work, spread over
+ * `segments` times more blocks; it pays when those blocks would otherwise
+ * leave SMs idle.
+ *
+ *   segments : 0 = choose automatically (what gdn_prefill does; see
+ *              gdn_prefill_auto_segments), 1 = no split, 2 ..
+ *              GDN_MAX_PREFILL_SEGMENTS = that many pieces per sequence.
+ *   workspace: at least gdn_prefill_segmented_workspace_size(..., segments)
+ *              bytes, 256-byte aligned.  A split adds (N x segments) record
+ *              slots, N x segments + 1 int32 segment starts and three
+ *              fp32 states per (piece, value head).
+ * Other arguments, results and errors as gdn_prefill; GDN_ERR_INVALID_ARG also
+ * for `segments` out of range.
+ */
+GDN_API gdn_status gdn_prefill_segmented(const void *q, const void *k, const void *v,
+                                 const float *log_alpha, const float *beta,
+                                 const float *S0, const int32_t *cu_seqlens,
+                                 int32_t N, int32_t T, int32_t H_qk, int32_t H_v,
+                                 int32_t dk, int32_t dv, gdn_dtype io_dtype,
+                                 void *o, float *S_final, int32_t segments,
+                                 void *workspace, size_t workspace_bytes, void *stream);
+
+/* Workspace bytes of gdn_prefill_segmented with these arguments (0 when T == 0
+ * or the arguments are invalid). */
+GDN_API size_t gdn_prefill_segmented_workspace_size(int32_t N, int32_t T, int32_t H_qk,
+                                            int32_t H_v, int32_t dk, int32_t dv,
+                                            gdn_dtype io_dtype, int32_t segments);
+
+/* Segments per sequence gdn_prefill uses for these sizes on the current device:
+ * 1 unless a split fills more SMs (a cost model over the SM count, the
+ * sequences x value heads and the average sequence length; pieces of at least
+ * 8 chunks, at most 16 pieces).  Returns 1 for invalid arguments. */
+GDN_API int32_t gdn_prefill_auto_segments(int32_t N, int32_t T, int32_t H_qk, int32_t H_v);
 
 /*
  * gdn_prefill_noalloc -- gdn_prefill for callers that cannot allocate device

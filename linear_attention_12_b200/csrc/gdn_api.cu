@@ -87,10 +87,25 @@ const char* gdn_status_string(gdn_status s) {
 
 int32_t gdn_version(void) { return 100; }
 
+int32_t gdn_prefill_auto_segments(int32_t N, int32_t T, int32_t H_qk, int32_t H_v) {
+    if (N <= 0 || T < 0 || H_qk <= 0 || H_v <= 0 || H_v % H_qk != 0) return 1;
+    return gdn::choose_segments(N, T, H_v, gdn::device_sms());
+}
+
+size_t gdn_prefill_segmented_workspace_size(int32_t N, int32_t T, int32_t H_qk, int32_t H_v,
+                                            int32_t dk, int32_t dv, gdn_dtype io_dtype,
+                                            int32_t segments) {
+    if (N <= 0 || T < 0 || segments < 0 || segments > GDN_MAX_PREFILL_SEGMENTS ||
+        check_heads(H_qk, H_v, dk, dv, io_dtype) != GDN_OK)
+        return 0;
+    if ((long long)N * (segments > 0 ? segments : 1) >= (1ll << 30)) return 0;
+    const int P = segments > 0 ? segments : gdn_prefill_auto_segments(N, T, H_qk, H_v);
+    return gdn::prefill_workspace_bytes(N, T, H_qk, H_v, io_dtype == GDN_BF16, P);
+}
+
 size_t gdn_prefill_workspace_size(int32_t N, int32_t T, int32_t H_qk, int32_t H_v, int32_t dk,
                                   int32_t dv, gdn_dtype io_dtype) {
-    if (N <= 0 || T < 0 || check_heads(H_qk, H_v, dk, dv, io_dtype) != GDN_OK) return 0;
-    return gdn::prefill_workspace_bytes(N, T, H_qk, H_v, io_dtype == GDN_BF16);
+    return gdn_prefill_segmented_workspace_size(N, T, H_qk, H_v, dk, dv, io_dtype, 0);
 }
 
 }  // extern "C"
@@ -124,24 +139,37 @@ gdn_status check_prefill_args(const void* q, const void* k, const void* v, const
 
 extern "C" {
 
-gdn_status gdn_prefill(const void* q, const void* k, const void* v, const float* log_alpha,
-                       const float* beta, const float* S0, const int32_t* cu_seqlens, int32_t N,
-                       int32_t T, int32_t H_qk, int32_t H_v, int32_t dk, int32_t dv,
-                       gdn_dtype io_dtype, void* o, float* S_final, void* workspace,
-                       size_t workspace_bytes, void* stream) {
+gdn_status gdn_prefill_segmented(const void* q, const void* k, const void* v,
+                                 const float* log_alpha, const float* beta, const float* S0,
+                                 const int32_t* cu_seqlens, int32_t N, int32_t T, int32_t H_qk,
+                                 int32_t H_v, int32_t dk, int32_t dv, gdn_dtype io_dtype, void* o,
+                                 float* S_final, int32_t segments, void* workspace,
+                                 size_t workspace_bytes, void* stream) {
     gdn_status st = check_prefill_args(q, k, v, log_alpha, beta, S0, cu_seqlens, N, T, H_qk, H_v,
                                        dk, dv, io_dtype, o, S_final);
     if (st != GDN_OK) return st;
+    if (segments < 0 || segments > GDN_MAX_PREFILL_SEGMENTS) return GDN_ERR_INVALID_ARG;
+    if ((long long)N * (segments > 0 ? segments : 1) >= (1ll << 30)) return GDN_ERR_INVALID_ARG;
     const bool bf16 = io_dtype == GDN_BF16;
-    const size_t need = gdn::prefill_workspace_bytes(N, T, H_qk, H_v, bf16);
+    const int P = segments > 0 ? segments : gdn_prefill_auto_segments(N, T, H_qk, H_v);
+    const size_t need = gdn::prefill_workspace_bytes(N, T, H_qk, H_v, bf16, P);
     if (need > 0 && (!workspace || workspace_bytes < need || !aligned(workspace, 256)))
         return GDN_ERR_WORKSPACE;
     st = check_device();
     if (st != GDN_OK) return st;
     cudaError_t e = gdn::launch_prefill(q, k, v, log_alpha, beta, S0, cu_seqlens, N, T, H_qk,
-                                        H_v, bf16, o, S_final, workspace,
+                                        H_v, bf16, o, S_final, workspace, P,
                                         static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+}
+
+gdn_status gdn_prefill(const void* q, const void* k, const void* v, const float* log_alpha,
+                       const float* beta, const float* S0, const int32_t* cu_seqlens, int32_t N,
+                       int32_t T, int32_t H_qk, int32_t H_v, int32_t dk, int32_t dv,
+                       gdn_dtype io_dtype, void* o, float* S_final, void* workspace,
+                       size_t workspace_bytes, void* stream) {
+    return gdn_prefill_segmented(q, k, v, log_alpha, beta, S0, cu_seqlens, N, T, H_qk, H_v, dk,
+                                 dv, io_dtype, o, S_final, 0, workspace, workspace_bytes, stream);
 }
 
 gdn_status gdn_prefill_noalloc(const void* q, const void* k, const void* v,

@@ -15,13 +15,22 @@ cudaError_t launch_decode_multi(const void* q, const void* k, const void* v,
                                 float* S_steps, int B, int M, int H_qk, int H_v, bool bf16,
                                 void* o, cudaStream_t stream);
 
-// Workspace bytes the prefill needs (fp32 I/O stages bf16 copies of q, k, v).
-size_t prefill_workspace_bytes(int N, int T, int H_qk, int H_v, bool bf16);
+// Workspace bytes the prefill needs with P segments per sequence (fp32 I/O
+// also stages bf16 copies of q, k, v).
+size_t prefill_workspace_bytes(int N, int T, int H_qk, int H_v, bool bf16, int P);
 
+// SM count of the current device (148 when there is none).
+int device_sms();
+
+// Segments per sequence the prefill uses when the caller leaves it to the
+// library: 1 unless splitting the sequences fills more of the SMs.
+int choose_segments(int N, int T, int H_v, int sms);
+
+// P segments per sequence (P <= 0: choose_segments).
 cudaError_t launch_prefill(const void* q, const void* k, const void* v, const float* log_alpha,
                            const float* beta, const float* S0, const int32_t* cu_seqlens, int N,
                            int T, int H_qk, int H_v, bool bf16, void* o, float* S_final,
-                           void* workspace, cudaStream_t stream);
+                           void* workspace, int P, cudaStream_t stream);
 
 cudaError_t launch_frontend(const void* q_raw, const void* k_raw, const void* v_raw,
                             const float* conv_w, const float* a, const float* b,

@@ -45,6 +45,7 @@
 #include <cudaTypedefs.h>
 
 #include <algorithm>
+#include <cmath>
 #include <mutex>
 
 #include "gdn_common.cuh"
@@ -54,6 +55,7 @@ namespace gdn {
 
 namespace {
 
+constexpr int kMaxSegments = 16;  // most segments per sequence the automatic choice takes
 constexpr int C = 64;            // chunk length
 constexpr int D = 128;           // head dim (d_k = d_v)
 constexpr uint32_t HALF = 8192;  // one 64 x 64 bf16 tile: 64 rows x 128 B
@@ -260,6 +262,7 @@ struct PrefillParams {
     void* o;
     float* S_final;
     uint8_t* records;  // chunk operator records, REC_BYTES each
+    float* S_prop;     // segmented prefill, phase A: the segment propagators
     int H_qk, H_v;
     int N, T;
 };
@@ -612,7 +615,14 @@ __device__ __forceinline__ void delta_half(uint8_t* sm, uint32_t tb, uint32_t xt
 // ============================================================================
 // Pass 2: state pass.  Grid (d_v slices, H_v, N).
 // ============================================================================
-template <int NS, typename IO>
+// MODE P2_OUT: the prefill proper (outputs, final states).  MODE P2_SEGMENT:
+// phase A of the segmented prefill -- no outputs; blocks x < slices carry the
+// state from zero (final state to S_final), blocks x >= slices carry the
+// identity with V taken as zero, so that their final state is the segment's
+// propagator P (to S_prop): S_end = P S_start + (state from zero).
+constexpr int P2_OUT = 0, P2_SEGMENT = 1;
+
+template <int NS, typename IO, int MODE>
 __global__ void __launch_bounds__(P2_THREADS, 1)
     state_pass_kernel(const __grid_constant__ CUtensorMap map_q,
                       const __grid_constant__ CUtensorMap map_k,
@@ -620,6 +630,7 @@ __global__ void __launch_bounds__(P2_THREADS, 1)
     static_assert(NS == 32 || NS == 48 || NS == 64, "slice width");
     constexpr int NT = NS / 8;  // n-tiles of a slice
     constexpr int NP = NT / 2;  // n-tile pairs
+    constexpr int NSL = (D + NS - 1) / NS;  // slices of a head
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
@@ -633,7 +644,8 @@ __global__ void __launch_bounds__(P2_THREADS, 1)
     const int h = blockIdx.y;
     const int n = blockIdx.z;
     const int hq = h / (p.H_v / p.H_qk);
-    const int col0 = blockIdx.x * NS;
+    const bool prop = MODE == P2_SEGMENT && blockIdx.x >= NSL;  // propagator block
+    const int col0 = (blockIdx.x - (prop ? NSL : 0)) * NS;
     const int ncols = min(NS, D - col0);
     const int t_beg = p.cu_seqlens[n];
     const int t_end = p.cu_seqlens[n + 1];
@@ -654,12 +666,12 @@ __global__ void __launch_bounds__(P2_THREADS, 1)
         uint8_t* st = sm + s * STAGE_BYTES;
         const int y = t_beg + c * C;
         uint64_t* full = &bars[B2_FULL + s];
-        mbar_arrive_expect_tx(full, STAGE_TX);
+        mbar_arrive_expect_tx(full, prop ? STAGE_TX - HALF : STAGE_TX);
         tma_load_2d(st + ST_K, &map_k, hq * D, y, full);
         tma_load_2d(st + ST_K + HALF, &map_k, hq * D + 64, y, full);
         tma_load_2d(st + ST_Q, &map_q, hq * D, y, full);
         tma_load_2d(st + ST_Q + HALF, &map_q, hq * D + 64, y, full);
-        tma_load_2d(st + ST_V, &map_v, h * D + col0, y, full);
+        if (!prop) tma_load_2d(st + ST_V, &map_v, h * D + col0, y, full);
         bulk_load(st + ST_REC, p.records + (size_t)(record_slot(n, y) * p.H_v + h) * REC_BYTES,
                   REC_BYTES, full);
     };
@@ -683,7 +695,10 @@ __global__ void __launch_bounds__(P2_THREADS, 1)
                 for (int e = 0; e < 4; ++e) {
                     const int row = r0 + g + ((e >> 1) << 3);
                     const int col = 8 * nt + 2 * t4 + (e & 1);
-                    Sacc[nt][e] = (s0 && col < ncols) ? s0[(size_t)row * D + col0 + col] : 0.f;
+                    if (prop)  // the identity's columns col0 .. col0 + NS - 1
+                        Sacc[nt][e] = (col < ncols && row == col0 + col) ? 1.f : 0.f;
+                    else
+                        Sacc[nt][e] = (s0 && col < ncols) ? s0[(size_t)row * D + col0 + col] : 0.f;
                 }
             store_acc_bf16<NT>(sm, P2_SB, 0, r0, Sacc, lane, 1.f, 1.f);
         }
@@ -710,15 +725,17 @@ __global__ void __launch_bounds__(P2_THREADS, 1)
                 for (int ks = 0; ks < 8; ++ks) {
                     uint32_t ak[4], aq[4];
                     lda_k(st + ST_K, HALF, m0, 16 * ks, lane, ak);
-                    lda_k(st + ST_Q, HALF, m0, 16 * ks, lane, aq);
+                    if constexpr (MODE == P2_OUT) lda_k(st + ST_Q, HALF, m0, 16 * ks, lane, aq);
 #pragma unroll
                     for (int np = 0; np < NP; ++np) {
                         uint32_t b[4];
                         ldb_mn(sb + P2_SB, 0, 16 * np, 16 * ks, lane, b);
                         mma16816(accK[2 * np], ak, b[0], b[1]);
                         mma16816(accK[2 * np + 1], ak, b[2], b[3]);
-                        mma16816(accQ[2 * np], aq, b[0], b[1]);
-                        mma16816(accQ[2 * np + 1], aq, b[2], b[3]);
+                        if constexpr (MODE == P2_OUT) {
+                            mma16816(accQ[2 * np], aq, b[0], b[1]);
+                            mma16816(accQ[2 * np + 1], aq, b[2], b[3]);
+                        }
                     }
                 }
                 // X = V - gamma o (K S)   (rows past the sequence end are zero: V and K are);
@@ -728,10 +745,13 @@ __global__ void __launch_bounds__(P2_THREADS, 1)
 #pragma unroll
                 for (int nt = 0; nt < NT; ++nt) {
                     const int col = 8 * nt + 2 * t4;
-                    const float2 v_lo = __bfloat1622float2(
-                        *reinterpret_cast<const __nv_bfloat162*>(vt + taddr_e(0, m0 + g, col, 0)));
-                    const float2 v_hi = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(
-                        vt + taddr_e(0, m0 + g + 8, col, 0)));
+                    float2 v_lo = make_float2(0.f, 0.f), v_hi = v_lo;
+                    if (!prop) {
+                        v_lo = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(
+                            vt + taddr_e(0, m0 + g, col, 0)));
+                        v_hi = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(
+                            vt + taddr_e(0, m0 + g + 8, col, 0)));
+                    }
                     accK[nt][0] = v_lo.x - gm_lo * accK[nt][0];
                     accK[nt][1] = v_lo.y - gm_lo * accK[nt][1];
                     accK[nt][2] = v_hi.x - gm_hi * accK[nt][2];
@@ -778,7 +798,7 @@ __global__ void __launch_bounds__(P2_THREADS, 1)
                 }
             }
             // ---- O = gamma o (Q S) + (M o Q K^T) Delta   (warps 0-3), stored
-            if (mw) {
+            if (MODE == P2_OUT && mw) {
 #pragma unroll
                 for (int ks = 0; ks < 4; ++ks) {
                     if (ks <= warp) {
@@ -813,8 +833,9 @@ __global__ void __launch_bounds__(P2_THREADS, 1)
             // this ring stage is free again: refill it with the chunk NSTAGE ahead
             if (tid == P2_LOADER && c + NSTAGE < nchunks) issue_chunk(issued++);
         }
-        if (p.S_final && !*abort_flag) {
-            float* sf = p.S_final + ((size_t)n * p.H_v + h) * D * D;
+        float* const s_out = prop ? p.S_prop : p.S_final;
+        if (s_out && !*abort_flag) {
+            float* sf = s_out + ((size_t)n * p.H_v + h) * D * D;
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
@@ -885,14 +906,111 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols) {
            CUDA_SUCCESS;
 }
 
-template <int NS, typename IO>
+// ---- segmented prefill (sequence parallelism within one GPU) -------------
+// Each sequence is cut into P segments of whole chunks, run as P "virtual"
+// sequences.  Phase A carries every segment's state from zero (R) and its
+// propagator (P_s, the map of the segment on the entering state); a scan over
+// the segments gives the true entering states, S <- P_s S + R_s; phase C reruns
+// the segments from those states and writes the outputs.
+
+// cu_v[n P + i] = start of segment i of sequence n (chunk-aligned), cu_v[N P] = T.
+__global__ void segment_cu_kernel(const int32_t* __restrict__ cu, int N, int P,
+                                  int32_t* __restrict__ cu_v) {
+    const int idx = blockIdx.x * blockDim.x + threadIdx.x;
+    if (idx > N * P) return;
+    if (idx == N * P) {
+        cu_v[idx] = cu[N];
+        return;
+    }
+    const int n = idx / P, i = idx - n * P;
+    const int len = cu[n + 1] - cu[n];
+    const int per = ((len + C - 1) / C + P - 1) / P;  // chunks per segment
+    cu_v[idx] = cu[n] + min(i * per * C, len);
+}
+
+// Block (column block cb of 32, value head h, sequence n): S_entry[n P + s] is
+// the state entering segment s, S_final[n] the state after the last one;
+// S <- P_s S + R_s from S0[n] (or zero), in fp32.  Each step stages P_s in
+// shared memory (all its loads in flight at once; rows padded to 132 floats
+// so that the row-wise float4 reads below hit distinct banks).
+constexpr int SCAN_COLS = 32;
+constexpr int SCAN_LD = D + 4;
+constexpr uint32_t SCAN_SMEM = (D * SCAN_LD + D * SCAN_COLS) * sizeof(float);  // 83,968 B
+__global__ void __launch_bounds__(256)
+    segment_scan_kernel(const float* __restrict__ S0, const float* __restrict__ R,
+                        const float* __restrict__ Pm, float* __restrict__ S_entry,
+                        float* S_final, int P, int H_v) {
+    extern __shared__ float4 scan_sm4[];
+    float* Ps = reinterpret_cast<float*>(scan_sm4);  // [D][SCAN_LD]
+    float* cur = Ps + D * SCAN_LD;                   // [D][SCAN_COLS]
+    const int cb = blockIdx.x, h = blockIdx.y, n = blockIdx.z;
+    const int t = threadIdx.x, i = t >> 1, j0 = (t & 1) * 16;
+    const size_t hs = (size_t)D * D;
+    const size_t c0 = (size_t)cb * SCAN_COLS;
+    for (int e = t; e < D * SCAN_COLS; e += blockDim.x) {
+        const int r = e / SCAN_COLS, c = e % SCAN_COLS;
+        cur[e] = S0 ? S0[((size_t)n * H_v + h) * hs + (size_t)r * D + c0 + c] : 0.f;
+    }
+    for (int sg = 0; sg < P; ++sg) {
+        const size_t base = (((size_t)n * P + sg) * H_v + h) * hs;
+        const float4* P4 = reinterpret_cast<const float4*>(Pm + base);
+        for (int e = t; e < D * D / 4; e += blockDim.x) {
+            const int r = e / (D / 4), c4 = e % (D / 4);
+            *reinterpret_cast<float4*>(Ps + r * SCAN_LD + 4 * c4) = P4[e];
+        }
+        float acc[16];
+        const float4* R4 = reinterpret_cast<const float4*>(R + base + (size_t)i * D + c0 + j0);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const float4 rv = R4[q];
+            acc[4 * q] = rv.x;
+            acc[4 * q + 1] = rv.y;
+            acc[4 * q + 2] = rv.z;
+            acc[4 * q + 3] = rv.w;
+        }
+        __syncthreads();  // P_s staged; cur holds the entering state
+        for (int e = t; e < D * SCAN_COLS; e += blockDim.x) {
+            const int r = e / SCAN_COLS, c = e % SCAN_COLS;
+            S_entry[base + (size_t)r * D + c0 + c] = cur[e];
+        }
+        for (int kk = 0; kk < D; kk += 4) {
+            const float4 pv = *reinterpret_cast<const float4*>(Ps + i * SCAN_LD + kk);
+            const float pk[4] = {pv.x, pv.y, pv.z, pv.w};
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const float4* cr = reinterpret_cast<const float4*>(cur + (kk + u) * SCAN_COLS + j0);
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const float4 cv = cr[q];
+                    acc[4 * q] = fmaf(pk[u], cv.x, acc[4 * q]);
+                    acc[4 * q + 1] = fmaf(pk[u], cv.y, acc[4 * q + 1]);
+                    acc[4 * q + 2] = fmaf(pk[u], cv.z, acc[4 * q + 2]);
+                    acc[4 * q + 3] = fmaf(pk[u], cv.w, acc[4 * q + 3]);
+                }
+            }
+        }
+        __syncthreads();  // every thread has read the entering state and P_s
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+            *reinterpret_cast<float4*>(cur + i * SCAN_COLS + j0 + 4 * q) =
+                make_float4(acc[4 * q], acc[4 * q + 1], acc[4 * q + 2], acc[4 * q + 3]);
+        __syncthreads();
+    }
+    if (S_final)
+        for (int e = t; e < D * SCAN_COLS; e += blockDim.x) {
+            const int r = e / SCAN_COLS, c = e % SCAN_COLS;
+            S_final[((size_t)n * H_v + h) * hs + (size_t)r * D + c0 + c] = cur[e];
+        }
+}
+
+template <int NS, typename IO, int MODE>
 cudaError_t launch_pass2(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                          const PrefillParams& prm, int N, cudaStream_t stream) {
-    auto kern = state_pass_kernel<NS, IO>;
+    auto kern = state_pass_kernel<NS, IO, MODE>;
     cudaError_t e =
         cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, P2_SMEM);
     if (e != cudaSuccess) return e;
-    dim3 grid((D + NS - 1) / NS, prm.H_v, N);
+    dim3 grid((D + NS - 1) / NS * (MODE == P2_SEGMENT ? 2 : 1), prm.H_v, N);
     kern<<<grid, P2_THREADS, P2_SMEM, stream>>>(mq, mk, mv, prm);
     return cudaGetLastError();
 }
@@ -940,15 +1058,93 @@ cudaError_t noalloc_scratch_address(void** out) {
     return cudaSuccess;
 }
 
-size_t prefill_workspace_bytes(int N, int T, int H_qk, int H_v, bool bf16) {
+// per-segment states of the segmented prefill: R, P_s and the entering states
+size_t segment_state_bytes(int N, int P, int H_v) {
+    return up256((size_t)N * P * H_v * D * D * sizeof(float));
+}
+size_t segment_cu_bytes(int N, int P) { return up256(((size_t)N * P + 1) * sizeof(int32_t)); }
+
+size_t prefill_workspace_bytes(int N, int T, int H_qk, int H_v, bool bf16, int P) {
     if (T == 0) return 0;
-    return staging_bytes(T, H_qk, H_v, bf16) + record_bytes(N, T, H_v);
+    if (P <= 1) return staging_bytes(T, H_qk, H_v, bf16) + record_bytes(N, T, H_v);
+    return staging_bytes(T, H_qk, H_v, bf16) + record_bytes(N * P, T, H_v) +
+           segment_cu_bytes(N, P) + 3 * segment_state_bytes(N, P, H_v);
+}
+
+int device_sms() {
+    int dev = 0, sms = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+        sms <= 0) {
+        cudaGetLastError();  // no device: clear the error, assume a B200
+        return 148;
+    }
+    return sms;
+}
+
+// d_v slices per head for `units` (sequence, value head) chains: as many as fit
+// in one wave of one block per SM (4 x 32, 3 x 48 or 2 x 64 columns)
+static int pass2_slices(long long units, int sms) {
+    return units * 4 <= sms ? 4 : (units * 3 <= sms ? 3 : 2);
+}
+
+int choose_segments(int N, int T, int H_v, int sms) {
+    if (N <= 0 || T <= 0 || H_v <= 0) return 1;
+    // Cost model in microseconds, from B200 measurements of one chunk step of a
+    // state-pass block (one block per SM) by slice width -- with outputs (the
+    // prefill proper, phase C) and without (phase A) -- and of one scan step.
+    const double chunks = (double)T / N / C;
+    auto waves = [&](long long blocks) { return (double)((blocks + sms - 1) / sms); };
+    auto t_out = [](int slices) { return slices == 4 ? 1.50 : (slices == 3 ? 1.94 : 2.67); };
+    auto t_seg = [](int slices) { return slices == 4 ? 1.11 : (slices == 3 ? 1.48 : 1.80); };
+    const double t_scan = 3.0, t_fixed = 20.0;  // per segment; segment launches and scan setup
+    const long long u1 = (long long)N * H_v;
+    const int s1 = pass2_slices(u1, sms);
+    double best = waves(u1 * s1) * t_out(s1) * chunks;
+    int best_p = 1;
+    for (int P = 2; P <= kMaxSegments; ++P) {
+        const double per = std::ceil(chunks / P);
+        if (per < 8) break;  // segments of at least 8 chunks
+        const long long u = u1 * P;
+        const int sa = pass2_slices(2 * u, sms), sc = pass2_slices(u, sms);
+        const double cost = (waves(2 * u * sa) * t_seg(sa) + waves(u * sc) * t_out(sc)) * per +
+                            t_scan * P + t_fixed;
+        if (cost < 0.9 * best) {  // a split must win clearly
+            best = cost;
+            best_p = P;
+        }
+    }
+    return best_p;
+}
+
+template <typename IO, int MODE>
+static cudaError_t run_pass2(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+                             const PrefillParams& prm, int sms, cudaStream_t stream) {
+    // one block per SM at most (each holds ~212 KB of shared memory): split every
+    // value head into as many d_v slices as still fit in one wave
+    const long long units = (long long)prm.N * prm.H_v * (MODE == P2_SEGMENT ? 2 : 1);
+    const int slices = pass2_slices(units, sms);
+    if (slices == 4) return launch_pass2<32, IO, MODE>(mq, mk, mv, prm, prm.N, stream);
+    if (slices == 3) return launch_pass2<48, IO, MODE>(mq, mk, mv, prm, prm.N, stream);
+    return launch_pass2<64, IO, MODE>(mq, mk, mv, prm, prm.N, stream);
+}
+
+static cudaError_t run_pass1(const CUtensorMap& mq, const CUtensorMap& mk,
+                             const PrefillParams& prm, cudaStream_t stream) {
+    cudaError_t e =
+        cudaFuncSetAttribute(chunk_ops_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, P1_SMEM);
+    if (e != cudaSuccess) return e;
+    const int group = prm.H_v / prm.H_qk;
+    const long long slots = (long long)prm.N + ((long long)prm.T + C - 1) / C;
+    dim3 grid((unsigned)slots, prm.H_qk, (group + P1_MAX_GROUP - 1) / P1_MAX_GROUP);
+    chunk_ops_kernel<<<grid, P1_THREADS, P1_SMEM, stream>>>(mq, mk, prm);
+    return cudaGetLastError();
 }
 
 cudaError_t launch_prefill(const void* q, const void* k, const void* v, const float* log_alpha,
                            const float* beta, const float* S0, const int32_t* cu_seqlens, int N,
                            int T, int H_qk, int H_v, bool bf16, void* o, float* S_final,
-                           void* workspace, cudaStream_t stream) {
+                           void* workspace, int P, cudaStream_t stream) {
     if (T == 0) {  // every sequence is empty: S_final = S0 (or zeros)
         if (!S_final) return cudaSuccess;
         copy_state_kernel<<<592, 256, 0, stream>>>(S0, S_final, (size_t)N * H_v * D * D / 4);
@@ -975,37 +1171,51 @@ cudaError_t launch_prefill(const void* q, const void* k, const void* v, const fl
     if (!make_map(&mq, qb, T, (uint64_t)H_qk * D) || !make_map(&mk, kb, T, (uint64_t)H_qk * D) ||
         !make_map(&mv, vb, T, (uint64_t)H_v * D))
         return cudaErrorInvalidValue;
-    PrefillParams prm{log_alpha, beta, S0, cu_seqlens, o, S_final, records, H_qk, H_v, N, T};
-
-    // pass 1: every chunk's operators, all chunks at once
-    int num_sms = 148, dev = 0;
-    if (cudaGetDevice(&dev) == cudaSuccess)
-        cudaDeviceGetAttribute(&num_sms, cudaDevAttrMultiProcessorCount, dev);
-    {
-        cudaError_t e = cudaFuncSetAttribute(chunk_ops_kernel,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize, P1_SMEM);
-        if (e != cudaSuccess) return e;
-        const int group = H_v / H_qk;
-        const long long slots = (long long)N + ((long long)T + C - 1) / C;
-        dim3 grid((unsigned)slots, H_qk, (group + P1_MAX_GROUP - 1) / P1_MAX_GROUP);
-        chunk_ops_kernel<<<grid, P1_THREADS, P1_SMEM, stream>>>(mq, mk, prm);
-        e = cudaGetLastError();
-        if (e != cudaSuccess) return e;
+    const int sms = device_sms();
+    if (P <= 0) P = choose_segments(N, T, H_v, sms);
+    cudaError_t e;
+    if (P == 1) {
+        // pass 1: every chunk's operators, all chunks at once; pass 2: the state
+        // through the chunks
+        const PrefillParams prm{log_alpha, beta, S0,      cu_seqlens, o, S_final,
+                                records,   nullptr, H_qk, H_v,        N, T};
+        if ((e = run_pass1(mq, mk, prm, stream)) != cudaSuccess) return e;
+        return bf16 ? run_pass2<__nv_bfloat16, P2_OUT>(mq, mk, mv, prm, sms, stream)
+                    : run_pass2<float, P2_OUT>(mq, mk, mv, prm, sms, stream);
     }
-    // pass 2: the state through the chunks.  One CTA per SM at most (each holds
-    // ~212 KB of shared memory): split every value head into as many d_v slices
-    // (4 x 32, 3 x 48 or 2 x 64 columns) as still fit in one wave, so few long
-    // sequences still cover the SMs.
-    const long long units = (long long)N * H_v;
-    const int ns = units * 4 <= num_sms ? 32 : (units * 3 <= num_sms ? 48 : 64);
-    if (bf16) {
-        if (ns == 64) return launch_pass2<64, __nv_bfloat16>(mq, mk, mv, prm, N, stream);
-        if (ns == 48) return launch_pass2<48, __nv_bfloat16>(mq, mk, mv, prm, N, stream);
-        return launch_pass2<32, __nv_bfloat16>(mq, mk, mv, prm, N, stream);
-    }
-    if (ns == 64) return launch_pass2<64, float>(mq, mk, mv, prm, N, stream);
-    if (ns == 48) return launch_pass2<48, float>(mq, mk, mv, prm, N, stream);
-    return launch_pass2<32, float>(mq, mk, mv, prm, N, stream);
+    // segmented: N P virtual sequences
+    const int Nv = N * P;
+    uint8_t* w = records + record_bytes(Nv, T, H_v);
+    int32_t* cu_v = reinterpret_cast<int32_t*>(w);
+    w += segment_cu_bytes(N, P);
+    float* R = reinterpret_cast<float*>(w);
+    w += segment_state_bytes(N, P, H_v);
+    float* Pm = reinterpret_cast<float*>(w);
+    w += segment_state_bytes(N, P, H_v);
+    float* S_entry = reinterpret_cast<float*>(w);
+    segment_cu_kernel<<<(Nv + 1 + 255) / 256, 256, 0, stream>>>(cu_seqlens, N, P, cu_v);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    // pass 1 over the segments (chunks never cross one, so the operators are those
+    // of the unsegmented sequences)
+    const PrefillParams pa{log_alpha, beta, nullptr, cu_v, nullptr, R, records, Pm, H_qk, H_v,
+                           Nv,        T};
+    if ((e = run_pass1(mq, mk, pa, stream)) != cudaSuccess) return e;
+    // phase A: R (from zero) and P_s (from the identity, V = 0) of every segment
+    e = bf16 ? run_pass2<__nv_bfloat16, P2_SEGMENT>(mq, mk, mv, pa, sms, stream)
+             : run_pass2<float, P2_SEGMENT>(mq, mk, mv, pa, sms, stream);
+    if (e != cudaSuccess) return e;
+    // the entering state of every segment, and the final states
+    if ((e = cudaFuncSetAttribute(segment_scan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  SCAN_SMEM)) != cudaSuccess)
+        return e;
+    segment_scan_kernel<<<dim3(D / SCAN_COLS, H_v, N), 256, SCAN_SMEM, stream>>>(
+        S0, R, Pm, S_entry, S_final, P, H_v);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    // phase C: every segment from its entering state, writing the outputs
+    const PrefillParams pc{log_alpha, beta, S_entry, cu_v, o, nullptr, records, nullptr,
+                           H_qk,      H_v,  Nv,      T};
+    return bf16 ? run_pass2<__nv_bfloat16, P2_OUT>(mq, mk, mv, pc, sms, stream)
+                : run_pass2<float, P2_OUT>(mq, mk, mv, pc, sms, stream);
 }
 
 }  // namespace gdn

@@ -35,6 +35,12 @@ SIGNATURES = {
                                _c.c_int32, _c.c_int32, _c.c_int32, _c.c_int, _c.c_void_p,
                                _c.c_void_p, _c.c_void_p, _c.c_size_t, _c.c_void_p]),
     "gdn_prefill_workspace_size": (_c.c_size_t, [_c.c_int32] * 6 + [_c.c_int]),
+    "gdn_prefill_segmented": (_c.c_int, [_c.c_void_p] * 7 + [_c.c_int32] * 6 +
+                              [_c.c_int, _c.c_void_p, _c.c_void_p, _c.c_int32, _c.c_void_p,
+                               _c.c_size_t, _c.c_void_p]),
+    "gdn_prefill_segmented_workspace_size": (_c.c_size_t,
+                                             [_c.c_int32] * 6 + [_c.c_int, _c.c_int32]),
+    "gdn_prefill_auto_segments": (_c.c_int32, [_c.c_int32] * 4),
     "gdn_prefill_noalloc": (_c.c_int, [_c.c_void_p, _c.c_void_p, _c.c_void_p, _c.c_void_p,
                                        _c.c_void_p, _c.c_void_p, _c.c_void_p, _c.c_int32,
                                        _c.c_int32, _c.c_int32, _c.c_int32, _c.c_int32,
@@ -117,13 +123,26 @@ def _check(t, name, dtype=None, shape=None):
         raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
 
 
-def workspace_size(N, T, H_qk, H_v, d=128, io_dtype=GDN_BF16) -> int:
-    return int(lib().gdn_prefill_workspace_size(N, T, H_qk, H_v, d, d, io_dtype))
+def workspace_size(N, T, H_qk, H_v, d=128, io_dtype=GDN_BF16, segments=0) -> int:
+    return int(lib().gdn_prefill_segmented_workspace_size(N, T, H_qk, H_v, d, d, io_dtype,
+                                                          segments))
+
+
+MAX_PREFILL_SEGMENTS = 64  # GDN_MAX_PREFILL_SEGMENTS
+
+
+def auto_segments(N, T, H_qk, H_v) -> int:
+    """Segments per sequence ``prefill`` uses for these sizes on the current device."""
+    return int(lib().gdn_prefill_auto_segments(N, T, H_qk, H_v))
 
 
 def prefill(q, k, v, log_alpha, beta, S0=None, cu_seqlens=None, *, o=None, S_final=None,
-            want_state=True, workspace=None, stream=None):
-    """Chunked prefill.  Returns ``(o, S_final)`` (``S_final`` None if not wanted)."""
+            want_state=True, workspace=None, segments=None, stream=None):
+    """Chunked prefill.  Returns ``(o, S_final)`` (``S_final`` None if not wanted).
+
+    ``segments``: None or 0 lets the library split long sequences when that
+    fills more SMs; 1 disables the split; 2 .. 64 forces that many pieces per
+    sequence (gdn_prefill_segmented)."""
     T, H_qk, dk = q.shape
     H_v, dv = v.shape[1], v.shape[2]
     dt = q.dtype
@@ -146,15 +165,17 @@ def prefill(q, k, v, log_alpha, beta, S0=None, cu_seqlens=None, *, o=None, S_fin
     if S_final is not None:
         _check(S_final, "S_final", torch.float32, (N, H_v, dk, dv))
     io = _io_dtype(q)
-    need = workspace_size(N, T, H_qk, H_v, dk, io)
+    seg = 0 if segments is None else int(segments)
+    need = workspace_size(N, T, H_qk, H_v, dk, io, segments=seg)
     if need and workspace is None:
         workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
     wbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
-    st = lib().gdn_prefill(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _ptr(S0),
-                           _ptr(cu_seqlens), N, T, H_qk, H_v, dk, dv, io, _ptr(o), _ptr(S_final),
-                           _ptr(workspace), wbytes, _stream_handle(stream))
+    st = lib().gdn_prefill_segmented(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta),
+                                     _ptr(S0), _ptr(cu_seqlens), N, T, H_qk, H_v, dk, dv, io,
+                                     _ptr(o), _ptr(S_final), seg, _ptr(workspace), wbytes,
+                                     _stream_handle(stream))
     if st != GDN_OK:
-        raise GDNError(st, "gdn_prefill")
+        raise GDNError(st, "gdn_prefill_segmented")
     return o, S_final
 
 
