@@ -9,6 +9,8 @@ Workloads (synthetic, seeded; see linear_attention_12_b200/inputs.py):
     place (805 MB) -- reported in the ``decode`` object (GB/s);
   * multi-token decode: 4 tokens per sequence for the same 256 x 48 heads, a
     state checkpoint after each (4.0 GB moved) -- the ``decode_multi`` object;
+  * prefill of one 8-way tensor-parallel shard (2 QK / 6 V heads, L=32768),
+    with and without the library's sequence split -- the ``prefill_shard`` object;
   * front end: the short convolution, q/k normalisation and gate activations
     over the raw inputs of the L=32768 prefill (1.37 GB moved) -- reported in
     the ``frontend`` object (GB/s).
@@ -272,6 +274,41 @@ def run_decode_multi(args, dev, stream, world):
     return ms, DM_BYTES / (ms / 1e3) / 1e9
 
 
+def run_prefill_shard(args, dev, stream, world, L):
+    """The prefill of one tensor-parallel shard (1/8 of the heads: 2 QK, 6 V),
+    with the library's automatic sequence split and without it; returns
+    (segments, ms with the split, ms without)."""
+    import torch
+    from linear_attention_12_b200 import gdn, inputs
+    hq, hv = H_QK // 8, H_V // 8
+    case = inputs.make_prefill(f"prefill_shard_L{L}", [L], hq, hv, seed=6)
+    q, k, v = case.q.to(dev), case.k.to(dev), case.v.to(dev)
+    la, be, cu = case.log_alpha.to(dev), case.beta.to(dev), case.cu_seqlens.to(dev)
+    o = torch.empty((L, hv, D), dtype=torch.bfloat16, device=dev)
+    Sf = torch.empty((1, hv, D, D), dtype=torch.float32, device=dev)
+    seg = gdn.auto_segments(1, L, hq, hv)
+    out = []
+    for s in (0, 1):
+        ws = torch.empty(max(gdn.workspace_size(1, L, hq, hv, segments=s), 256),
+                         dtype=torch.uint8, device=dev)
+        for _ in range(max(args.warmup, 3)):
+            gdn.prefill(q, k, v, la, be, None, cu, o=o, S_final=Sf, workspace=ws, segments=s)
+        torch.cuda.synchronize()
+        barrier(world)
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        n = max(args.steps, 10)
+        e0.record(stream)
+        for _ in range(n):
+            gdn.prefill(q, k, v, la, be, None, cu, o=o, S_final=Sf, workspace=ws, segments=s)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        barrier(world)
+        out.append(max_over_ranks(e0.elapsed_time(e1), world) / n)
+        assert gdn.last_device_error() == gdn.GDN_OK
+    return seg, out[0], out[1]
+
+
 def run_frontend(args, dev, stream, world, L):
     """Time the front end on raw inputs of the prefill's shape; returns
     (ms per call, GB/s)."""
@@ -423,6 +460,11 @@ def run_ours(args):
     if not args.no_decode:
         dm_ms, dm_gbs = run_decode_multi(args, dev, stream, world)
 
+    # ---------------- prefill of a tensor-parallel shard (few heads: sequence split)
+    shard = None
+    if not args.no_shard:
+        shard = run_prefill_shard(args, dev, stream, world, L)
+
     # ---------------- front end on raw inputs of the same shape
     fe_ms = fe_gbs = None
     if not args.no_frontend:
@@ -497,6 +539,17 @@ def run_ours(args):
                 "frac": dm_gbs / hbm_peak,
                 "workload": f"decode of M={DM_M} tokens per sequence, B={DEC_B} H_qk={H_QK} "
                             f"H_v={H_V} d={D}, fp32 state read once, a checkpoint per token",
+                "steps": max(args.steps, 10),
+            },
+            "prefill_shard": None if shard is None else {
+                "value": L / (shard[1] / 1e3),
+                "unit": "tokens/s",
+                "ms_per_call": shard[1],
+                "segments": shard[0],
+                "ms_per_call_unsplit": shard[2],
+                "speedup_from_split": shard[2] / shard[1],
+                "workload": f"prefill B=1 L={L} H_qk={H_QK // 8} H_v={H_V // 8} d={D} bf16 "
+                            "(one shard of 8-way tensor parallelism)",
                 "steps": max(args.steps, 10),
             },
             "frontend": None if fe_gbs is None else {
@@ -598,6 +651,8 @@ def main():
     ap.add_argument("--no-decode", action="store_true", help="skip the decode measurement")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer measurement")
     ap.add_argument("--no-frontend", action="store_true", help="skip the front-end measurement")
+    ap.add_argument("--no-shard", action="store_true",
+                    help="skip the tensor-parallel-shard prefill measurement")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

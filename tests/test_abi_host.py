@@ -90,6 +90,47 @@ def test_prefill_rejects_bad_arguments_on_host(L, kw, expect):
     assert _prefill(L, **kw) == expect
 
 
+def _prefill_seg(L, segments, **kw):
+    a = dict(q=P, k=P, v=P, la=P, be=P, S0=None, cu=P, N=1, T=4096, H_qk=1, H_v=1, dk=128,
+             dv=128, dt=gdn.GDN_BF16, o=P, Sf=None, ws=P, wsb=1 << 40, stream=None)
+    a.update(kw)
+    return L.gdn_prefill_segmented(a["q"], a["k"], a["v"], a["la"], a["be"], a["S0"], a["cu"],
+                                   a["N"], a["T"], a["H_qk"], a["H_v"], a["dk"], a["dv"], a["dt"],
+                                   a["o"], a["Sf"], segments, a["ws"], a["wsb"], a["stream"])
+
+
+@pytest.mark.parametrize("segments", [-1, 65])
+def test_segmented_prefill_rejects_segment_counts_out_of_range(L, segments):
+    assert _prefill_seg(L, segments) == gdn.GDN_ERR_INVALID_ARG
+
+
+def test_segmented_prefill_checks_its_workspace(L):
+    need = L.gdn_prefill_segmented_workspace_size(1, 4096, 1, 1, 128, 128, gdn.GDN_BF16, 4)
+    assert _prefill_seg(L, 4, wsb=need - 1) == gdn.GDN_ERR_WORKSPACE
+    assert _prefill_seg(L, 4, ws=P + 16, wsb=need) == gdn.GDN_ERR_WORKSPACE  # not 256-aligned
+
+
+def test_segmented_workspace_adds_the_pieces_states(L):
+    ws = lambda seg: L.gdn_prefill_segmented_workspace_size(1, 32768, 2, 6, 128, 128,
+                                                            gdn.GDN_BF16, seg)
+    one, four = ws(1), ws(4)
+    rec = 16912 * 6  # one more record slot per extra piece, per value head
+    states = 3 * 4 * 6 * 128 * 128 * 4  # R, P_s and the entering state of every piece
+    assert four - one >= 3 * rec + states
+    assert four - one <= 3 * rec + states + 4 * 256 + 256  # plus the piece starts and rounding
+    assert ws(0) == ws(L.gdn_prefill_auto_segments(1, 32768, 2, 6))
+    assert L.gdn_prefill_segmented_workspace_size(1, 32768, 2, 6, 128, 128, gdn.GDN_BF16, 65) == 0
+
+
+def test_automatic_split_only_for_few_chains(L):
+    assert L.gdn_prefill_auto_segments(1, 32768, 16, 48) == 1   # 48 heads fill the SMs
+    assert L.gdn_prefill_auto_segments(8, 65536, 16, 48) == 1
+    assert L.gdn_prefill_auto_segments(1, 256, 1, 1) == 1        # too short to split
+    assert L.gdn_prefill_auto_segments(1, 32768, 2, 6) > 1       # a tensor-parallel shard
+    assert L.gdn_prefill_auto_segments(1, 32768, 1, 1) > 1
+    assert L.gdn_prefill_auto_segments(0, 32768, 1, 1) == 1      # invalid: no split
+
+
 def _decode(L, **kw):
     a = dict(q=P, k=P, v=P, la=P, be=P, S=P, B=4, H_qk=1, H_v=3, dk=128, dv=128,
              dt=gdn.GDN_BF16, o=P, stream=None)
