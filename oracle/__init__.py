@@ -18,6 +18,9 @@ Two independent formulations live here:
   with numpy.  Slow (O(d^3) per token); for tiny cases only.  It exists to pin
   the C oracle against a differently-written evaluation of the page's formula.
 
+``oracle.backward`` holds the prefill's gradients (reverse mode of the same
+recurrence, fp64 numpy); see its header.
+
 ``oracle.frontend`` holds the front end (short causal convolution, L2
 normalisation of q and k, gate activations) in fp64 numpy; see its header.
 
