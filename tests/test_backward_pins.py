@@ -80,3 +80,27 @@ def test_pure_decay_closed_form():
     np.testing.assert_allclose(dS0[0, 0], want, rtol=1e-12)
     np.testing.assert_array_equal(dv, 0.0)
     np.testing.assert_allclose(dk, 0.0, atol=1e-15)  # k only enters through beta k k^T and beta k v^T
+
+
+@pytest.mark.parametrize("C,lens,H_qk,H_v", [(4, (13, 0, 9), 1, 2), (8, (17,), 2, 4),
+                                              (16, (5, 40), 1, 3)])
+def test_chunk_form_of_the_gradients_equals_the_oracle(C, lens, H_qk, H_v):
+    # the chunked backward the kernels follow (tests/chunk_form.py) against the
+    # token-by-token reverse mode, on ragged and empty sequences with grouped heads
+    from tests.chunk_form import chunked_backward
+    rng = np.random.default_rng(C)
+    T, N, d = sum(lens), len(lens), 8
+    cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int64)
+    q = rng.standard_normal((T, H_qk, d))
+    k = rng.standard_normal((T, H_qk, d))
+    k /= np.linalg.norm(k, axis=-1, keepdims=True)
+    v = rng.standard_normal((T, H_v, d))
+    la = -np.log1p(np.exp(rng.standard_normal((T, H_v))))
+    be = 1 / (1 + np.exp(-rng.standard_normal((T, H_v))))
+    S0 = 0.3 * rng.standard_normal((N, H_v, d, d))
+    dO = rng.standard_normal((T, H_v, d))
+    dSf = rng.standard_normal((N, H_v, d, d))
+    ref = backward.prefill_backward(q, k, v, la, be, dO, S0=S0, dS_final=dSf, cu_seqlens=cu)
+    got = chunked_backward(q, k, v, la, be, dO, S0=S0, dS_final=dSf, cu_seqlens=cu, C=C)
+    for name, a, b in zip(["dq", "dk", "dv", "dlog_alpha", "dbeta", "dS0"], got, ref):
+        np.testing.assert_allclose(a, b, rtol=1e-10, atol=1e-12, err_msg=name)
