@@ -50,12 +50,18 @@ STATE_BYTES = H_V * D * D * 4                                                 # 
 # (three triangular C x C x d products at half) + 2 C d / 3 (grams at half,
 # shared by the 3 V heads of a QK head), C = 64.
 FLOP_PER_TOKEN = H_V * (6 * D * D + 3 * 64 * D + (2 * 64 * D) // 3)
-DEC_BYTES = 2 * DEC_B * H_V * D * D * 4 + DEC_B * (2 * H_QK * D * 2 + 2 * H_V * D * 2 + 2 * H_V * 4)
+def dec_bytes(B):
+    """One decode step: the fp32 states read and written, plus the tokens."""
+    return 2 * B * H_V * D * D * 4 + B * (2 * H_QK * D * 2 + 2 * H_V * D * 2 + 2 * H_V * 4)
+
+
+DEC_BYTES = dec_bytes(DEC_B)
 # multi-token decode (speculative verification, M = 4 tokens: 3 drafted + 1):
 # the state read once and written after each token, plus the tokens' inputs/outputs
 DM_M = 4
-DM_BYTES = ((1 + DM_M) * DEC_B * H_V * D * D * 4
-            + DEC_B * DM_M * (2 * H_QK * D * 2 + 2 * H_V * D * 2 + 2 * H_V * 4))
+def dm_bytes(B):
+    return ((1 + DM_M) * B * H_V * D * D * 4
+            + B * DM_M * (2 * H_QK * D * 2 + 2 * H_V * D * 2 + 2 * H_V * 4))
 # front end, per token: raw q, k, v read and normalised q, k, v written (bf16),
 # a, b read and log_alpha, beta written (fp32); plus the conv weight once
 FE_BYTES_PER_TOKEN = 2 * (2 * H_QK + H_V) * D * 2 + 4 * H_V * 4                # 41,728
@@ -224,10 +230,11 @@ def run_decode(args, dev, stream, world):
     """Time decode steps on the 256-sequence workload; returns (ms per step, GB/s)."""
     import torch
     from linear_attention_12_b200 import gdn, inputs
-    dc = inputs.batched_decode_256()
+    B = args.decode_batch
+    dc = inputs.make_decode(B, H_QK, H_V, D, seed=4)
     S = dc.S0.to(dev)
     dq, dk_, dv_, dla, dbe = (x.to(dev) for x in dc.step(0))
-    do = torch.empty((DEC_B, H_V, D), dtype=torch.bfloat16, device=dev)
+    do = torch.empty((B, H_V, D), dtype=torch.bfloat16, device=dev)
     dec_steps = max(args.steps, 20)
     for _ in range(max(args.warmup, 3)):
         gdn.decode_step(dq, dk_, dv_, dla, dbe, S, o=do)
@@ -243,7 +250,7 @@ def run_decode(args, dev, stream, world):
     barrier(world)
     dec_ms = max_over_ranks(d0.elapsed_time(d1), world) / dec_steps
     assert gdn.last_device_error() == gdn.GDN_OK
-    return dec_ms, DEC_BYTES / (dec_ms / 1e3) / 1e9
+    return dec_ms, dec_bytes(B) / (dec_ms / 1e3) / 1e9
 
 
 def run_decode_multi(args, dev, stream, world):
@@ -251,11 +258,12 @@ def run_decode_multi(args, dev, stream, world):
     returns (ms per call, GB/s)."""
     import torch
     from linear_attention_12_b200 import gdn, inputs
-    dc = inputs.batched_decode_256()
+    B = args.decode_batch
+    dc = inputs.make_decode(B, H_QK, H_V, D, seed=4)
     S_in = dc.S0.to(dev)
     win = [x.to(dev) for x in dc.window(0, DM_M)]
-    o = torch.empty((DEC_B, DM_M, H_V, D), dtype=torch.bfloat16, device=dev)
-    S_steps = torch.empty((DEC_B, DM_M, H_V, D, D), dtype=torch.float32, device=dev)
+    o = torch.empty((B, DM_M, H_V, D), dtype=torch.bfloat16, device=dev)
+    S_steps = torch.empty((B, DM_M, H_V, D, D), dtype=torch.float32, device=dev)
     n = max(args.steps, 10)
     for _ in range(max(args.warmup, 3)):
         gdn.decode_multi(*win, S_in, o=o, S_steps=S_steps)
@@ -271,7 +279,7 @@ def run_decode_multi(args, dev, stream, world):
     barrier(world)
     ms = max_over_ranks(e0.elapsed_time(e1), world) / n
     assert gdn.last_device_error() == gdn.GDN_OK
-    return ms, DM_BYTES / (ms / 1e3) / 1e9
+    return ms, dm_bytes(B) / (ms / 1e3) / 1e9
 
 
 def run_prefill_shard(args, dev, stream, world, L):
@@ -523,21 +531,22 @@ def run_ours(args):
                 "value": dec_gbs,
                 "unit": "GB/s",
                 "us_per_step": dec_ms * 1e3,
-                "bytes_per_step": DEC_BYTES,
+                "bytes_per_step": dec_bytes(args.decode_batch),
                 "peak": hbm_peak,
                 "frac": dec_gbs / hbm_peak,
-                "workload": f"decode B={DEC_B} H_qk={H_QK} H_v={H_V} d={D}, fp32 state in place",
+                "workload": f"decode B={args.decode_batch} H_qk={H_QK} H_v={H_V} d={D}, "
+                            "fp32 state in place",
                 "steps": max(args.steps, 20),
             },
             "decode_multi": None if dm_gbs is None else {
                 "value": dm_gbs,
                 "unit": "GB/s",
                 "us_per_call": dm_ms * 1e3,
-                "tokens_per_s": DEC_B * DM_M / (dm_ms / 1e3),
-                "bytes_per_call": DM_BYTES,
+                "tokens_per_s": args.decode_batch * DM_M / (dm_ms / 1e3),
+                "bytes_per_call": dm_bytes(args.decode_batch),
                 "peak": hbm_peak,
                 "frac": dm_gbs / hbm_peak,
-                "workload": f"decode of M={DM_M} tokens per sequence, B={DEC_B} H_qk={H_QK} "
+                "workload": f"decode of M={DM_M} tokens per sequence, B={args.decode_batch} H_qk={H_QK} "
                             f"H_v={H_V} d={D}, fp32 state read once, a checkpoint per token",
                 "steps": max(args.steps, 10),
             },
@@ -649,6 +658,8 @@ def main():
     ap.add_argument("--seq-len", type=int, default=L,
                     help="prefill length (the benchmark is L=32768; smaller only for profiling)")
     ap.add_argument("--no-decode", action="store_true", help="skip the decode measurement")
+    ap.add_argument("--decode-batch", type=int, default=DEC_B,
+                    help="sequences of the decode workloads (256; smaller only for profiling)")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer measurement")
     ap.add_argument("--no-frontend", action="store_true", help="skip the front-end measurement")
     ap.add_argument("--no-shard", action="store_true",

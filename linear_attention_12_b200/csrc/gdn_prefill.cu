@@ -928,29 +928,48 @@ __global__ void segment_cu_kernel(const int32_t* __restrict__ cu, int N, int P,
     cu_v[idx] = cu[n] + min(i * per * C, len);
 }
 
+// x = hi + lo with both parts tf32: three tf32 products (hi hi, hi lo, lo hi)
+// keep an fp32 product's accuracy.
+__device__ __forceinline__ void split_tf32(float x, uint32_t& hi, uint32_t& lo) {
+    hi = to_tf32(x);
+    lo = to_tf32(x - __uint_as_float(hi));
+}
+__device__ __forceinline__ void mma_tf32_frag(float* d, const uint32_t (&a)[4], uint32_t b0,
+                                              uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 "
+        "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
 // Block (column block cb of 32, value head h, sequence n): S_entry[n P + s] is
 // the state entering segment s, S_final[n] the state after the last one;
-// S <- P_s S + R_s from S0[n] (or zero), in fp32.  Each step stages P_s in
-// shared memory (all its loads in flight at once; rows padded to 132 floats
-// so that the row-wise float4 reads below hit distinct banks).
+// S <- P_s S + R_s from S0[n] (or zero).  Each step stages P_s in shared
+// memory (all its loads in flight at once) and multiplies on the tensor cores
+// in split tf32 (three products per term: fp32 accuracy); warp w owns rows
+// 16 w .. +15 of the 32 columns.  Row strides (132 and 40 floats) keep the
+// fragment loads free of bank conflicts.
 constexpr int SCAN_COLS = 32;
 constexpr int SCAN_LD = D + 4;
-constexpr uint32_t SCAN_SMEM = (D * SCAN_LD + D * SCAN_COLS) * sizeof(float);  // 83,968 B
+constexpr int CUR_LD = SCAN_COLS + 8;
+constexpr uint32_t SCAN_SMEM = (D * SCAN_LD + D * CUR_LD) * sizeof(float);  // 88,064 B
 __global__ void __launch_bounds__(256)
     segment_scan_kernel(const float* __restrict__ S0, const float* __restrict__ R,
                         const float* __restrict__ Pm, float* __restrict__ S_entry,
                         float* S_final, int P, int H_v) {
     extern __shared__ float4 scan_sm4[];
     float* Ps = reinterpret_cast<float*>(scan_sm4);  // [D][SCAN_LD]
-    float* cur = Ps + D * SCAN_LD;                   // [D][SCAN_COLS]
+    float* cur = Ps + D * SCAN_LD;                   // [D][CUR_LD]
     const int cb = blockIdx.x, h = blockIdx.y, n = blockIdx.z;
-    const int t = threadIdx.x, i = t >> 1, j0 = (t & 1) * 16;
+    const int t = threadIdx.x, warp = t >> 5, lane = t & 31, g = lane >> 2, t4 = lane & 3;
     const size_t hs = (size_t)D * D;
     const size_t c0 = (size_t)cb * SCAN_COLS;
     for (int e = t; e < D * SCAN_COLS; e += blockDim.x) {
         const int r = e / SCAN_COLS, c = e % SCAN_COLS;
-        cur[e] = S0 ? S0[((size_t)n * H_v + h) * hs + (size_t)r * D + c0 + c] : 0.f;
+        cur[r * CUR_LD + c] = S0 ? S0[((size_t)n * H_v + h) * hs + (size_t)r * D + c0 + c] : 0.f;
     }
+    const int r0 = 16 * warp;
     for (int sg = 0; sg < P; ++sg) {
         const size_t base = (((size_t)n * P + sg) * H_v + h) * hs;
         const float4* P4 = reinterpret_cast<const float4*>(Pm + base);
@@ -958,48 +977,57 @@ __global__ void __launch_bounds__(256)
             const int r = e / (D / 4), c4 = e % (D / 4);
             *reinterpret_cast<float4*>(Ps + r * SCAN_LD + 4 * c4) = P4[e];
         }
-        float acc[16];
-        const float4* R4 = reinterpret_cast<const float4*>(R + base + (size_t)i * D + c0 + j0);
+        // accumulators start from R_s: rows r0 + g (+8), columns 8 nt + 2 t4 (+1)
+        float d[4][4];
+        const float* Rb = R + base + c0;
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-            const float4 rv = R4[q];
-            acc[4 * q] = rv.x;
-            acc[4 * q + 1] = rv.y;
-            acc[4 * q + 2] = rv.z;
-            acc[4 * q + 3] = rv.w;
+        for (int nt = 0; nt < 4; ++nt) {
+            const int col = 8 * nt + 2 * t4;
+            const float2 lo = *reinterpret_cast<const float2*>(Rb + (size_t)(r0 + g) * D + col);
+            const float2 hi = *reinterpret_cast<const float2*>(Rb + (size_t)(r0 + g + 8) * D + col);
+            d[nt][0] = lo.x;
+            d[nt][1] = lo.y;
+            d[nt][2] = hi.x;
+            d[nt][3] = hi.y;
         }
         __syncthreads();  // P_s staged; cur holds the entering state
         for (int e = t; e < D * SCAN_COLS; e += blockDim.x) {
             const int r = e / SCAN_COLS, c = e % SCAN_COLS;
-            S_entry[base + (size_t)r * D + c0 + c] = cur[e];
+            S_entry[base + (size_t)r * D + c0 + c] = cur[r * CUR_LD + c];
         }
-        for (int kk = 0; kk < D; kk += 4) {
-            const float4 pv = *reinterpret_cast<const float4*>(Ps + i * SCAN_LD + kk);
-            const float pk[4] = {pv.x, pv.y, pv.z, pv.w};
+#pragma unroll 4
+        for (int ks = 0; ks < D / 8; ++ks) {
+            uint32_t ah[4], al[4];
+            const float* Ar = Ps + (r0 + g) * SCAN_LD + 8 * ks + t4;
+            split_tf32(Ar[0], ah[0], al[0]);
+            split_tf32(Ar[8 * SCAN_LD], ah[1], al[1]);
+            split_tf32(Ar[4], ah[2], al[2]);
+            split_tf32(Ar[8 * SCAN_LD + 4], ah[3], al[3]);
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                const float4* cr = reinterpret_cast<const float4*>(cur + (kk + u) * SCAN_COLS + j0);
-#pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    const float4 cv = cr[q];
-                    acc[4 * q] = fmaf(pk[u], cv.x, acc[4 * q]);
-                    acc[4 * q + 1] = fmaf(pk[u], cv.y, acc[4 * q + 1]);
-                    acc[4 * q + 2] = fmaf(pk[u], cv.z, acc[4 * q + 2]);
-                    acc[4 * q + 3] = fmaf(pk[u], cv.w, acc[4 * q + 3]);
-                }
+            for (int nt = 0; nt < 4; ++nt) {
+                uint32_t b0h, b0l, b1h, b1l;
+                const float* Br = cur + (8 * ks + t4) * CUR_LD + 8 * nt + g;
+                split_tf32(Br[0], b0h, b0l);
+                split_tf32(Br[4 * CUR_LD], b1h, b1l);
+                mma_tf32_frag(d[nt], ah, b0h, b1h);
+                mma_tf32_frag(d[nt], ah, b0l, b1l);
+                mma_tf32_frag(d[nt], al, b0h, b1h);
             }
         }
-        __syncthreads();  // every thread has read the entering state and P_s
+        __syncthreads();  // every warp has read the entering state and P_s
 #pragma unroll
-        for (int q = 0; q < 4; ++q)
-            *reinterpret_cast<float4*>(cur + i * SCAN_COLS + j0 + 4 * q) =
-                make_float4(acc[4 * q], acc[4 * q + 1], acc[4 * q + 2], acc[4 * q + 3]);
+        for (int nt = 0; nt < 4; ++nt) {
+            const int col = 8 * nt + 2 * t4;
+            *reinterpret_cast<float2*>(cur + (r0 + g) * CUR_LD + col) = make_float2(d[nt][0], d[nt][1]);
+            *reinterpret_cast<float2*>(cur + (r0 + g + 8) * CUR_LD + col) =
+                make_float2(d[nt][2], d[nt][3]);
+        }
         __syncthreads();
     }
     if (S_final)
         for (int e = t; e < D * SCAN_COLS; e += blockDim.x) {
             const int r = e / SCAN_COLS, c = e % SCAN_COLS;
-            S_final[((size_t)n * H_v + h) * hs + (size_t)r * D + c0 + c] = cur[e];
+            S_final[((size_t)n * H_v + h) * hs + (size_t)r * D + c0 + c] = cur[r * CUR_LD + c];
         }
 }
 
