@@ -15,7 +15,7 @@
 // k, v; the weight is [(2 H_qk + H_v) d, 4] fp32.
 //
 // The work is HBM-bound.  The prefill form stages each block's rows in shared
-// memory with bulk copies (up to 70 KB in flight per block, three blocks per
+// memory with bulk copies (up to 35 KB in flight per block, six blocks per
 // SM), then one warp per head convolves them with a rolling window, each lane
 // holding 4 channels; outputs leave as one coalesced 256-byte (bf16) or
 // 512-byte (fp32) row segment per warp.
@@ -128,15 +128,16 @@ struct FrontendParams {
 // ---- prefill front end: rows staged in shared memory by bulk copies ----
 //
 // A block handles FE_TC consecutive tokens of a group of HG heads of one
-// kind (HG = 8 for bf16, 4 for fp32: 2 KB of each token row).  One thread
+// kind (HG = 4 for bf16, 2 for fp32: 1 KB of each token row).  One thread
 // issues one bulk copy per token row -- the three rows of history before the
-// tile and its FE_TC tokens -- so that the whole tile (up to 70 KB) is in
+// tile and its FE_TC tokens -- so that the whole tile (up to 35 KB) is in
 // flight at once; warp w then convolves head w of the group from shared
 // memory with a rolling window, each lane holding 4 channels.
 constexpr int FE_TC = 32;                         // tokens per block
 constexpr int FE_ROWS = FE_TC + 3;                // staged rows: history + tile
-constexpr uint32_t FE_ROWB = 2048;                // shared-memory bytes of one staged row
+constexpr uint32_t FE_ROWB = 1024;                // shared-memory bytes of one staged row
 constexpr uint32_t FE_SMEM = FE_ROWS * FE_ROWB + 16;  // + mbarrier and abort flag
+static_assert(FE_TC <= 32, "lane j handles token j of a tile (gates, sequence starts)");
 
 template <typename IO>
 __host__ __device__ constexpr int fe_heads() { return FE_ROWB / (FD * sizeof(IO)); }
