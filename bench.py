@@ -9,6 +9,8 @@ Workloads (synthetic, seeded; see linear_attention_12_b200/inputs.py):
     place (805 MB) -- reported in the ``decode`` object (GB/s);
   * multi-token decode: 4 tokens per sequence for the same 256 x 48 heads, a
     state checkpoint after each (4.0 GB moved) -- the ``decode_multi`` object;
+  * gradients of the same prefill (dq, dk, dv and the gate gradients) -- the
+    ``backward`` object (tokens/s and the tensor roofline);
   * prefill of one 8-way tensor-parallel shard (2 QK / 6 V heads, L=32768),
     with and without the library's sequence split -- the ``prefill_shard`` object;
   * front end: the short convolution, q/k normalisation and gate activations
@@ -62,6 +64,13 @@ DM_M = 4
 def dm_bytes(B):
     return ((1 + DM_M) * B * H_V * D * D * 4
             + B * DM_M * (2 * H_QK * D * 2 + 2 * H_V * D * 2 + 2 * H_V * 4))
+# gradients of the prefill, per token: q, k, v, dO and the gates read, dq, dk, dv and
+# the gate gradients written; FLOPs of the chunk form per (chunk, value head):
+# forward re-run 4 C d^2 + 2 C^2 d, reverse chain 6 C d^2 + 4 C^2 d, per-chunk
+# gradients 12 C d^2 + 20 C^2 d + 4 C^3  (C = 64)
+BW_BYTES_PER_TOKEN = (2 * H_QK * D * 2 + 2 * H_V * D * 2 + 2 * H_V * 4) + \
+                     (2 * H_QK * D * 2 + H_V * D * 2 + 2 * H_V * 4)                  # 53,504
+BW_FLOP_PER_TOKEN = H_V * (22 * D * D + 26 * 64 * D + 4 * 64 * 64)                  # 28.3 M
 # front end, per token: raw q, k, v read and normalised q, k, v written (bf16),
 # a, b read and log_alpha, beta written (fp32); plus the conv weight once
 FE_BYTES_PER_TOKEN = 2 * (2 * H_QK + H_V) * D * 2 + 4 * H_V * 4                # 41,728
@@ -317,6 +326,34 @@ def run_prefill_shard(args, dev, stream, world, L):
     return seg, out[0], out[1]
 
 
+def run_backward(args, case, dev, stream, world, L):
+    """Time the gradients of the L-token prefill (the same inputs); returns ms per call."""
+    import torch
+    from linear_attention_12_b200 import gdn
+    q, k, v = case.q.to(dev), case.k.to(dev), case.v.to(dev)
+    la, be, cu = case.log_alpha.to(dev), case.beta.to(dev), case.cu_seqlens.to(dev)
+    gen = torch.Generator().manual_seed(7)
+    dO = torch.randn((L, H_V, D), generator=gen).to(torch.bfloat16).to(dev)
+    ws = torch.empty(int(gdn.lib().gdn_prefill_backward_workspace_size(1, L, H_QK, H_V, D, D,
+                                                                      gdn.GDN_BF16)),
+                     dtype=torch.uint8, device=dev)
+    n = max(3, min(args.steps, 10))
+    for _ in range(max(args.warmup, 3)):
+        gdn.prefill_backward(q, k, v, la, be, dO, cu_seqlens=cu, workspace=ws)
+    torch.cuda.synchronize()
+    barrier(world)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(n):
+        gdn.prefill_backward(q, k, v, la, be, dO, cu_seqlens=cu, workspace=ws)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    assert gdn.last_device_error() == gdn.GDN_OK
+    return max_over_ranks(e0.elapsed_time(e1), world) / n, n
+
+
 def run_frontend(args, dev, stream, world, L):
     """Time the front end on raw inputs of the prefill's shape; returns
     (ms per call, GB/s)."""
@@ -497,6 +534,11 @@ def run_ours(args):
     if not args.no_decode:
         dm_ms, dm_gbs = run_decode_multi(args, dev, stream, world)
 
+    # ---------------- gradients of the same prefill
+    bw = None
+    if not args.no_backward:
+        bw = run_backward(args, case, dev, stream, world, L)
+
     # ---------------- prefill of a tensor-parallel shard (few heads: sequence split)
     shard = None
     if not args.no_shard:
@@ -577,6 +619,25 @@ def run_ours(args):
                 "workload": f"decode of M={DM_M} tokens per sequence, B={args.decode_batch} H_qk={H_QK} "
                             f"H_v={H_V} d={D}, fp32 state read once, a checkpoint per token",
                 "steps": max(args.steps, 10),
+            },
+            "backward": None if bw is None else {
+                "value": L / (bw[0] / 1e3),
+                "unit": "tokens/s",
+                "ms_per_call": bw[0],
+                "roofline": {
+                    "bound": "tensor",
+                    "achieved": BW_FLOP_PER_TOKEN * L / (bw[0] / 1e3) / 1e12,
+                    "peak": tf_peak,
+                    "unit": "TFLOP/s",
+                    "frac": BW_FLOP_PER_TOKEN * L / (bw[0] / 1e3) / 1e12 / tf_peak,
+                    "flop_per_call": BW_FLOP_PER_TOKEN * L,
+                    "hbm_bytes_per_call": BW_BYTES_PER_TOKEN * L,
+                    "hbm_term_us": BW_BYTES_PER_TOKEN * L / (hbm_peak * 1e9) * 1e6,
+                    "tensor_term_us": BW_FLOP_PER_TOKEN * L / (tf_peak * 1e12) * 1e6,
+                },
+                "workload": f"gradients of the prefill B=1 L={L} H_qk={H_QK} H_v={H_V} d={D} bf16 "
+                            "(dq, dk, dv, dlog_alpha, dbeta; S0 = 0, no state gradient)",
+                "steps": bw[1],
             },
             "prefill_shard": None if shard is None else {
                 "value": L / (shard[1] / 1e3),
@@ -691,6 +752,7 @@ def main():
                     help="sequences of the decode workloads (256; smaller only for profiling)")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer measurement")
     ap.add_argument("--no-frontend", action="store_true", help="skip the front-end measurement")
+    ap.add_argument("--no-backward", action="store_true", help="skip the gradient measurement")
     ap.add_argument("--no-shard", action="store_true",
                     help="skip the tensor-parallel-shard prefill measurement")
     args = ap.parse_args()

@@ -220,6 +220,54 @@ GDN_API gdn_status gdn_decode_step(const void *q, const void *k, const void *v,
                            int32_t dk, int32_t dv, gdn_dtype io_dtype,
                            void *o, void *stream);
 
+/*
+ * gdn_prefill_backward -- gradients of gdn_prefill for training.
+ *
+ * The Qwen3.8-Flash-Next article of alwayszhang (section 九) lists a chunked
+ * prefill backward among the FlashQLA kernels and prints nothing about it.
+ * This computes the gradients of
+ *
+ *     L = <dO, o> + <dS_final, S_final>
+ *
+ * by the chain rule of the state-update formula (bjdmk.com.cn article, section
+ * 2.1), taken through the chunk form of the forward kernels:
+ *   1. It reruns the forward pass, saving the state entering every chunk.
+ *   2. It carries the state gradient backwards through the chunks (one block
+ *      per sequence, value head and d_v slice).
+ *   3. It computes every chunk's gradients in parallel.
+ *
+ *   q, k, v, log_alpha, beta, S0, cu_seqlens: the prefill's inputs, as for
+ *              gdn_prefill (S0 may be NULL).
+ *   dO       : [T, H_v, dv] in io_dtype, the gradient of o.
+ *   dS_final : [N, H_v, dk, dv] fp32, the gradient of S_final, or NULL for zero.
+ *   dq, dk   : [T, H_qk, dk] in io_dtype (written; the value heads of a
+ *              query/key head are summed).
+ *   dv       : [T, H_v, dv] in io_dtype (written).
+ *   dlog_alpha, dbeta: [T, H_v] fp32 (written).
+ *   dS0      : [N, H_v, dk, dv] fp32 (written), or NULL to skip it.
+ *   workspace: at least gdn_prefill_backward_workspace_size(...) bytes,
+ *              256-byte aligned.  It holds the chunk-operator records and two
+ *              fp32 states per (chunk slot, value head): 144 KB each, about
+ *              3.6 GB for T = 32,768 and 48 value heads.
+ * io_dtype must be GDN_BF16 (GDN_ERR_UNSUPPORTED otherwise).  Returns GDN_OK,
+ * GDN_ERR_INVALID_ARG, GDN_ERR_UNSUPPORTED, GDN_ERR_WORKSPACE or GDN_ERR_CUDA.
+ */
+GDN_API gdn_status gdn_prefill_backward(const void *q, const void *k, const void *v,
+                                const float *log_alpha, const float *beta,
+                                const float *S0, const int32_t *cu_seqlens,
+                                const void *dO, const float *dS_final,
+                                int32_t N, int32_t T, int32_t H_qk, int32_t H_v,
+                                int32_t dk, int32_t dv, gdn_dtype io_dtype,
+                                void *dq, void *dk_out, void *dv_out,
+                                float *dlog_alpha, float *dbeta, float *dS0,
+                                void *workspace, size_t workspace_bytes, void *stream);
+
+/* Workspace bytes of gdn_prefill_backward (0 when T == 0 or the arguments are
+ * invalid). */
+GDN_API size_t gdn_prefill_backward_workspace_size(int32_t N, int32_t T, int32_t H_qk,
+                                           int32_t H_v, int32_t dk, int32_t dv,
+                                           gdn_dtype io_dtype);
+
 /* Most tokens per sequence that one gdn_decode_multi call takes. */
 #define GDN_MAX_DECODE_TOKENS 8
 

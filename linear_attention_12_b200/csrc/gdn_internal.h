@@ -32,6 +32,23 @@ cudaError_t launch_prefill(const void* q, const void* k, const void* v, const fl
                            int T, int H_qk, int H_v, bool bf16, void* o, float* S_final,
                            void* workspace, int P, cudaStream_t stream);
 
+// Records and chunk-entering states of a bf16 prefill, for its gradients.
+cudaError_t launch_prefill_save(const void* q, const void* k, const void* v,
+                                const float* log_alpha, const float* beta, const float* S0,
+                                const int32_t* cu_seqlens, int N, int T, int H_qk, int H_v,
+                                uint8_t* records, float* S_saved, cudaStream_t stream);
+size_t prefill_record_bytes(int N, int T, int H_v);
+
+// Gradients of a bf16 prefill: workspace bytes, and the launches (the forward
+// pass saving every chunk's state, the reverse chain, the per-chunk gradients).
+size_t prefill_backward_workspace_bytes(int N, int T, int H_v);
+cudaError_t launch_prefill_backward(const void* q, const void* k, const void* v,
+                                    const float* log_alpha, const float* beta, const float* S0,
+                                    const int32_t* cu_seqlens, const void* dO,
+                                    const float* dS_final, int N, int T, int H_qk, int H_v,
+                                    void* dq, void* dk, void* dv, float* dlog_alpha, float* dbeta,
+                                    float* dS0, void* workspace, cudaStream_t stream);
+
 cudaError_t launch_frontend(const void* q_raw, const void* k_raw, const void* v_raw,
                             const float* conv_w, const float* a, const float* b,
                             const int32_t* cu_seqlens, int N, int T, int H_qk, int H_v,

@@ -50,32 +50,13 @@
 
 #include "gdn_common.cuh"
 #include "gdn_internal.h"
+#include "gdn_tiles.cuh"
 
 namespace gdn {
 
 namespace {
 
 constexpr int kMaxSegments = 16;  // most segments per sequence the automatic choice takes
-constexpr int C = 64;            // chunk length
-constexpr int D = 128;           // head dim (d_k = d_v)
-constexpr uint32_t HALF = 8192;  // one 64 x 64 bf16 tile: 64 rows x 128 B
-constexpr float LOG2E = 1.4426950408889634f;
-
-// ---- chunk operator record (workspace), also its image in shared memory ----
-constexpr uint32_t REC_TB = 0;                 // T diag(beta), 64 x 64 bf16, swizzled
-constexpr uint32_t REC_MQ = HALF;              // M o Q K^T,    64 x 64 bf16, swizzled
-constexpr uint32_t REC_VEC = 2 * HALF;         // gamma[64], d[64], gamma_C, pad -> 132 floats
-constexpr uint32_t REC_VEC_FLOATS = 132;
-constexpr uint32_t REC_BYTES = REC_VEC + REC_VEC_FLOATS * 4;  // 16,912
-static_assert(REC_BYTES % 16 == 0, "bulk copies move multiples of 16 bytes");
-
-// Record slot of chunk c of sequence n (first token t0 = cu[n] + 64 c):
-// j = n + floor(t0 / 64).  Distinct chunks get distinct slots, all below
-// N + ceil(T / 64), without reading cu_seqlens on the host.
-__host__ __device__ __forceinline__ long long record_slot(int n, int t0) {
-    return (long long)n + t0 / C;
-}
-
 // ---- pass 1 shared memory ----
 constexpr int P1_THREADS = 256;
 constexpr int P1_MAX_GROUP = 4;                                // value heads per work item
@@ -115,145 +96,6 @@ constexpr uint32_t P2_MISC = P2_BAR + NBAR2 * 8;
 constexpr uint32_t P2_SMEM = P2_MISC + 16 + 1024;
 static_assert(P2_SMEM <= 232448, "pass 2 shared memory budget");
 
-__device__ __forceinline__ float ex2(float x) {
-    float y;
-    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-    return y;
-}
-
-template <int ID, int N>
-__device__ __forceinline__ void bar_sync() {
-    asm volatile("bar.sync %0, %1;" ::"n"(ID), "n"(N) : "memory");
-}
-// Named barrier that also returns the AND of every participant's `ok`.
-template <int ID, int N>
-__device__ __forceinline__ bool bar_and(bool ok) {
-    uint32_t r;
-    asm volatile(
-        "{\n\t.reg .pred pi, po;\n\t"
-        "setp.ne.u32 pi, %1, 0;\n\t"
-        "bar.red.and.pred po, %2, %3, pi;\n\t"
-        "selp.u32 %0, 1, 0, po;\n\t}"
-        : "=r"(r)
-        : "r"((uint32_t)ok), "n"(ID), "n"(N)
-        : "memory");
-    return r != 0;
-}
-
-// Wait bounded in time only (used to drain in-flight copies after an abort).
-__device__ __forceinline__ void mbar_wait_drain(uint64_t* bar, uint32_t parity) {
-    const uint32_t addr = smem_u32(bar);
-    const unsigned long long t0 = globaltimer();
-    while (!mbar_try_wait(addr, parity)) {
-        if (globaltimer() - t0 > kWaitLimitNs) {
-            atomicOr(&g_status, GDN_DEV_TIMEOUT);
-            return;
-        }
-    }
-}
-
-// Address of element (row, col) of a 128B-swizzled tile whose 64-column
-// halves lie `half` bytes apart; col is a multiple of 8.
-__device__ __forceinline__ uint32_t taddr(uint32_t base, int row, int col, uint32_t half) {
-    return base + (col >> 6) * half + row * 128 + ((((col & 63) >> 3) ^ (row & 7)) << 4);
-}
-__device__ __forceinline__ uint32_t taddr_e(uint32_t base, int row, int col, uint32_t half) {
-    return taddr(base, row, col & ~7, half) + (col & 7) * 2;  // any column
-}
-
-__device__ __forceinline__ void ldsm_x4(uint32_t a, uint32_t* r) {
-    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
-                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
-                 : "r"(a));
-}
-__device__ __forceinline__ void ldsm_x4_t(uint32_t a, uint32_t* r) {
-    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
-                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
-                 : "r"(a));
-}
-// D += A * B, m16n8k16, bf16 inputs, fp32 accumulate.
-__device__ __forceinline__ void mma16816(float* d, const uint32_t* a, uint32_t b0, uint32_t b1) {
-    asm volatile(
-        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 "
-        "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
-        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
-}
-
-// A fragment (16 x 16 at rows m0, cols k0) of a K-major tile (rows m, cols k).
-__device__ __forceinline__ void lda_k(uint32_t base, uint32_t half, int m0, int k0, int lane,
-                                      uint32_t* a) {
-    ldsm_x4(taddr(base, m0 + (lane & 15), k0 + ((lane >> 4) << 3), half), a);
-}
-// A fragment of an MN-major tile (stored rows k, cols m).
-__device__ __forceinline__ void lda_mn(uint32_t base, uint32_t half, int m0, int k0, int lane,
-                                       uint32_t* a) {
-    const int j = lane >> 3;
-    ldsm_x4_t(taddr(base, k0 + (lane & 7) + ((j >> 1) << 3), m0 + ((j & 1) << 3), half), a);
-}
-// B fragments of two n-tiles (n0, n0+8) x (k0..k0+15) from a K-major tile (rows n, cols k).
-__device__ __forceinline__ void ldb_k(uint32_t base, uint32_t half, int n0, int k0, int lane,
-                                      uint32_t* b) {
-    const int j = lane >> 3;
-    ldsm_x4(taddr(base, n0 + (lane & 7) + ((j >> 1) << 3), k0 + ((j & 1) << 3), half), b);
-}
-// B fragments of two n-tiles from an MN-major tile (stored rows k, cols n).
-__device__ __forceinline__ void ldb_mn(uint32_t base, uint32_t half, int n0, int k0, int lane,
-                                       uint32_t* b) {
-    const int j = lane >> 3;
-    ldsm_x4_t(taddr(base, k0 + (lane & 7) + ((j & 1) << 3), n0 + ((j >> 1) << 3), half), b);
-}
-
-__device__ __forceinline__ uint32_t pack2(float lo, float hi) { return pack_bf16x2(lo, hi); }
-
-__device__ __forceinline__ uint32_t to_tf32(float x) {
-    uint32_t r;
-    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
-    return r;
-}
-// D += A (16 x 8, fp32 rows of stride lda) * B (8 x 8, fp32 rows of stride ldb), both
-// rounded to tf32, fp32 accumulate (m16n8k8).
-__device__ __forceinline__ void mma_tf32(float* d, const float* A, int lda, const float* B,
-                                         int ldb, int lane) {
-    const int g = lane >> 2, t = lane & 3;
-    const uint32_t a0 = to_tf32(A[g * lda + t]), a1 = to_tf32(A[(g + 8) * lda + t]);
-    const uint32_t a2 = to_tf32(A[g * lda + t + 4]), a3 = to_tf32(A[(g + 8) * lda + t + 4]);
-    const uint32_t b0 = to_tf32(B[t * ldb + g]), b1 = to_tf32(B[(t + 4) * ldb + g]);
-    asm volatile(
-        "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 "
-        "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
-        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
-}
-
-// Store an accumulator tile (rows m0.., NT n-tiles from column 0) as bf16 into a
-// swizzled tile, scaled per row by rs_lo (row g) and rs_hi (row g+8).
-template <int NT>
-__device__ __forceinline__ void store_acc_bf16(uint8_t* smem, uint32_t base_off, uint32_t half,
-                                               int m0, const float (*acc)[4], int lane,
-                                               float rs_lo, float rs_hi) {
-    const int g = lane >> 2, t = lane & 3;
-#pragma unroll
-    for (int nt = 0; nt < NT; ++nt) {
-        const int col = 8 * nt + 2 * t;
-        *reinterpret_cast<uint32_t*>(smem + taddr_e(base_off, m0 + g, col, half)) =
-            pack2(acc[nt][0] * rs_lo, acc[nt][1] * rs_lo);
-        *reinterpret_cast<uint32_t*>(smem + taddr_e(base_off, m0 + g + 8, col, half)) =
-            pack2(acc[nt][2] * rs_hi, acc[nt][3] * rs_hi);
-    }
-}
-
-template <typename IO>
-__device__ __forceinline__ void store2(IO* p, float a, float b);
-template <>
-__device__ __forceinline__ void store2<float>(float* p, float a, float b) {
-    *reinterpret_cast<float2*>(p) = make_float2(a, b);
-}
-template <>
-__device__ __forceinline__ void store2<__nv_bfloat16>(__nv_bfloat16* p, float a, float b) {
-    *reinterpret_cast<uint32_t*>(p) = pack2(a, b);
-}
-
 struct PrefillParams {
     const float* log_alpha;
     const float* beta;
@@ -262,25 +104,11 @@ struct PrefillParams {
     void* o;
     float* S_final;
     uint8_t* records;  // chunk operator records, REC_BYTES each
-    float* S_prop;     // segmented prefill, phase A: the segment propagators
+    float* S_aux;      // P2_SEGMENT: the segment propagators; P2_SAVE: every
+                       // chunk's entering state, [record slot, H_v, 128, 128]
     int H_qk, H_v;
     int N, T;
 };
-
-// Sequence n and chunk c of record slot j, or n = -1 if no chunk maps to j.
-// The first slot of sequence n, n + floor(cu[n] / 64), increases strictly with
-// n, so the owner of j is the last sequence whose first slot is <= j.
-__device__ __forceinline__ void slot_owner(const int32_t* cu, int N, int j, int& n, int& c) {
-    int lo = 0, hi = N - 1;
-    while (lo < hi) {
-        const int mid = (lo + hi + 1) >> 1;
-        if (record_slot(mid, cu[mid]) <= j) lo = mid; else hi = mid - 1;
-    }
-    n = lo;
-    c = j - (int)record_slot(lo, cu[lo]);
-    const int nch = (cu[lo + 1] - cu[lo] + C - 1) / C;
-    if (c < 0 || c >= nch) n = -1;
-}
 
 // ============================================================================
 // Pass 1: chunk operators.  Grid (record slots, H_qk, batches of up to 4 value
@@ -522,10 +350,15 @@ __global__ void __launch_bounds__(P1_THREADS, 3)
             *reinterpret_cast<float2*>(to + (g + 24) * AF_LD) = make_float2(-y1[2], -y1[3]);
         }
         __syncthreads();
-        // ---- T diag(beta) as a bf16 tile (lower blocks; the upper ones are never read)
+        // ---- T diag(beta) as a bf16 tile.  The 16 x 16 blocks above the diagonal of
+        // it and of M o Q K^T are written as zeros, so that every byte of the record
+        // is defined (the gradients read both tiles whole).
         for (int idx = pt; idx < 64 * 8; idx += P1_THREADS) {
             const int r = idx >> 3, ch = idx & 7;
-            if ((ch >> 1) <= (r >> 4)) {
+            if ((ch >> 1) > (r >> 4)) {
+                *reinterpret_cast<uint4*>(rec + REC_TB + taddr(0, r, 8 * ch, 0)) = make_uint4(0, 0, 0, 0);
+                *reinterpret_cast<uint4*>(rec + REC_MQ + taddr(0, r, 8 * ch, 0)) = make_uint4(0, 0, 0, 0);
+            } else {
                 const float4 t0v = *reinterpret_cast<const float4*>(Tf + r * AF_LD + 8 * ch);
                 const float4 t1v = *reinterpret_cast<const float4*>(Tf + r * AF_LD + 8 * ch + 4);
                 const float4 b0 = *reinterpret_cast<const float4*>(s_b + 8 * ch);
@@ -556,16 +389,6 @@ __global__ void __launch_bounds__(P1_THREADS, 3)
 }
 
 
-
-__device__ __forceinline__ void ldsm_x2_t(uint32_t a, uint32_t* r) {
-    asm volatile("ldmatrix.sync.aligned.m8n8.x2.trans.shared.b16 {%0,%1}, [%2];"
-                 : "=r"(r[0]), "=r"(r[1])
-                 : "r"(a));
-}
-// B fragment of one n-tile (n0) x (k0..k0+15) from an MN-major tile (stored rows k, cols n).
-__device__ __forceinline__ void ldb_mn1(uint32_t base, int n0, int k0, int lane, uint32_t* b) {
-    ldsm_x2_t(taddr(base, k0 + (lane & 7) + (((lane >> 3) & 1) << 3), n0, 0), b);
-}
 
 // Delta = T_b X for row block rb (rows 16 rb .. +15) and n-tiles of column half H
 // of an NT-tile slice, stored as bf16 Delta and d o Delta.
@@ -619,8 +442,10 @@ __device__ __forceinline__ void delta_half(uint8_t* sm, uint32_t tb, uint32_t xt
 // phase A of the segmented prefill -- no outputs; blocks x < slices carry the
 // state from zero (final state to S_final), blocks x >= slices carry the
 // identity with V taken as zero, so that their final state is the segment's
-// propagator P (to S_prop): S_end = P S_start + (state from zero).
-constexpr int P2_OUT = 0, P2_SEGMENT = 1;
+// propagator P (to S_aux): S_end = P S_start + (state from zero).  MODE
+// P2_SAVE: no outputs; every chunk's entering state is stored to S_aux (for
+// the gradients).
+constexpr int P2_OUT = 0, P2_SEGMENT = 1, P2_SAVE = 2;
 
 template <int NS, typename IO, int MODE>
 __global__ void __launch_bounds__(P2_THREADS, 1)
@@ -713,6 +538,19 @@ __global__ void __launch_bounds__(P2_THREADS, 1)
             const int valid = min(C, t_end - tc0);
             const bool ok = mbar_wait(&bars[B2_FULL + s], (c / NSTAGE) & 1, abort_flag);
             __syncwarp();
+            if constexpr (MODE == P2_SAVE) {  // the state entering this chunk
+                float* sv = p.S_aux + ((size_t)record_slot(n, tc0) * p.H_v + h) * D * D;
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                    for (int hl = 0; hl < 2; ++hl) {
+                        const int row = r0 + g + 8 * hl;
+                        const int col = 8 * nt + 2 * t4;
+                        if (col < ncols)
+                            *reinterpret_cast<float2*>(sv + (size_t)row * D + col0 + col) =
+                                make_float2(Sacc[nt][2 * hl], Sacc[nt][2 * hl + 1]);
+                    }
+            }
 
             // ---- warps 0-3: K S and Q S for rows m0 .. m0+15 (one pass over S)
             float accK[NT][4], accQ[NT][4];
@@ -833,7 +671,7 @@ __global__ void __launch_bounds__(P2_THREADS, 1)
             // this ring stage is free again: refill it with the chunk NSTAGE ahead
             if (tid == P2_LOADER && c + NSTAGE < nchunks) issue_chunk(issued++);
         }
-        float* const s_out = prop ? p.S_prop : p.S_final;
+        float* const s_out = prop ? p.S_aux : p.S_final;
         if (s_out && !*abort_flag) {
             float* sf = s_out + ((size_t)n * p.H_v + h) * D * D;
 #pragma unroll
@@ -878,33 +716,6 @@ __global__ void copy_state_kernel(const float* __restrict__ S0, float* __restric
     }
 }
 
-PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
-    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-    static std::once_flag once;
-    std::call_once(once, [] {
-        void* f = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &f, 12000,
-                                             cudaEnableDefault, &q) == cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
-    });
-    return fn;
-}
-
-// 2-D bf16 tensor map over a [rows, cols] row-major matrix, 64 x 64 boxes, 128B swizzle.
-bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols) {
-    auto enc = get_encode_fn();
-    if (!enc) return false;
-    cuuint64_t dims[2] = {cols, rows > 0 ? rows : 1};
-    cuuint64_t strides[1] = {cols * 2};
-    cuuint32_t box[2] = {64, 64};
-    cuuint32_t estr[2] = {1, 1};
-    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
-               box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
-           CUDA_SUCCESS;
-}
 
 // ---- segmented prefill (sequence parallelism within one GPU) -------------
 // Each sequence is cut into P segments of whole chunks, run as P "virtual"
@@ -1245,5 +1056,25 @@ cudaError_t launch_prefill(const void* q, const void* k, const void* v, const fl
     return bf16 ? run_pass2<__nv_bfloat16, P2_OUT>(mq, mk, mv, pc, sms, stream)
                 : run_pass2<float, P2_OUT>(mq, mk, mv, pc, sms, stream);
 }
+
+// The forward pass the gradients start from (bf16 q, k, v): every chunk's
+// operator record (records, N + ceil(T/64) slots x H_v) and entering state
+// (S_saved, [slot, H_v, 128, 128] fp32).
+cudaError_t launch_prefill_save(const void* q, const void* k, const void* v,
+                                const float* log_alpha, const float* beta, const float* S0,
+                                const int32_t* cu_seqlens, int N, int T, int H_qk, int H_v,
+                                uint8_t* records, float* S_saved, cudaStream_t stream) {
+    CUtensorMap mq, mk, mv;
+    if (!make_map(&mq, q, T, (uint64_t)H_qk * D) || !make_map(&mk, k, T, (uint64_t)H_qk * D) ||
+        !make_map(&mv, v, T, (uint64_t)H_v * D))
+        return cudaErrorInvalidValue;
+    const PrefillParams prm{log_alpha, beta, S0,      cu_seqlens, nullptr, nullptr,
+                            records,   S_saved, H_qk, H_v,        N,       T};
+    cudaError_t e = run_pass1(mq, mk, prm, stream);
+    if (e != cudaSuccess) return e;
+    return run_pass2<__nv_bfloat16, P2_SAVE>(mq, mk, mv, prm, device_sms(), stream);
+}
+
+size_t prefill_record_bytes(int N, int T, int H_v) { return record_bytes(N, T, H_v); }
 
 }  // namespace gdn

@@ -41,6 +41,9 @@ SIGNATURES = {
     "gdn_prefill_segmented_workspace_size": (_c.c_size_t,
                                              [_c.c_int32] * 6 + [_c.c_int, _c.c_int32]),
     "gdn_prefill_auto_segments": (_c.c_int32, [_c.c_int32] * 4),
+    "gdn_prefill_backward": (_c.c_int, [_c.c_void_p] * 9 + [_c.c_int32] * 6 +
+                             [_c.c_int] + [_c.c_void_p] * 7 + [_c.c_size_t, _c.c_void_p]),
+    "gdn_prefill_backward_workspace_size": (_c.c_size_t, [_c.c_int32] * 6 + [_c.c_int]),
     "gdn_prefill_noalloc": (_c.c_int, [_c.c_void_p, _c.c_void_p, _c.c_void_p, _c.c_void_p,
                                        _c.c_void_p, _c.c_void_p, _c.c_void_p, _c.c_int32,
                                        _c.c_int32, _c.c_int32, _c.c_int32, _c.c_int32,
@@ -199,6 +202,48 @@ def decode_step(q, k, v, log_alpha, beta, S, *, o=None, stream=None):
     if st != GDN_OK:
         raise GDNError(st, "gdn_decode_step")
     return o
+
+
+def prefill_backward(q, k, v, log_alpha, beta, dO, S0=None, dS_final=None, cu_seqlens=None, *,
+                     want_dS0=True, workspace=None, stream=None):
+    """Gradients of ``L = <dO, o> + <dS_final, S_final>`` for gdn_prefill (bf16).
+
+    Returns ``(dq, dk, dv, dlog_alpha, dbeta, dS0)`` (``dS0`` None if not wanted)."""
+    T, H_qk, dk_ = q.shape
+    H_v, dv_ = v.shape[1], v.shape[2]
+    dt = q.dtype
+    _check(q, "q", dt)
+    _check(k, "k", dt, q.shape)
+    _check(v, "v", dt, (T, H_v, dv_))
+    _check(dO, "dO", dt, (T, H_v, dv_))
+    _check(log_alpha, "log_alpha", torch.float32, (T, H_v))
+    _check(beta, "beta", torch.float32, (T, H_v))
+    if cu_seqlens is None:
+        cu_seqlens = torch.tensor([0, T], dtype=torch.int32, device=q.device)
+    _check(cu_seqlens, "cu_seqlens", torch.int32)
+    N = cu_seqlens.numel() - 1
+    if S0 is not None:
+        _check(S0, "S0", torch.float32, (N, H_v, dk_, dv_))
+    if dS_final is not None:
+        _check(dS_final, "dS_final", torch.float32, (N, H_v, dk_, dv_))
+    dq, dk = torch.empty_like(q), torch.empty_like(k)
+    dv = torch.empty_like(v)
+    dla, dbe = torch.empty_like(log_alpha), torch.empty_like(beta)
+    dS0 = (torch.empty((N, H_v, dk_, dv_), dtype=torch.float32, device=q.device)
+           if want_dS0 else None)
+    io = _io_dtype(q)
+    need = int(lib().gdn_prefill_backward_workspace_size(N, T, H_qk, H_v, dk_, dv_, io))
+    if need and workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    wbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    st = lib().gdn_prefill_backward(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta),
+                                    _ptr(S0), _ptr(cu_seqlens), _ptr(dO), _ptr(dS_final), N, T,
+                                    H_qk, H_v, dk_, dv_, io, _ptr(dq), _ptr(dk), _ptr(dv),
+                                    _ptr(dla), _ptr(dbe), _ptr(dS0), _ptr(workspace), wbytes,
+                                    _stream_handle(stream))
+    if st != GDN_OK:
+        raise GDNError(st, "gdn_prefill_backward")
+    return dq, dk, dv, dla, dbe, dS0
 
 
 MAX_DECODE_TOKENS = 8  # GDN_MAX_DECODE_TOKENS

@@ -131,6 +131,41 @@ def test_automatic_split_only_for_few_chains(L):
     assert L.gdn_prefill_auto_segments(0, 32768, 1, 1) == 1      # invalid: no split
 
 
+def _backward(L, **kw):
+    a = dict(q=P, k=P, v=P, la=P, be=P, S0=None, cu=P, dO=P, dSf=None, N=1, T=64, H_qk=1, H_v=1,
+             dk=128, dv=128, dt=gdn.GDN_BF16, dq=P, dk_out=P, dv_out=P, dla=P, dbe=P, dS0=None,
+             ws=P, wsb=1 << 40, stream=None)
+    a.update(kw)
+    return L.gdn_prefill_backward(a["q"], a["k"], a["v"], a["la"], a["be"], a["S0"], a["cu"],
+                                  a["dO"], a["dSf"], a["N"], a["T"], a["H_qk"], a["H_v"], a["dk"],
+                                  a["dv"], a["dt"], a["dq"], a["dk_out"], a["dv_out"], a["dla"],
+                                  a["dbe"], a["dS0"], a["ws"], a["wsb"], a["stream"])
+
+
+@pytest.mark.parametrize("kw,expect", [
+    (dict(dt=gdn.GDN_F32), gdn.GDN_ERR_UNSUPPORTED),
+    (dict(dO=None), gdn.GDN_ERR_INVALID_ARG),
+    (dict(dq=None), gdn.GDN_ERR_INVALID_ARG),
+    (dict(dv_out=P + 8), gdn.GDN_ERR_INVALID_ARG),
+    (dict(dla=None), gdn.GDN_ERR_INVALID_ARG),
+    (dict(dS0=BAD), gdn.GDN_ERR_INVALID_ARG),
+    (dict(wsb=16), gdn.GDN_ERR_WORKSPACE),
+    (dict(ws=P + 64), gdn.GDN_ERR_WORKSPACE),   # not 256-byte aligned
+    (dict(H_qk=2, H_v=3), gdn.GDN_ERR_INVALID_ARG),
+])
+def test_backward_rejects_bad_arguments_on_host(L, kw, expect):
+    assert _backward(L, **kw) == expect
+
+
+def test_backward_workspace_holds_records_and_two_states_per_chunk(L):
+    N, T, H_v = 1, 4096, 3
+    ws = L.gdn_prefill_backward_workspace_size(N, T, 1, H_v, 128, 128, gdn.GDN_BF16)
+    slots = N + T // 64
+    assert ws >= slots * H_v * (16912 + 2 * 128 * 128 * 4)
+    assert ws <= slots * H_v * (16912 + 2 * 128 * 128 * 4) + 3 * 256
+    assert L.gdn_prefill_backward_workspace_size(N, T, 1, H_v, 128, 128, gdn.GDN_F32) == 0
+
+
 def _decode(L, **kw):
     a = dict(q=P, k=P, v=P, la=P, be=P, S=P, B=4, H_qk=1, H_v=3, dk=128, dv=128,
              dt=gdn.GDN_BF16, o=P, stream=None)
