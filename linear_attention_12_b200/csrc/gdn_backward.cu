@@ -346,24 +346,43 @@ constexpr uint32_t GC_SMEM = GC_MISC + 16 + 1024;
 static_assert(GC_SMEM <= 232448, "per-chunk gradient shared memory budget");
 
 // fp32 [128][128] state -> 128B-swizzled bf16 tile (two 128-row halves);
-// returns this thread's part of sum(a o b) when b is given.
+// returns this thread's part of sum(src o other) when other is given.  Each
+// thread converts 8 groups of 8 values, loading two groups before storing.
 __device__ __forceinline__ float stage_state(uint8_t* sm, uint32_t dst, const float* src,
                                              const float* other, int tid) {
     float dot = 0.f;
-    for (int e = tid; e < D * D / 8; e += 256) {
-        const int row = e / 16, c8 = (e % 16) * 8;
-        const float4 a = *reinterpret_cast<const float4*>(src + (size_t)row * D + c8);
-        const float4 b = *reinterpret_cast<const float4*>(src + (size_t)row * D + c8 + 4);
-        *reinterpret_cast<uint4*>(sm + taddr(dst, row, c8, SHALF)) =
-            make_uint4(pack2(a.x, a.y), pack2(a.z, a.w), pack2(b.x, b.y), pack2(b.z, b.w));
-        if (other) {
-            const float4 x = *reinterpret_cast<const float4*>(other + (size_t)row * D + c8);
-            const float4 y = *reinterpret_cast<const float4*>(other + (size_t)row * D + c8 + 4);
-            dot += a.x * x.x + a.y * x.y + a.z * x.z + a.w * x.w + b.x * y.x + b.y * y.y +
-                   b.z * y.z + b.w * y.w;
+#pragma unroll 1
+    for (int e0 = tid; e0 < D * D / 8; e0 += 512) {
+        float4 a[2], b[2], x[2], y[2];
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+            const int e = e0 + 256 * u, row = e / 16, c8 = (e % 16) * 8;
+            a[u] = *reinterpret_cast<const float4*>(src + (size_t)row * D + c8);
+            b[u] = *reinterpret_cast<const float4*>(src + (size_t)row * D + c8 + 4);
+            if (other) {
+                x[u] = *reinterpret_cast<const float4*>(other + (size_t)row * D + c8);
+                y[u] = *reinterpret_cast<const float4*>(other + (size_t)row * D + c8 + 4);
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+            const int e = e0 + 256 * u, row = e / 16, c8 = (e % 16) * 8;
+            *reinterpret_cast<uint4*>(sm + taddr(dst, row, c8, SHALF)) =
+                make_uint4(pack2(a[u].x, a[u].y), pack2(a[u].z, a[u].w), pack2(b[u].x, b[u].y),
+                           pack2(b[u].z, b[u].w));
+            if (other)
+                dot += a[u].x * x[u].x + a[u].y * x[u].y + a[u].z * x[u].z + a[u].w * x[u].w +
+                       b[u].x * y[u].x + b[u].y * y[u].y + b[u].z * y[u].z + b[u].w * y[u].w;
         }
     }
     return dot;
+}
+
+// Bring a 64 KiB fp32 state (512 lines of 128 B) into L2 ahead of its use.
+__device__ __forceinline__ void prefetch_state(const float* src, int tid) {
+#pragma unroll
+    for (int i = 0; i < 2; ++i)
+        asm volatile("prefetch.global.L2 [%0];" ::"l"(src + (size_t)(tid + 256 * i) * 32));
 }
 
 // Row sums (over the accumulator's columns) of acc o w, into dst[row] (smem,
@@ -436,6 +455,11 @@ __global__ void __launch_bounds__(256, 1)
     const int valid = min(C, t_end - tc0);
     const long long slot = record_slot(n, tc0);
 
+    {  // the first value head's states, into L2 while K and Q arrive
+        const size_t so = ((size_t)slot * p.H_v + hq * group) * D * D;
+        prefetch_state(p.S_saved + so, tid);
+        prefetch_state(p.dS_saved + so, tid);
+    }
     if (tid == 0) {
         mbar_init(&bars[0], 1);
         mbar_init(&bars[1], 1);
@@ -481,8 +505,13 @@ __global__ void __launch_bounds__(256, 1)
             bulk_load(sm + GC_REC, p.records + (size_t)(slot * p.H_v + h) * REC_BYTES, REC_BYTES,
                       &bars[1]);
         }
-        // meanwhile: the states in bf16, <dS', S>, the gates
+        // meanwhile: the states in bf16, <dS', S>, the gates; the next value
+        // head's states into L2
         const size_t so = ((size_t)slot * p.H_v + h) * D * D;
+        if (vh + 1 < group) {
+            prefetch_state(p.S_saved + so + D * D, tid);
+            prefetch_state(p.dS_saved + so + D * D, tid);
+        }
         stage_state(sm, GC_S, p.S_saved + so, nullptr, tid);
         float dot = stage_state(sm, GC_DS, p.dS_saved + so, p.S_saved + so, tid);
 #pragma unroll
