@@ -248,9 +248,11 @@ GDN_API gdn_status gdn_decode_step(const void *q, const void *k, const void *v,
  *   workspace: at least gdn_prefill_backward_workspace_size(...) bytes,
  *              256-byte aligned.  It holds the chunk-operator records and two
  *              fp32 states per (chunk slot, value head): 144 KB each, about
- *              3.6 GB for T = 32,768 and 48 value heads.
- * io_dtype must be GDN_BF16 (GDN_ERR_UNSUPPORTED otherwise).  Returns GDN_OK,
- * GDN_ERR_INVALID_ARG, GDN_ERR_UNSUPPORTED, GDN_ERR_WORKSPACE or GDN_ERR_CUDA.
+ *              3.6 GB for T = 32,768 and 48 value heads.  For GDN_F32 it also
+ *              holds bf16 copies of q, k, v and dO (the products read bf16
+ *              operands, as in the forward pass).
+ * Returns GDN_OK, GDN_ERR_INVALID_ARG, GDN_ERR_UNSUPPORTED, GDN_ERR_WORKSPACE
+ * or GDN_ERR_CUDA.
  */
 GDN_API gdn_status gdn_prefill_backward(const void *q, const void *k, const void *v,
                                 const float *log_alpha, const float *beta,

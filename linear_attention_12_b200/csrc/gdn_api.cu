@@ -216,10 +216,8 @@ gdn_status gdn_decode_step(const void* q, const void* k, const void* v, const fl
 
 size_t gdn_prefill_backward_workspace_size(int32_t N, int32_t T, int32_t H_qk, int32_t H_v,
                                            int32_t dk, int32_t dv, gdn_dtype io_dtype) {
-    if (N <= 0 || T < 0 || io_dtype != GDN_BF16 ||
-        check_heads(H_qk, H_v, dk, dv, io_dtype) != GDN_OK)
-        return 0;
-    return gdn::prefill_backward_workspace_bytes(N, T, H_v);
+    if (N <= 0 || T < 0 || check_heads(H_qk, H_v, dk, dv, io_dtype) != GDN_OK) return 0;
+    return gdn::prefill_backward_workspace_bytes(N, T, H_qk, H_v, io_dtype == GDN_BF16);
 }
 
 gdn_status gdn_prefill_backward(const void* q, const void* k, const void* v,
@@ -232,7 +230,6 @@ gdn_status gdn_prefill_backward(const void* q, const void* k, const void* v,
     gdn_status st = check_prefill_args(q, k, v, log_alpha, beta, S0, cu_seqlens, N, T, H_qk, H_v,
                                        dk, dv, io_dtype, dq, nullptr);
     if (st != GDN_OK) return st;
-    if (io_dtype != GDN_BF16) return GDN_ERR_UNSUPPORTED;
     if (T > 0) {
         const void* p16[] = {dO, dk_out, dv_out};
         for (const void* ptr : p16)
@@ -242,13 +239,14 @@ gdn_status gdn_prefill_backward(const void* q, const void* k, const void* v,
     }
     if ((dS_final && !aligned(dS_final, 16)) || (dS0 && !aligned(dS0, 16)))
         return GDN_ERR_INVALID_ARG;
-    const size_t need = gdn::prefill_backward_workspace_bytes(N, T, H_v);
+    const size_t need = gdn::prefill_backward_workspace_bytes(N, T, H_qk, H_v, io_dtype == GDN_BF16);
     if (need > 0 && (!workspace || workspace_bytes < need || !aligned(workspace, 256)))
         return GDN_ERR_WORKSPACE;
     st = check_device();
     if (st != GDN_OK) return st;
     cudaError_t e = gdn::launch_prefill_backward(q, k, v, log_alpha, beta, S0, cu_seqlens, dO,
-                                                 dS_final, N, T, H_qk, H_v, dq, dk_out, dv_out,
+                                                 dS_final, N, T, H_qk, H_v,
+                                                 io_dtype == GDN_BF16, dq, dk_out, dv_out,
                                                  dlog_alpha, dbeta, dS0, workspace,
                                                  static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;

@@ -790,31 +790,52 @@ __global__ void __launch_bounds__(256, 1)
         }
 }
 
-template <int NS>
+template <int NS, typename IO>
 cudaError_t launch_grad_state(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mo,
                               const GradParams& prm, cudaStream_t stream) {
-    auto kern = grad_state_kernel<NS, __nv_bfloat16>;
+    auto kern = grad_state_kernel<NS, IO>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, GS_SMEM);
     if (e != cudaSuccess) return e;
     kern<<<dim3((D + NS - 1) / NS, prm.H_v, prm.N), 256, GS_SMEM, stream>>>(mq, mk, mo, prm);
     return cudaGetLastError();
 }
 
+// The reverse chain (as many d_v slices as fit in one wave of one block per
+// SM), then the per-chunk gradients; IO is the type of dq, dk and dv.
+template <typename IO>
+cudaError_t launch_grads(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+                         const CUtensorMap& mo, const GradParams& prm, long long units, int sms,
+                         size_t slots, cudaStream_t stream) {
+    cudaError_t e = units * 4 <= sms ? launch_grad_state<32, IO>(mq, mk, mo, prm, stream)
+                    : units * 3 <= sms ? launch_grad_state<48, IO>(mq, mk, mo, prm, stream)
+                                       : launch_grad_state<64, IO>(mq, mk, mo, prm, stream);
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(grad_chunk_kernel<IO>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             GC_SMEM);
+    if (e != cudaSuccess) return e;
+    grad_chunk_kernel<IO><<<dim3((unsigned)slots, prm.H_qk), 256, GC_SMEM, stream>>>(mq, mk, mv, mo,
+                                                                                    prm);
+    return cudaGetLastError();
+}
+
 }  // namespace
 
-size_t prefill_backward_workspace_bytes(int N, int T, int H_v) {
+size_t prefill_backward_workspace_bytes(int N, int T, int H_qk, int H_v, bool bf16) {
     if (T == 0) return 0;
     const size_t slots = (size_t)N + ((size_t)T + C - 1) / C;
-    const size_t states = (slots * H_v * D * D * sizeof(float) + 255) & ~size_t(255);
-    return prefill_record_bytes(N, T, H_v) + 2 * states;
+    const size_t states = up256(slots * H_v * D * D * sizeof(float));
+    const size_t staging =
+        bf16 ? 0 : 2 * up256((size_t)T * H_qk * D * 2) + 2 * up256((size_t)T * H_v * D * 2);
+    return prefill_record_bytes(N, T, H_v) + 2 * states + staging;
 }
 
 cudaError_t launch_prefill_backward(const void* q, const void* k, const void* v,
                                     const float* log_alpha, const float* beta, const float* S0,
                                     const int32_t* cu_seqlens, const void* dO,
                                     const float* dS_final, int N, int T, int H_qk, int H_v,
-                                    void* dq, void* dk, void* dv, float* dlog_alpha, float* dbeta,
-                                    float* dS0, void* workspace, cudaStream_t stream) {
+                                    bool bf16, void* dq, void* dk, void* dv, float* dlog_alpha,
+                                    float* dbeta, float* dS0, void* workspace,
+                                    cudaStream_t stream) {
     if (T == 0) {  // nothing ran: dS0 = dS_final (or zero)
         if (dS0) {
             const size_t bytes = (size_t)N * H_v * D * D * sizeof(float);
@@ -825,12 +846,32 @@ cudaError_t launch_prefill_backward(const void* q, const void* k, const void* v,
     }
     uint8_t* ws = static_cast<uint8_t*>(workspace);
     const size_t slots = (size_t)N + ((size_t)T + C - 1) / C;
-    const size_t states = (slots * H_v * D * D * sizeof(float) + 255) & ~size_t(255);
+    const size_t states = up256(slots * H_v * D * D * sizeof(float));
     uint8_t* records = ws;
     float* S_saved = reinterpret_cast<float*>(ws + prefill_record_bytes(N, T, H_v));
     float* dS_saved = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(S_saved) + states);
-    cudaError_t e = launch_prefill_save(q, k, v, log_alpha, beta, S0, cu_seqlens, N, T, H_qk, H_v,
-                                        records, S_saved, stream);
+    cudaError_t e;
+    if (!bf16) {  // bf16 copies of q, k, v and dO after the states
+        uint8_t* st = reinterpret_cast<uint8_t*>(dS_saved) + states;
+        const size_t nqk = (size_t)T * H_qk * D, nv = (size_t)T * H_v * D;
+        const void* src[4] = {q, k, v, dO};
+        const size_t cnt[4] = {nqk, nqk, nv, nv};
+        const void* dst[4];
+        for (int i = 0; i < 4; ++i) {
+            f32_to_bf16_kernel<<<592, 256, 0, stream>>>(static_cast<const float*>(src[i]),
+                                                       reinterpret_cast<__nv_bfloat16*>(st),
+                                                       cnt[i] / 4);
+            dst[i] = st;
+            st += up256(cnt[i] * 2);
+        }
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        q = dst[0];
+        k = dst[1];
+        v = dst[2];
+        dO = dst[3];
+    }
+    e = launch_prefill_save(q, k, v, log_alpha, beta, S0, cu_seqlens, N, T, H_qk, H_v, records,
+                            S_saved, stream);
     if (e != cudaSuccess) return e;
     CUtensorMap mq, mk, mv, mo;
     if (!make_map(&mq, q, T, (uint64_t)H_qk * D) || !make_map(&mk, k, T, (uint64_t)H_qk * D) ||
@@ -838,19 +879,10 @@ cudaError_t launch_prefill_backward(const void* q, const void* k, const void* v,
         return cudaErrorInvalidValue;
     const GradParams prm{log_alpha, beta, cu_seqlens, records, S_saved, dS_saved, dS_final, dS0,
                          dq,        dk,   dv,         dlog_alpha, dbeta, H_qk, H_v, N, T};
-    // the reverse chain: one block per SM at most, as many d_v slices as fit in a wave
     const long long units = (long long)N * H_v;
     const int sms = device_sms();
-    e = units * 4 <= sms ? launch_grad_state<32>(mq, mk, mo, prm, stream)
-                         : (units * 3 <= sms ? launch_grad_state<48>(mq, mk, mo, prm, stream)
-                                             : launch_grad_state<64>(mq, mk, mo, prm, stream));
-    if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(grad_chunk_kernel<__nv_bfloat16>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize, GC_SMEM);
-    if (e != cudaSuccess) return e;
-    grad_chunk_kernel<__nv_bfloat16><<<dim3((unsigned)slots, H_qk), 256, GC_SMEM, stream>>>(
-        mq, mk, mv, mo, prm);
-    return cudaGetLastError();
+    return bf16 ? launch_grads<__nv_bfloat16>(mq, mk, mv, mo, prm, units, sms, slots, stream)
+                : launch_grads<float>(mq, mk, mv, mo, prm, units, sms, slots, stream);
 }
 
 }  // namespace gdn

@@ -41,13 +41,14 @@ size_t prefill_record_bytes(int N, int T, int H_v);
 
 // Gradients of a bf16 prefill: workspace bytes, and the launches (the forward
 // pass saving every chunk's state, the reverse chain, the per-chunk gradients).
-size_t prefill_backward_workspace_bytes(int N, int T, int H_v);
+size_t prefill_backward_workspace_bytes(int N, int T, int H_qk, int H_v, bool bf16);
 cudaError_t launch_prefill_backward(const void* q, const void* k, const void* v,
                                     const float* log_alpha, const float* beta, const float* S0,
                                     const int32_t* cu_seqlens, const void* dO,
                                     const float* dS_final, int N, int T, int H_qk, int H_v,
-                                    void* dq, void* dk, void* dv, float* dlog_alpha, float* dbeta,
-                                    float* dS0, void* workspace, cudaStream_t stream);
+                                    bool bf16, void* dq, void* dk, void* dv, float* dlog_alpha,
+                                    float* dbeta, float* dS0, void* workspace,
+                                    cudaStream_t stream);
 
 cudaError_t launch_frontend(const void* q_raw, const void* k_raw, const void* v_raw,
                             const float* conv_w, const float* a, const float* b,

@@ -693,19 +693,6 @@ __global__ void __launch_bounds__(P2_THREADS, 1)
     __syncthreads();
 }
 
-// fp32 -> bf16 staging of q, k, v for fp32 I/O.
-__global__ void f32_to_bf16_kernel(const float* __restrict__ src, __nv_bfloat16* __restrict__ dst,
-                                   size_t n4) {
-    for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n4;
-         i += (size_t)gridDim.x * blockDim.x) {
-        const float4 v = reinterpret_cast<const float4*>(src)[i];
-        uint2 u;
-        u.x = pack2(v.x, v.y);
-        u.y = pack2(v.z, v.w);
-        reinterpret_cast<uint2*>(dst)[i] = u;
-    }
-}
-
 // S_final = S0, or zeros when S0 is NULL (used when no sequence has tokens).
 __global__ void copy_state_kernel(const float* __restrict__ S0, float* __restrict__ S_final,
                                   size_t n4) {
@@ -854,7 +841,6 @@ cudaError_t launch_pass2(const CUtensorMap& mq, const CUtensorMap& mk, const CUt
     return cudaGetLastError();
 }
 
-size_t up256(size_t b) { return (b + 255) & ~size_t(255); }
 
 size_t staging_bytes(int T, int H_qk, int H_v, bool bf16) {
     if (bf16) return 0;

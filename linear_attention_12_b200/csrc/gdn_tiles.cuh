@@ -126,6 +126,19 @@ __device__ __forceinline__ void ldb_mn(uint32_t base, uint32_t half, int n0, int
 
 __device__ __forceinline__ uint32_t pack2(float lo, float hi) { return pack_bf16x2(lo, hi); }
 
+// fp32 -> bf16 copies of row-major operands for fp32 I/O (the tensor maps
+// read bf16); n4 = elements / 4.
+__global__ void f32_to_bf16_kernel(const float* __restrict__ src, __nv_bfloat16* __restrict__ dst,
+                                   size_t n4) {
+    for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n4;
+         i += (size_t)gridDim.x * blockDim.x) {
+        const float4 v = reinterpret_cast<const float4*>(src)[i];
+        reinterpret_cast<uint2*>(dst)[i] = make_uint2(pack2(v.x, v.y), pack2(v.z, v.w));
+    }
+}
+
+inline size_t up256(size_t b) { return (b + 255) & ~size_t(255); }
+
 __device__ __forceinline__ uint32_t to_tf32(float x) {
     uint32_t r;
     asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));

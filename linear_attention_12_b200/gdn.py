@@ -206,7 +206,8 @@ def decode_step(q, k, v, log_alpha, beta, S, *, o=None, stream=None):
 
 def prefill_backward(q, k, v, log_alpha, beta, dO, S0=None, dS_final=None, cu_seqlens=None, *,
                      want_dS0=True, workspace=None, stream=None):
-    """Gradients of ``L = <dO, o> + <dS_final, S_final>`` for gdn_prefill (bf16).
+    """Gradients of ``L = <dO, o> + <dS_final, S_final>`` for gdn_prefill (bf16 or
+    fp32 q, k, v, dO; the gradients of q, k, v in the same type).
 
     Returns ``(dq, dk, dv, dlog_alpha, dbeta, dS0)`` (``dS0`` None if not wanted)."""
     T, H_qk, dk_ = q.shape

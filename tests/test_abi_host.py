@@ -143,7 +143,6 @@ def _backward(L, **kw):
 
 
 @pytest.mark.parametrize("kw,expect", [
-    (dict(dt=gdn.GDN_F32), gdn.GDN_ERR_UNSUPPORTED),
     (dict(dO=None), gdn.GDN_ERR_INVALID_ARG),
     (dict(dq=None), gdn.GDN_ERR_INVALID_ARG),
     (dict(dv_out=P + 8), gdn.GDN_ERR_INVALID_ARG),
@@ -157,13 +156,23 @@ def test_backward_rejects_bad_arguments_on_host(L, kw, expect):
     assert _backward(L, **kw) == expect
 
 
+def test_backward_fp32_needs_room_for_bf16_copies(L):
+    ws16 = L.gdn_prefill_backward_workspace_size(1, 64, 1, 1, 128, 128, gdn.GDN_BF16)
+    ws32 = L.gdn_prefill_backward_workspace_size(1, 64, 1, 1, 128, 128, gdn.GDN_F32)
+    assert ws32 > ws16
+    assert _backward(L, dt=gdn.GDN_F32, wsb=ws16) == gdn.GDN_ERR_WORKSPACE
+    assert _backward(L, dt=gdn.GDN_BF16, wsb=ws16) == gdn.GDN_ERR_CUDA  # host checks pass; no device
+
+
 def test_backward_workspace_holds_records_and_two_states_per_chunk(L):
     N, T, H_v = 1, 4096, 3
     ws = L.gdn_prefill_backward_workspace_size(N, T, 1, H_v, 128, 128, gdn.GDN_BF16)
     slots = N + T // 64
     assert ws >= slots * H_v * (16912 + 2 * 128 * 128 * 4)
     assert ws <= slots * H_v * (16912 + 2 * 128 * 128 * 4) + 3 * 256
-    assert L.gdn_prefill_backward_workspace_size(N, T, 1, H_v, 128, 128, gdn.GDN_F32) == 0
+    # fp32 I/O adds bf16 copies of q, k (1 head) and v, dO (H_v heads)
+    ws32 = L.gdn_prefill_backward_workspace_size(N, T, 1, H_v, 128, 128, gdn.GDN_F32)
+    assert ws32 == ws + 2 * T * 128 * 2 * (1 + H_v)
 
 
 def _decode(L, **kw):

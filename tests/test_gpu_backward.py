@@ -1,4 +1,4 @@
-"""GPU parity of gdn_prefill_backward (bf16) against the fp64 backward oracle
+"""GPU parity of gdn_prefill_backward (bf16 and fp32 I/O) against the fp64 backward oracle
 (oracle/backward.py), through the C ABI: every gradient on ragged packed
 sequences, many-chunk sequences, grouped heads and long-memory gates.
 
@@ -15,16 +15,18 @@ pytestmark = pytest.mark.gpu
 TOL = 1e-2
 
 
-def _case(name, lens, H_qk, H_v, seed, s0=True, with_dsf=True, alpha_mu=0.0):
-    case = inputs.make_prefill(name, lens, H_qk, H_v, seed=seed, s0=s0, alpha_mu=alpha_mu)
+def _case(name, lens, H_qk, H_v, seed, s0=True, with_dsf=True, alpha_mu=0.0,
+          dtype=torch.bfloat16):
+    case = inputs.make_prefill(name, lens, H_qk, H_v, seed=seed, s0=s0, alpha_mu=alpha_mu,
+                               dtype=dtype)
     gen = torch.Generator().manual_seed(seed + 1000)
     T, N = case.q.shape[0], len(lens)
-    dO = torch.randn((T, H_v, 128), generator=gen).to(torch.bfloat16)
+    dO = torch.randn((T, H_v, 128), generator=gen).to(dtype)
     dSf = 0.1 * torch.randn((N, H_v, 128, 128), generator=gen) if with_dsf else None
     return case, dO, dSf
 
 
-def _check(case, dO, dSf):
+def _check(case, dO, dSf, dtype=torch.bfloat16):
     d = lambda x: None if x is None else x.cuda()
     got = gdn.prefill_backward(d(case.q), d(case.k), d(case.v), d(case.log_alpha), d(case.beta),
                                d(dO), S0=d(case.S0), dS_final=d(dSf),
@@ -36,6 +38,7 @@ def _check(case, dO, dSf):
                                     S0=None if case.S0 is None else case.S0.numpy(),
                                     dS_final=None if dSf is None else dSf.numpy(),
                                     cu_seqlens=case.cu_seqlens.numpy())
+    assert got[0].dtype == got[1].dtype == got[2].dtype == dtype
     for name, a, b in zip(["dq", "dk", "dv", "dlog_alpha", "dbeta", "dS0"], got, ref):
         a = a.float().cpu().double().numpy()
         err = np.abs(a - b).max() / max(np.abs(b).max(), 1e-300)
@@ -61,3 +64,11 @@ def test_backward_sixteen_heads_4k_packed():
     # a mid-size packed case with the benchmark's head layout on a quarter of the heads
     case, dO, dSf = _case("bw_4k", [1500, 2596], 4, 12, seed=9)
     _check(case, dO, dSf)
+
+
+@pytest.mark.parametrize("lens,H_qk,H_v", [([100, 0, 37, 64], 2, 6), ([1100], 1, 3)])
+def test_backward_fp32_io(lens, H_qk, H_v):
+    # fp32 inputs and gradients (the products read bf16 copies of q, k, v and dO)
+    case, dO, dSf = _case("bw_f32", lens, H_qk, H_v, seed=11, alpha_mu=-6.0,
+                          dtype=torch.float32)
+    _check(case, dO, dSf, dtype=torch.float32)
