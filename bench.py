@@ -524,6 +524,25 @@ def run_ours(args):
     t_hbm = bytes_per_launch / (hbm_peak * 1e9)
     t_tc = flops_per_launch / (tf_peak * 1e12)
 
+    # ---------------- the same prefill with its output state pass on tcgen05
+    tc_ms = None
+    if not args.no_tc:
+        def tc_step():
+            gdn.prefill(q, k, v, la, be, None, cu, o=o, S_final=Sf, workspace=ws, tcgen05=True)
+        for _ in range(args.warmup):
+            tc_step()
+        torch.cuda.synchronize()
+        barrier(world)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(args.steps):
+            tc_step()
+        b.record(stream)
+        torch.cuda.synchronize()
+        barrier(world)
+        assert gdn.last_device_error() == gdn.GDN_OK
+        tc_ms = max_over_ranks(a.elapsed_time(b), world) / args.steps
+
     # ---------------- decode workload (states in place)
     dec_ms = dec_gbs = None
     if not args.no_decode:
@@ -596,6 +615,16 @@ def run_ours(args):
                 "tensor_term_us": t_tc * 1e6,
                 "frac_of_roofline_time": max(t_hbm, t_tc) / (kern_avg_ms / 1e3),
                 "tflops": flops_per_launch / (kern_avg_ms / 1e3) / 1e12,
+            },
+            "prefill_tcgen05": None if tc_ms is None else {
+                "value": L / (tc_ms / 1e3),
+                "unit": "tokens/s",
+                "ms_per_call": tc_ms,
+                "ms_per_call_default": ms_per_step,
+                "ratio_to_default": ms_per_step / tc_ms,
+                "workload": "the headline prefill with its output state pass on tcgen05 "
+                            "(gdn_prefill_tc); not the default path",
+                "steps": args.steps,
             },
             "decode": None if dec_gbs is None else {
                 "value": dec_gbs,
@@ -753,6 +782,8 @@ def main():
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer measurement")
     ap.add_argument("--no-frontend", action="store_true", help="skip the front-end measurement")
     ap.add_argument("--no-backward", action="store_true", help="skip the gradient measurement")
+    ap.add_argument("--no-tc", action="store_true",
+                    help="skip the prefill with the tcgen05 state pass")
     ap.add_argument("--no-shard", action="store_true",
                     help="skip the tensor-parallel-shard prefill measurement")
     args = ap.parse_args()

@@ -158,6 +158,25 @@ GDN_API gdn_status gdn_prefill_segmented(const void *q, const void *k, const voi
                                  void *o, float *S_final, int32_t segments,
                                  void *workspace, size_t workspace_bytes, void *stream);
 
+/*
+ * gdn_prefill_tc -- gdn_prefill with the state pass that writes the outputs
+ * on the fifth-generation tensor cores (tcgen05.mma, accumulators in tensor
+ * memory) instead of mma.sync.  Same arguments, layouts, workspace
+ * (gdn_prefill_workspace_size), results within rounding, and errors as
+ * gdn_prefill; the automatic segment choice applies as there.  Per chunk the
+ * pass runs four dependent tensor-memory products ([K; Q] S, T_b X,
+ * K^T (d o Delta) and [T_b; M o Q K^T] Delta, the chunk form of the
+ * bjdmk.com.cn article's recurrence, section 2.1) with a read-back between
+ * them; at 16/48 heads and 32,768 tokens it is slower than gdn_prefill's
+ * mma.sync pass, which stays the default.
+ */
+GDN_API gdn_status gdn_prefill_tc(const void *q, const void *k, const void *v,
+                                  const float *log_alpha, const float *beta, const float *S0,
+                                  const int32_t *cu_seqlens, int32_t N, int32_t T, int32_t H_qk,
+                                  int32_t H_v, int32_t dk, int32_t dv, gdn_dtype io_dtype,
+                                  void *o, float *S_final, void *workspace,
+                                  size_t workspace_bytes, void *stream);
+
 /* Workspace bytes of gdn_prefill_segmented with these arguments (0 when T == 0
  * or the arguments are invalid). */
 GDN_API size_t gdn_prefill_segmented_workspace_size(int32_t N, int32_t T, int32_t H_qk,

@@ -135,6 +135,12 @@ gdn_status check_prefill_args(const void* q, const void* k, const void* v, const
     return GDN_OK;
 }
 
+gdn_status prefill_call(const void* q, const void* k, const void* v, const float* log_alpha,
+                        const float* beta, const float* S0, const int32_t* cu_seqlens, int32_t N,
+                        int32_t T, int32_t H_qk, int32_t H_v, int32_t dk, int32_t dv,
+                        gdn_dtype io_dtype, void* o, float* S_final, int32_t segments,
+                        void* workspace, size_t workspace_bytes, bool tc, void* stream);
+
 }  // namespace
 
 extern "C" {
@@ -145,6 +151,28 @@ gdn_status gdn_prefill_segmented(const void* q, const void* k, const void* v,
                                  int32_t H_v, int32_t dk, int32_t dv, gdn_dtype io_dtype, void* o,
                                  float* S_final, int32_t segments, void* workspace,
                                  size_t workspace_bytes, void* stream) {
+    return prefill_call(q, k, v, log_alpha, beta, S0, cu_seqlens, N, T, H_qk, H_v, dk, dv,
+                        io_dtype, o, S_final, segments, workspace, workspace_bytes, false, stream);
+}
+
+gdn_status gdn_prefill_tc(const void* q, const void* k, const void* v, const float* log_alpha,
+                          const float* beta, const float* S0, const int32_t* cu_seqlens, int32_t N,
+                          int32_t T, int32_t H_qk, int32_t H_v, int32_t dk, int32_t dv,
+                          gdn_dtype io_dtype, void* o, float* S_final, void* workspace,
+                          size_t workspace_bytes, void* stream) {
+    return prefill_call(q, k, v, log_alpha, beta, S0, cu_seqlens, N, T, H_qk, H_v, dk, dv,
+                        io_dtype, o, S_final, 0, workspace, workspace_bytes, true, stream);
+}
+
+}  // extern "C"
+
+namespace {
+
+gdn_status prefill_call(const void* q, const void* k, const void* v, const float* log_alpha,
+                        const float* beta, const float* S0, const int32_t* cu_seqlens, int32_t N,
+                        int32_t T, int32_t H_qk, int32_t H_v, int32_t dk, int32_t dv,
+                        gdn_dtype io_dtype, void* o, float* S_final, int32_t segments,
+                        void* workspace, size_t workspace_bytes, bool tc, void* stream) {
     gdn_status st = check_prefill_args(q, k, v, log_alpha, beta, S0, cu_seqlens, N, T, H_qk, H_v,
                                        dk, dv, io_dtype, o, S_final);
     if (st != GDN_OK) return st;
@@ -158,10 +186,14 @@ gdn_status gdn_prefill_segmented(const void* q, const void* k, const void* v,
     st = check_device();
     if (st != GDN_OK) return st;
     cudaError_t e = gdn::launch_prefill(q, k, v, log_alpha, beta, S0, cu_seqlens, N, T, H_qk,
-                                        H_v, bf16, o, S_final, workspace, P,
+                                        H_v, bf16, o, S_final, workspace, P, tc,
                                         static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
 }
+
+}  // namespace
+
+extern "C" {
 
 gdn_status gdn_prefill(const void* q, const void* k, const void* v, const float* log_alpha,
                        const float* beta, const float* S0, const int32_t* cu_seqlens, int32_t N,

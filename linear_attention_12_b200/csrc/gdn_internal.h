@@ -26,11 +26,12 @@ int device_sms();
 // library: 1 unless splitting the sequences fills more of the SMs.
 int choose_segments(int N, int T, int H_v, int sms);
 
-// P segments per sequence (P <= 0: choose_segments).
+// P segments per sequence (P <= 0: choose_segments); tc: the state pass that
+// writes the outputs runs on tcgen05 instead of mma.sync.
 cudaError_t launch_prefill(const void* q, const void* k, const void* v, const float* log_alpha,
                            const float* beta, const float* S0, const int32_t* cu_seqlens, int N,
                            int T, int H_qk, int H_v, bool bf16, void* o, float* S_final,
-                           void* workspace, int P, cudaStream_t stream);
+                           void* workspace, int P, bool tc, cudaStream_t stream);
 
 // Records and chunk-entering states of a bf16 prefill, for its gradients.
 cudaError_t launch_prefill_save(const void* q, const void* k, const void* v,

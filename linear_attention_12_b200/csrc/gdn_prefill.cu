@@ -693,6 +693,326 @@ __global__ void __launch_bounds__(P2_THREADS, 1)
     __syncthreads();
 }
 
+// ============================================================================
+// Pass 2 on the fifth-generation tensor cores: the prefill's outputs and final
+// states.  Grid (d_v slices, H_v, N); 256 threads; one thread issues every
+// tcgen05.mma, accumulators live in tensor memory.  Per chunk:
+//   MMA1  [K; Q] S          M = 128: lanes 0-63 K S, lanes 64-127 Q S
+//   MMA2  T_b X             M = 64: Delta, row r in lane (r % 16) + 32 (r / 16)
+//   MMA3  K^T (d o Delta)   M = 128: the state increment, lane = d_k index
+//   MMA4  [T_b; M_Q] Delta  M = 128: lanes 64-127 (M o Q K^T) Delta, beside Q S
+// (M_Q = M o Q K^T; the record stores T_b and M_Q as adjacent 64-row K-major
+// tiles, so [T_b; M_Q] is one 128-row operand.)  Between the products every
+// warp reads one TMEM lane per thread and half of the slice's columns (warps
+// w and w + 4 share lane quadrant w): X and Delta go back to shared memory in
+// bf16 as the next product's B operand; each thread keeps half a row of the
+// fp32 state and writes its bf16 copy (MMA1's B operand); the warps on lanes
+// 64-127 also combine gamma o (Q S) with (M o Q K^T) Delta into the output.
+// Warp 4's thread 0 streams K, Q, the V slice and the record into a 3-stage
+// ring; it refills the previous chunk's stage while MMA1 runs.
+// ============================================================================
+constexpr int TC_THREADS = 256;
+constexpr int TC_LOADER = 128;
+constexpr int BAR_TC = 1;
+// ring stage: [K h0 | Q h0 | K h1 | Q h1] -- [K; Q] is one 128-row K-major tile
+// per 64-column half, and K alone an MN-major one with its halves 16 KB apart
+constexpr uint32_t TS_KQ = 0, TS_V = 4 * HALF, TS_REC = 5 * HALF;
+constexpr uint32_t TS_STAGE = ((TS_REC + REC_BYTES + 1023) / 1024) * 1024;
+constexpr uint32_t TS_TX = 5 * HALF + REC_BYTES;
+constexpr uint32_t TC_SB = NSTAGE * TS_STAGE;  // S in bf16: 128 k-rows x 64 columns, MN-major
+constexpr uint32_t TC_X = TC_SB + 2 * HALF;    // X, 64 token rows x 64 columns, MN-major
+constexpr uint32_t TC_DU = TC_X + HALF;        // Delta
+constexpr uint32_t TC_DD = TC_DU + HALF;       // d o Delta
+constexpr uint32_t TC_BAR = TC_DD + HALF;      // full[NSTAGE], mma, drain
+constexpr uint32_t TC_MISC = TC_BAR + 64;      // abort flag, TMEM base
+constexpr uint32_t TC_SMEM = TC_MISC + 16 + 1024;
+static_assert(TS_STAGE % 1024 == 0 && TC_SB % 1024 == 0, "swizzled tiles sit on 1 KB");
+static_assert(TC_SMEM <= 232448, "tcgen05 state pass shared memory budget");
+// TMEM columns (256 allocated)
+constexpr uint32_t TM_KQ = 0, TM_DL = 64, TM_U = 128, TM_O = 192, TM_COLS = 256;
+
+__device__ __forceinline__ void tmem_ld8(uint32_t taddr, float* r) {
+    uint32_t* u = reinterpret_cast<uint32_t*>(r);
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+                 : "=r"(u[0]), "=r"(u[1]), "=r"(u[2]), "=r"(u[3]), "=r"(u[4]), "=r"(u[5]),
+                   "=r"(u[6]), "=r"(u[7])
+                 : "r"(taddr));
+}
+
+// N columns (a multiple of 8) of this thread's TMEM lane, fp32.  The values are
+// pinned behind the wait so that no use moves above it.
+template <int N>
+__device__ __forceinline__ void tmem_cols(uint32_t ta, float* v) {
+#pragma unroll
+    for (int i = 0; i < N / 8; ++i) tmem_ld8(ta + 8 * i, v + 8 * i);
+    tmem_ld_wait();
+#pragma unroll
+    for (int i = 0; i < N; ++i) asm volatile("" : "+f"(v[i]));
+}
+
+// Columns c0 .. c0 + N - 1 (c0, N multiples of 8) of row r of an MN-major
+// 128B-swizzled bf16 tile (one 64-column block), scaled by s.
+template <int N>
+__device__ __forceinline__ void put_cols(uint8_t* sm, uint32_t tile, int r, int c0, const float* v,
+                                         float s) {
+#pragma unroll
+    for (int i = 0; i < N / 8; ++i) {
+        const int j = c0 / 8 + i;
+        *reinterpret_cast<uint4*>(sm + tile + r * 128 + ((j ^ (r & 7)) << 4)) =
+            make_uint4(pack2(s * v[8 * i], s * v[8 * i + 1]), pack2(s * v[8 * i + 2], s * v[8 * i + 3]),
+                       pack2(s * v[8 * i + 4], s * v[8 * i + 5]),
+                       pack2(s * v[8 * i + 6], s * v[8 * i + 7]));
+    }
+}
+
+template <typename IO>
+__device__ __forceinline__ void store8(IO* p, const float* v);
+template <>
+__device__ __forceinline__ void store8<float>(float* p, const float* v) {
+    reinterpret_cast<float4*>(p)[0] = make_float4(v[0], v[1], v[2], v[3]);
+    reinterpret_cast<float4*>(p)[1] = make_float4(v[4], v[5], v[6], v[7]);
+}
+template <>
+__device__ __forceinline__ void store8<__nv_bfloat16>(__nv_bfloat16* p, const float* v) {
+    *reinterpret_cast<uint4*>(p) = make_uint4(pack2(v[0], v[1]), pack2(v[2], v[3]),
+                                              pack2(v[4], v[5]), pack2(v[6], v[7]));
+}
+
+template <int NS, typename IO>
+__global__ void __launch_bounds__(TC_THREADS, 1)
+    state_tc_kernel(const __grid_constant__ CUtensorMap map_q,
+                    const __grid_constant__ CUtensorMap map_k,
+                    const __grid_constant__ CUtensorMap map_v, const PrefillParams p) {
+    static_assert(NS == 32 || NS == 48 || NS == 64, "slice width");
+    constexpr int HN = NS / 2;                              // columns per half
+    constexpr uint32_t ID_KQ = idesc_bf16(128, NS, 0, 1);   // K-major A, MN-major B
+    constexpr uint32_t ID_TB = idesc_bf16(64, NS, 0, 1);    // T_b X
+    constexpr uint32_t ID_KT = idesc_bf16(128, NS, 1, 1);   // MN-major A (K^T), MN-major B
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+    const uint32_t sb = smem_u32(sm);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(sm + TC_BAR);
+    uint64_t* mma_bar = bars + NSTAGE;
+    uint64_t* drain_bar = bars + NSTAGE + 1;
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + TC_MISC);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + TC_MISC + 4);
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int quad = warp & 3;       // TMEM lanes 32 quad .. 32 quad + 31
+    const int c_lo = (warp >> 2) * HN;  // this warp's half of the slice's columns
+    const int row = 32 * quad + lane;   // this thread's TMEM lane
+    const int h = blockIdx.y, n = blockIdx.z;
+    const int hq = h / (p.H_v / p.H_qk);
+    const int col0 = blockIdx.x * NS;
+    const int ncols = min(NS, D - col0);
+    const int t_beg = p.cu_seqlens[n];
+    const int t_end = p.cu_seqlens[n + 1];
+    const int nchunks = (t_end - t_beg + C - 1) / C;
+
+    if (tid == 0) {
+        for (int i = 0; i < NSTAGE + 2; ++i) mbar_init(&bars[i], 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 0) {
+        tmem_alloc(tmem_slot, TM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const uint32_t tl = tmem + ((uint32_t)(32 * quad) << 16) + c_lo;  // my lane, my columns
+
+    auto issue_chunk = [&](int c) {
+        const int s = c % NSTAGE;
+        uint8_t* st = sm + s * TS_STAGE;
+        const int y = t_beg + c * C;
+        uint64_t* full = &bars[s];
+        mbar_arrive_expect_tx(full, TS_TX);
+        tma_load_2d(st + TS_KQ, &map_k, hq * D, y, full);
+        tma_load_2d(st + TS_KQ + HALF, &map_q, hq * D, y, full);
+        tma_load_2d(st + TS_KQ + 2 * HALF, &map_k, hq * D + 64, y, full);
+        tma_load_2d(st + TS_KQ + 3 * HALF, &map_q, hq * D + 64, y, full);
+        tma_load_2d(st + TS_V, &map_v, h * D + col0, y, full);
+        bulk_load(st + TS_REC, p.records + (size_t)(record_slot(n, y) * p.H_v + h) * REC_BYTES,
+                  REC_BYTES, full);
+    };
+    int issued = 0;
+    if (tid == TC_LOADER)
+        for (; issued < min(NSTAGE, nchunks); ++issued) issue_chunk(issued);
+
+    // row `row` of the state, columns col0 + c_lo .. + HN - 1, fp32
+    float Sr[HN];
+    {
+        const float* s0 =
+            p.S0 ? p.S0 + (((size_t)n * p.H_v + h) * D + row) * D + col0 + c_lo : nullptr;
+#pragma unroll
+        for (int j = 0; j < HN; ++j) Sr[j] = (s0 && c_lo + j < ncols) ? s0[j] : 0.f;
+        put_cols<HN>(sm, TC_SB, row, c_lo, Sr, 1.f);
+        fence_proxy_async_smem();
+    }
+
+    uint32_t mph = 0;  // completed phases of mma_bar
+    for (int c = 0; c < nchunks; ++c) {
+        const int s = c % NSTAGE;
+        const uint32_t st = sb + s * TS_STAGE;
+        const uint8_t* stp = sm + s * TS_STAGE;
+        const int tc0 = t_beg + c * C;
+        const int valid = min(C, t_end - tc0);
+        bool ok = mbar_wait(&bars[s], (c / NSTAGE) & 1, abort_flag);
+        tc_fence_before();
+        if (!bar_and<BAR_TC, TC_THREADS>(ok)) break;
+
+        // MMA1: [K; Q] S
+        if (tid == 0) {
+            tc_fence_after();
+#pragma unroll
+            for (int ks = 0; ks < 8; ++ks)
+                mma_bf16_ss(tmem + TM_KQ,
+                            sdesc_sw128(st + TS_KQ + (ks >> 2) * 2 * HALF + (ks & 3) * 32, 16, 1024),
+                            sdesc_sw128(sb + TC_SB + ks * 2048, 8192, 1024), ID_KQ, ks > 0);
+            mma_commit(mma_bar);
+        }
+        // meanwhile: the previous chunk's stage gets the chunk NSTAGE after it, and the
+        // chunk's scalars come into registers
+        if (tid == TC_LOADER && c >= 1 && c - 1 + NSTAGE < nchunks) issue_chunk(issued++);
+        const float* rv = reinterpret_cast<const float*>(stp + TS_REC + REC_VEC);
+        const float g_row = quad < 2 ? rv[row] : rv[row - 64];  // gamma of my K / Q row
+        const float d_row = rv[64 + 16 * quad + (lane & 15)];   // d of my Delta row
+        const float g_C = rv[128];
+        ok = mbar_wait(mma_bar, mph & 1, abort_flag);
+        ++mph;
+        tc_fence_after();
+        if (quad < 2) {  // X = V - gamma o (K S), token row `row`
+            float x[HN];
+            tmem_cols<HN>(tl + TM_KQ, x);
+#pragma unroll
+            for (int i = 0; i < HN / 8; ++i) {
+                const int j = c_lo / 8 + i;
+                const uint4 u = *reinterpret_cast<const uint4*>(stp + TS_V + row * 128 +
+                                                                ((j ^ (row & 7)) << 4));
+                const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float2 v2 =
+                        __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[e]));
+                    x[8 * i + 2 * e] = v2.x - g_row * x[8 * i + 2 * e];
+                    x[8 * i + 2 * e + 1] = v2.y - g_row * x[8 * i + 2 * e + 1];
+                }
+            }
+            put_cols<HN>(sm, TC_X, row, c_lo, x, 1.f);
+            fence_proxy_async_smem();
+        }
+        tc_fence_before();
+        if (!bar_and<BAR_TC, TC_THREADS>(ok)) break;
+
+        // MMA2: Delta = T_b X (M = 64)
+        if (tid == 0) {
+            tc_fence_after();
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks)
+                mma_bf16_ss(tmem + TM_DL, sdesc_sw128(st + TS_REC + ks * 32, 16, 1024),
+                            sdesc_sw128(sb + TC_X + ks * 2048, 8192, 1024), ID_TB, ks > 0);
+            mma_commit(mma_bar);
+        }
+        ok = mbar_wait(mma_bar, mph & 1, abort_flag);
+        ++mph;
+        tc_fence_after();
+        {  // Delta and d o Delta: token row 16 quad + lane on lanes 0-15 of each quadrant
+            float dl[HN];
+            tmem_cols<HN>(tl + TM_DL, dl);  // warp-collective; lanes 16-31 read unused lanes
+            if (lane < 16) {
+                const int r = 16 * quad + lane;
+                put_cols<HN>(sm, TC_DU, r, c_lo, dl, 1.f);
+                put_cols<HN>(sm, TC_DD, r, c_lo, dl, d_row);
+                fence_proxy_async_smem();
+            }
+        }
+        tc_fence_before();
+        if (!bar_and<BAR_TC, TC_THREADS>(ok)) break;
+
+        // MMA3: K^T (d o Delta);  MMA4: [T_b; M_Q] Delta
+        if (tid == 0) {
+            tc_fence_after();
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks) {
+                mma_bf16_ss(tmem + TM_U, sdesc_sw128(st + TS_KQ + ks * 2048, 2 * HALF, 1024),
+                            sdesc_sw128(sb + TC_DD + ks * 2048, 8192, 1024), ID_KT, ks > 0);
+                mma_bf16_ss(tmem + TM_O, sdesc_sw128(st + TS_REC + ks * 32, 16, 1024),
+                            sdesc_sw128(sb + TC_DU + ks * 2048, 8192, 1024), ID_KQ, ks > 0);
+            }
+            mma_commit(mma_bar);
+        }
+        ok = mbar_wait(mma_bar, mph & 1, abort_flag);
+        ++mph;
+        tc_fence_after();
+        {  // S <- gamma_C S + K^T (d o Delta), state row `row`; bf16 copy for MMA1
+            float u[HN];
+            tmem_cols<HN>(tl + TM_U, u);
+#pragma unroll
+            for (int j = 0; j < HN; ++j) Sr[j] = fmaf(g_C, Sr[j], u[j]);
+            put_cols<HN>(sm, TC_SB, row, c_lo, Sr, 1.f);
+            fence_proxy_async_smem();
+        }
+        if (quad >= 2) {  // O = gamma o (Q S) + (M o Q K^T) Delta, token row i = row - 64
+            const int i = row - 64;
+            float qs[HN], oi[HN];
+            tmem_cols<HN>(tl + TM_KQ, qs);
+            tmem_cols<HN>(tl + TM_O, oi);
+            if (i < valid) {
+                IO* orow = static_cast<IO*>(p.o) + ((size_t)(tc0 + i) * p.H_v + h) * D + col0 + c_lo;
+#pragma unroll
+                for (int j = 0; j < HN / 8; ++j) {
+                    if (c_lo + 8 * j < ncols) {
+                        float ov[8];
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) ov[e] = fmaf(g_row, qs[8 * j + e], oi[8 * j + e]);
+                        store8<IO>(orow + 8 * j, ov);
+                    }
+                }
+            }
+        }
+        tc_fence_before();
+        if (!bar_and<BAR_TC, TC_THREADS>(ok)) break;
+    }
+    if (p.S_final && !*abort_flag) {
+        float* sf = p.S_final + (((size_t)n * p.H_v + h) * D + row) * D + col0 + c_lo;
+#pragma unroll
+        for (int j = 0; j < HN / 4; ++j)
+            if (c_lo + 4 * j < ncols)
+                reinterpret_cast<float4*>(sf)[j] =
+                    make_float4(Sr[4 * j], Sr[4 * j + 1], Sr[4 * j + 2], Sr[4 * j + 3]);
+    }
+    // Drain: no product may still run and no copy still land when TMEM is freed
+    // and the CTA exits (both waits bounded).
+    if (tid == 0) {
+        mma_commit(drain_bar);
+        mbar_wait_drain(drain_bar, 0);
+    }
+    if (tid == TC_LOADER)
+        for (int c = max(0, issued - NSTAGE); c < issued; ++c)
+            mbar_wait_drain(&bars[c % NSTAGE], (c / NSTAGE) & 1);
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, TM_COLS);
+    }
+}
+
+template <int NS, typename IO>
+cudaError_t launch_state_tc(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+                            const PrefillParams& prm, cudaStream_t stream) {
+    auto kern = state_tc_kernel<NS, IO>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, TC_SMEM);
+    if (e != cudaSuccess) return e;
+    dim3 grid((D + NS - 1) / NS, prm.H_v, prm.N);
+    kern<<<grid, TC_THREADS, TC_SMEM, stream>>>(mq, mk, mv, prm);
+    return cudaGetLastError();
+}
+
 // S_final = S0, or zeros when S0 is NULL (used when no sequence has tokens).
 __global__ void copy_state_kernel(const float* __restrict__ S0, float* __restrict__ S_final,
                                   size_t n4) {
@@ -944,11 +1264,19 @@ int choose_segments(int N, int T, int H_v, int sms) {
 
 template <typename IO, int MODE>
 static cudaError_t run_pass2(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
-                             const PrefillParams& prm, int sms, cudaStream_t stream) {
+                             const PrefillParams& prm, int sms, cudaStream_t stream,
+                             bool tc = false) {
     // one block per SM at most (each holds ~212 KB of shared memory): split every
     // value head into as many d_v slices as still fit in one wave
     const long long units = (long long)prm.N * prm.H_v * (MODE == P2_SEGMENT ? 2 : 1);
     const int slices = pass2_slices(units, sms);
+    if constexpr (MODE == P2_OUT) {
+        if (tc) {
+            if (slices == 4) return launch_state_tc<32, IO>(mq, mk, mv, prm, stream);
+            if (slices == 3) return launch_state_tc<48, IO>(mq, mk, mv, prm, stream);
+            return launch_state_tc<64, IO>(mq, mk, mv, prm, stream);
+        }
+    }
     if (slices == 4) return launch_pass2<32, IO, MODE>(mq, mk, mv, prm, prm.N, stream);
     if (slices == 3) return launch_pass2<48, IO, MODE>(mq, mk, mv, prm, prm.N, stream);
     return launch_pass2<64, IO, MODE>(mq, mk, mv, prm, prm.N, stream);
@@ -969,7 +1297,7 @@ static cudaError_t run_pass1(const CUtensorMap& mq, const CUtensorMap& mk,
 cudaError_t launch_prefill(const void* q, const void* k, const void* v, const float* log_alpha,
                            const float* beta, const float* S0, const int32_t* cu_seqlens, int N,
                            int T, int H_qk, int H_v, bool bf16, void* o, float* S_final,
-                           void* workspace, int P, cudaStream_t stream) {
+                           void* workspace, int P, bool tc, cudaStream_t stream) {
     if (T == 0) {  // every sequence is empty: S_final = S0 (or zeros)
         if (!S_final) return cudaSuccess;
         copy_state_kernel<<<592, 256, 0, stream>>>(S0, S_final, (size_t)N * H_v * D * D / 4);
@@ -1005,8 +1333,8 @@ cudaError_t launch_prefill(const void* q, const void* k, const void* v, const fl
         const PrefillParams prm{log_alpha, beta, S0,      cu_seqlens, o, S_final,
                                 records,   nullptr, H_qk, H_v,        N, T};
         if ((e = run_pass1(mq, mk, prm, stream)) != cudaSuccess) return e;
-        return bf16 ? run_pass2<__nv_bfloat16, P2_OUT>(mq, mk, mv, prm, sms, stream)
-                    : run_pass2<float, P2_OUT>(mq, mk, mv, prm, sms, stream);
+        return bf16 ? run_pass2<__nv_bfloat16, P2_OUT>(mq, mk, mv, prm, sms, stream, tc)
+                    : run_pass2<float, P2_OUT>(mq, mk, mv, prm, sms, stream, tc);
     }
     // segmented: N P virtual sequences
     const int Nv = N * P;
@@ -1039,8 +1367,8 @@ cudaError_t launch_prefill(const void* q, const void* k, const void* v, const fl
     // phase C: every segment from its entering state, writing the outputs
     const PrefillParams pc{log_alpha, beta, S_entry, cu_v, o, nullptr, records, nullptr,
                            H_qk,      H_v,  Nv,      T};
-    return bf16 ? run_pass2<__nv_bfloat16, P2_OUT>(mq, mk, mv, pc, sms, stream)
-                : run_pass2<float, P2_OUT>(mq, mk, mv, pc, sms, stream);
+    return bf16 ? run_pass2<__nv_bfloat16, P2_OUT>(mq, mk, mv, pc, sms, stream, tc)
+                : run_pass2<float, P2_OUT>(mq, mk, mv, pc, sms, stream, tc);
 }
 
 // The forward pass the gradients start from (bf16 q, k, v): every chunk's

@@ -35,6 +35,10 @@ SIGNATURES = {
                                _c.c_int32, _c.c_int32, _c.c_int32, _c.c_int, _c.c_void_p,
                                _c.c_void_p, _c.c_void_p, _c.c_size_t, _c.c_void_p]),
     "gdn_prefill_workspace_size": (_c.c_size_t, [_c.c_int32] * 6 + [_c.c_int]),
+    "gdn_prefill_tc": (_c.c_int, [_c.c_void_p, _c.c_void_p, _c.c_void_p, _c.c_void_p, _c.c_void_p,
+                                  _c.c_void_p, _c.c_void_p, _c.c_int32, _c.c_int32, _c.c_int32,
+                                  _c.c_int32, _c.c_int32, _c.c_int32, _c.c_int, _c.c_void_p,
+                                  _c.c_void_p, _c.c_void_p, _c.c_size_t, _c.c_void_p]),
     "gdn_prefill_segmented": (_c.c_int, [_c.c_void_p] * 7 + [_c.c_int32] * 6 +
                               [_c.c_int, _c.c_void_p, _c.c_void_p, _c.c_int32, _c.c_void_p,
                                _c.c_size_t, _c.c_void_p]),
@@ -140,12 +144,14 @@ def auto_segments(N, T, H_qk, H_v) -> int:
 
 
 def prefill(q, k, v, log_alpha, beta, S0=None, cu_seqlens=None, *, o=None, S_final=None,
-            want_state=True, workspace=None, segments=None, stream=None):
+            want_state=True, workspace=None, segments=None, tcgen05=False, stream=None):
     """Chunked prefill.  Returns ``(o, S_final)`` (``S_final`` None if not wanted).
 
     ``segments``: None or 0 lets the library split long sequences when that
     fills more SMs; 1 disables the split; 2 .. 64 forces that many pieces per
-    sequence (gdn_prefill_segmented)."""
+    sequence (gdn_prefill_segmented).  ``tcgen05=True`` runs the output state
+    pass on the fifth-generation tensor cores (gdn_prefill_tc; automatic
+    segments only)."""
     T, H_qk, dk = q.shape
     H_v, dv = v.shape[1], v.shape[2]
     dt = q.dtype
@@ -173,12 +179,20 @@ def prefill(q, k, v, log_alpha, beta, S0=None, cu_seqlens=None, *, o=None, S_fin
     if need and workspace is None:
         workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
     wbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
-    st = lib().gdn_prefill_segmented(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta),
-                                     _ptr(S0), _ptr(cu_seqlens), N, T, H_qk, H_v, dk, dv, io,
-                                     _ptr(o), _ptr(S_final), seg, _ptr(workspace), wbytes,
-                                     _stream_handle(stream))
+    if tcgen05:
+        if seg != 0:
+            raise ValueError("tcgen05=True takes the automatic segment choice only")
+        st = lib().gdn_prefill_tc(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta),
+                                  _ptr(S0), _ptr(cu_seqlens), N, T, H_qk, H_v, dk, dv, io,
+                                  _ptr(o), _ptr(S_final), _ptr(workspace), wbytes,
+                                  _stream_handle(stream))
+    else:
+        st = lib().gdn_prefill_segmented(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta),
+                                         _ptr(S0), _ptr(cu_seqlens), N, T, H_qk, H_v, dk, dv, io,
+                                         _ptr(o), _ptr(S_final), seg, _ptr(workspace), wbytes,
+                                         _stream_handle(stream))
     if st != GDN_OK:
-        raise GDNError(st, "gdn_prefill_segmented")
+        raise GDNError(st, "gdn_prefill_tc" if tcgen05 else "gdn_prefill_segmented")
     return o, S_final
 
 
