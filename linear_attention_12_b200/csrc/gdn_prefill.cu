@@ -697,25 +697,29 @@ __global__ void __launch_bounds__(P2_THREADS, 1)
 // Pass 2 on the fifth-generation tensor cores: the prefill's outputs and final
 // states.  Grid (d_v slices, H_v, N); 256 threads; one thread issues every
 // tcgen05.mma, accumulators live in tensor memory.  Per chunk:
-//   MMA1  [K; Q] S          M = 128: lanes 0-63 K S, lanes 64-127 Q S
-//   MMA2  T_b X             M = 64: Delta, row r in lane (r % 16) + 32 (r / 16)
-//   MMA3  K^T (d o Delta)   M = 128: the state increment, lane = d_k index
-//   MMA4  [T_b; M_Q] Delta  M = 128: lanes 64-127 (M o Q K^T) Delta, beside Q S
+//   [K; Q] S             M = 128: lanes 0-63 K S, lanes 64-127 Q S
+//   Delta = T_b X        M = 64:  row r in lane (r % 16) + 32 (r / 16)
+//   K^T (d o Delta)      M = 128: the state increment, lane = d_k index
+//   [T_b; M_Q] Delta     M = 128: lanes 64-127 (M o Q K^T) Delta, beside Q S
 // (M_Q = M o Q K^T; the record stores T_b and M_Q as adjacent 64-row K-major
 // tiles, so [T_b; M_Q] is one 128-row operand.)  Between the products every
-// warp reads one TMEM lane per thread and half of the slice's columns (warps
-// w and w + 4 share lane quadrant w): X and Delta go back to shared memory in
-// bf16 as the next product's B operand; each thread keeps half a row of the
-// fp32 state and writes its bf16 copy (MMA1's B operand); the warps on lanes
-// 64-127 also combine gamma o (Q S) with (M o Q K^T) Delta into the output.
-// Warp 4's thread 0 streams K, Q, the V slice and the record into a 3-stage
-// ring; it refills the previous chunk's stage while MMA1 runs.
+// warp reads its TMEM lanes and half of the slice's columns (warps w and w + 4
+// share lane quadrant w): X and Delta go back to shared memory in bf16 as the
+// next product's B operand (MN-major); each thread keeps half a row of the
+// fp32 state and writes its bf16 copy, the next [K; Q] S's B operand.  The
+// output rows O = gamma o (Q S) + (M o Q K^T) Delta of a chunk are formed by
+// the warps on lanes 64-127 while the next chunk's [K; Q] S runs ([K; Q] S
+// and [T_b; M_Q] Delta are double-buffered in TMEM).  Every product commits
+// to an mbarrier of its own, once per chunk.  Warp 6's thread 0 streams K, Q,
+// the V slice and the record into a 3-stage ring; it refills the previous
+// chunk's stage while X is formed.
 // ============================================================================
 constexpr int TC_THREADS = 256;
-constexpr int TC_LOADER = 128;
+constexpr int TC_LOADER = 192;  // warp 6: idle while warps 0, 1, 4, 5 form X
 constexpr int BAR_TC = 1;
-// ring stage: [K h0 | Q h0 | K h1 | Q h1] -- [K; Q] is one 128-row K-major tile
-// per 64-column half, and K alone an MN-major one with its halves 16 KB apart
+// ring stage: K h0 | Q h0 | K h1 | Q h1 -- [K; Q] is one 128-row K-major tile
+// per 64-column half, and K alone an MN-major one with its halves 16 KB apart --
+// then the V slice and the record (T_b, then M o Q K^T)
 constexpr uint32_t TS_KQ = 0, TS_V = 4 * HALF, TS_REC = 5 * HALF;
 constexpr uint32_t TS_STAGE = ((TS_REC + REC_BYTES + 1023) / 1024) * 1024;
 constexpr uint32_t TS_TX = 5 * HALF + REC_BYTES;
@@ -723,13 +727,14 @@ constexpr uint32_t TC_SB = NSTAGE * TS_STAGE;  // S in bf16: 128 k-rows x 64 col
 constexpr uint32_t TC_X = TC_SB + 2 * HALF;    // X, 64 token rows x 64 columns, MN-major
 constexpr uint32_t TC_DU = TC_X + HALF;        // Delta
 constexpr uint32_t TC_DD = TC_DU + HALF;       // d o Delta
-constexpr uint32_t TC_BAR = TC_DD + HALF;      // full[NSTAGE], mma, drain
-constexpr uint32_t TC_MISC = TC_BAR + 64;      // abort flag, TMEM base
+constexpr uint32_t TC_BAR = TC_DD + HALF;      // full[NSTAGE], ks, dl, u, o, drain
+constexpr uint32_t TC_MISC = TC_BAR + 128;     // abort flag, TMEM base
 constexpr uint32_t TC_SMEM = TC_MISC + 16 + 1024;
 static_assert(TS_STAGE % 1024 == 0 && TC_SB % 1024 == 0, "swizzled tiles sit on 1 KB");
 static_assert(TC_SMEM <= 232448, "tcgen05 state pass shared memory budget");
-// TMEM columns (256 allocated)
-constexpr uint32_t TM_KQ = 0, TM_DL = 64, TM_U = 128, TM_O = 192, TM_COLS = 256;
+// TMEM columns (512 allocated): [K; Q] S (two buffers), Delta, the state
+// increment, [T_b; M_Q] Delta (two buffers)
+constexpr uint32_t TM_KQ = 0, TM_DL = 128, TM_U = 192, TM_O = 256, TM_COLS = 512;
 
 __device__ __forceinline__ void tmem_ld8(uint32_t taddr, float* r) {
     uint32_t* u = reinterpret_cast<uint32_t*>(r);
@@ -785,23 +790,27 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
                     const __grid_constant__ CUtensorMap map_v, const PrefillParams p) {
     static_assert(NS == 32 || NS == 48 || NS == 64, "slice width");
     constexpr int HN = NS / 2;                              // columns per half
-    constexpr uint32_t ID_KQ = idesc_bf16(128, NS, 0, 1);   // K-major A, MN-major B
-    constexpr uint32_t ID_TB = idesc_bf16(64, NS, 0, 1);    // T_b X
+    constexpr uint32_t ID_128 = idesc_bf16(128, NS, 0, 1);  // K-major A, MN-major B
+    constexpr uint32_t ID_64 = idesc_bf16(64, NS, 0, 1);    // the same, M = 64
     constexpr uint32_t ID_KT = idesc_bf16(128, NS, 1, 1);   // MN-major A (K^T), MN-major B
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
     const uint32_t sb = smem_u32(sm);
     uint64_t* bars = reinterpret_cast<uint64_t*>(sm + TC_BAR);
-    uint64_t* mma_bar = bars + NSTAGE;
-    uint64_t* drain_bar = bars + NSTAGE + 1;
+    uint64_t* bar_ks = bars + NSTAGE;
+    uint64_t* bar_dl = bars + NSTAGE + 1;
+    uint64_t* bar_u = bars + NSTAGE + 2;
+    uint64_t* bar_o = bars + NSTAGE + 3;
+    uint64_t* drain_bar = bars + NSTAGE + 4;
     volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + TC_MISC);
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + TC_MISC + 4);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int quad = warp & 3;       // TMEM lanes 32 quad .. 32 quad + 31
+    const int quad = warp & 3;          // TMEM lanes 32 quad .. 32 quad + 31
     const int c_lo = (warp >> 2) * HN;  // this warp's half of the slice's columns
-    const int row = 32 * quad + lane;   // this thread's TMEM lane
+    const int row = 32 * quad + lane;   // my row of an M = 128 product (a state row)
+    const int r64 = 16 * quad + lane;   // my row of an M = 64 product, when lane < 16
     const int h = blockIdx.y, n = blockIdx.z;
     const int hq = h / (p.H_v / p.H_qk);
     const int col0 = blockIdx.x * NS;
@@ -811,7 +820,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     const int nchunks = (t_end - t_beg + C - 1) / C;
 
     if (tid == 0) {
-        for (int i = 0; i < NSTAGE + 2; ++i) mbar_init(&bars[i], 1);
+        for (int i = 0; i < NSTAGE + 5; ++i) mbar_init(&bars[i], 1);
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -823,7 +832,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    const uint32_t tl = tmem + ((uint32_t)(32 * quad) << 16) + c_lo;  // my lane, my columns
+    const uint32_t tl = tmem + ((uint32_t)(32 * quad) << 16) + c_lo;  // my lanes, my columns
 
     auto issue_chunk = [&](int c) {
         const int s = c % NSTAGE;
@@ -853,102 +862,129 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         put_cols<HN>(sm, TC_SB, row, c_lo, Sr, 1.f);
         fence_proxy_async_smem();
     }
+    __syncthreads();  // the first K S reads the whole tile
 
-    uint32_t mph = 0;  // completed phases of mma_bar
+    // O rows of chunk c (warps on lanes 64-127: token row row - 64), once
+    // (M o Q K^T) Delta is done
+    auto output = [&](int c, float g_o) -> bool {
+        const bool ok = mbar_wait(bar_o, c & 1, abort_flag);
+        tc_fence_after();
+        float qs[HN], oi[HN];
+        tmem_cols<HN>(tl + TM_KQ + 64 * (c & 1), qs);
+        tmem_cols<HN>(tl + TM_O + 64 * (c & 1), oi);
+        const int tc0 = t_beg + c * C, i = row - 64;
+        if (ok && i < t_end - tc0) {
+            IO* orow = static_cast<IO*>(p.o) + ((size_t)(tc0 + i) * p.H_v + h) * D + col0 + c_lo;
+#pragma unroll
+            for (int j = 0; j < HN / 8; ++j) {
+                if (c_lo + 8 * j < ncols) {
+                    float ov[8];
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) ov[e] = fmaf(g_o, qs[8 * j + e], oi[8 * j + e]);
+                    store8<IO>(orow + 8 * j, ov);
+                }
+            }
+        }
+        return ok;
+    };
+
+    float g_prev = 0.f;  // gamma of my output row in the previous chunk
+    bool ok = true;
     for (int c = 0; c < nchunks; ++c) {
         const int s = c % NSTAGE;
         const uint32_t st = sb + s * TS_STAGE;
         const uint8_t* stp = sm + s * TS_STAGE;
-        const int tc0 = t_beg + c * C;
-        const int valid = min(C, t_end - tc0);
-        bool ok = mbar_wait(&bars[s], (c / NSTAGE) & 1, abort_flag);
-        tc_fence_before();
-        if (!bar_and<BAR_TC, TC_THREADS>(ok)) break;
-
-        // MMA1: [K; Q] S
+        const uint32_t par = c & 1;
+        ok = mbar_wait(&bars[s], (c / NSTAGE) & 1, abort_flag);
+        // [K; Q] S (the S tile and every read of the TMEM region it overwrites
+        // were ordered by the previous chunk's last barrier)
         if (tid == 0) {
             tc_fence_after();
 #pragma unroll
             for (int ks = 0; ks < 8; ++ks)
-                mma_bf16_ss(tmem + TM_KQ,
+                mma_bf16_ss(tmem + TM_KQ + 64 * par,
                             sdesc_sw128(st + TS_KQ + (ks >> 2) * 2 * HALF + (ks & 3) * 32, 16, 1024),
-                            sdesc_sw128(sb + TC_SB + ks * 2048, 8192, 1024), ID_KQ, ks > 0);
-            mma_commit(mma_bar);
+                            sdesc_sw128(sb + TC_SB + ks * 2048, 8192, 1024), ID_128, ks > 0);
+            mma_commit(bar_ks);
         }
-        // meanwhile: the previous chunk's stage gets the chunk NSTAGE after it, and the
-        // chunk's scalars come into registers
-        if (tid == TC_LOADER && c >= 1 && c - 1 + NSTAGE < nchunks) issue_chunk(issued++);
+        // meanwhile: this chunk's scalars come into registers; the previous chunk's
+        // outputs
         const float* rv = reinterpret_cast<const float*>(stp + TS_REC + REC_VEC);
-        const float g_row = quad < 2 ? rv[row] : rv[row - 64];  // gamma of my K / Q row
-        const float d_row = rv[64 + 16 * quad + (lane & 15)];   // d of my Delta row
+        const float g_row = rv[row & 63];         // gamma of my K row (quads 0-1) or Q row (2-3)
+        const float d_row = rv[64 + (r64 & 63)];  // d of my Delta row (lanes < 16)
         const float g_C = rv[128];
-        ok = mbar_wait(mma_bar, mph & 1, abort_flag);
-        ++mph;
+        if (c >= 1 && quad >= 2) ok = output(c - 1, g_prev) && ok;
+        g_prev = g_row;
+        ok = mbar_wait(bar_ks, par, abort_flag) && ok;
         tc_fence_after();
+        // the previous chunk's stage gets the chunk NSTAGE after it (issued while the
+        // tensor pipe waits for X, so that the copies land outside [K; Q] S)
+        if (tid == TC_LOADER && c >= 1 && c - 1 + NSTAGE < nchunks) issue_chunk(issued++);
         if (quad < 2) {  // X = V - gamma o (K S), token row `row`
             float x[HN];
-            tmem_cols<HN>(tl + TM_KQ, x);
+            tmem_cols<HN>(tl + TM_KQ + 64 * par, x);
+            {
 #pragma unroll
-            for (int i = 0; i < HN / 8; ++i) {
-                const int j = c_lo / 8 + i;
-                const uint4 u = *reinterpret_cast<const uint4*>(stp + TS_V + row * 128 +
-                                                                ((j ^ (row & 7)) << 4));
-                const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+                for (int i = 0; i < HN / 8; ++i) {
+                    const int j = c_lo / 8 + i;
+                    const uint4 u = *reinterpret_cast<const uint4*>(stp + TS_V + row * 128 +
+                                                                    ((j ^ (row & 7)) << 4));
+                    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const float2 v2 =
-                        __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[e]));
-                    x[8 * i + 2 * e] = v2.x - g_row * x[8 * i + 2 * e];
-                    x[8 * i + 2 * e + 1] = v2.y - g_row * x[8 * i + 2 * e + 1];
+                    for (int e = 0; e < 4; ++e) {
+                        const float2 v2 =
+                            __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[e]));
+                        x[8 * i + 2 * e] = v2.x - g_row * x[8 * i + 2 * e];
+                        x[8 * i + 2 * e + 1] = v2.y - g_row * x[8 * i + 2 * e + 1];
+                    }
                 }
-            }
-            put_cols<HN>(sm, TC_X, row, c_lo, x, 1.f);
-            fence_proxy_async_smem();
-        }
-        tc_fence_before();
-        if (!bar_and<BAR_TC, TC_THREADS>(ok)) break;
-
-        // MMA2: Delta = T_b X (M = 64)
-        if (tid == 0) {
-            tc_fence_after();
-#pragma unroll
-            for (int ks = 0; ks < 4; ++ks)
-                mma_bf16_ss(tmem + TM_DL, sdesc_sw128(st + TS_REC + ks * 32, 16, 1024),
-                            sdesc_sw128(sb + TC_X + ks * 2048, 8192, 1024), ID_TB, ks > 0);
-            mma_commit(mma_bar);
-        }
-        ok = mbar_wait(mma_bar, mph & 1, abort_flag);
-        ++mph;
-        tc_fence_after();
-        {  // Delta and d o Delta: token row 16 quad + lane on lanes 0-15 of each quadrant
-            float dl[HN];
-            tmem_cols<HN>(tl + TM_DL, dl);  // warp-collective; lanes 16-31 read unused lanes
-            if (lane < 16) {
-                const int r = 16 * quad + lane;
-                put_cols<HN>(sm, TC_DU, r, c_lo, dl, 1.f);
-                put_cols<HN>(sm, TC_DD, r, c_lo, dl, d_row);
+                put_cols<HN>(sm, TC_X, row, c_lo, x, 1.f);
                 fence_proxy_async_smem();
             }
         }
         tc_fence_before();
         if (!bar_and<BAR_TC, TC_THREADS>(ok)) break;
 
-        // MMA3: K^T (d o Delta);  MMA4: [T_b; M_Q] Delta
+        // Delta = T_b X
         if (tid == 0) {
             tc_fence_after();
 #pragma unroll
-            for (int ks = 0; ks < 4; ++ks) {
+            for (int ks = 0; ks < 4; ++ks)
+                mma_bf16_ss(tmem + TM_DL, sdesc_sw128(st + TS_REC + ks * 32, 16, 1024),
+                            sdesc_sw128(sb + TC_X + ks * 2048, 8192, 1024), ID_64, ks > 0);
+            mma_commit(bar_dl);
+        }
+        ok = mbar_wait(bar_dl, par, abort_flag);
+        tc_fence_after();
+        {  // Delta and d o Delta, token row r64 on lanes < 16
+            float dl[HN];
+            tmem_cols<HN>(tl + TM_DL, dl);
+            if (lane < 16) {
+                put_cols<HN>(sm, TC_DU, r64, c_lo, dl, 1.f);
+                put_cols<HN>(sm, TC_DD, r64, c_lo, dl, d_row);
+                fence_proxy_async_smem();
+            }
+        }
+        tc_fence_before();
+        if (!bar_and<BAR_TC, TC_THREADS>(ok)) break;
+
+        // K^T (d o Delta), then [T_b; M_Q] Delta
+        if (tid == 0) {
+            tc_fence_after();
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks)
                 mma_bf16_ss(tmem + TM_U, sdesc_sw128(st + TS_KQ + ks * 2048, 2 * HALF, 1024),
                             sdesc_sw128(sb + TC_DD + ks * 2048, 8192, 1024), ID_KT, ks > 0);
-                mma_bf16_ss(tmem + TM_O, sdesc_sw128(st + TS_REC + ks * 32, 16, 1024),
-                            sdesc_sw128(sb + TC_DU + ks * 2048, 8192, 1024), ID_KQ, ks > 0);
-            }
-            mma_commit(mma_bar);
+            mma_commit(bar_u);
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks)
+                mma_bf16_ss(tmem + TM_O + 64 * par, sdesc_sw128(st + TS_REC + ks * 32, 16, 1024),
+                            sdesc_sw128(sb + TC_DU + ks * 2048, 8192, 1024), ID_128, ks > 0);
+            mma_commit(bar_o);
         }
-        ok = mbar_wait(mma_bar, mph & 1, abort_flag);
-        ++mph;
+        ok = mbar_wait(bar_u, par, abort_flag);
         tc_fence_after();
-        {  // S <- gamma_C S + K^T (d o Delta), state row `row`; bf16 copy for MMA1
+        {  // S <- gamma_C S + K^T (d o Delta), state row `row`; bf16 copy for K S and Q S
             float u[HN];
             tmem_cols<HN>(tl + TM_U, u);
 #pragma unroll
@@ -956,26 +992,12 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
             put_cols<HN>(sm, TC_SB, row, c_lo, Sr, 1.f);
             fence_proxy_async_smem();
         }
-        if (quad >= 2) {  // O = gamma o (Q S) + (M o Q K^T) Delta, token row i = row - 64
-            const int i = row - 64;
-            float qs[HN], oi[HN];
-            tmem_cols<HN>(tl + TM_KQ, qs);
-            tmem_cols<HN>(tl + TM_O, oi);
-            if (i < valid) {
-                IO* orow = static_cast<IO*>(p.o) + ((size_t)(tc0 + i) * p.H_v + h) * D + col0 + c_lo;
-#pragma unroll
-                for (int j = 0; j < HN / 8; ++j) {
-                    if (c_lo + 8 * j < ncols) {
-                        float ov[8];
-#pragma unroll
-                        for (int e = 0; e < 8; ++e) ov[e] = fmaf(g_row, qs[8 * j + e], oi[8 * j + e]);
-                        store8<IO>(orow + 8 * j, ov);
-                    }
-                }
-            }
-        }
         tc_fence_before();
         if (!bar_and<BAR_TC, TC_THREADS>(ok)) break;
+    }
+    if (nchunks > 0 && !*abort_flag && quad >= 2) {  // the last chunk's outputs
+        output(nchunks - 1, g_prev);
+        tc_fence_before();
     }
     if (p.S_final && !*abort_flag) {
         float* sf = p.S_final + (((size_t)n * p.H_v + h) * D + row) * D + col0 + c_lo;
