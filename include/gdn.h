@@ -266,8 +266,10 @@ GDN_API gdn_status gdn_decode_step(const void *q, const void *k, const void *v,
  *   dS0      : [N, H_v, dk, dv] fp32 (written), or NULL to skip it.
  *   workspace: at least gdn_prefill_backward_workspace_size(...) bytes,
  *              256-byte aligned.  It holds the chunk-operator records and two
- *              fp32 states per (chunk slot, value head): 144 KB each, about
- *              3.6 GB for T = 32,768 and 48 value heads.  For GDN_F32 it also
+ *              bf16 states per (chunk slot, value head) -- the state entering
+ *              the chunk and the gradient of the state after it, each a 32 KB
+ *              128B-swizzled tile image: about 2.0 GB for T = 32,768 and 48
+ *              value heads.  For GDN_F32 it also
  *              holds bf16 copies of q, k, v and dO (the products read bf16
  *              operands, as in the forward pass).
  * Returns GDN_OK, GDN_ERR_INVALID_ARG, GDN_ERR_UNSUPPORTED, GDN_ERR_WORKSPACE

@@ -41,8 +41,8 @@ struct GradParams {
     const float* beta;        // [T, H_v]
     const int32_t* cu_seqlens;
     const uint8_t* records;   // chunk-operator records of the forward pass
-    const float* S_saved;     // [slot, H_v, 128, 128]: state entering each chunk
-    float* dS_saved;          // [slot, H_v, 128, 128]: gradient of the state after each chunk
+    const uint8_t* S_saved;   // [slot, H_v] bf16 images: state entering each chunk
+    uint8_t* dS_saved;        // [slot, H_v] bf16 images: gradient of the state after it
     const float* dS_final;    // [N, H_v, 128, 128] or null
     float* dS0;               // [N, H_v, 128, 128] or null
     void* dq;                 // [T, H_qk, 128]
@@ -241,16 +241,16 @@ __global__ void __launch_bounds__(256, 1)
         const int valid = min(C, t_end - tc0);
         const bool ok = mbar_wait(&bars[s], (i / GS_STAGES) & 1, abort_flag);
         __syncwarp();
-        {  // the gradient of the state after this chunk, for the per-chunk gradients
-            float* sv = p.dS_saved + ((size_t)record_slot(n, tc0) * p.H_v + h) * D * D;
+        {  // the gradient of the state after this chunk (bf16 image), for the per-chunk gradients
+            uint8_t* sv = p.dS_saved + ((size_t)record_slot(n, tc0) * p.H_v + h) * STATE_IMAGE_BYTES;
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
                 for (int hl = 0; hl < 2; ++hl) {
                     const int row = r0 + g + 8 * hl, col = 8 * nt + 2 * t4;
                     if (col < ncols)
-                        *reinterpret_cast<float2*>(sv + (size_t)row * D + col0 + col) =
-                            make_float2(G[nt][2 * hl], G[nt][2 * hl + 1]);
+                        *reinterpret_cast<uint32_t*>(sv + taddr_e(0, row, col0 + col, 2 * HALF)) =
+                            pack2(G[nt][2 * hl], G[nt][2 * hl + 1]);
                 }
         }
         if (mw) {
@@ -340,49 +340,29 @@ constexpr uint32_t GC_DX = GC_DDEL + 2 * HALF;                           // dX
 constexpr uint32_t GC_PY = GC_DX + 2 * HALF;    // P (then Y), 64 x 64
 constexpr uint32_t GC_TE = GC_PY + HALF;        // dT_b (then E), 64 x 64
 constexpr uint32_t GC_F = GC_TE + HALF;         // fp32: g2[64], dg[64], dbeta[64], misc[64]
-constexpr uint32_t GC_BAR = GC_F + 4 * 64 * 4;  // two mbarriers
-constexpr uint32_t GC_MISC = GC_BAR + 16;
+constexpr uint32_t GC_BAR = GC_F + 4 * 64 * 4;  // three mbarriers
+constexpr uint32_t GC_MISC = GC_BAR + 24;
 constexpr uint32_t GC_SMEM = GC_MISC + 16 + 1024;
 static_assert(GC_SMEM <= 232448, "per-chunk gradient shared memory budget");
 
-// fp32 [128][128] state -> 128B-swizzled bf16 tile (two 128-row halves);
-// returns this thread's part of sum(src o other) when other is given.  Each
-// thread converts 8 groups of 8 values, loading two groups before storing.
-__device__ __forceinline__ float stage_state(uint8_t* sm, uint32_t dst, const float* src,
-                                             const float* other, int tid) {
+// This thread's part of sum(S o dS') over two bf16 state tiles of the same
+// layout (each thread 128 bytes of each).
+__device__ __forceinline__ float tile_dot(const uint8_t* a, const uint8_t* b, int tid) {
     float dot = 0.f;
-#pragma unroll 1
-    for (int e0 = tid; e0 < D * D / 8; e0 += 512) {
-        float4 a[2], b[2], x[2], y[2];
 #pragma unroll
-        for (int u = 0; u < 2; ++u) {
-            const int e = e0 + 256 * u, row = e / 16, c8 = (e % 16) * 8;
-            a[u] = *reinterpret_cast<const float4*>(src + (size_t)row * D + c8);
-            b[u] = *reinterpret_cast<const float4*>(src + (size_t)row * D + c8 + 4);
-            if (other) {
-                x[u] = *reinterpret_cast<const float4*>(other + (size_t)row * D + c8);
-                y[u] = *reinterpret_cast<const float4*>(other + (size_t)row * D + c8 + 4);
-            }
-        }
+    for (int i = 0; i < 8; ++i) {
+        const uint32_t off = (uint32_t)(tid + 256 * i) * 16;
+        const uint4 x = *reinterpret_cast<const uint4*>(a + off);
+        const uint4 y = *reinterpret_cast<const uint4*>(b + off);
+        const uint32_t xs[4] = {x.x, x.y, x.z, x.w}, ys[4] = {y.x, y.y, y.z, y.w};
 #pragma unroll
-        for (int u = 0; u < 2; ++u) {
-            const int e = e0 + 256 * u, row = e / 16, c8 = (e % 16) * 8;
-            *reinterpret_cast<uint4*>(sm + taddr(dst, row, c8, SHALF)) =
-                make_uint4(pack2(a[u].x, a[u].y), pack2(a[u].z, a[u].w), pack2(b[u].x, b[u].y),
-                           pack2(b[u].z, b[u].w));
-            if (other)
-                dot += a[u].x * x[u].x + a[u].y * x[u].y + a[u].z * x[u].z + a[u].w * x[u].w +
-                       b[u].x * y[u].x + b[u].y * y[u].y + b[u].z * y[u].z + b[u].w * y[u].w;
+        for (int e = 0; e < 4; ++e) {
+            const float2 u = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&xs[e]));
+            const float2 v = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&ys[e]));
+            dot = fmaf(u.x, v.x, fmaf(u.y, v.y, dot));
         }
     }
     return dot;
-}
-
-// Bring a 64 KiB fp32 state (512 lines of 128 B) into L2 ahead of its use.
-__device__ __forceinline__ void prefetch_state(const float* src, int tid) {
-#pragma unroll
-    for (int i = 0; i < 2; ++i)
-        asm volatile("prefetch.global.L2 [%0];" ::"l"(src + (size_t)(tid + 256 * i) * 32));
 }
 
 // Row sums (over the accumulator's columns) of acc o w, into dst[row] (smem,
@@ -455,29 +435,54 @@ __global__ void __launch_bounds__(256, 1)
     const int valid = min(C, t_end - tc0);
     const long long slot = record_slot(n, tc0);
 
-    {  // the first value head's states, into L2 while K and Q arrive
-        const size_t so = ((size_t)slot * p.H_v + hq * group) * D * D;
-        prefetch_state(p.S_saved + so, tid);
-        prefetch_state(p.dS_saved + so, tid);
-    }
     if (tid == 0) {
-        mbar_init(&bars[0], 1);
-        mbar_init(&bars[1], 1);
+        for (int i = 0; i < 3; ++i) mbar_init(&bars[i], 1);
         *abort_flag = 0;
         fence_mbar_init();
     }
     __syncthreads();
+    // value head vh's V, dO and saved states (bf16 images, straight into their
+    // tiles) on bars[1]; its record on bars[2]
+    auto issue_head = [&](int vh) {
+        const int h = hq * group + vh;
+        const size_t so = ((size_t)slot * p.H_v + h) * STATE_IMAGE_BYTES;
+        mbar_arrive_expect_tx(&bars[1], 4 * HALF + 2 * STATE_IMAGE_BYTES);
+        tma_load_2d(sm + GC_V, &map_v, h * D, tc0, &bars[1]);
+        tma_load_2d(sm + GC_V + HALF, &map_v, h * D + 64, tc0, &bars[1]);
+        tma_load_2d(sm + GC_O, &map_do, h * D, tc0, &bars[1]);
+        tma_load_2d(sm + GC_O + HALF, &map_do, h * D + 64, tc0, &bars[1]);
+        bulk_load(sm + GC_S, p.S_saved + so, STATE_IMAGE_BYTES, &bars[1]);
+        bulk_load(sm + GC_DS, p.dS_saved + so, STATE_IMAGE_BYTES, &bars[1]);
+    };
+    auto issue_rec = [&](int vh) {
+        const int h = hq * group + vh;
+        mbar_arrive_expect_tx(&bars[2], REC_BYTES);
+        bulk_load(sm + GC_REC, p.records + (size_t)(slot * p.H_v + h) * REC_BYTES, REC_BYTES,
+                  &bars[2]);
+    };
+    int heads = 0, recs = 0;  // copies issued (thread 0)
+    // after a failed wait: let every copy in flight land (bounded), then leave
+    auto drain = [&]() {
+        if (tid == 0) {
+            mbar_wait_drain(&bars[0], 0);
+            if (heads > 0) mbar_wait_drain(&bars[1], (heads - 1) & 1);
+            if (recs > 0) mbar_wait_drain(&bars[2], (recs - 1) & 1);
+        }
+        __syncthreads();
+    };
     if (tid == 0) {
         mbar_arrive_expect_tx(&bars[0], 4 * HALF);
         tma_load_2d(sm + GC_K, &map_k, hq * D, tc0, &bars[0]);
         tma_load_2d(sm + GC_K + HALF, &map_k, hq * D + 64, tc0, &bars[0]);
         tma_load_2d(sm + GC_Q, &map_q, hq * D, tc0, &bars[0]);
         tma_load_2d(sm + GC_Q + HALF, &map_q, hq * D + 64, tc0, &bars[0]);
+        issue_head(0);
+        issue_rec(0);
+        heads = recs = 1;
     }
     bool ok = mbar_wait(&bars[0], 0, abort_flag);
     if (!__syncthreads_and(ok)) {
-        if (tid == 0) mbar_wait_drain(&bars[0], 0);
-        __syncthreads();
+        drain();
         return;
     }
     if (valid < C) {  // rows past the sequence end belong to the next sequence: zero them
@@ -496,26 +501,7 @@ __global__ void __launch_bounds__(256, 1)
 
     for (int vh = 0; vh < group; ++vh) {
         const int h = hq * group + vh;
-        if (tid == 0) {
-            mbar_arrive_expect_tx(&bars[1], 4 * HALF + REC_BYTES);
-            tma_load_2d(sm + GC_V, &map_v, h * D, tc0, &bars[1]);
-            tma_load_2d(sm + GC_V + HALF, &map_v, h * D + 64, tc0, &bars[1]);
-            tma_load_2d(sm + GC_O, &map_do, h * D, tc0, &bars[1]);
-            tma_load_2d(sm + GC_O + HALF, &map_do, h * D + 64, tc0, &bars[1]);
-            bulk_load(sm + GC_REC, p.records + (size_t)(slot * p.H_v + h) * REC_BYTES, REC_BYTES,
-                      &bars[1]);
-        }
-        // meanwhile: the states in bf16, <dS', S>, the gates; the next value
-        // head's states into L2
-        const size_t so = ((size_t)slot * p.H_v + h) * D * D;
-        if (vh + 1 < group) {
-            prefetch_state(p.S_saved + so + D * D, tid);
-            prefetch_state(p.dS_saved + so + D * D, tid);
-        }
-        stage_state(sm, GC_S, p.S_saved + so, nullptr, tid);
-        float dot = stage_state(sm, GC_DS, p.dS_saved + so, p.S_saved + so, tid);
-#pragma unroll
-        for (int off = 16; off > 0; off >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, off);
+        // the gates (while this head's copies land)
         if (tid < 64) {
             dg[tid] = 0.f;
             dbt[tid] = 0.f;
@@ -537,12 +523,17 @@ __global__ void __launch_bounds__(256, 1)
             g2[2 * lane + 1] = incl;
         }
         __syncthreads();
-        if (lane == 0) atomicAdd(&misc[1], dot);
         ok = mbar_wait(&bars[1], vh & 1, abort_flag);
+        ok = mbar_wait(&bars[2], vh & 1, abort_flag) && ok;
         if (!__syncthreads_and(ok)) {
-            if (tid == 0) mbar_wait_drain(&bars[1], vh & 1);
-            __syncthreads();
+            drain();
             return;
+        }
+        {  // <dS', S>, for the gate gradient of the chunk's last row
+            float dot = tile_dot(sm + GC_S, sm + GC_DS, tid);
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, off);
+            if (lane == 0) atomicAdd(&misc[1], dot);
         }
         if (valid < C) {  // V and dO rows past the sequence end
             for (int i = tid; i < 4 * 64 * 8; i += 256) {
@@ -558,6 +549,7 @@ __global__ void __launch_bounds__(256, 1)
         const int n0 = 64 * hh;  // this warp's columns of the 128-wide products
         const float gm_lo = rv[m0 + g], gm_hi = rv[m0 + g + 8];
         const float d_lo = rv[64 + m0 + g], d_hi = rv[64 + m0 + g + 8];
+        const float gam_C = rv[128];
 
         // 1. K S (kept for dg), Q S -> dg += gamma_r dO_r . (QS)_r; X = V - gamma o KS
         float KS[8][4];
@@ -710,6 +702,11 @@ __global__ void __launch_bounds__(256, 1)
             add_col_sums<4>(dbt, p0, tt, lane, 1.f);
         }
         __syncthreads();
+        // V (X), dO and both states are free: the next head's copies land during steps 9-12
+        if (tid == 0 && vh + 1 < group) {
+            issue_head(vh + 1);
+            ++heads;
+        }
         // 9. Y = dT_b T_b^T
         {
             const int p0 = 32 * hh;
@@ -742,6 +739,11 @@ __global__ void __launch_bounds__(256, 1)
             add_col_sums<4>(dg, p0, kk, lane, -1.f);
         }
         __syncthreads();
+        // the record is free too (gamma_C is in a register)
+        if (tid == 0 && vh + 1 < group) {
+            issue_rec(vh + 1);
+            ++recs;
+        }
         // 11. dK += E K + E^T K
         mma_rows<4, true, false>(dK, sb + GC_TE, 0, m0, sb + GC_K, HALF, n0, 0, rb + 1, lane);
         mma_rows<4, false, false>(dK, sb + GC_TE, 0, m0, sb + GC_K, HALF, n0, rb, 4, lane);
@@ -749,7 +751,7 @@ __global__ void __launch_bounds__(256, 1)
         // dlog_alpha_t = sum_{r >= t} dg_r (dg holds the gradient w.r.t. g in
         // natural-log units); dbeta_j = (dbeta * beta)_j / beta_j
         if (warp == 0) {
-            const float last = misc[0] + rv[128] * misc[1];
+            const float last = misc[0] + gam_C * misc[1];
             // reverse inclusive scan of dg over 64 rows, 2 per lane (rows 2l, 2l+1)
             float d0 = dg[2 * lane], d1 = dg[2 * lane + 1];
             if (lane == 31) d1 += last;
@@ -772,7 +774,7 @@ __global__ void __launch_bounds__(256, 1)
                 }
             }
         }
-        __syncthreads();  // the next value head refills V, dO, the record and the states
+        __syncthreads();  // the next head's gates overwrite dg, dbt and misc
     }
     // dQ, dK of this chunk and query/key head (every value head of the group summed)
     IO* dq = static_cast<IO*>(p.dq);
@@ -823,7 +825,7 @@ cudaError_t launch_grads(const CUtensorMap& mq, const CUtensorMap& mk, const CUt
 size_t prefill_backward_workspace_bytes(int N, int T, int H_qk, int H_v, bool bf16) {
     if (T == 0) return 0;
     const size_t slots = (size_t)N + ((size_t)T + C - 1) / C;
-    const size_t states = up256(slots * H_v * D * D * sizeof(float));
+    const size_t states = up256(slots * H_v * STATE_IMAGE_BYTES);
     const size_t staging =
         bf16 ? 0 : 2 * up256((size_t)T * H_qk * D * 2) + 2 * up256((size_t)T * H_v * D * 2);
     return prefill_record_bytes(N, T, H_v) + 2 * states + staging;
@@ -846,13 +848,13 @@ cudaError_t launch_prefill_backward(const void* q, const void* k, const void* v,
     }
     uint8_t* ws = static_cast<uint8_t*>(workspace);
     const size_t slots = (size_t)N + ((size_t)T + C - 1) / C;
-    const size_t states = up256(slots * H_v * D * D * sizeof(float));
+    const size_t states = up256(slots * H_v * STATE_IMAGE_BYTES);
     uint8_t* records = ws;
-    float* S_saved = reinterpret_cast<float*>(ws + prefill_record_bytes(N, T, H_v));
-    float* dS_saved = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(S_saved) + states);
+    uint8_t* S_saved = ws + prefill_record_bytes(N, T, H_v);  // bf16 state images
+    uint8_t* dS_saved = S_saved + states;
     cudaError_t e;
     if (!bf16) {  // bf16 copies of q, k, v and dO after the states
-        uint8_t* st = reinterpret_cast<uint8_t*>(dS_saved) + states;
+        uint8_t* st = dS_saved + states;
         const size_t nqk = (size_t)T * H_qk * D, nv = (size_t)T * H_v * D;
         const void* src[4] = {q, k, v, dO};
         const size_t cnt[4] = {nqk, nqk, nv, nv};
@@ -871,7 +873,7 @@ cudaError_t launch_prefill_backward(const void* q, const void* k, const void* v,
         dO = dst[3];
     }
     e = launch_prefill_save(q, k, v, log_alpha, beta, S0, cu_seqlens, N, T, H_qk, H_v, records,
-                            S_saved, stream);
+                            reinterpret_cast<float*>(S_saved), stream);
     if (e != cudaSuccess) return e;
     CUtensorMap mq, mk, mv, mo;
     if (!make_map(&mq, q, T, (uint64_t)H_qk * D) || !make_map(&mk, k, T, (uint64_t)H_qk * D) ||

@@ -105,7 +105,7 @@ struct PrefillParams {
     float* S_final;
     uint8_t* records;  // chunk operator records, REC_BYTES each
     float* S_aux;      // P2_SEGMENT: the segment propagators; P2_SAVE: every
-                       // chunk's entering state, [record slot, H_v, 128, 128]
+                       // chunk's entering state as a bf16 image [record slot, H_v]
     int H_qk, H_v;
     int N, T;
 };
@@ -538,8 +538,9 @@ __global__ void __launch_bounds__(P2_THREADS, 1)
             const int valid = min(C, t_end - tc0);
             const bool ok = mbar_wait(&bars[B2_FULL + s], (c / NSTAGE) & 1, abort_flag);
             __syncwarp();
-            if constexpr (MODE == P2_SAVE) {  // the state entering this chunk
-                float* sv = p.S_aux + ((size_t)record_slot(n, tc0) * p.H_v + h) * D * D;
+            if constexpr (MODE == P2_SAVE) {  // the state entering this chunk, as a bf16 image
+                uint8_t* sv = reinterpret_cast<uint8_t*>(p.S_aux) +
+                              ((size_t)record_slot(n, tc0) * p.H_v + h) * STATE_IMAGE_BYTES;
 #pragma unroll
                 for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
@@ -547,8 +548,8 @@ __global__ void __launch_bounds__(P2_THREADS, 1)
                         const int row = r0 + g + 8 * hl;
                         const int col = 8 * nt + 2 * t4;
                         if (col < ncols)
-                            *reinterpret_cast<float2*>(sv + (size_t)row * D + col0 + col) =
-                                make_float2(Sacc[nt][2 * hl], Sacc[nt][2 * hl + 1]);
+                            *reinterpret_cast<uint32_t*>(sv + taddr_e(0, row, col0 + col, 2 * HALF)) =
+                                pack2(Sacc[nt][2 * hl], Sacc[nt][2 * hl + 1]);
                     }
             }
 

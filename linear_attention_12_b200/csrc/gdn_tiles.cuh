@@ -26,6 +26,10 @@ constexpr uint32_t REC_MQ = HALF;              // M o Q K^T,    64 x 64 bf16, sw
 constexpr uint32_t REC_VEC = 2 * HALF;         // gamma[64], d[64], gamma_C, pad -> 132 floats
 constexpr uint32_t REC_VEC_FLOATS = 132;
 constexpr uint32_t REC_BYTES = REC_VEC + REC_VEC_FLOATS * 4;  // 16,912
+// A 128 x 128 state saved for the gradients: bf16, two 128-row halves of 64
+// columns (16 KB apart), 128B-swizzled -- element (r, c) at
+// taddr_e(0, r, c, 2 * HALF); the tile layout the gradient kernel multiplies.
+constexpr uint32_t STATE_IMAGE_BYTES = D * D * 2;
 static_assert(REC_BYTES % 16 == 0, "bulk copies move multiples of 16 bytes");
 
 // Record slot of chunk c of sequence n (first token t0 = cu[n] + 64 c):

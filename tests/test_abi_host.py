@@ -165,11 +165,12 @@ def test_backward_fp32_needs_room_for_bf16_copies(L):
 
 
 def test_backward_workspace_holds_records_and_two_states_per_chunk(L):
+    # per (chunk slot, value head): the 16,912-byte record and two bf16 state images
     N, T, H_v = 1, 4096, 3
     ws = L.gdn_prefill_backward_workspace_size(N, T, 1, H_v, 128, 128, gdn.GDN_BF16)
     slots = N + T // 64
-    assert ws >= slots * H_v * (16912 + 2 * 128 * 128 * 4)
-    assert ws <= slots * H_v * (16912 + 2 * 128 * 128 * 4) + 3 * 256
+    assert ws >= slots * H_v * (16912 + 2 * 128 * 128 * 2)
+    assert ws <= slots * H_v * (16912 + 2 * 128 * 128 * 2) + 3 * 256
     # fp32 I/O adds bf16 copies of q, k (1 head) and v, dO (H_v heads)
     ws32 = L.gdn_prefill_backward_workspace_size(N, T, 1, H_v, 128, 128, gdn.GDN_F32)
     assert ws32 == ws + 2 * T * 128 * 2 * (1 + H_v)
