@@ -327,7 +327,10 @@ def run_prefill_shard(args, dev, stream, world, L):
 
 
 def run_backward(args, case, dev, stream, world, L):
-    """Time the gradients of the L-token prefill (the same inputs); returns ms per call."""
+    """Time the gradients of the L-token prefill (the same inputs): the recomputing
+    backward, and the training pair (saving forward, backward from the saved
+    states).  Returns (ms per backward, calls, ms per training forward, ms per
+    saved backward)."""
     import torch
     from linear_attention_12_b200 import gdn
     q, k, v = case.q.to(dev), case.k.to(dev), case.v.to(dev)
@@ -351,7 +354,40 @@ def run_backward(args, case, dev, stream, world, L):
     torch.cuda.synchronize()
     barrier(world)
     assert gdn.last_device_error() == gdn.GDN_OK
-    return max_over_ranks(e0.elapsed_time(e1), world) / n, n
+    bw_ms = max_over_ranks(e0.elapsed_time(e1), world) / n
+
+    # a training step: the saving forward, then the gradients from its saved states
+    o, Sf = torch.empty_like(v), torch.empty((1, H_V, D, D), dtype=torch.float32, device=dev)
+
+    def train_fwd():
+        st = gdn.lib().gdn_prefill_train(
+            gdn._ptr(q), gdn._ptr(k), gdn._ptr(v), gdn._ptr(la), gdn._ptr(be), None, gdn._ptr(cu),
+            1, L, H_QK, H_V, D, D, gdn.GDN_BF16, gdn._ptr(o), gdn._ptr(Sf), gdn._ptr(ws),
+            ws.numel(), gdn._stream_handle(None))
+        assert st == gdn.GDN_OK
+
+    def train_bwd():
+        gdn.prefill_backward(q, k, v, la, be, dO, cu_seqlens=cu, workspace=ws, saved=True)
+
+    for _ in range(max(args.warmup, 3)):
+        train_fwd()
+        train_bwd()
+    torch.cuda.synchronize()
+    barrier(world)
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+    fwd_ms = bwd_ms = 0.0
+    for _ in range(n):
+        ev[0].record(stream)
+        train_fwd()
+        ev[1].record(stream)
+        train_bwd()
+        ev[2].record(stream)
+        torch.cuda.synchronize()
+        fwd_ms += ev[0].elapsed_time(ev[1])
+        bwd_ms += ev[1].elapsed_time(ev[2])
+    barrier(world)
+    assert gdn.last_device_error() == gdn.GDN_OK
+    return (bw_ms, n, max_over_ranks(fwd_ms / n, world), max_over_ranks(bwd_ms / n, world))
 
 
 def run_frontend(args, dev, stream, world, L):
@@ -667,6 +703,16 @@ def run_ours(args):
                 "workload": f"gradients of the prefill B=1 L={L} H_qk={H_QK} H_v={H_V} d={D} bf16 "
                             "(dq, dk, dv, dlog_alpha, dbeta; S0 = 0, no state gradient)",
                 "steps": bw[1],
+                "train_step": {
+                    "ms_forward": bw[2],
+                    "ms_backward": bw[3],
+                    "ms_per_step": bw[2] + bw[3],
+                    "tokens_per_s": L / ((bw[2] + bw[3]) / 1e3),
+                    "ms_per_step_recomputing": ms_per_step + bw[0],
+                    "what": "gdn_prefill_train (outputs + saved states) then "
+                            "gdn_prefill_backward_saved, against gdn_prefill then "
+                            "gdn_prefill_backward (which re-runs the forward)",
+                },
             },
             "prefill_shard": None if shard is None else {
                 "value": L / (shard[1] / 1e3),

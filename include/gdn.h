@@ -285,6 +285,36 @@ GDN_API gdn_status gdn_prefill_backward(const void *q, const void *k, const void
                                 float *dlog_alpha, float *dbeta, float *dS0,
                                 void *workspace, size_t workspace_bytes, void *stream);
 
+/*
+ * gdn_prefill_train -- gdn_prefill for a training step: the same outputs o
+ * and S_final (same arguments, layouts and errors; no sequence split), and in
+ * `workspace` -- at least gdn_prefill_backward_workspace_size(...) bytes,
+ * 256-byte aligned, owned by the caller -- the chunk-operator records and
+ * every chunk's entering state that the gradients read.  Pass the same
+ * inputs and the untouched workspace to gdn_prefill_backward_saved, which
+ * then skips re-running the forward pass.
+ */
+GDN_API gdn_status gdn_prefill_train(const void *q, const void *k, const void *v,
+                                     const float *log_alpha, const float *beta, const float *S0,
+                                     const int32_t *cu_seqlens, int32_t N, int32_t T,
+                                     int32_t H_qk, int32_t H_v, int32_t dk, int32_t dv,
+                                     gdn_dtype io_dtype, void *o, float *S_final,
+                                     void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * gdn_prefill_backward_saved -- gdn_prefill_backward (same arguments, outputs
+ * and errors) reading the records and entering states that gdn_prefill_train
+ * left in `workspace` for the same q, k, v, gates, S0 and cu_seqlens, instead
+ * of recomputing them.  Behaviour is undefined if the workspace was not filled
+ * that way (the library cannot tell).
+ */
+GDN_API gdn_status gdn_prefill_backward_saved(
+    const void *q, const void *k, const void *v, const float *log_alpha, const float *beta,
+    const float *S0, const int32_t *cu_seqlens, const void *dO, const float *dS_final, int32_t N,
+    int32_t T, int32_t H_qk, int32_t H_v, int32_t dk, int32_t dv, gdn_dtype io_dtype, void *dq,
+    void *dk_out, void *dv_out, float *dlog_alpha, float *dbeta, float *dS0, void *workspace,
+    size_t workspace_bytes, void *stream);
+
 /* Workspace bytes of gdn_prefill_backward (0 when T == 0 or the arguments are
  * invalid). */
 GDN_API size_t gdn_prefill_backward_workspace_size(int32_t N, int32_t T, int32_t H_qk,

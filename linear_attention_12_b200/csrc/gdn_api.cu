@@ -168,6 +168,40 @@ gdn_status gdn_prefill_tc(const void* q, const void* k, const void* v, const flo
 
 namespace {
 
+gdn_status backward_call(const void* q, const void* k, const void* v,
+                         const float* log_alpha, const float* beta, const float* S0,
+                         const int32_t* cu_seqlens, const void* dO, const float* dS_final,
+                         int32_t N, int32_t T, int32_t H_qk, int32_t H_v, int32_t dk,
+                         int32_t dv, gdn_dtype io_dtype, void* dq, void* dk_out,
+                         void* dv_out, float* dlog_alpha, float* dbeta, float* dS0,
+                         void* workspace, size_t workspace_bytes, bool recompute,
+                         void* stream) {
+    gdn_status st = check_prefill_args(q, k, v, log_alpha, beta, S0, cu_seqlens, N, T, H_qk, H_v,
+                                       dk, dv, io_dtype, dq, nullptr);
+    if (st != GDN_OK) return st;
+    if (T > 0) {
+        const void* p16[] = {dO, dk_out, dv_out};
+        for (const void* ptr : p16)
+            if (!ptr || !aligned(ptr, 16)) return GDN_ERR_INVALID_ARG;
+        if (!dlog_alpha || !dbeta || !aligned(dlog_alpha, 4) || !aligned(dbeta, 4))
+            return GDN_ERR_INVALID_ARG;
+    }
+    if ((dS_final && !aligned(dS_final, 16)) || (dS0 && !aligned(dS0, 16)))
+        return GDN_ERR_INVALID_ARG;
+    const size_t need = gdn::prefill_backward_workspace_bytes(N, T, H_qk, H_v, io_dtype == GDN_BF16);
+    if (need > 0 && (!workspace || workspace_bytes < need || !aligned(workspace, 256)))
+        return GDN_ERR_WORKSPACE;
+    st = check_device();
+    if (st != GDN_OK) return st;
+    cudaError_t e = gdn::launch_prefill_backward(q, k, v, log_alpha, beta, S0, cu_seqlens, dO,
+                                                 dS_final, N, T, H_qk, H_v,
+                                                 io_dtype == GDN_BF16, dq, dk_out, dv_out,
+                                                 dlog_alpha, dbeta, dS0, workspace, recompute,
+                                                 static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+}
+
+
 gdn_status prefill_call(const void* q, const void* k, const void* v, const float* log_alpha,
                         const float* beta, const float* S0, const int32_t* cu_seqlens, int32_t N,
                         int32_t T, int32_t H_qk, int32_t H_v, int32_t dk, int32_t dv,
@@ -259,28 +293,41 @@ gdn_status gdn_prefill_backward(const void* q, const void* k, const void* v,
                                 int32_t dv, gdn_dtype io_dtype, void* dq, void* dk_out,
                                 void* dv_out, float* dlog_alpha, float* dbeta, float* dS0,
                                 void* workspace, size_t workspace_bytes, void* stream) {
+    return backward_call(q, k, v, log_alpha, beta, S0, cu_seqlens, dO, dS_final, N, T, H_qk, H_v,
+                         dk, dv, io_dtype, dq, dk_out, dv_out, dlog_alpha, dbeta, dS0, workspace,
+                         workspace_bytes, true, stream);
+}
+
+gdn_status gdn_prefill_backward_saved(const void* q, const void* k, const void* v,
+                                      const float* log_alpha, const float* beta, const float* S0,
+                                      const int32_t* cu_seqlens, const void* dO,
+                                      const float* dS_final, int32_t N, int32_t T, int32_t H_qk,
+                                      int32_t H_v, int32_t dk, int32_t dv, gdn_dtype io_dtype,
+                                      void* dq, void* dk_out, void* dv_out, float* dlog_alpha,
+                                      float* dbeta, float* dS0, void* workspace,
+                                      size_t workspace_bytes, void* stream) {
+    return backward_call(q, k, v, log_alpha, beta, S0, cu_seqlens, dO, dS_final, N, T, H_qk, H_v,
+                         dk, dv, io_dtype, dq, dk_out, dv_out, dlog_alpha, dbeta, dS0, workspace,
+                         workspace_bytes, false, stream);
+}
+
+gdn_status gdn_prefill_train(const void* q, const void* k, const void* v, const float* log_alpha,
+                             const float* beta, const float* S0, const int32_t* cu_seqlens,
+                             int32_t N, int32_t T, int32_t H_qk, int32_t H_v, int32_t dk,
+                             int32_t dv, gdn_dtype io_dtype, void* o, float* S_final,
+                             void* workspace, size_t workspace_bytes, void* stream) {
     gdn_status st = check_prefill_args(q, k, v, log_alpha, beta, S0, cu_seqlens, N, T, H_qk, H_v,
-                                       dk, dv, io_dtype, dq, nullptr);
+                                       dk, dv, io_dtype, o, S_final);
     if (st != GDN_OK) return st;
-    if (T > 0) {
-        const void* p16[] = {dO, dk_out, dv_out};
-        for (const void* ptr : p16)
-            if (!ptr || !aligned(ptr, 16)) return GDN_ERR_INVALID_ARG;
-        if (!dlog_alpha || !dbeta || !aligned(dlog_alpha, 4) || !aligned(dbeta, 4))
-            return GDN_ERR_INVALID_ARG;
-    }
-    if ((dS_final && !aligned(dS_final, 16)) || (dS0 && !aligned(dS0, 16)))
-        return GDN_ERR_INVALID_ARG;
-    const size_t need = gdn::prefill_backward_workspace_bytes(N, T, H_qk, H_v, io_dtype == GDN_BF16);
+    const size_t need =
+        gdn::prefill_backward_workspace_bytes(N, T, H_qk, H_v, io_dtype == GDN_BF16);
     if (need > 0 && (!workspace || workspace_bytes < need || !aligned(workspace, 256)))
         return GDN_ERR_WORKSPACE;
     st = check_device();
     if (st != GDN_OK) return st;
-    cudaError_t e = gdn::launch_prefill_backward(q, k, v, log_alpha, beta, S0, cu_seqlens, dO,
-                                                 dS_final, N, T, H_qk, H_v,
-                                                 io_dtype == GDN_BF16, dq, dk_out, dv_out,
-                                                 dlog_alpha, dbeta, dS0, workspace,
-                                                 static_cast<cudaStream_t>(stream));
+    cudaError_t e = gdn::launch_prefill_train(q, k, v, log_alpha, beta, S0, cu_seqlens, N, T,
+                                              H_qk, H_v, io_dtype == GDN_BF16, o, S_final,
+                                              workspace, static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
 }
 

@@ -831,12 +831,47 @@ size_t prefill_backward_workspace_bytes(int N, int T, int H_qk, int H_v, bool bf
     return prefill_record_bytes(N, T, H_v) + 2 * states + staging;
 }
 
+cudaError_t launch_prefill_train(const void* q, const void* k, const void* v,
+                                 const float* log_alpha, const float* beta, const float* S0,
+                                 const int32_t* cu_seqlens, int N, int T, int H_qk, int H_v,
+                                 bool bf16, void* o, float* S_final, void* workspace,
+                                 cudaStream_t stream) {
+    if (T == 0) return launch_prefill(q, k, v, log_alpha, beta, S0, cu_seqlens, N, T, H_qk, H_v,
+                                      bf16, o, S_final, nullptr, 1, false, stream);
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    const size_t slots = (size_t)N + ((size_t)T + C - 1) / C;
+    const size_t states = up256(slots * H_v * STATE_IMAGE_BYTES);
+    uint8_t* records = ws;
+    uint8_t* S_saved = ws + prefill_record_bytes(N, T, H_v);
+    if (!bf16) {  // bf16 copies of q, k and v where the gradients stage them too
+        uint8_t* st = S_saved + 2 * states;
+        const size_t nqk = (size_t)T * H_qk * D, nv = (size_t)T * H_v * D;
+        const void* src[3] = {q, k, v};
+        const size_t cnt[3] = {nqk, nqk, nv};
+        const void* dst[3];
+        for (int i = 0; i < 3; ++i) {
+            f32_to_bf16_kernel<<<592, 256, 0, stream>>>(static_cast<const float*>(src[i]),
+                                                        reinterpret_cast<__nv_bfloat16*>(st),
+                                                        cnt[i] / 4);
+            dst[i] = st;
+            st += up256(cnt[i] * 2);
+        }
+        cudaError_t e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+        q = dst[0];
+        k = dst[1];
+        v = dst[2];
+    }
+    return launch_prefill_save(q, k, v, log_alpha, beta, S0, cu_seqlens, N, T, H_qk, H_v, records,
+                               S_saved, o, S_final, bf16, stream);
+}
+
 cudaError_t launch_prefill_backward(const void* q, const void* k, const void* v,
                                     const float* log_alpha, const float* beta, const float* S0,
                                     const int32_t* cu_seqlens, const void* dO,
                                     const float* dS_final, int N, int T, int H_qk, int H_v,
                                     bool bf16, void* dq, void* dk, void* dv, float* dlog_alpha,
-                                    float* dbeta, float* dS0, void* workspace,
+                                    float* dbeta, float* dS0, void* workspace, bool recompute,
                                     cudaStream_t stream) {
     if (T == 0) {  // nothing ran: dS0 = dS_final (or zero)
         if (dS0) {
@@ -872,9 +907,11 @@ cudaError_t launch_prefill_backward(const void* q, const void* k, const void* v,
         v = dst[2];
         dO = dst[3];
     }
-    e = launch_prefill_save(q, k, v, log_alpha, beta, S0, cu_seqlens, N, T, H_qk, H_v, records,
-                            reinterpret_cast<float*>(S_saved), stream);
-    if (e != cudaSuccess) return e;
+    if (recompute) {  // the records and entering states, unless a training forward left them
+        e = launch_prefill_save(q, k, v, log_alpha, beta, S0, cu_seqlens, N, T, H_qk, H_v, records,
+                                S_saved, nullptr, nullptr, true, stream);
+        if (e != cudaSuccess) return e;
+    }
     CUtensorMap mq, mk, mv, mo;
     if (!make_map(&mq, q, T, (uint64_t)H_qk * D) || !make_map(&mk, k, T, (uint64_t)H_qk * D) ||
         !make_map(&mv, v, T, (uint64_t)H_v * D) || !make_map(&mo, dO, T, (uint64_t)H_v * D))

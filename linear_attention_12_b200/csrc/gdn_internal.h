@@ -33,11 +33,14 @@ cudaError_t launch_prefill(const void* q, const void* k, const void* v, const fl
                            int T, int H_qk, int H_v, bool bf16, void* o, float* S_final,
                            void* workspace, int P, bool tc, cudaStream_t stream);
 
-// Records and chunk-entering states of a bf16 prefill, for its gradients.
+// Records and chunk-entering states (bf16 images) of a prefill with bf16
+// q, k, v, for its gradients; with o non-null also its outputs (bf16 or fp32)
+// and final states.
 cudaError_t launch_prefill_save(const void* q, const void* k, const void* v,
                                 const float* log_alpha, const float* beta, const float* S0,
                                 const int32_t* cu_seqlens, int N, int T, int H_qk, int H_v,
-                                uint8_t* records, float* S_saved, cudaStream_t stream);
+                                uint8_t* records, uint8_t* S_saved, void* o, float* S_final,
+                                bool out_bf16, cudaStream_t stream);
 size_t prefill_record_bytes(int N, int T, int H_v);
 
 // Gradients of a bf16 prefill: workspace bytes, and the launches (the forward
@@ -48,8 +51,17 @@ cudaError_t launch_prefill_backward(const void* q, const void* k, const void* v,
                                     const int32_t* cu_seqlens, const void* dO,
                                     const float* dS_final, int N, int T, int H_qk, int H_v,
                                     bool bf16, void* dq, void* dk, void* dv, float* dlog_alpha,
-                                    float* dbeta, float* dS0, void* workspace,
+                                    float* dbeta, float* dS0, void* workspace, bool recompute,
                                     cudaStream_t stream);
+// The prefill (outputs, final states) that also leaves in `workspace` (laid
+// out as launch_prefill_backward's) the records and entering states its
+// gradients read; launch_prefill_backward with recompute = false then skips
+// the forward re-run.
+cudaError_t launch_prefill_train(const void* q, const void* k, const void* v,
+                                 const float* log_alpha, const float* beta, const float* S0,
+                                 const int32_t* cu_seqlens, int N, int T, int H_qk, int H_v,
+                                 bool bf16, void* o, float* S_final, void* workspace,
+                                 cudaStream_t stream);
 
 cudaError_t launch_frontend(const void* q_raw, const void* k_raw, const void* v_raw,
                             const float* conv_w, const float* a, const float* b,

@@ -445,7 +445,9 @@ __device__ __forceinline__ void delta_half(uint8_t* sm, uint32_t tb, uint32_t xt
 // propagator P (to S_aux): S_end = P S_start + (state from zero).  MODE
 // P2_SAVE: no outputs; every chunk's entering state is stored to S_aux (for
 // the gradients).
-constexpr int P2_OUT = 0, P2_SEGMENT = 1, P2_SAVE = 2;
+// MODE P2_OUT_SAVE: the outputs and final states of P2_OUT, and the entering
+// states of P2_SAVE (a training forward whose gradients follow).
+constexpr int P2_OUT = 0, P2_SEGMENT = 1, P2_SAVE = 2, P2_OUT_SAVE = 3;
 
 template <int NS, typename IO, int MODE>
 __global__ void __launch_bounds__(P2_THREADS, 1)
@@ -456,6 +458,7 @@ __global__ void __launch_bounds__(P2_THREADS, 1)
     constexpr int NT = NS / 8;  // n-tiles of a slice
     constexpr int NP = NT / 2;  // n-tile pairs
     constexpr int NSL = (D + NS - 1) / NS;  // slices of a head
+    constexpr bool OUTS = MODE == P2_OUT || MODE == P2_OUT_SAVE;  // writes the outputs
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
@@ -538,7 +541,7 @@ __global__ void __launch_bounds__(P2_THREADS, 1)
             const int valid = min(C, t_end - tc0);
             const bool ok = mbar_wait(&bars[B2_FULL + s], (c / NSTAGE) & 1, abort_flag);
             __syncwarp();
-            if constexpr (MODE == P2_SAVE) {  // the state entering this chunk, as a bf16 image
+            if constexpr (MODE == P2_SAVE || MODE == P2_OUT_SAVE) {  // the entering state, bf16 image
                 uint8_t* sv = reinterpret_cast<uint8_t*>(p.S_aux) +
                               ((size_t)record_slot(n, tc0) * p.H_v + h) * STATE_IMAGE_BYTES;
 #pragma unroll
@@ -564,14 +567,14 @@ __global__ void __launch_bounds__(P2_THREADS, 1)
                 for (int ks = 0; ks < 8; ++ks) {
                     uint32_t ak[4], aq[4];
                     lda_k(st + ST_K, HALF, m0, 16 * ks, lane, ak);
-                    if constexpr (MODE == P2_OUT) lda_k(st + ST_Q, HALF, m0, 16 * ks, lane, aq);
+                    if constexpr (OUTS) lda_k(st + ST_Q, HALF, m0, 16 * ks, lane, aq);
 #pragma unroll
                     for (int np = 0; np < NP; ++np) {
                         uint32_t b[4];
                         ldb_mn(sb + P2_SB, 0, 16 * np, 16 * ks, lane, b);
                         mma16816(accK[2 * np], ak, b[0], b[1]);
                         mma16816(accK[2 * np + 1], ak, b[2], b[3]);
-                        if constexpr (MODE == P2_OUT) {
+                        if constexpr (OUTS) {
                             mma16816(accQ[2 * np], aq, b[0], b[1]);
                             mma16816(accQ[2 * np + 1], aq, b[2], b[3]);
                         }
@@ -637,7 +640,7 @@ __global__ void __launch_bounds__(P2_THREADS, 1)
                 }
             }
             // ---- O = gamma o (Q S) + (M o Q K^T) Delta   (warps 0-3), stored
-            if (MODE == P2_OUT && mw) {
+            if (OUTS && mw) {
 #pragma unroll
                 for (int ks = 0; ks < 4; ++ks) {
                     if (ks <= warp) {
@@ -1400,16 +1403,20 @@ cudaError_t launch_prefill(const void* q, const void* k, const void* v, const fl
 cudaError_t launch_prefill_save(const void* q, const void* k, const void* v,
                                 const float* log_alpha, const float* beta, const float* S0,
                                 const int32_t* cu_seqlens, int N, int T, int H_qk, int H_v,
-                                uint8_t* records, float* S_saved, cudaStream_t stream) {
+                                uint8_t* records, uint8_t* S_saved, void* o, float* S_final,
+                                bool out_bf16, cudaStream_t stream) {
     CUtensorMap mq, mk, mv;
     if (!make_map(&mq, q, T, (uint64_t)H_qk * D) || !make_map(&mk, k, T, (uint64_t)H_qk * D) ||
         !make_map(&mv, v, T, (uint64_t)H_v * D))
         return cudaErrorInvalidValue;
-    const PrefillParams prm{log_alpha, beta, S0,      cu_seqlens, nullptr, nullptr,
-                            records,   S_saved, H_qk, H_v,        N,       T};
+    const PrefillParams prm{log_alpha, beta, S0,   cu_seqlens, o, S_final, records,
+                            reinterpret_cast<float*>(S_saved), H_qk, H_v, N, T};
     cudaError_t e = run_pass1(mq, mk, prm, stream);
     if (e != cudaSuccess) return e;
-    return run_pass2<__nv_bfloat16, P2_SAVE>(mq, mk, mv, prm, device_sms(), stream);
+    const int sms = device_sms();
+    if (!o) return run_pass2<__nv_bfloat16, P2_SAVE>(mq, mk, mv, prm, sms, stream);
+    return out_bf16 ? run_pass2<__nv_bfloat16, P2_OUT_SAVE>(mq, mk, mv, prm, sms, stream)
+                    : run_pass2<float, P2_OUT_SAVE>(mq, mk, mv, prm, sms, stream);
 }
 
 size_t prefill_record_bytes(int N, int T, int H_v) { return record_bytes(N, T, H_v); }

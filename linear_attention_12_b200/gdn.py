@@ -47,6 +47,11 @@ SIGNATURES = {
     "gdn_prefill_auto_segments": (_c.c_int32, [_c.c_int32] * 4),
     "gdn_prefill_backward": (_c.c_int, [_c.c_void_p] * 9 + [_c.c_int32] * 6 +
                              [_c.c_int] + [_c.c_void_p] * 7 + [_c.c_size_t, _c.c_void_p]),
+    "gdn_prefill_backward_saved": (_c.c_int, [_c.c_void_p] * 9 + [_c.c_int32] * 6 +
+                                   [_c.c_int] + [_c.c_void_p] * 7 + [_c.c_size_t, _c.c_void_p]),
+    "gdn_prefill_train": (_c.c_int, [_c.c_void_p] * 7 + [_c.c_int32] * 6 +
+                          [_c.c_int, _c.c_void_p, _c.c_void_p, _c.c_void_p, _c.c_size_t,
+                           _c.c_void_p]),
     "gdn_prefill_backward_workspace_size": (_c.c_size_t, [_c.c_int32] * 6 + [_c.c_int]),
     "gdn_prefill_noalloc": (_c.c_int, [_c.c_void_p, _c.c_void_p, _c.c_void_p, _c.c_void_p,
                                        _c.c_void_p, _c.c_void_p, _c.c_void_p, _c.c_int32,
@@ -218,12 +223,59 @@ def decode_step(q, k, v, log_alpha, beta, S, *, o=None, stream=None):
     return o
 
 
+def backward_workspace(q, v, cu_seqlens=None):
+    """A workspace tensor of gdn_prefill_backward_workspace_size bytes for these inputs
+    (also what ``prefill_train`` fills)."""
+    T, H_qk, dk_ = q.shape
+    N = 1 if cu_seqlens is None else cu_seqlens.numel() - 1
+    need = int(lib().gdn_prefill_backward_workspace_size(N, T, H_qk, v.shape[1], dk_,
+                                                         v.shape[2], _io_dtype(q)))
+    return torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
+
+
+def prefill_train(q, k, v, log_alpha, beta, S0=None, cu_seqlens=None, *, workspace=None,
+                  stream=None):
+    """The prefill of a training step (gdn_prefill_train): returns ``(o, S_final,
+    workspace)``, the workspace holding what ``prefill_backward(..., saved=True)``
+    reads for the same inputs."""
+    T, H_qk, dk_ = q.shape
+    H_v, dv_ = v.shape[1], v.shape[2]
+    dt = q.dtype
+    _check(q, "q", dt)
+    _check(k, "k", dt, q.shape)
+    _check(v, "v", dt, (T, H_v, dv_))
+    _check(log_alpha, "log_alpha", torch.float32, (T, H_v))
+    _check(beta, "beta", torch.float32, (T, H_v))
+    if cu_seqlens is None:
+        cu_seqlens = torch.tensor([0, T], dtype=torch.int32, device=q.device)
+    _check(cu_seqlens, "cu_seqlens", torch.int32)
+    N = cu_seqlens.numel() - 1
+    if S0 is not None:
+        _check(S0, "S0", torch.float32, (N, H_v, dk_, dv_))
+    o = torch.empty((T, H_v, dv_), dtype=dt, device=q.device)
+    S_final = torch.empty((N, H_v, dk_, dv_), dtype=torch.float32, device=q.device)
+    if workspace is None:
+        workspace = backward_workspace(q, v, cu_seqlens)
+    wbytes = workspace.numel() * workspace.element_size()
+    st = lib().gdn_prefill_train(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta),
+                                 _ptr(S0), _ptr(cu_seqlens), N, T, H_qk, H_v, dk_, dv_,
+                                 _io_dtype(q), _ptr(o), _ptr(S_final), _ptr(workspace), wbytes,
+                                 _stream_handle(stream))
+    if st != GDN_OK:
+        raise GDNError(st, "gdn_prefill_train")
+    return o, S_final, workspace
+
+
 def prefill_backward(q, k, v, log_alpha, beta, dO, S0=None, dS_final=None, cu_seqlens=None, *,
-                     want_dS0=True, workspace=None, stream=None):
+                     want_dS0=True, workspace=None, saved=False, stream=None):
     """Gradients of ``L = <dO, o> + <dS_final, S_final>`` for gdn_prefill (bf16 or
-    fp32 q, k, v, dO; the gradients of q, k, v in the same type).
+    fp32 q, k, v, dO; the gradients of q, k, v in the same type).  ``saved=True``:
+    ``workspace`` is the one ``prefill_train`` filled for the same inputs, and the
+    forward pass is not re-run (gdn_prefill_backward_saved).
 
     Returns ``(dq, dk, dv, dlog_alpha, dbeta, dS0)`` (``dS0`` None if not wanted)."""
+    if saved and workspace is None:
+        raise ValueError("saved=True needs the workspace prefill_train filled")
     T, H_qk, dk_ = q.shape
     H_v, dv_ = v.shape[1], v.shape[2]
     dt = q.dtype
@@ -251,13 +303,13 @@ def prefill_backward(q, k, v, log_alpha, beta, dO, S0=None, dS_final=None, cu_se
     if need and workspace is None:
         workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
     wbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
-    st = lib().gdn_prefill_backward(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta),
-                                    _ptr(S0), _ptr(cu_seqlens), _ptr(dO), _ptr(dS_final), N, T,
-                                    H_qk, H_v, dk_, dv_, io, _ptr(dq), _ptr(dk), _ptr(dv),
-                                    _ptr(dla), _ptr(dbe), _ptr(dS0), _ptr(workspace), wbytes,
-                                    _stream_handle(stream))
+    fn = lib().gdn_prefill_backward_saved if saved else lib().gdn_prefill_backward
+    st = fn(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _ptr(S0),
+            _ptr(cu_seqlens), _ptr(dO), _ptr(dS_final), N, T, H_qk, H_v, dk_, dv_, io, _ptr(dq),
+            _ptr(dk), _ptr(dv), _ptr(dla), _ptr(dbe), _ptr(dS0), _ptr(workspace), wbytes,
+            _stream_handle(stream))
     if st != GDN_OK:
-        raise GDNError(st, "gdn_prefill_backward")
+        raise GDNError(st, "gdn_prefill_backward_saved" if saved else "gdn_prefill_backward")
     return dq, dk, dv, dla, dbe, dS0
 
 

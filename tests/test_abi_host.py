@@ -164,6 +164,21 @@ def test_backward_fp32_needs_room_for_bf16_copies(L):
     assert _backward(L, dt=gdn.GDN_BF16, wsb=ws16) == gdn.GDN_ERR_CUDA  # host checks pass; no device
 
 
+def test_training_forward_checks_its_workspace(L):
+    ws = L.gdn_prefill_backward_workspace_size(1, 64, 1, 1, 128, 128, gdn.GDN_BF16)
+    args = lambda wsb, dt=gdn.GDN_BF16, o=P: (P, P, P, P, P, None, P, 1, 64, 1, 1, 128, 128, dt,
+                                                o, None, P, wsb, None)
+    assert L.gdn_prefill_train(*args(ws - 256)) == gdn.GDN_ERR_WORKSPACE
+    assert L.gdn_prefill_train(*args(ws, gdn.GDN_F32)) == gdn.GDN_ERR_WORKSPACE  # + bf16 copies
+    assert L.gdn_prefill_train(*args(ws, o=None)) == gdn.GDN_ERR_INVALID_ARG
+    assert L.gdn_prefill_train(*args(ws)) == gdn.GDN_ERR_CUDA  # host checks pass; no device
+    assert _backward(L, wsb=16) == gdn.GDN_ERR_WORKSPACE
+    b = dict(q=P, k=P, v=P, la=P, be=P, S0=None, cu=P, dO=P, dSf=None, N=1, T=64, H_qk=1, H_v=1,
+             dk=128, dv=128, dt=gdn.GDN_BF16, dq=P, dk_out=P, dv_out=P, dla=P, dbe=P, dS0=None,
+             ws=P, wsb=16, stream=None)
+    assert L.gdn_prefill_backward_saved(*b.values()) == gdn.GDN_ERR_WORKSPACE
+
+
 def test_backward_workspace_holds_records_and_two_states_per_chunk(L):
     # per (chunk slot, value head): the 16,912-byte record and two bf16 state images
     N, T, H_v = 1, 4096, 3

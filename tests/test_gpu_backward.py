@@ -1,4 +1,5 @@
-"""GPU parity of gdn_prefill_backward (bf16 and fp32 I/O) against the fp64 backward oracle
+"""GPU parity of gdn_prefill_backward (bf16 and fp32 I/O), and of the
+training pair gdn_prefill_train + gdn_prefill_backward_saved, against the fp64 backward oracle
 (oracle/backward.py), through the C ABI: every gradient on ragged packed
 sequences, many-chunk sequences, grouped heads and long-memory gates.
 
@@ -72,3 +73,37 @@ def test_backward_fp32_io(lens, H_qk, H_v):
     case, dO, dSf = _case("bw_f32", lens, H_qk, H_v, seed=11, alpha_mu=-6.0,
                           dtype=torch.float32)
     _check(case, dO, dSf, dtype=torch.float32)
+
+
+@pytest.mark.parametrize("lens,H_qk,H_v,dtype", [([100, 0, 37, 64], 2, 6, torch.bfloat16),
+                                                 ([1100], 1, 3, torch.bfloat16),
+                                                 ([300, 65], 2, 4, torch.float32)])
+def test_training_forward_then_saved_backward(lens, H_qk, H_v, dtype):
+    # the training forward's outputs match the oracle's forward; the backward that
+    # reads its saved states matches the oracle's gradients
+    import oracle
+    case, dO, dSf = _case("train", lens, H_qk, H_v, seed=13 + len(lens), alpha_mu=-3.0,
+                          dtype=dtype)
+    d = lambda x: None if x is None else x.cuda()
+    o, S, ws = gdn.prefill_train(d(case.q), d(case.k), d(case.v), d(case.log_alpha),
+                                 d(case.beta), S0=d(case.S0), cu_seqlens=d(case.cu_seqlens))
+    torch.cuda.synchronize()
+    assert o.dtype == dtype
+    o_ref, S_ref = oracle.prefill(case.q, case.k, case.v, case.log_alpha, case.beta, S0=case.S0,
+                                  cu_seqlens=case.cu_seqlens)
+    assert np.abs(o.float().cpu().double().numpy() - o_ref).max() / np.abs(o_ref).max() <= TOL
+    assert np.linalg.norm(S.cpu().double().numpy() - S_ref) / np.linalg.norm(S_ref) <= TOL
+    got = gdn.prefill_backward(d(case.q), d(case.k), d(case.v), d(case.log_alpha), d(case.beta),
+                               d(dO), S0=d(case.S0), dS_final=d(dSf),
+                               cu_seqlens=d(case.cu_seqlens), workspace=ws, saved=True)
+    torch.cuda.synchronize()
+    assert gdn.last_device_error() == gdn.GDN_OK
+    ref = backward.prefill_backward(case.q, case.k, case.v, case.log_alpha, case.beta,
+                                    dO.float().numpy(),
+                                    S0=None if case.S0 is None else case.S0.numpy(),
+                                    dS_final=None if dSf is None else dSf.numpy(),
+                                    cu_seqlens=case.cu_seqlens.numpy())
+    for name, a, b in zip(["dq", "dk", "dv", "dlog_alpha", "dbeta", "dS0"], got, ref):
+        a = a.float().cpu().double().numpy()
+        err = np.abs(a - b).max() / max(np.abs(b).max(), 1e-300)
+        assert err <= TOL, (name, err)
