@@ -159,16 +159,23 @@ GDN_API gdn_status gdn_prefill_segmented(const void *q, const void *k, const voi
                                  void *workspace, size_t workspace_bytes, void *stream);
 
 /*
- * gdn_prefill_tc -- gdn_prefill with the state pass that writes the outputs
- * on the fifth-generation tensor cores (tcgen05.mma, accumulators in tensor
- * memory) instead of mma.sync.  Same arguments, layouts, workspace
- * (gdn_prefill_workspace_size), results within rounding, and errors as
- * gdn_prefill; the automatic segment choice applies as there.  Per chunk the
- * pass runs four dependent tensor-memory products ([K; Q] S, T_b X,
- * K^T (d o Delta) and [T_b; M o Q K^T] Delta, the chunk form of the
- * bjdmk.com.cn article's recurrence, section 2.1) with a read-back between
- * them; at 16/48 heads and 32,768 tokens it is slower than gdn_prefill's
- * mma.sync pass, which stays the default.
+ * gdn_prefill_tc / gdn_prefill_mma -- gdn_prefill with the implementation of
+ * the state pass that writes the outputs fixed.
+ *
+ * There are two, of the same chunk form of the bjdmk.com.cn article's
+ * recurrence, section 2.1:
+ *   - gdn_prefill_tc: the fifth-generation tensor cores (tcgen05.mma,
+ *     accumulators in tensor memory);
+ *   - gdn_prefill_mma: warp-level mma.sync with the state in registers.
+ *
+ * gdn_prefill picks per d_v slice width.  It takes tcgen05 for the 48-column
+ * slices it uses at 38-49 (sequence, value head) units, e.g. 16/48 heads and
+ * one sequence: 1.31-1.32 against 1.32-1.34 ms at 32,768 tokens.  It takes
+ * mma.sync otherwise (at 32-column slices mma.sync measured faster).
+ *
+ * Same arguments, layouts, workspace (gdn_prefill_workspace_size), results
+ * within rounding, and errors as gdn_prefill; the automatic segment choice
+ * applies as there.
  */
 GDN_API gdn_status gdn_prefill_tc(const void *q, const void *k, const void *v,
                                   const float *log_alpha, const float *beta, const float *S0,
@@ -176,6 +183,12 @@ GDN_API gdn_status gdn_prefill_tc(const void *q, const void *k, const void *v,
                                   int32_t H_v, int32_t dk, int32_t dv, gdn_dtype io_dtype,
                                   void *o, float *S_final, void *workspace,
                                   size_t workspace_bytes, void *stream);
+GDN_API gdn_status gdn_prefill_mma(const void *q, const void *k, const void *v,
+                                   const float *log_alpha, const float *beta, const float *S0,
+                                   const int32_t *cu_seqlens, int32_t N, int32_t T, int32_t H_qk,
+                                   int32_t H_v, int32_t dk, int32_t dv, gdn_dtype io_dtype,
+                                   void *o, float *S_final, void *workspace,
+                                   size_t workspace_bytes, void *stream);
 
 /* Workspace bytes of gdn_prefill_segmented with these arguments (0 when T == 0
  * or the arguments are invalid). */

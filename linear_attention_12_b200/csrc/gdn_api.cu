@@ -139,7 +139,7 @@ gdn_status prefill_call(const void* q, const void* k, const void* v, const float
                         const float* beta, const float* S0, const int32_t* cu_seqlens, int32_t N,
                         int32_t T, int32_t H_qk, int32_t H_v, int32_t dk, int32_t dv,
                         gdn_dtype io_dtype, void* o, float* S_final, int32_t segments,
-                        void* workspace, size_t workspace_bytes, bool tc, void* stream);
+                        void* workspace, size_t workspace_bytes, int state_pass, void* stream);
 
 }  // namespace
 
@@ -152,7 +152,18 @@ gdn_status gdn_prefill_segmented(const void* q, const void* k, const void* v,
                                  float* S_final, int32_t segments, void* workspace,
                                  size_t workspace_bytes, void* stream) {
     return prefill_call(q, k, v, log_alpha, beta, S0, cu_seqlens, N, T, H_qk, H_v, dk, dv,
-                        io_dtype, o, S_final, segments, workspace, workspace_bytes, false, stream);
+                        io_dtype, o, S_final, segments, workspace, workspace_bytes,
+                        gdn::STATE_PASS_AUTO, stream);
+}
+
+gdn_status gdn_prefill_mma(const void* q, const void* k, const void* v, const float* log_alpha,
+                           const float* beta, const float* S0, const int32_t* cu_seqlens, int32_t N,
+                           int32_t T, int32_t H_qk, int32_t H_v, int32_t dk, int32_t dv,
+                           gdn_dtype io_dtype, void* o, float* S_final, void* workspace,
+                           size_t workspace_bytes, void* stream) {
+    return prefill_call(q, k, v, log_alpha, beta, S0, cu_seqlens, N, T, H_qk, H_v, dk, dv,
+                        io_dtype, o, S_final, 0, workspace, workspace_bytes, gdn::STATE_PASS_MMA,
+                        stream);
 }
 
 gdn_status gdn_prefill_tc(const void* q, const void* k, const void* v, const float* log_alpha,
@@ -161,7 +172,8 @@ gdn_status gdn_prefill_tc(const void* q, const void* k, const void* v, const flo
                           gdn_dtype io_dtype, void* o, float* S_final, void* workspace,
                           size_t workspace_bytes, void* stream) {
     return prefill_call(q, k, v, log_alpha, beta, S0, cu_seqlens, N, T, H_qk, H_v, dk, dv,
-                        io_dtype, o, S_final, 0, workspace, workspace_bytes, true, stream);
+                        io_dtype, o, S_final, 0, workspace, workspace_bytes, gdn::STATE_PASS_TC,
+                        stream);
 }
 
 }  // extern "C"
@@ -206,7 +218,7 @@ gdn_status prefill_call(const void* q, const void* k, const void* v, const float
                         const float* beta, const float* S0, const int32_t* cu_seqlens, int32_t N,
                         int32_t T, int32_t H_qk, int32_t H_v, int32_t dk, int32_t dv,
                         gdn_dtype io_dtype, void* o, float* S_final, int32_t segments,
-                        void* workspace, size_t workspace_bytes, bool tc, void* stream) {
+                        void* workspace, size_t workspace_bytes, int state_pass, void* stream) {
     gdn_status st = check_prefill_args(q, k, v, log_alpha, beta, S0, cu_seqlens, N, T, H_qk, H_v,
                                        dk, dv, io_dtype, o, S_final);
     if (st != GDN_OK) return st;
@@ -220,7 +232,7 @@ gdn_status prefill_call(const void* q, const void* k, const void* v, const float
     st = check_device();
     if (st != GDN_OK) return st;
     cudaError_t e = gdn::launch_prefill(q, k, v, log_alpha, beta, S0, cu_seqlens, N, T, H_qk,
-                                        H_v, bf16, o, S_final, workspace, P, tc,
+                                        H_v, bf16, o, S_final, workspace, P, state_pass,
                                         static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
 }

@@ -837,7 +837,7 @@ cudaError_t launch_prefill_train(const void* q, const void* k, const void* v,
                                  bool bf16, void* o, float* S_final, void* workspace,
                                  cudaStream_t stream) {
     if (T == 0) return launch_prefill(q, k, v, log_alpha, beta, S0, cu_seqlens, N, T, H_qk, H_v,
-                                      bf16, o, S_final, nullptr, 1, false, stream);
+                                      bf16, o, S_final, nullptr, 1, STATE_PASS_MMA, stream);
     uint8_t* ws = static_cast<uint8_t*>(workspace);
     const size_t slots = (size_t)N + ((size_t)T + C - 1) / C;
     const size_t states = up256(slots * H_v * STATE_IMAGE_BYTES);

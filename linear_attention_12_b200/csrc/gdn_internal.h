@@ -26,12 +26,16 @@ int device_sms();
 // library: 1 unless splitting the sequences fills more of the SMs.
 int choose_segments(int N, int T, int H_v, int sms);
 
-// P segments per sequence (P <= 0: choose_segments); tc: the state pass that
-// writes the outputs runs on tcgen05 instead of mma.sync.
+// Which implementation runs the state pass that writes the prefill's outputs.
+constexpr int STATE_PASS_AUTO = 0;  // the faster one for the slice width
+constexpr int STATE_PASS_TC = 1;    // tcgen05, accumulators in tensor memory
+constexpr int STATE_PASS_MMA = 2;   // warp-level mma.sync, accumulators in registers
+
+// P segments per sequence (P <= 0: choose_segments).
 cudaError_t launch_prefill(const void* q, const void* k, const void* v, const float* log_alpha,
                            const float* beta, const float* S0, const int32_t* cu_seqlens, int N,
                            int T, int H_qk, int H_v, bool bf16, void* o, float* S_final,
-                           void* workspace, int P, bool tc, cudaStream_t stream);
+                           void* workspace, int P, int state_pass, cudaStream_t stream);
 
 // Records and chunk-entering states (bf16 images) of a prefill with bf16
 // q, k, v, for its gradients; with o non-null also its outputs (bf16 or fp32)

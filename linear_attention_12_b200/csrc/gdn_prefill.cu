@@ -1291,13 +1291,16 @@ int choose_segments(int N, int T, int H_v, int sms) {
 template <typename IO, int MODE>
 static cudaError_t run_pass2(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                              const PrefillParams& prm, int sms, cudaStream_t stream,
-                             bool tc = false) {
+                             int state_pass = STATE_PASS_MMA) {
     // one block per SM at most (each holds ~212 KB of shared memory): split every
     // value head into as many d_v slices as still fit in one wave
     const long long units = (long long)prm.N * prm.H_v * (MODE == P2_SEGMENT ? 2 : 1);
     const int slices = pass2_slices(units, sms);
     if constexpr (MODE == P2_OUT) {
-        if (tc) {
+        // the tcgen05 pass where it measured faster (48-column slices: 1.31-1.32 vs
+        // 1.32-1.34 ms at 16/48 heads and 32K tokens), mma.sync at the other widths
+        // (32-column slices: 0.95 vs 0.82 ms on a 2/6-head shard)
+        if (state_pass == STATE_PASS_TC || (state_pass == STATE_PASS_AUTO && slices == 3)) {
             if (slices == 4) return launch_state_tc<32, IO>(mq, mk, mv, prm, stream);
             if (slices == 3) return launch_state_tc<48, IO>(mq, mk, mv, prm, stream);
             return launch_state_tc<64, IO>(mq, mk, mv, prm, stream);
@@ -1323,7 +1326,7 @@ static cudaError_t run_pass1(const CUtensorMap& mq, const CUtensorMap& mk,
 cudaError_t launch_prefill(const void* q, const void* k, const void* v, const float* log_alpha,
                            const float* beta, const float* S0, const int32_t* cu_seqlens, int N,
                            int T, int H_qk, int H_v, bool bf16, void* o, float* S_final,
-                           void* workspace, int P, bool tc, cudaStream_t stream) {
+                           void* workspace, int P, int state_pass, cudaStream_t stream) {
     if (T == 0) {  // every sequence is empty: S_final = S0 (or zeros)
         if (!S_final) return cudaSuccess;
         copy_state_kernel<<<592, 256, 0, stream>>>(S0, S_final, (size_t)N * H_v * D * D / 4);
@@ -1359,8 +1362,8 @@ cudaError_t launch_prefill(const void* q, const void* k, const void* v, const fl
         const PrefillParams prm{log_alpha, beta, S0,      cu_seqlens, o, S_final,
                                 records,   nullptr, H_qk, H_v,        N, T};
         if ((e = run_pass1(mq, mk, prm, stream)) != cudaSuccess) return e;
-        return bf16 ? run_pass2<__nv_bfloat16, P2_OUT>(mq, mk, mv, prm, sms, stream, tc)
-                    : run_pass2<float, P2_OUT>(mq, mk, mv, prm, sms, stream, tc);
+        return bf16 ? run_pass2<__nv_bfloat16, P2_OUT>(mq, mk, mv, prm, sms, stream, state_pass)
+                    : run_pass2<float, P2_OUT>(mq, mk, mv, prm, sms, stream, state_pass);
     }
     // segmented: N P virtual sequences
     const int Nv = N * P;
@@ -1393,8 +1396,8 @@ cudaError_t launch_prefill(const void* q, const void* k, const void* v, const fl
     // phase C: every segment from its entering state, writing the outputs
     const PrefillParams pc{log_alpha, beta, S_entry, cu_v, o, nullptr, records, nullptr,
                            H_qk,      H_v,  Nv,      T};
-    return bf16 ? run_pass2<__nv_bfloat16, P2_OUT>(mq, mk, mv, pc, sms, stream, tc)
-                : run_pass2<float, P2_OUT>(mq, mk, mv, pc, sms, stream, tc);
+    return bf16 ? run_pass2<__nv_bfloat16, P2_OUT>(mq, mk, mv, pc, sms, stream, state_pass)
+                : run_pass2<float, P2_OUT>(mq, mk, mv, pc, sms, stream, state_pass);
 }
 
 // The forward pass the gradients start from (bf16 q, k, v): every chunk's

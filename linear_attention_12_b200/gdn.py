@@ -35,6 +35,10 @@ SIGNATURES = {
                                _c.c_int32, _c.c_int32, _c.c_int32, _c.c_int, _c.c_void_p,
                                _c.c_void_p, _c.c_void_p, _c.c_size_t, _c.c_void_p]),
     "gdn_prefill_workspace_size": (_c.c_size_t, [_c.c_int32] * 6 + [_c.c_int]),
+    "gdn_prefill_mma": (_c.c_int, [_c.c_void_p, _c.c_void_p, _c.c_void_p, _c.c_void_p, _c.c_void_p,
+                                   _c.c_void_p, _c.c_void_p, _c.c_int32, _c.c_int32, _c.c_int32,
+                                   _c.c_int32, _c.c_int32, _c.c_int32, _c.c_int, _c.c_void_p,
+                                   _c.c_void_p, _c.c_void_p, _c.c_size_t, _c.c_void_p]),
     "gdn_prefill_tc": (_c.c_int, [_c.c_void_p, _c.c_void_p, _c.c_void_p, _c.c_void_p, _c.c_void_p,
                                   _c.c_void_p, _c.c_void_p, _c.c_int32, _c.c_int32, _c.c_int32,
                                   _c.c_int32, _c.c_int32, _c.c_int32, _c.c_int, _c.c_void_p,
@@ -149,14 +153,14 @@ def auto_segments(N, T, H_qk, H_v) -> int:
 
 
 def prefill(q, k, v, log_alpha, beta, S0=None, cu_seqlens=None, *, o=None, S_final=None,
-            want_state=True, workspace=None, segments=None, tcgen05=False, stream=None):
+            want_state=True, workspace=None, segments=None, state_pass="auto", stream=None):
     """Chunked prefill.  Returns ``(o, S_final)`` (``S_final`` None if not wanted).
 
     ``segments``: None or 0 lets the library split long sequences when that
     fills more SMs; 1 disables the split; 2 .. 64 forces that many pieces per
-    sequence (gdn_prefill_segmented).  ``tcgen05=True`` runs the output state
-    pass on the fifth-generation tensor cores (gdn_prefill_tc; automatic
-    segments only)."""
+    sequence (gdn_prefill_segmented).  ``state_pass``: "auto" (the library's
+    choice per slice width), "tcgen05" (gdn_prefill_tc) or "mma_sync"
+    (gdn_prefill_mma); the last two take the automatic segment choice only."""
     T, H_qk, dk = q.shape
     H_v, dv = v.shape[1], v.shape[2]
     dt = q.dtype
@@ -184,20 +188,23 @@ def prefill(q, k, v, log_alpha, beta, S0=None, cu_seqlens=None, *, o=None, S_fin
     if need and workspace is None:
         workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
     wbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
-    if tcgen05:
+    if state_pass not in ("auto", "tcgen05", "mma_sync"):
+        raise ValueError(f"state_pass: 'auto', 'tcgen05' or 'mma_sync', not {state_pass!r}")
+    if state_pass != "auto":
         if seg != 0:
-            raise ValueError("tcgen05=True takes the automatic segment choice only")
-        st = lib().gdn_prefill_tc(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta),
-                                  _ptr(S0), _ptr(cu_seqlens), N, T, H_qk, H_v, dk, dv, io,
-                                  _ptr(o), _ptr(S_final), _ptr(workspace), wbytes,
-                                  _stream_handle(stream))
+            raise ValueError("a fixed state_pass takes the automatic segment choice only")
+        fn = lib().gdn_prefill_tc if state_pass == "tcgen05" else lib().gdn_prefill_mma
+        st = fn(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _ptr(S0),
+                _ptr(cu_seqlens), N, T, H_qk, H_v, dk, dv, io, _ptr(o), _ptr(S_final),
+                _ptr(workspace), wbytes, _stream_handle(stream))
     else:
         st = lib().gdn_prefill_segmented(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta),
                                          _ptr(S0), _ptr(cu_seqlens), N, T, H_qk, H_v, dk, dv, io,
                                          _ptr(o), _ptr(S_final), seg, _ptr(workspace), wbytes,
                                          _stream_handle(stream))
     if st != GDN_OK:
-        raise GDNError(st, "gdn_prefill_tc" if tcgen05 else "gdn_prefill_segmented")
+        raise GDNError(st, {"auto": "gdn_prefill_segmented", "tcgen05": "gdn_prefill_tc",
+                            "mma_sync": "gdn_prefill_mma"}[state_pass])
     return o, S_final
 
 

@@ -1,6 +1,7 @@
 """GPU parity of gdn_prefill_tc -- the prefill with its output state pass on
-the fifth-generation tensor cores -- against the fp64 oracle, through the C
-ABI.  The cases reach all three slice widths of the pass (32, 48 and 64
+the fifth-generation tensor cores at every slice width -- and of
+gdn_prefill_mma (the same pass on mma.sync, which gdn_prefill does not pick at
+48-column slices) against the fp64 oracle, through the C ABI.  The cases reach all three slice widths of the pass (32, 48 and 64
 columns: the width follows the number of (sequence, value head) units),
 ragged and empty sequences, partial chunks, fp32 I/O, long-memory gates and
 the segmented prefill, whose last phase also runs this pass."""
@@ -18,7 +19,7 @@ pytestmark = pytest.mark.gpu
 def _tc(case):
     c = to_cuda(case)
     o, S = gdn.prefill(c["q"], c["k"], c["v"], c["log_alpha"], c["beta"], S0=c["S0"],
-                       cu_seqlens=c["cu_seqlens"], tcgen05=True)
+                       cu_seqlens=c["cu_seqlens"], state_pass="tcgen05")
     torch.cuda.synchronize()
     assert gdn.last_device_error() == gdn.GDN_OK
     return o, S
@@ -79,3 +80,22 @@ def test_tc_equals_default_within_rounding():
     o1, S1 = _tc(case)
     assert o_err(o1, o0.float().cpu().double().numpy()) <= O_TOL
     assert s_err(S1, S0.cpu().double().numpy()) <= S_TOL
+
+
+@pytest.mark.parametrize("lens,H_qk,H_v", [([300] * 8, 2, 6), ([4096], 16, 48)])
+def test_mma_pass_at_48_column_slices(lens, H_qk, H_v):
+    # 48 units: gdn_prefill takes the tcgen05 pass here; the mma.sync one stays checked
+    case = inputs.make_prefill("mma48", lens, H_qk, H_v, seed=17, s0=True)
+    c = to_cuda(case)
+    o, S = gdn.prefill(c["q"], c["k"], c["v"], c["log_alpha"], c["beta"], S0=c["S0"],
+                       cu_seqlens=c["cu_seqlens"], state_pass="mma_sync")
+    torch.cuda.synchronize()
+    assert gdn.last_device_error() == gdn.GDN_OK
+    heads = None if H_v <= 6 else [0, 25, 47]
+    o_ref, S_ref = oracle.prefill(case.q, case.k, case.v, case.log_alpha, case.beta, S0=case.S0,
+                                  cu_seqlens=case.cu_seqlens, heads=heads)
+    if heads is None:
+        assert o_err(o, o_ref) <= O_TOL and s_err(S, S_ref) <= S_TOL
+    else:
+        assert o_err(o[:, heads], o_ref[:, heads]) <= O_TOL
+        assert s_err(S[:, heads], S_ref[:, heads]) <= S_TOL
