@@ -362,11 +362,7 @@ def run_backward(args, case, dev, stream, world, L):
     o, Sf = torch.empty_like(v), torch.empty((1, H_V, D, D), dtype=torch.float32, device=dev)
 
     def train_fwd():
-        st = gdn.lib().gdn_prefill_train(
-            gdn._ptr(q), gdn._ptr(k), gdn._ptr(v), gdn._ptr(la), gdn._ptr(be), None, gdn._ptr(cu),
-            1, L, H_QK, H_V, D, D, gdn.GDN_BF16, gdn._ptr(o), gdn._ptr(Sf), gdn._ptr(ws),
-            ws.numel(), gdn._stream_handle(None))
-        assert st == gdn.GDN_OK
+        gdn.prefill_train(q, k, v, la, be, cu_seqlens=cu, o=o, S_final=Sf, workspace=ws)
 
     def train_bwd():
         gdn.prefill_backward(q, k, v, la, be, dO, cu_seqlens=cu, workspace=ws, saved=True)

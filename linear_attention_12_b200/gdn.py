@@ -240,8 +240,8 @@ def backward_workspace(q, v, cu_seqlens=None):
     return torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
 
 
-def prefill_train(q, k, v, log_alpha, beta, S0=None, cu_seqlens=None, *, workspace=None,
-                  stream=None):
+def prefill_train(q, k, v, log_alpha, beta, S0=None, cu_seqlens=None, *, o=None, S_final=None,
+                  workspace=None, stream=None):
     """The prefill of a training step (gdn_prefill_train): returns ``(o, S_final,
     workspace)``, the workspace holding what ``prefill_backward(..., saved=True)``
     reads for the same inputs."""
@@ -259,8 +259,12 @@ def prefill_train(q, k, v, log_alpha, beta, S0=None, cu_seqlens=None, *, workspa
     N = cu_seqlens.numel() - 1
     if S0 is not None:
         _check(S0, "S0", torch.float32, (N, H_v, dk_, dv_))
-    o = torch.empty((T, H_v, dv_), dtype=dt, device=q.device)
-    S_final = torch.empty((N, H_v, dk_, dv_), dtype=torch.float32, device=q.device)
+    if o is None:
+        o = torch.empty((T, H_v, dv_), dtype=dt, device=q.device)
+    _check(o, "o", dt, (T, H_v, dv_))
+    if S_final is None:
+        S_final = torch.empty((N, H_v, dk_, dv_), dtype=torch.float32, device=q.device)
+    _check(S_final, "S_final", torch.float32, (N, H_v, dk_, dv_))
     if workspace is None:
         workspace = backward_workspace(q, v, cu_seqlens)
     wbytes = workspace.numel() * workspace.element_size()
