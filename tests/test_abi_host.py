@@ -90,6 +90,21 @@ def test_prefill_rejects_bad_arguments_on_host(L, kw, expect):
     assert _prefill(L, **kw) == expect
 
 
+@pytest.mark.parametrize("entry", ["gdn_prefill_tc", "gdn_prefill_mma"])
+@pytest.mark.parametrize("kw,expect", [
+    (dict(q=None), gdn.GDN_ERR_INVALID_ARG),
+    (dict(H_qk=3, H_v=4), gdn.GDN_ERR_INVALID_ARG),
+    (dict(dk=64, dv=64), gdn.GDN_ERR_UNSUPPORTED),
+    (dict(wsb=16), gdn.GDN_ERR_WORKSPACE),
+    (dict(), gdn.GDN_ERR_CUDA),  # host checks pass; no device here
+])
+def test_fixed_state_pass_entries_check_like_the_prefill(L, entry, kw, expect):
+    a = dict(q=P, k=P, v=P, la=P, be=P, S0=None, cu=P, N=1, T=64, H_qk=1, H_v=1, dk=128,
+             dv=128, dt=gdn.GDN_BF16, o=P, Sf=None, ws=P, wsb=1 << 40, stream=None)
+    a.update(kw)
+    assert getattr(L, entry)(*a.values()) == expect
+
+
 def _prefill_seg(L, segments, **kw):
     a = dict(q=P, k=P, v=P, la=P, be=P, S0=None, cu=P, N=1, T=4096, H_qk=1, H_v=1, dk=128,
              dv=128, dt=gdn.GDN_BF16, o=P, Sf=None, ws=P, wsb=1 << 40, stream=None)
