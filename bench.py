@@ -828,8 +828,9 @@ def main():
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer measurement")
     ap.add_argument("--no-frontend", action="store_true", help="skip the front-end measurement")
     ap.add_argument("--no-backward", action="store_true", help="skip the gradient measurement")
-    ap.add_argument("--no-tc", action="store_true",
-                    help="skip the prefill with the mma.sync state pass (the comparison leg)")
+    ap.add_argument("--no-alt", "--no-tc", dest="no_tc", action="store_true",
+                    help="skip the comparison leg: the prefill through the state pass the "
+                         "library does not pick at this shape (mma.sync)")
     ap.add_argument("--no-shard", action="store_true",
                     help="skip the tensor-parallel-shard prefill measurement")
     args = ap.parse_args()
