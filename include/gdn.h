@@ -212,11 +212,16 @@ GDN_API int32_t gdn_prefill_auto_segments(int32_t N, int32_t T, int32_t H_qk, in
  * (which may synchronise the device or fail on a fragmented heap) is not
  * allowed.  This entry point takes the same arguments as gdn_prefill minus the
  * workspace and allocates nothing: the scratch it needs (what
- * gdn_prefill_workspace_size reports for the same sizes) lives in a fixed device array
- * inside the library, of gdn_prefill_noalloc_max_scratch_bytes() bytes
- * (16 MiB), which every GPU that loads the library holds until the process
- * exits.  Calls whose scratch would exceed it return GDN_ERR_WORKSPACE and
- * launch nothing; use gdn_prefill with a caller-owned workspace instead.
+ * gdn_prefill_workspace_size reports for the same sizes: the chunk-operator
+ * records, 16,912 bytes per chunk and value head, plus bf16 copies of fp32
+ * q, k, v) lives in a fixed device array inside the library, of
+ * gdn_prefill_noalloc_max_scratch_bytes() bytes (16 MiB), which every GPU that
+ * loads the library holds until the process exits.  When the automatic split
+ * of long sequences (gdn_prefill_auto_segments) would need more scratch than
+ * that, the call runs the prefill unsplit (gdn_prefill_segmented with
+ * segments = 1, the least scratch; same results, fewer SMs busy).  Calls whose
+ * scratch would still exceed the array return GDN_ERR_WORKSPACE and launch
+ * nothing; use gdn_prefill with a caller-owned workspace instead.
  *
  * The first call on each device looks up the array's device address
  * (cudaGetSymbolAddress, with that device current); make that first call

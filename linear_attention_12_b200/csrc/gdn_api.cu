@@ -259,14 +259,22 @@ gdn_status gdn_prefill_noalloc(const void* q, const void* k, const void* v,
                                        dk, dv, io_dtype, o, S_final);
     if (st != GDN_OK) return st;
     // The scratch this call needs is the workspace gdn_prefill would take; it
-    // comes from the library's fixed device array instead of the caller.
-    const size_t need = gdn_prefill_workspace_size(N, T, H_qk, H_v, dk, dv, io_dtype);
-    if (need > gdn::noalloc_scratch_bytes()) return GDN_ERR_WORKSPACE;
+    // comes from the library's fixed device array instead of the caller.  When
+    // the automatic split of the sequences needs more than the array holds, the
+    // unsplit prefill (one piece per sequence, the least scratch) runs instead.
+    const size_t cap = gdn::noalloc_scratch_bytes();
+    int32_t segments = 0;
+    size_t need = gdn_prefill_workspace_size(N, T, H_qk, H_v, dk, dv, io_dtype);
+    if (need > cap) {
+        segments = 1;
+        need = gdn_prefill_segmented_workspace_size(N, T, H_qk, H_v, dk, dv, io_dtype, 1);
+        if (need > cap) return GDN_ERR_WORKSPACE;
+    }
     void* scratch = nullptr;
     if (need > 0 && gdn::noalloc_scratch_address(&scratch) != cudaSuccess) return GDN_ERR_CUDA;
-    return gdn_prefill(q, k, v, log_alpha, beta, S0, cu_seqlens, N, T, H_qk, H_v, dk, dv,
-                       io_dtype, o, S_final, scratch, need > 0 ? gdn::noalloc_scratch_bytes() : 0,
-                       stream);
+    return gdn_prefill_segmented(q, k, v, log_alpha, beta, S0, cu_seqlens, N, T, H_qk, H_v, dk,
+                                 dv, io_dtype, o, S_final, segments, scratch,
+                                 need > 0 ? cap : 0, stream);
 }
 
 size_t gdn_prefill_noalloc_max_scratch_bytes(void) { return gdn::noalloc_scratch_bytes(); }
