@@ -54,6 +54,10 @@ STATE_BYTES = H_V * D * D * 4                                                 # 
 # (three triangular C x C x d products at half) + 2 C d / 3 (grams at half,
 # shared by the 3 V heads of a QK head), C = 64.
 FLOP_PER_TOKEN = H_V * (6 * D * D + 3 * 64 * D + (2 * 64 * D) // 3)
+# B200 HBM3e bandwidth as specified (HGX), beside the measured copy peak
+HBM_SPEC_GBS = 7700.0
+
+
 def dec_bytes(B):
     """One decode step: the fp32 states read and written, plus the tokens."""
     return 2 * B * H_V * D * D * 4 + B * (2 * H_QK * D * 2 + 2 * H_V * D * 2 + 2 * H_V * 4)
@@ -485,6 +489,64 @@ def run_e2e(args, case, cu, ws, stream, world, L):
     return world * L / (e2e_ms / 1e3), e2e_ms, h2d, d2h
 
 
+def run_prefill_workload(args, case, dev, stream, world):
+    """Time gdn_prefill on one workload (inputs resident in HBM, workspace
+    allocated outside the timing); returns ms per call (max over ranks)."""
+    import torch
+    from linear_attention_12_b200 import gdn
+    q, k, v = case.q.to(dev), case.k.to(dev), case.v.to(dev)
+    la, be = case.log_alpha.to(dev), case.beta.to(dev)
+    S0 = None if case.S0 is None else case.S0.to(dev)
+    cu = case.cu_seqlens.to(dev)
+    o = torch.empty((case.T, H_V, D), dtype=torch.bfloat16, device=dev)
+    Sf = torch.empty((case.N, H_V, D, D), dtype=torch.float32, device=dev)
+    ws = torch.empty(gdn.workspace_size(case.N, case.T, H_QK, H_V, D, gdn.GDN_BF16),
+                     dtype=torch.uint8, device=dev)
+
+    def step():
+        gdn.prefill(q, k, v, la, be, S0, cu, o=o, S_final=Sf, workspace=ws)
+
+    n = max(3, min(args.steps, 10))
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    barrier(world)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(n):
+        step()
+    b.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    assert gdn.last_device_error() == gdn.GDN_OK
+    ms = max_over_ranks(a.elapsed_time(b), world) / n
+    del q, k, v, la, be, S0, o, Sf, ws
+    torch.cuda.empty_cache()
+    return ms, n
+
+
+def prefill_workload_line(case, ms, steps, hbm_peak, tf_peak, workload, cpu):
+    """Throughput and roofline of one prefill workload (bf16 q/k/v, o; fp32 gates,
+    states): bytes = the tokens' algorithmic bytes + S0 (if given) + S_final."""
+    T, N = case.T, case.N
+    nbytes = BYTES_PER_TOKEN * T + (2 if case.S0 is not None else 1) * N * STATE_BYTES
+    flops = FLOP_PER_TOKEN * T
+    t_hbm = nbytes / (hbm_peak * 1e9)
+    t_tc = flops / (tf_peak * 1e12)
+    gbs = nbytes / (ms / 1e3) / 1e9
+    line = {
+        "value": T / (ms / 1e3), "unit": "tokens/s", "ms_per_call": ms, "tokens": T,
+        "sequences": N, "workload": workload, "steps": steps,
+        "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm_peak, "unit": "GB/s",
+                     "frac": gbs / hbm_peak, "bytes_per_call": nbytes,
+                     "roofline_us": max(t_hbm, t_tc) * 1e6, "hbm_term_us": t_hbm * 1e6,
+                     "tensor_term_us": t_tc * 1e6},
+    }
+    if cpu is not None:
+        line["cpu_baseline"] = cpu
+    return line
+
+
 def traffic_from_profile(L):
     """DRAM bytes per prefill launch from the committed ncu summary, if it was
     taken on the current kernel source; else None."""
@@ -598,6 +660,31 @@ def run_ours(args):
     if not args.no_shard:
         shard = run_prefill_shard(args, dev, stream, world, L)
 
+    # ---------------- the other prefill workloads: packed varlen batch with S0, and
+    # the long-context prefill (each timed alone; inputs resident)
+    varlen = long_ctx = None
+    if not args.no_workloads:
+        vcase = inputs.varlen_8seq()
+        ms, n = run_prefill_workload(args, vcase, dev, stream, world)
+        vcpu = None
+        if world == 1 and not args.no_cpu_baseline:
+            vcpu = cpu_baseline(vcase, args.cpu_tokens)
+        varlen = prefill_workload_line(
+            vcase, ms, n, hbm_peak, tf_peak,
+            f"packed varlen prefill: {vcase.N} sequences, lengths uniform in [1024, 8192] "
+            f"(T={vcase.T}), H_qk={H_QK} H_v={H_V} d={D} bf16, S0 ~ N(0, 0.02^2)", vcpu)
+        del vcase
+        lcase = inputs.long_256k(args.long_len)
+        ms, n = run_prefill_workload(args, lcase, dev, stream, world)
+        lcpu = None
+        if world == 1 and not args.no_cpu_baseline:
+            lcpu = cpu_baseline(lcase, args.cpu_tokens)
+        long_ctx = prefill_workload_line(
+            lcase, ms, n, hbm_peak, tf_peak,
+            f"long-context prefill B=1 L={lcase.T} H_qk={H_QK} H_v={H_V} d={D} bf16, "
+            "long-memory gates log_alpha = -softplus(N(-2, 1)), S0 = 0", lcpu)
+        del lcase
+
     # ---------------- front end on raw inputs of the same shape
     fe_ms = fe_gbs = None
     if not args.no_frontend:
@@ -610,9 +697,11 @@ def run_ours(args):
         e2e_value, e2e_ms, h2d, d2h = run_e2e(args, case, cu, ws, stream, world, L)
 
     # ---------------- CPU baseline (the oracle as it stands), rank 0 at N=1 only
-    cpu = None
+    cpu = dec_cpu = None
     if world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(case, args.cpu_baseline_tokens)
+        if not args.no_decode:
+            dec_cpu = decode_cpu_baseline(args.decode_batch, args.cpu_decode_seqs)
     if rank == 0:
         line = {
             "metric": METRIC,
@@ -641,6 +730,7 @@ def run_ours(args):
                 "peak": hbm_peak,
                 "unit": "GB/s",
                 "frac": achieved_gbs / hbm_peak,
+                "frac_of_spec": achieved_gbs / HBM_SPEC_GBS,
                 "traffic": traffic_from_profile(L),
                 "peak_source": peak_src,
                 "kernel": "prefill path: chunk_ops_kernel + state_tc_kernel (tcgen05)",
@@ -669,10 +759,16 @@ def run_ours(args):
                 "bytes_per_step": dec_bytes(args.decode_batch),
                 "peak": hbm_peak,
                 "frac": dec_gbs / hbm_peak,
+                "frac_of_copy_peak": dec_gbs / hbm_peak,
+                "frac_of_spec": dec_gbs / HBM_SPEC_GBS,
+                "spec_gbs": HBM_SPEC_GBS,
                 "workload": f"decode B={args.decode_batch} H_qk={H_QK} H_v={H_V} d={D}, "
                             "fp32 state in place",
                 "steps": max(args.steps, 20),
+                **({"cpu_baseline": dec_cpu} if dec_cpu is not None else {}),
             },
+            "prefill_varlen": varlen,
+            "prefill_long": long_ctx,
             "decode_multi": None if dm_gbs is None else {
                 "value": dm_gbs,
                 "unit": "GB/s",
@@ -753,17 +849,38 @@ def run_ours(args):
 
 
 def cpu_baseline(case, tokens):
-    """The fp64 oracle on all 48 V heads of the first ``tokens`` tokens."""
+    """The fp64 oracle on all 48 V heads of the first ``tokens`` tokens of the
+    first sequence (from its S0 when the workload has one)."""
     import oracle
-    T = min(tokens, case.T)
+    T = min(tokens, int(case.cu_seqlens[1]))
     n_threads = oracle.default_threads()
     args = (case.q[:T], case.k[:T], case.v[:T], case.log_alpha[:T], case.beta[:T])
+    S0 = None if case.S0 is None else case.S0[:1]
     t0 = time.perf_counter()
-    oracle.prefill(*args, want_o=True, n_threads=n_threads)
+    oracle.prefill(*args, S0=S0, want_o=True, n_threads=n_threads)
     dt = time.perf_counter() - t0
     return {"value": T / dt, "unit": "tokens/s", "cores": min(n_threads, H_V),
             "kind": "oracle",
-            "sample": f"first {T} of {case.T} tokens, all {H_V} V heads, fp64, {dt:.1f} s"}
+            "sample": f"first {T} tokens of sequence 0 (of {case.T} tokens in {case.N} "
+                      f"sequences), all {H_V} V heads, fp64, {dt:.1f} s"}
+
+
+def decode_cpu_baseline(B, seqs):
+    """The fp64 oracle's decode step on the first ``seqs`` sequences of the decode
+    batch (all 48 V heads), scaled to GB/s by the same algorithmic bytes."""
+    import oracle
+    from linear_attention_12_b200 import inputs
+    dc = inputs.make_decode(B, H_QK, H_V, D, seed=4)
+    n = min(seqs, B)
+    q, k, v, la, be = (x[:n] for x in dc.step(0))
+    n_threads = oracle.default_threads()
+    t0 = time.perf_counter()
+    oracle.decode_step(q, k, v, la, be, dc.S0[:n], n_threads=n_threads)
+    dt = time.perf_counter() - t0
+    return {"value": dec_bytes(n) / dt / 1e9, "unit": "GB/s", "cores": n_threads,
+            "kind": "oracle", "us_per_step_sample": dt * 1e6,
+            "sample": f"one step of the first {n} of {B} sequences, all {H_V} V heads, fp64, "
+                      f"{dt:.2f} s"}
 
 
 def run_reference(args):
@@ -831,6 +948,12 @@ def main():
     ap.add_argument("--no-alt", "--no-tc", dest="no_tc", action="store_true",
                     help="skip the comparison leg: the prefill through the state pass the "
                          "library does not pick at this shape (mma.sync)")
+    ap.add_argument("--no-workloads", action="store_true",
+                    help="skip the packed-varlen and long-context prefill workloads")
+    ap.add_argument("--long-len", type=int, default=262144,
+                    help="length of the long-context prefill workload (262144)")
+    ap.add_argument("--cpu-decode-seqs", type=int, default=16,
+                    help="sequences of the decode batch in the decode cpu_baseline sample")
     ap.add_argument("--no-shard", action="store_true",
                     help="skip the tensor-parallel-shard prefill measurement")
     args = ap.parse_args()
