@@ -4,6 +4,9 @@ The bar (bf16 q/k/v, fp32 gates and state) is
     max|o_gpu - o_ref| / max|o_ref|                <= 1e-2
     ||S_gpu - S_ref||_F / ||S_ref||_F               <= 1e-2
 """
+import json
+import os
+
 import numpy as np
 import torch
 
@@ -33,3 +36,25 @@ def to_cuda(case):
     return dict(q=case.q.to(d), k=case.k.to(d), v=case.v.to(d), log_alpha=case.log_alpha.to(d),
                 beta=case.beta.to(d), S0=None if case.S0 is None else case.S0.to(d),
                 cu_seqlens=case.cu_seqlens.to(d))
+
+
+def record(test, workload, **errors):
+    """Append one line of measured errors to the file named by GDN_PARITY_LOG
+    (if set), so that a GPU run leaves a table of its parity margins."""
+    path = os.environ.get("GDN_PARITY_LOG")
+    if not path:
+        return
+    with open(path, "a") as f:
+        f.write(json.dumps({"test": test, "workload": workload, **errors}) + "\n")
+
+
+def per_head_o(o_gpu, o_ref, heads):
+    """Worst o error of each listed value head (o is [T, H_v, d])."""
+    a = o_gpu.float().cpu().double().numpy() if isinstance(o_gpu, torch.Tensor) else o_gpu
+    return {int(h): o_err(a[:, h], np.asarray(o_ref)[:, h]) for h in heads}
+
+
+def per_head_s(S_gpu, S_ref, heads):
+    """Relative Frobenius S error of each listed value head (S is [N, H_v, d, d])."""
+    a = S_gpu.cpu().double().numpy() if isinstance(S_gpu, torch.Tensor) else S_gpu
+    return {int(h): s_err(a[:, h], np.asarray(S_ref)[:, h]) for h in heads}

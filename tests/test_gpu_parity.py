@@ -11,7 +11,8 @@ import torch
 
 import oracle
 from linear_attention_12_b200 import gdn, inputs
-from tests.gpu_util import O_TOL, S_TOL, o_err, s_err, to_cuda
+from tests.gpu_util import (O_TOL, S_TOL, o_err, per_head_o, per_head_s, record, s_err,
+                            to_cuda)
 
 pytestmark = pytest.mark.gpu
 
@@ -67,9 +68,12 @@ def test_decode_batched_256_full_512_steps_sampled():
         o_ref, S_ref = oracle.decode_step(q, k, v, la, be, S_ref, units_bh=pairs)
         og = o.float().cpu().numpy()
         worst_o = max(worst_o, o_err(np.stack([og[b, h] for b, h in pairs]), o_ref))
-    assert worst_o <= O_TOL
     Sg = S.cpu().double().numpy()
-    assert s_err(np.stack([Sg[b, h] for b, h in pairs]), S_ref) <= S_TOL
+    se = s_err(np.stack([Sg[b, h] for b, h in pairs]), S_ref)
+    record("decode_batched_256", "config 4: decode 256 x 16/48 heads, 512 steps", o_err=worst_o,
+           s_err=se, units="24 sampled (sequence, head) units")
+    assert worst_o <= O_TOL
+    assert se <= S_TOL
 
 
 # ------------------------------------------------------------------ prefill, small
@@ -78,8 +82,10 @@ def test_prefill_tiny_fp32_L256():
     case = inputs.tiny_fp32()
     o, S, o_ref, S_ref = _run_case(case)
     assert o.dtype == torch.float32
-    assert o_err(o, o_ref) <= O_TOL
-    assert s_err(S, S_ref) <= S_TOL
+    oe, se = o_err(o, o_ref), s_err(S, S_ref)
+    record("prefill_tiny_fp32_L256", "config 0: L=256, 1/1 heads, fp32", o_err=oe, s_err=se)
+    assert oe <= O_TOL
+    assert se <= S_TOL
 
 
 @pytest.mark.parametrize("lens", [[1], [63], [64], [65], [200], [17, 64, 1, 0, 130], [0]])
@@ -180,8 +186,11 @@ def test_prefill_qwen_32k_sampled_heads():
     case = inputs.qwen_prefill_32k()
     heads = [0, 25, 47]
     o, S, o_ref, S_ref = _run_case(case, heads=heads)
-    assert o_err(o[:, heads], o_ref[:, heads]) <= O_TOL
-    assert s_err(S[:, heads], S_ref[:, heads]) <= S_TOL
+    oe, se = o_err(o[:, heads], o_ref[:, heads]), s_err(S[:, heads], S_ref[:, heads])
+    record("prefill_qwen_32k", "config 1: L=32768, 16/48 heads", o_err=oe, s_err=se,
+           o_per_head=per_head_o(o, o_ref, heads), s_per_head=per_head_s(S, S_ref, heads))
+    assert oe <= O_TOL
+    assert se <= S_TOL
     assert torch.isfinite(o.float()).all()
 
 
@@ -189,8 +198,11 @@ def test_prefill_varlen_8seq_sampled_heads():
     case = inputs.varlen_8seq()
     heads = [5, 40]
     o, S, o_ref, S_ref = _run_case(case, heads=heads)
-    assert o_err(o[:, heads], o_ref[:, heads]) <= O_TOL
-    assert s_err(S[:, heads], S_ref[:, heads]) <= S_TOL
+    oe, se = o_err(o[:, heads], o_ref[:, heads]), s_err(S[:, heads], S_ref[:, heads])
+    record("prefill_varlen_8seq", "config 2: 8 packed sequences, S0 != 0", o_err=oe, s_err=se,
+           o_per_head=per_head_o(o, o_ref, heads), s_per_head=per_head_s(S, S_ref, heads))
+    assert oe <= O_TOL
+    assert se <= S_TOL
 
 
 @pytest.mark.slow
@@ -199,5 +211,23 @@ def test_prefill_long_256k_final_state_sampled_heads():
     case = inputs.long_256k()
     heads = [7, 31]
     o, S, o_ref, S_ref = _run_case(case, heads=heads, want_o=False)
-    assert s_err(S[:, heads], S_ref[:, heads]) <= S_TOL
+    se = s_err(S[:, heads], S_ref[:, heads])
+    record("prefill_long_256k", "config 3: L=262144, long-memory gates", s_err=se,
+           s_per_head=per_head_s(S, S_ref, heads))
+    assert se <= S_TOL
     assert torch.isfinite(o.float()).all()
+
+
+def test_prefill_long_memory_gates_bench_layout_sampled_heads():
+    """Gates that remember across many chunks (log_alpha = -softplus(N(-6, 1)),
+    alpha ~ 0.9975 per token) at the benchmark's head layout (16/48 heads,
+    48-column slices of the state), 8192 tokens: o and S on sampled heads."""
+    case = inputs.make_prefill("longmem_bench_layout", [8192], 16, 48, seed=12, alpha_mu=-6.0)
+    heads = [1, 22, 46]
+    o, S, o_ref, S_ref = _run_case(case, heads=heads)
+    oe, se = o_err(o[:, heads], o_ref[:, heads]), s_err(S[:, heads], S_ref[:, heads])
+    record("prefill_longmem_bench_layout", "L=8192, 16/48 heads, log_alpha=-softplus(N(-6,1))",
+           o_err=oe, s_err=se, o_per_head=per_head_o(o, o_ref, heads),
+           s_per_head=per_head_s(S, S_ref, heads))
+    assert oe <= O_TOL
+    assert se <= S_TOL
