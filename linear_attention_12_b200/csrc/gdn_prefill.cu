@@ -1,10 +1,8 @@
 // gdn_prefill.cu -- chunked GDN prefill (sm_100a) in two kernels: a fully
 // parallel pass over all chunks that computes each chunk's state-independent
 // operators, and a sequential pass that carries the state through the chunks.
-// Both use TMA / bulk copies into 128-byte-swizzled shared-memory tiles and
-// warp-level bf16 tensor-core products (ldmatrix + mma.sync m16n8k16, fp32
-// accumulate); the triangular solve runs in fp32 (tf32 tensor-core block
-// products); the state stays in registers for the whole sequence.
+// Both stage their tiles with TMA / bulk copies into 128-byte-swizzled shared
+// memory.
 //
 // Operation: the gated delta rule of the bjdmk.com.cn article (section 2.1,
 // state-update formula) over packed sequences, with readout o_t = S_t^T q_t.
@@ -24,19 +22,21 @@
 // (Delta equals U - W S of the WY form with U = T_b V and W = T_b diag(gamma) K.)
 //
 // Pass 1, chunk_ops_kernel: one CTA per (chunk, query/key head).  Both grams
-// K K^T and Q K^T (lower 16x16 blocks only) are computed once and shared by
-// the value heads of that query/key head; per value head the CTA builds the
-// masks, solves for T and writes one "chunk operator" record to the
-// workspace: T_b and M o Q K^T as 128-byte-swizzled bf16 tiles plus gamma, d
-// and gamma_C.  A record is written by one bulk copy and read by one.
+// K K^T and Q K^T come from one tcgen05 product [K; Q] K^T accumulated in
+// tensor memory and are shared by the value heads of that query/key head; per
+// value head the CTA builds the masks (running products of the gates), solves
+// for T (fp32 forward substitution on the diagonal 16 x 16 blocks, tf32
+// tensor-core block products for the rest) and writes one "chunk operator"
+// record to the workspace: T_b and M o Q K^T as 128-byte-swizzled bf16 tiles
+// plus gamma, d and gamma_C.  A record is written by one bulk copy.
 //
-// Pass 2, state_pass_kernel: one CTA per (sequence, value head, d_v slice of
-// NS columns); the columns of S evolve independently, so slices need no
-// communication.  Eight warps each own 16 rows of S as fp32 mma accumulators;
-// warps 0-3 compute K S and Q S (one pass over S) and the output rows; all
-// eight compute Delta and update the state.  One thread streams each chunk's K, Q, V tiles and
-// operator record into a 3-stage ring, refilling a stage as soon as the chain
-// releases it.
+// Pass 2 (the prefill's outputs): one CTA per (sequence, value head, d_v slice
+// of NS columns); the columns of S evolve independently, so slices need no
+// communication.  state_tc_kernel runs the products on the fifth-generation
+// tensor cores with the accumulators in tensor memory (the 48-column slices of
+// the 16/48-head workload); state_pass_kernel runs them as warp-level mma.sync
+// with the state in registers (other slice widths, the segmented prefill's
+// first phase and the gradients' forward).
 //
 // Every mbarrier wait is bounded (gdn_common.cuh); every named barrier inside
 // the chunk loop also votes on whether all of its threads are still healthy,
@@ -57,23 +57,11 @@ namespace gdn {
 namespace {
 
 constexpr int kMaxSegments = 16;  // most segments per sequence the automatic choice takes
-// ---- pass 1 shared memory ----
-constexpr int P1_THREADS = 256;
-constexpr int P1_MAX_GROUP = 4;                                // value heads per work item
-constexpr int AF_LD = 68;                                      // fp32 row stride of A and T
-constexpr uint32_t P1_K = 0;                                   // K, 64 x 128 (two halves)
-constexpr uint32_t P1_Q = 2 * HALF;                            // Q
-constexpr uint32_t P1_AF = 0;                                  // after the grams: A, fp32 64 x 68
-constexpr uint32_t P1_TF = 64 * AF_LD * 4;                     //                  T, fp32 64 x 68
-constexpr uint32_t P1_REC = ((2 * 64 * AF_LD * 4 + 1023) / 1024) * 1024;  // one record
-constexpr uint32_t P1_REC_STRIDE = 17408;                      // REC_BYTES rounded to 1 KB
-constexpr uint32_t P1_XS = P1_REC + P1_REC_STRIDE;             // 256 floats per warp (warps 0-3)
-constexpr uint32_t P1_VEC = P1_XS + 4 * 256 * 4;               // per value head: g[64], beta[64]
-constexpr uint32_t P1_BAR = P1_VEC + P1_MAX_GROUP * 128 * 4;
-constexpr uint32_t P1_MISC = P1_BAR + 8;
-constexpr uint32_t P1_SMEM = P1_MISC + 16 + 1024;
-static_assert(P1_REC_STRIDE >= REC_BYTES && P1_REC >= 4 * HALF, "pass 1 layout");
-static_assert(3 * (P1_SMEM + 1024) <= 233472, "three pass-1 CTAs per SM");
+// ---- pass 1 ----
+constexpr int P1_MAX_GROUP = 4;       // value heads per work item
+constexpr int AF_LD = 68;             // fp32 row stride of A and T (conflict-free row writes)
+constexpr uint32_t P1_REC_STRIDE = 17408;  // REC_BYTES rounded up to 1 KB
+static_assert(P1_REC_STRIDE >= REC_BYTES, "record staging");
 
 // ---- pass 2 shared memory ----
 constexpr int NSTAGE = 3;
@@ -112,25 +100,146 @@ struct PrefillParams {
 
 // ============================================================================
 // Pass 1: chunk operators.  Grid (record slots, H_qk, batches of up to 4 value
-// heads of that head); three CTAs per SM.  A and T reuse the K and Q tiles'
-// shared memory once the grams are in registers.
+// heads of that head); 128 threads, four CTAs per SM.  The grams come from one
+// tcgen05 product [K; Q] K^T (M = 128, N = 64, K = 128) accumulated in tensor
+// memory: TMEM lane r holds row r of K K^T (r < 64) or of Q K^T (r >= 64), and
+// thread r reads it into registers.  Per value head the masks are applied in
+// registers, T = (I + A)^{-1} is solved in fp32 on the CUDA cores (diagonal
+// 16 x 16 blocks by forward substitution, then the off-diagonal blocks from
+// block products), and the record is bulk-stored.  Once the grams are in
+// registers the K and Q tiles' shared memory holds A and T.
 // ============================================================================
-__global__ void __launch_bounds__(P1_THREADS, 3)
+constexpr int CO_THREADS = 128;
+constexpr uint32_t CO_KQ = 0;                       // [K h0 | Q h0 | K h1 | Q h1], 32 KB
+constexpr uint32_t CO_AF = 0;                       // after the grams: A, fp32 64 x AF_LD
+constexpr uint32_t CO_TF = 64 * AF_LD * 4;          //                  T, fp32 64 x AF_LD
+constexpr uint32_t CO_REC = ((2 * 64 * AF_LD * 4 + 1023) / 1024) * 1024;  // record staging
+constexpr uint32_t CO_XS = CO_REC + REC_TB;         // block-product scratch, in T_b's bytes
+constexpr uint32_t CO_VEC = CO_REC + ((REC_BYTES + 15) / 16) * 16;  // per value head:
+                                                    // g[64] (log2), beta[64], alpha[64]
+constexpr int CO_VEC_FLOATS = 192;
+constexpr uint32_t CO_BAR = CO_VEC + P1_MAX_GROUP * CO_VEC_FLOATS * 4;  // K/Q copies, grams
+constexpr uint32_t CO_MISC = CO_BAR + 16;           // abort flag, TMEM base
+constexpr uint32_t CO_SMEM = CO_MISC + 16 + 1024;
+constexpr uint32_t CO_TM_COLS = 64;
+static_assert(CO_REC >= 4 * HALF && CO_TF + 64 * AF_LD * 4 <= CO_REC, "pass 1 layout");
+static_assert(4 * 256 * 4 <= HALF, "block-product scratch fits in the T_b tile's bytes");
+static_assert(4 * (CO_SMEM + 1024) <= 233472, "four pass-1 CTAs per SM");
+
+// tf32 rounding of an fp32 value, kept as fp32 (the low mantissa bits cleared)
+__device__ __forceinline__ float tf32r(float x) { return __uint_as_float(to_tf32(x)); }
+// mma_tf32 for operands already rounded to tf32 in shared memory (no conversions)
+__device__ __forceinline__ void mma_tf32_pre(float* d, const float* A, int lda, const float* B,
+                                             int ldb, int lane) {
+    const int g = lane >> 2, t = lane & 3;
+    const uint32_t a0 = __float_as_uint(A[g * lda + t]), a1 = __float_as_uint(A[(g + 8) * lda + t]);
+    const uint32_t a2 = __float_as_uint(A[g * lda + t + 4]);
+    const uint32_t a3 = __float_as_uint(A[(g + 8) * lda + t + 4]);
+    const uint32_t b0 = __float_as_uint(B[t * ldb + g]), b1 = __float_as_uint(B[(t + 4) * ldb + g]);
+    asm volatile(
+        "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 "
+        "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// T = (I + A)^{-1} for the strictly lower 64 x 64 A in Af (row stride AF_LD),
+// into the lower 16 x 16 blocks of Tf (the diagonal blocks with their zeros
+// above the diagonal; the blocks above the diagonal are not written).  All
+// CO_THREADS threads (four warps) take part; Xs is scratch (256 floats per warp).
+// The diagonal blocks come from fp32 forward substitution, the off-diagonal
+// ones from tf32 tensor-core block products:
+//   T_10 = -T_11 (A_10 T_00),  T_32 = -T_33 (A_32 T_22),  T_ba = -T_bb (A_ba T_aa)
+// (a = rows/columns 0..31, b = 32..63).  A, the diagonal blocks, the level-1
+// blocks and the scratch hold tf32-rounded values (the block products read them
+// as they are).
+__device__ __forceinline__ void solve_unit_lower(const float* Af, float* Tf, float* Xs, int tid) {
+    const int warp = tid >> 5, lane = tid & 31, g = lane >> 2, t4 = lane & 3;
+    if (tid < 64) {  // diagonal blocks: thread (b, cc) solves column cc of block b
+        const int b = tid >> 4, cc = tid & 15;
+        const float* Ab = Af + (16 * b) * AF_LD + 16 * b;
+        float x[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) x[i] = (i == cc) ? 1.f : 0.f;
+#pragma unroll
+        for (int jj = 0; jj < 15; ++jj) {
+            const float xj = x[jj];
+#pragma unroll
+            for (int i = jj + 1; i < 16; ++i) x[i] = fmaf(-Ab[i * AF_LD + jj], xj, x[i]);
+        }
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+            Tf[(16 * b + i) * AF_LD + 16 * b + cc] = __uint_as_float(to_tf32(x[i]));
+    }
+    __syncthreads();
+    float* xw = Xs + warp * 256;
+    {  // level 1: warp = (block, n-tile)
+        const int blk = warp >> 1, nt = warp & 1, bi = 1 + 2 * blk, bj = 2 * blk;
+        float d[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int ks = 0; ks < 2; ++ks)
+            mma_tf32_pre(d, Af + (16 * bi) * AF_LD + 16 * bj + 8 * ks, AF_LD,
+                     Tf + (16 * bj + 8 * ks) * AF_LD + 16 * bj + 8 * nt, AF_LD, lane);
+        *reinterpret_cast<float2*>(xw + g * 8 + 2 * t4) = make_float2(tf32r(d[0]), tf32r(d[1]));
+        *reinterpret_cast<float2*>(xw + (g + 8) * 8 + 2 * t4) = make_float2(tf32r(d[2]), tf32r(d[3]));
+        __syncwarp();
+        float e[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int ks = 0; ks < 2; ++ks)
+            mma_tf32_pre(e, Tf + (16 * bi) * AF_LD + 16 * bi + 8 * ks, AF_LD, xw + 8 * ks * 8, 8, lane);
+        float* to = Tf + (16 * bi) * AF_LD + 16 * bj + 8 * nt + 2 * t4;
+        *reinterpret_cast<float2*>(to + g * AF_LD) = make_float2(tf32r(-e[0]), tf32r(-e[1]));
+        *reinterpret_cast<float2*>(to + (g + 8) * AF_LD) = make_float2(tf32r(-e[2]), tf32r(-e[3]));
+    }
+    __syncthreads();
+    {  // level 2: warp qn owns n-tile qn of both m-tiles; T_aa's and T_bb's blocks
+       // above the diagonal are zero (T_aa's upper-right block is skipped)
+        const int qn = warp;
+        float x0[4] = {0.f, 0.f, 0.f, 0.f}, x1[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int ks = 0; ks < 4; ++ks)
+            if (qn < 2 || ks >= 2) {
+                mma_tf32_pre(x0, Af + 32 * AF_LD + 8 * ks, AF_LD, Tf + (8 * ks) * AF_LD + 8 * qn,
+                         AF_LD, lane);
+                mma_tf32_pre(x1, Af + 48 * AF_LD + 8 * ks, AF_LD, Tf + (8 * ks) * AF_LD + 8 * qn,
+                         AF_LD, lane);
+            }
+        *reinterpret_cast<float2*>(xw + g * 8 + 2 * t4) = make_float2(tf32r(x0[0]), tf32r(x0[1]));
+        *reinterpret_cast<float2*>(xw + (g + 8) * 8 + 2 * t4) = make_float2(tf32r(x0[2]), tf32r(x0[3]));
+        *reinterpret_cast<float2*>(xw + (g + 16) * 8 + 2 * t4) = make_float2(tf32r(x1[0]), tf32r(x1[1]));
+        *reinterpret_cast<float2*>(xw + (g + 24) * 8 + 2 * t4) = make_float2(tf32r(x1[2]), tf32r(x1[3]));
+        __syncwarp();
+        float y0[4] = {0.f, 0.f, 0.f, 0.f}, y1[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int ks = 0; ks < 4; ++ks) {
+            if (ks < 2) mma_tf32_pre(y0, Tf + 32 * AF_LD + 32 + 8 * ks, AF_LD, xw + 8 * ks * 8, 8, lane);
+            mma_tf32_pre(y1, Tf + 48 * AF_LD + 32 + 8 * ks, AF_LD, xw + 8 * ks * 8, 8, lane);
+        }
+        float* to = Tf + 32 * AF_LD + 8 * qn + 2 * t4;
+        *reinterpret_cast<float2*>(to + g * AF_LD) = make_float2(-y0[0], -y0[1]);
+        *reinterpret_cast<float2*>(to + (g + 8) * AF_LD) = make_float2(-y0[2], -y0[3]);
+        *reinterpret_cast<float2*>(to + (g + 16) * AF_LD) = make_float2(-y1[0], -y1[1]);
+        *reinterpret_cast<float2*>(to + (g + 24) * AF_LD) = make_float2(-y1[2], -y1[3]);
+    }
+    __syncthreads();
+}
+
+__global__ void __launch_bounds__(CO_THREADS, 4)
     chunk_ops_kernel(const __grid_constant__ CUtensorMap map_q,
                      const __grid_constant__ CUtensorMap map_k, const PrefillParams p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
     const uint32_t sb = smem_u32(sm);
-    uint64_t* bar = reinterpret_cast<uint64_t*>(sm + P1_BAR);
-    volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + P1_MISC);
-    float* Af = reinterpret_cast<float*>(sm + P1_AF);
-    float* Tf = reinterpret_cast<float*>(sm + P1_TF);
-    float* Xs = reinterpret_cast<float*>(sm + P1_XS);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(sm + CO_BAR);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + CO_MISC);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + CO_MISC + 4);
+    float* Af = reinterpret_cast<float*>(sm + CO_AF);
+    float* Tf = reinterpret_cast<float*>(sm + CO_TF);
+    float* Xs = reinterpret_cast<float*>(sm + CO_XS);
+    uint8_t* rec = sm + CO_REC;
 
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int g = lane >> 2, t4 = lane & 3;
-    const int pt = threadIdx.x;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     int n, c;
     slot_owner(p.cu_seqlens, p.N, blockIdx.x, n, c);
     if (n < 0) return;  // uniform across the CTA
@@ -143,21 +252,29 @@ __global__ void __launch_bounds__(P1_THREADS, 3)
     const int valid = min(C, t_end - t0);
     const long long slot = record_slot(n, t0);
 
-    if (pt == 0) {
-        mbar_init(bar, 1);
+    if (tid == 0) {
+        mbar_init(&bars[0], 1);
+        mbar_init(&bars[1], 1);
         *abort_flag = 0;
         fence_mbar_init();
     }
-    __syncthreads();
-    if (pt == 0) {
-        mbar_arrive_expect_tx(bar, 4 * HALF);
-        tma_load_2d(sm + P1_K, &map_k, hq * D, t0, bar);
-        tma_load_2d(sm + P1_K + HALF, &map_k, hq * D + 64, t0, bar);
-        tma_load_2d(sm + P1_Q, &map_q, hq * D, t0, bar);
-        tma_load_2d(sm + P1_Q + HALF, &map_q, hq * D + 64, t0, bar);
+    if (warp == 0) {
+        tmem_alloc(tmem_slot, CO_TM_COLS);
+        tmem_relinquish();
     }
-    // decay scan per value head: warp w < nheads handles head hv0 + w
-    // (lane l: tokens 2l, 2l+1); T's upper blocks are zeroed meanwhile
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    if (tid == 0) {
+        mbar_arrive_expect_tx(&bars[0], 4 * HALF);
+        tma_load_2d(sm + CO_KQ, &map_k, hq * D, t0, &bars[0]);
+        tma_load_2d(sm + CO_KQ + HALF, &map_q, hq * D, t0, &bars[0]);
+        tma_load_2d(sm + CO_KQ + 2 * HALF, &map_k, hq * D + 64, t0, &bars[0]);
+        tma_load_2d(sm + CO_KQ + 3 * HALF, &map_q, hq * D + 64, t0, &bars[0]);
+    }
+    // decay scan per value head while the copies land: warp w < nheads handles
+    // head hv0 + w (lane l: tokens 2l, 2l+1); gates past the sequence end are 0
     if (warp < nheads) {
         const int h = hv0 + warp;
         float la[2] = {0.f, 0.f}, be[2] = {0.f, 0.f};
@@ -174,218 +291,154 @@ __global__ void __launch_bounds__(P1_THREADS, 3)
             const float y = __shfl_up_sync(0xffffffffu, incl, off);
             if (lane >= off) incl += y;
         }
-        float* v = reinterpret_cast<float*>(sm + P1_VEC) + warp * 128;
+        float* v = reinterpret_cast<float*>(sm + CO_VEC) + warp * CO_VEC_FLOATS;
         *reinterpret_cast<float2*>(v + 2 * lane) = make_float2(incl - x1, incl);
         *reinterpret_cast<float2*>(v + 64 + 2 * lane) = make_float2(be[0], be[1]);
+        *reinterpret_cast<float2*>(v + 128 + 2 * lane) = make_float2(ex2(x0), ex2(x1));
     }
-    const bool ok = mbar_wait(bar, 0, abort_flag);
-    __syncwarp();
-    if (!__syncthreads_and(ok)) {
-        // the copy may still land: wait for it (bounded) before the CTA exits
-        if (pt == 0) mbar_wait_drain(bar, 0);
+    bool ok = mbar_wait(&bars[0], 0, abort_flag);
+    if (!__syncthreads_and(ok)) {  // the copies may still land: wait (bounded), then leave
+        if (tid == 0) mbar_wait_drain(&bars[0], 0);
         __syncthreads();
+        if (warp == 0) tmem_dealloc(tmem, CO_TM_COLS);
         return;
     }
-    if (valid < C) {  // zero K and Q rows past the end of the sequence
-        for (int i = pt; i < 4 * 64 * 8; i += P1_THREADS) {
-            const int tile = i / 512, row = (i >> 3) & 63, ch = i & 7;
-            if (row >= valid)
-                *reinterpret_cast<uint4*>(sm + tile * HALF + row * 128 + ch * 16) =
-                    make_uint4(0, 0, 0, 0);
-        }
-        __syncthreads();
-    }
-
-    // ---- grams, lower 16x16 blocks only.  Warp: type (0: K K^T, 1: Q K^T) and
-    // up to three blocks (bi, bj), sorted by bi.
-    const int gtype = warp & 1;
-    int nblk, bi0, bj0, bi1, bj1, bi2, bj2;
-    switch (warp >> 1) {
-        case 0: nblk = 2; bi0 = 3; bj0 = 0; bi1 = 3; bj1 = 1; bi2 = 3; bj2 = 1; break;
-        case 1: nblk = 2; bi0 = 3; bj0 = 2; bi1 = 3; bj1 = 3; bi2 = 3; bj2 = 3; break;
-        case 2: nblk = 3; bi0 = 2; bj0 = 0; bi1 = 2; bj1 = 1; bi2 = 2; bj2 = 2; break;
-        default: nblk = 3; bi0 = 1; bj0 = 0; bi1 = 1; bj1 = 1; bi2 = 0; bj2 = 0; break;
-    }
-    const int gbi[3] = {bi0, bi1, bi2};
-    const int gbj[3] = {bj0, bj1, bj2};
-    float acc[3][2][4];
-#pragma unroll
-    for (int b = 0; b < 3; ++b)
-#pragma unroll
-        for (int i = 0; i < 2; ++i)
-#pragma unroll
-            for (int e = 0; e < 4; ++e) acc[b][i][e] = 0.f;
-    {
-        const uint32_t abase = sb + (gtype ? P1_Q : P1_K);
+    // [K; Q] K^T: A = the 128 rows K h | Q h of each 64-column half (K-major),
+    // B = K (K-major, N = 64 tokens); k step ks reads 16 columns of half ks / 4
+    if (tid == 0) {
+        tc_fence_after();
+        constexpr uint32_t ID_G = idesc_bf16(128, 64, 0, 0);
 #pragma unroll
         for (int ks = 0; ks < 8; ++ks) {
-            uint32_t a[4];
-#pragma unroll
-            for (int b = 0; b < 3; ++b) {
-                if (b < nblk) {
-                    if (b == 0 || gbi[b] != gbi[b - 1])
-                        lda_k(abase, HALF, 16 * gbi[b], 16 * ks, lane, a);
-                    uint32_t bb[4];
-                    ldb_k(sb + P1_K, HALF, 16 * gbj[b], 16 * ks, lane, bb);
-                    mma16816(acc[b][0], a, bb[0], bb[1]);
-                    mma16816(acc[b][1], a, bb[2], bb[3]);
-                }
-            }
+            const uint32_t a = sb + CO_KQ + (ks >> 2) * 2 * HALF + (ks & 3) * 32;
+            mma_bf16_ss(tmem, sdesc_sw128(a, 16, 1024), sdesc_sw128(a, 16, 1024), ID_G, ks > 0);
         }
+        mma_commit(&bars[1]);
     }
-    // K and Q are dead: their space now holds A and T.  T's blocks above the
-    // diagonal are read as zeros by the solve and never written.
-    __syncthreads();
-    for (int i = pt; i < 64 * AF_LD / 4; i += P1_THREADS)
-        reinterpret_cast<float4*>(Tf)[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+    ok = mbar_wait(&bars[1], 0, abort_flag);
+    if (!__syncthreads_and(ok)) {
+        if (tid == 0) mbar_wait_drain(&bars[1], 0);
+        tc_fence_before();
+        __syncthreads();
+        if (warp == 0) {
+            tc_fence_after();
+            tmem_dealloc(tmem, CO_TM_COLS);
+        }
+        return;
+    }
+    tc_fence_after();
+    // The product is complete, so K and Q are no longer read: their bytes become A
+    // and T.  The grams stay in tensor memory; each value head reads its row again.
+    const bool qrow = tid >= 64;
+    const int r = tid & 63;
+    const bool rvalid = r < valid;
 
     for (int vh = 0; vh < nheads; ++vh) {
         const int h = hv0 + vh;
-        const float* s_g = reinterpret_cast<const float*>(sm + P1_VEC) + vh * 128;
+        const float* s_g = reinterpret_cast<const float*>(sm + CO_VEC) + vh * CO_VEC_FLOATS;
         const float* s_b = s_g + 64;
-        uint8_t* rec = sm + P1_REC;  // refilled per value head (see the store below)
-        // ---- masks: A -> Af (fp32), M o Q K^T -> the record (bf16)
+        const float* s_a = s_g + 128;  // alpha of each token
+        if (vh > 0) {  // the previous head's record has left the staging buffer
+            if (tid == 0) bulk_wait_read<0>();
+            __syncthreads();
+        }
+        // ---- row tid of [K; Q] K^T (TMEM lane tid): K K^T row r for tid < 64, Q K^T
+        // row r after; masks: A (fp32, strictly lower) from K K^T, M o Q K^T (bf16,
+        // lower incl. the diagonal) from Q K^T; rows past the sequence end are zero
+        float gr[64];
 #pragma unroll
-        for (int b = 0; b < 3; ++b) {
-            if (b < nblk) {
+        for (int i = 0; i < 4; ++i)
+            tmem_ld16(tmem + ((uint32_t)(32 * warp) << 16) + 16 * i, gr + 16 * i);
+        tmem_ld_wait();
+        // The decay mask M_rj = exp(g_r - g_j) = alpha_{j+1} ... alpha_r (j <= r) is a
+        // running product over j, from j = r down (one multiply per entry, never an
+        // exponential of a positive number).  Rows 0-31 (warps 0 and 2) have no entries
+        // right of column 31.
+        const bool upper_half = (warp & 1) == 0;
+        if (!qrow) {  // A = strict_lower(diag(beta) (M o K K^T)), rounded to tf32
+            const float b_r = rvalid ? s_b[r] : 0.f;
+            float* arow = Af + r * AF_LD;
+            float m = 1.f;
 #pragma unroll
-                for (int hl = 0; hl < 2; ++hl) {
-                    const int r = 16 * gbi[b] + g + 8 * hl;
-                    const float gr = s_g[r], br = s_b[r];
+            for (int j4 = 15; j4 >= 0; --j4) {
+                float a4[4] = {0.f, 0.f, 0.f, 0.f};
+                if (!(upper_half && j4 >= 8)) {
+                    const float4 al = *reinterpret_cast<const float4*>(s_a + 4 * j4);
+                    const float av[4] = {al.x, al.y, al.z, al.w};
+                    const float anext = (j4 < 15) ? s_a[4 * j4 + 4] : 1.f;
 #pragma unroll
-                    for (int nt = 0; nt < 2; ++nt) {
-                        const int j = 16 * gbj[b] + 8 * nt + 2 * t4;
-                        const float2 gj = *reinterpret_cast<const float2*>(s_g + j);
-                        const float x0 = acc[b][nt][2 * hl], x1 = acc[b][nt][2 * hl + 1];
-                        const float e0 = (j <= r) ? ex2(gr - gj.x) : 0.f;
-                        const float e1 = (j + 1 <= r) ? ex2(gr - gj.y) : 0.f;
-                        if (gtype == 0) {
-                            const float a0 = (j < r) ? br * e0 * x0 : 0.f;
-                            const float a1 = (j + 1 < r) ? br * e1 * x1 : 0.f;
-                            *reinterpret_cast<float2*>(Af + r * AF_LD + j) = make_float2(a0, a1);
-                        } else {
-                            *reinterpret_cast<uint32_t*>(rec + REC_MQ + taddr_e(0, r, j, 0)) =
-                                pack2(e0 * x0, e1 * x1);
-                        }
+                    for (int e = 3; e >= 0; --e) {
+                        const int j = 4 * j4 + e;
+                        const float a_j1 = (e < 3) ? av[e + 1] : anext;  // alpha_{j+1}
+                        m = (j < r) ? m * a_j1 : 1.f;
+                        a4[e] = (j < r) ? __uint_as_float(to_tf32(b_r * m * gr[j])) : 0.f;
                     }
                 }
+                *reinterpret_cast<float4*>(arow + 4 * j4) = make_float4(a4[0], a4[1], a4[2], a4[3]);
             }
-        }
-        __syncthreads();
-
-        // ---- T = (I + A)^{-1}, fp32.  Diagonal 16x16 blocks by forward substitution
-        // (thread = column cc of block b), then the off-diagonal blocks from tf32
-        // tensor-core block products:
-        //   T_10 = -T_11 (A_10 T_00),  T_32 = -T_33 (A_32 T_22),
-        //   T_ba = -T_bb (A_ba T_aa)   (a = rows/columns 0..31, b = 32..63)
-        if (pt < C) {
-            const int b = pt >> 4, cc = pt & 15;
-            const float* Ab = Af + (16 * b) * AF_LD + 16 * b;
-            float x[16];
+        } else {  // M o Q K^T, bf16, lower triangle with the diagonal
+            float m = 1.f;
 #pragma unroll
-            for (int i = 0; i < 16; ++i) x[i] = (i == cc) ? 1.f : 0.f;
+            for (int ch = 7; ch >= 0; --ch) {
+                float m8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+                if (rvalid && !(upper_half && ch >= 4)) {
+                    const float4 la4 = *reinterpret_cast<const float4*>(s_a + 8 * ch);
+                    const float4 lb4 = *reinterpret_cast<const float4*>(s_a + 8 * ch + 4);
+                    const float av[8] = {la4.x, la4.y, la4.z, la4.w, lb4.x, lb4.y, lb4.z, lb4.w};
+                    const float anext = (ch < 7) ? s_a[8 * ch + 8] : 1.f;
 #pragma unroll
-            for (int jj = 0; jj < 15; ++jj) {
-                const float xj = x[jj];
-#pragma unroll
-                for (int i = jj + 1; i < 16; ++i) x[i] = fmaf(-Ab[i * AF_LD + jj], xj, x[i]);
-            }
-#pragma unroll
-            for (int i = 0; i < 16; ++i) Tf[(16 * b + i) * AF_LD + 16 * b + cc] = x[i];
-        }
-        __syncthreads();
-        // Off-diagonal blocks from tf32 tensor-core block products (warps 0-3; the
-        // intermediate goes through a per-warp scratch to become an operand):
-        //   T_10 = -T_11 (A_10 T_00),  T_32 = -T_33 (A_32 T_22)   (one n-tile per warp)
-        float* xw = Xs + warp * 256;
-        if (warp < 4) {
-            const int blk = warp >> 1, nt = warp & 1, bi = 1 + 2 * blk, bj = 2 * blk;
-            float d[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-            for (int ks = 0; ks < 2; ++ks)
-                mma_tf32(d, Af + (16 * bi) * AF_LD + 16 * bj + 8 * ks, AF_LD,
-                         Tf + (16 * bj + 8 * ks) * AF_LD + 16 * bj + 8 * nt, AF_LD, lane);
-            *reinterpret_cast<float2*>(xw + g * 8 + 2 * t4) = make_float2(d[0], d[1]);
-            *reinterpret_cast<float2*>(xw + (g + 8) * 8 + 2 * t4) = make_float2(d[2], d[3]);
-            __syncwarp();
-            float e[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-            for (int ks = 0; ks < 2; ++ks)
-                mma_tf32(e, Tf + (16 * bi) * AF_LD + 16 * bi + 8 * ks, AF_LD, xw + 8 * ks * 8, 8,
-                         lane);
-            float* to = Tf + (16 * bi) * AF_LD + 16 * bj + 8 * nt + 2 * t4;
-            *reinterpret_cast<float2*>(to + g * AF_LD) = make_float2(-e[0], -e[1]);
-            *reinterpret_cast<float2*>(to + (g + 8) * AF_LD) = make_float2(-e[2], -e[3]);
-        }
-        __syncthreads();
-        //   T_ba = -T_bb (A_ba T_aa)  (a = rows/columns 0..31, b = 32..63): warp qn owns
-        //   n-tile qn of both m-tiles; T_aa's and T_bb's upper-right blocks are zero
-        if (warp < 4) {
-            const int qn = warp;
-            float x0[4] = {0.f, 0.f, 0.f, 0.f}, x1[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-            for (int ks = 0; ks < 4; ++ks)
-                if (qn < 2 || ks >= 2) {
-                    mma_tf32(x0, Af + 32 * AF_LD + 8 * ks, AF_LD, Tf + (8 * ks) * AF_LD + 8 * qn,
-                             AF_LD, lane);
-                    mma_tf32(x1, Af + 48 * AF_LD + 8 * ks, AF_LD, Tf + (8 * ks) * AF_LD + 8 * qn,
-                             AF_LD, lane);
+                    for (int e = 7; e >= 0; --e) {
+                        const int j = 8 * ch + e;
+                        const float a_j1 = (e < 7) ? av[e + 1] : anext;
+                        m = (j < r) ? m * a_j1 : 1.f;
+                        m8[e] = (j <= r) ? m * gr[j] : 0.f;
+                    }
                 }
-            *reinterpret_cast<float2*>(xw + g * 8 + 2 * t4) = make_float2(x0[0], x0[1]);
-            *reinterpret_cast<float2*>(xw + (g + 8) * 8 + 2 * t4) = make_float2(x0[2], x0[3]);
-            *reinterpret_cast<float2*>(xw + (g + 16) * 8 + 2 * t4) = make_float2(x1[0], x1[1]);
-            *reinterpret_cast<float2*>(xw + (g + 24) * 8 + 2 * t4) = make_float2(x1[2], x1[3]);
-            __syncwarp();
-            float y0[4] = {0.f, 0.f, 0.f, 0.f}, y1[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-            for (int ks = 0; ks < 4; ++ks) {
-                if (ks < 2)
-                    mma_tf32(y0, Tf + 32 * AF_LD + 32 + 8 * ks, AF_LD, xw + 8 * ks * 8, 8, lane);
-                mma_tf32(y1, Tf + 48 * AF_LD + 32 + 8 * ks, AF_LD, xw + 8 * ks * 8, 8, lane);
+                *reinterpret_cast<uint4*>(rec + REC_MQ + taddr(0, r, 8 * ch, 0)) =
+                    make_uint4(pack2(m8[0], m8[1]), pack2(m8[2], m8[3]), pack2(m8[4], m8[5]),
+                               pack2(m8[6], m8[7]));
             }
-            float* to = Tf + 32 * AF_LD + 8 * qn + 2 * t4;
-            *reinterpret_cast<float2*>(to + g * AF_LD) = make_float2(-y0[0], -y0[1]);
-            *reinterpret_cast<float2*>(to + (g + 8) * AF_LD) = make_float2(-y0[2], -y0[3]);
-            *reinterpret_cast<float2*>(to + (g + 16) * AF_LD) = make_float2(-y1[0], -y1[1]);
-            *reinterpret_cast<float2*>(to + (g + 24) * AF_LD) = make_float2(-y1[2], -y1[3]);
         }
         __syncthreads();
-        // ---- T diag(beta) as a bf16 tile.  The 16 x 16 blocks above the diagonal of
-        // it and of M o Q K^T are written as zeros, so that every byte of the record
-        // is defined (the gradients read both tiles whole).
-        for (int idx = pt; idx < 64 * 8; idx += P1_THREADS) {
-            const int r = idx >> 3, ch = idx & 7;
-            if ((ch >> 1) > (r >> 4)) {
-                *reinterpret_cast<uint4*>(rec + REC_TB + taddr(0, r, 8 * ch, 0)) = make_uint4(0, 0, 0, 0);
-                *reinterpret_cast<uint4*>(rec + REC_MQ + taddr(0, r, 8 * ch, 0)) = make_uint4(0, 0, 0, 0);
-            } else {
-                const float4 t0v = *reinterpret_cast<const float4*>(Tf + r * AF_LD + 8 * ch);
-                const float4 t1v = *reinterpret_cast<const float4*>(Tf + r * AF_LD + 8 * ch + 4);
+        solve_unit_lower(Af, Tf, Xs, tid);
+        // ---- T diag(beta) as a bf16 tile; its 16 x 16 blocks above the diagonal are
+        // written as zeros so that every byte of the record is defined
+        for (int idx = tid; idx < 64 * 8; idx += CO_THREADS) {
+            const int rr = idx >> 3, ch = idx & 7;
+            uint4 w = make_uint4(0, 0, 0, 0);
+            if ((ch >> 1) <= (rr >> 4)) {
+                const float4 ta = *reinterpret_cast<const float4*>(Tf + rr * AF_LD + 8 * ch);
+                const float4 tb = *reinterpret_cast<const float4*>(Tf + rr * AF_LD + 8 * ch + 4);
                 const float4 b0 = *reinterpret_cast<const float4*>(s_b + 8 * ch);
                 const float4 b1 = *reinterpret_cast<const float4*>(s_b + 8 * ch + 4);
-                *reinterpret_cast<uint4*>(rec + REC_TB + taddr(0, r, 8 * ch, 0)) = make_uint4(
-                    pack2(t0v.x * b0.x, t0v.y * b0.y), pack2(t0v.z * b0.z, t0v.w * b0.w),
-                    pack2(t1v.x * b1.x, t1v.y * b1.y), pack2(t1v.z * b1.z, t1v.w * b1.w));
+                w = make_uint4(pack2(ta.x * b0.x, ta.y * b0.y), pack2(ta.z * b0.z, ta.w * b0.w),
+                               pack2(tb.x * b1.x, tb.y * b1.y), pack2(tb.z * b1.z, tb.w * b1.w));
             }
+            *reinterpret_cast<uint4*>(rec + REC_TB + taddr(0, rr, 8 * ch, 0)) = w;
         }
-        // gamma_r, d_r (zero past the sequence end) and gamma_C
-        if (pt < C) {
+        // gamma_r, d_r (zero past the sequence end), gamma_C, zero padding
+        if (tid < C) {
             float* rv = reinterpret_cast<float*>(rec + REC_VEC);
-            const float gr = s_g[pt], gC = s_g[C - 1];
-            rv[pt] = ex2(gr);
-            rv[64 + pt] = (pt < valid) ? ex2(gC - gr) : 0.f;
-            if (pt == 0) rv[128] = ex2(gC);
+            const float gC = s_g[C - 1];
+            const float g_t = s_g[tid];
+            rv[tid] = ex2(g_t);
+            rv[64 + tid] = (tid < valid) ? ex2(gC - g_t) : 0.f;
+            if (tid < REC_VEC_FLOATS - 128) rv[128 + tid] = (tid == 0) ? ex2(gC) : 0.f;
         }
         fence_proxy_async_smem();  // generic writes, read next by the bulk copy
         __syncthreads();
-        if (pt == 0) {
+        if (tid == 0) {
             bulk_store(p.records + (size_t)(slot * p.H_v + h) * REC_BYTES, rec, REC_BYTES);
             bulk_commit();
-            bulk_wait_read<0>();  // the record buffer is refilled by the next value head
         }
-        __syncthreads();
     }
-    if (pt == 0) bulk_wait_all();
+    if (tid == 0) bulk_wait_read<0>();  // the staging buffer is read before the CTA exits
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, CO_TM_COLS);
+    }
 }
 
 
@@ -1201,9 +1254,11 @@ size_t record_bytes(int N, int T, int H_v) {
 }  // namespace
 
 // ---- scratch for gdn_prefill_noalloc -------------------------------------
-// A file-scope device array that stands in for the caller's workspace (the bf16
-// copies of fp32 q, k, v).  Every GPU that loads the library holds it until the
-// process exits.  Its host-side name is not a device address: the address is
+// A file-scope device array that stands in for the caller's workspace: the
+// chunk-operator records (REC_BYTES per chunk slot and value head) and, for
+// fp32 q, k, v, their bf16 copies; with a split of the sequences also the
+// pieces' starts and states.  Every GPU that loads the library holds it until
+// the process exits.  Its host-side name is not a device address: the address is
 // obtained once per device with cudaGetSymbolAddress, with that device current.
 constexpr size_t kNoAllocScratchBytes = size_t(16) << 20;  // 16 MiB
 static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];
@@ -1297,9 +1352,9 @@ static cudaError_t run_pass2(const CUtensorMap& mq, const CUtensorMap& mk, const
     const long long units = (long long)prm.N * prm.H_v * (MODE == P2_SEGMENT ? 2 : 1);
     const int slices = pass2_slices(units, sms);
     if constexpr (MODE == P2_OUT) {
-        // the tcgen05 pass where it measured faster (48-column slices: 1.31-1.32 vs
-        // 1.32-1.34 ms at 16/48 heads and 32K tokens), mma.sync at the other widths
-        // (32-column slices: 0.95 vs 0.82 ms on a 2/6-head shard)
+        // the tcgen05 pass at 48-column slices (the 16/48-head workload, where it
+        // measured faster), mma.sync at the other widths (32-column slices: 0.82 vs
+        // 0.95 ms on a 2/6-head shard)
         if (state_pass == STATE_PASS_TC || (state_pass == STATE_PASS_AUTO && slices == 3)) {
             if (slices == 4) return launch_state_tc<32, IO>(mq, mk, mv, prm, stream);
             if (slices == 3) return launch_state_tc<48, IO>(mq, mk, mv, prm, stream);
@@ -1314,12 +1369,12 @@ static cudaError_t run_pass2(const CUtensorMap& mq, const CUtensorMap& mk, const
 static cudaError_t run_pass1(const CUtensorMap& mq, const CUtensorMap& mk,
                              const PrefillParams& prm, cudaStream_t stream) {
     cudaError_t e =
-        cudaFuncSetAttribute(chunk_ops_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, P1_SMEM);
+        cudaFuncSetAttribute(chunk_ops_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, CO_SMEM);
     if (e != cudaSuccess) return e;
     const int group = prm.H_v / prm.H_qk;
     const long long slots = (long long)prm.N + ((long long)prm.T + C - 1) / C;
     dim3 grid((unsigned)slots, prm.H_qk, (group + P1_MAX_GROUP - 1) / P1_MAX_GROUP);
-    chunk_ops_kernel<<<grid, P1_THREADS, P1_SMEM, stream>>>(mq, mk, prm);
+    chunk_ops_kernel<<<grid, CO_THREADS, CO_SMEM, stream>>>(mq, mk, prm);
     return cudaGetLastError();
 }
 
