@@ -23,12 +23,13 @@
 //
 // Pass 1, chunk_ops_kernel: one CTA per (chunk, query/key head).  Both grams
 // K K^T and Q K^T come from one tcgen05 product [K; Q] K^T accumulated in
-// tensor memory and are shared by the value heads of that query/key head; per
-// value head the CTA builds the masks (running products of the gates), solves
-// for T (fp32 forward substitution on the diagonal 16 x 16 blocks, tf32
-// tensor-core block products for the rest) and writes one "chunk operator"
-// record to the workspace: T_b and M o Q K^T as 128-byte-swizzled bf16 tiles
-// plus gamma, d and gamma_C.  A record is written by one bulk copy.
+// tensor memory and are shared by the value heads of that query/key head.  Per
+// value head two "solver" warps build A (the masks factor per 16-column block,
+// so each entry left of the diagonal block costs two multiplies) and solve for
+// T (fp32 forward substitution on the diagonal 16 x 16 blocks, tf32
+// tensor-core block products for the rest), while two "writer" warps store
+// M o Q K^T, then T diag(beta), as 128-byte-swizzled bf16 tiles of one "chunk
+// operator" record together with gamma, d and gamma_C, straight from registers.
 //
 // Pass 2 (the prefill's outputs): one CTA per (sequence, value head, d_v slice
 // of NS columns); the columns of S evolve independently, so slices need no
@@ -60,8 +61,6 @@ constexpr int kMaxSegments = 16;  // most segments per sequence the automatic ch
 // ---- pass 1 ----
 constexpr int P1_MAX_GROUP = 4;       // value heads per work item
 constexpr int AF_LD = 68;             // fp32 row stride of A and T (conflict-free row writes)
-constexpr uint32_t P1_REC_STRIDE = 17408;  // REC_BYTES rounded up to 1 KB
-static_assert(P1_REC_STRIDE >= REC_BYTES, "record staging");
 
 // ---- pass 2 shared memory ----
 constexpr int NSTAGE = 3;
@@ -100,131 +99,336 @@ struct PrefillParams {
 
 // ============================================================================
 // Pass 1: chunk operators.  Grid (record slots, H_qk, batches of up to 4 value
-// heads of that head); 128 threads, four CTAs per SM.  The grams come from one
+// heads of that head); 128 threads, five CTAs per SM.  The grams come from one
 // tcgen05 product [K; Q] K^T (M = 128, N = 64, K = 128) accumulated in tensor
-// memory: TMEM lane r holds row r of K K^T (r < 64) or of Q K^T (r >= 64), and
-// thread r reads it into registers.  Per value head the masks are applied in
-// registers, T = (I + A)^{-1} is solved in fp32 on the CUDA cores (diagonal
-// 16 x 16 blocks by forward substitution, then the off-diagonal blocks from
-// block products), and the record is bulk-stored.  Once the grams are in
-// registers the K and Q tiles' shared memory holds A and T.
+// memory: TMEM lane r holds row r of K K^T (r < 64) or of Q K^T (r >= 64).
+// Warps 0-1 (the
+// solvers) read the K K^T rows, build A and solve for T = (I + A)^{-1} in fp32
+// shared memory; warps 2-3 (the writers) read the Q K^T rows, store M o Q K^T
+// and the gate vectors of the record, then store T diag(beta) once the solvers
+// have finished T.  The solvers start the next value head's A while the
+// writers store the previous head's T_b.  Records go to global memory straight
+// from registers.  Once the grams are complete the K and Q tiles' shared memory
+// holds A and T.
 // ============================================================================
 constexpr int CO_THREADS = 128;
 constexpr uint32_t CO_KQ = 0;                       // [K h0 | Q h0 | K h1 | Q h1], 32 KB
 constexpr uint32_t CO_AF = 0;                       // after the grams: A, fp32 64 x AF_LD
 constexpr uint32_t CO_TF = 64 * AF_LD * 4;          //                  T, fp32 64 x AF_LD
-constexpr uint32_t CO_REC = ((2 * 64 * AF_LD * 4 + 1023) / 1024) * 1024;  // record staging
-constexpr uint32_t CO_XS = CO_REC + REC_TB;         // block-product scratch, in T_b's bytes
-constexpr uint32_t CO_VEC = CO_REC + ((REC_BYTES + 15) / 16) * 16;  // per value head:
-                                                    // g[64] (log2), beta[64], alpha[64]
+constexpr uint32_t CO_XS = 2 * 64 * AF_LD * 4;      // block-product scratch per solver warp
+constexpr int CO_XS_FLOATS = 16 * 36;
+constexpr uint32_t CO_VEC = CO_XS + 2 * CO_XS_FLOATS * 4;  // per value head: g[64] (log2), beta[64],
+                                                    // w[64] = exp2(g_{16J+15} - g_j), J = j / 16
 constexpr int CO_VEC_FLOATS = 192;
 constexpr uint32_t CO_BAR = CO_VEC + P1_MAX_GROUP * CO_VEC_FLOATS * 4;  // K/Q copies, grams
 constexpr uint32_t CO_MISC = CO_BAR + 16;           // abort flag, TMEM base
 constexpr uint32_t CO_SMEM = CO_MISC + 16 + 1024;
 constexpr uint32_t CO_TM_COLS = 64;
-static_assert(CO_REC >= 4 * HALF && CO_TF + 64 * AF_LD * 4 <= CO_REC, "pass 1 layout");
-static_assert(4 * 256 * 4 <= HALF, "block-product scratch fits in the T_b tile's bytes");
-static_assert(4 * (CO_SMEM + 1024) <= 233472, "four pass-1 CTAs per SM");
+static_assert(CO_XS >= 4 * HALF, "the K and Q tiles lie inside A and T");
+static_assert(5 * (CO_SMEM + 1024) <= 233472, "five pass-1 CTAs per SM");
+// named barriers of pass 1 (0 is __syncthreads)
+constexpr int CO_BAR_SOLVE = 1;  // the two solver warps
+constexpr int CO_BAR_TDONE = 2;  // solvers -> writers: T is complete
+constexpr int CO_BAR_TFREE = 3;  // writers -> solvers: T has been read
+
+template <int ID, int N>
+__device__ __forceinline__ void bar_arrive() {
+    asm volatile("bar.arrive %0, %1;" ::"n"(ID), "n"(N) : "memory");
+}
 
 // tf32 rounding of an fp32 value, kept as fp32 (the low mantissa bits cleared)
 __device__ __forceinline__ float tf32r(float x) { return __uint_as_float(to_tf32(x)); }
-// mma_tf32 for operands already rounded to tf32 in shared memory (no conversions)
-__device__ __forceinline__ void mma_tf32_pre(float* d, const float* A, int lda, const float* B,
-                                             int ldb, int lane) {
-    const int g = lane >> 2, t = lane & 3;
-    const uint32_t a0 = __float_as_uint(A[g * lda + t]), a1 = __float_as_uint(A[(g + 8) * lda + t]);
-    const uint32_t a2 = __float_as_uint(A[g * lda + t + 4]);
-    const uint32_t a3 = __float_as_uint(A[(g + 8) * lda + t + 4]);
-    const uint32_t b0 = __float_as_uint(B[t * ldb + g]), b1 = __float_as_uint(B[(t + 4) * ldb + g]);
+// The decay mask M_rj = exp2(g_r - g_j) (j <= r, g in log2 units) of a row r in
+// 16-row block R.  Left of the diagonal block (column block J < R) it factors as
+// exp2(g_r - g_e) * w_j with g_e = g_{16J+15} and w_j = exp2(g_e - g_j): both
+// factors are at most 1, so nothing overflows whatever the gates, and the row
+// pays one exponential per block.  In the diagonal block each entry takes its
+// own exponential of g_r - g_j <= 0.
+//
+// Row r = 32 W + lane of A = strict_lower(diag(beta) (M o K K^T)), rounded to
+// tf32, into Af: the blocks left of the diagonal block and the diagonal block
+// (zeros on and above the diagonal).  Blocks right of it are never read.
+// tm_row addresses row r of K K^T in tensor memory, read one 16-column block at
+// a time; lanes 16-31 lie in row block 2W + 1, lanes 0-15 in 2W.
+template <int W>
+__device__ __forceinline__ void build_a(float* Af, uint32_t tm_row, const float* s_g,
+                                        const float* s_b, const float* s_w, int lane) {
+    const int r = 32 * W + lane;
+    const bool hi = lane >= 16;
+    const float g_r = s_g[r], b_r = s_b[r];
+    float* arow = Af + r * AF_LD;
+    float gA[16], gB[16];  // gram columns 16 J .. 16 J + 15 of row r
+#pragma unroll
+    for (int J = 0; J <= 2 * W; ++J) {
+        tmem_ld16(tm_row + 16 * J, gA);
+        if (J == 2 * W) tmem_ld16(tm_row + 16 * J + 16, gB);
+        tmem_ld_wait();
+        if (J < 2 * W || hi) {
+            const float s = b_r * ex2(g_r - s_g[16 * J + 15]);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const float4 w4 = *reinterpret_cast<const float4*>(s_w + 16 * J + 4 * q);
+                const float* gq = gA + 4 * q;
+                *reinterpret_cast<float4*>(arow + 16 * J + 4 * q) =
+                    make_float4(tf32r(gq[0] * w4.x * s), tf32r(gq[1] * w4.y * s),
+                                tf32r(gq[2] * w4.z * s), tf32r(gq[3] * w4.w * s));
+            }
+        }
+    }
+    const int jb = 32 * W + (hi ? 16 : 0);  // the diagonal block's first column
+    const int rr = lane & 15;                // r - jb
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        const float4 g4 = *reinterpret_cast<const float4*>(s_g + jb + 4 * q);
+        const float gj[4] = {g4.x, g4.y, g4.z, g4.w};
+        float a[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const int c = 4 * q + e;
+            const float gv = hi ? gB[c] : gA[c];
+            a[e] = (c < rr) ? tf32r(gv * b_r * ex2(g_r - gj[e])) : 0.f;
+        }
+        *reinterpret_cast<float4*>(arow + jb + 4 * q) = make_float4(a[0], a[1], a[2], a[3]);
+    }
+}
+
+// Row r = 32 W + lane of M o Q K^T (lower triangle with the diagonal; zero past
+// the sequence end), as bf16 straight into the record's swizzled tile in global
+// memory; every byte of the row is written.  tm_row addresses row r of Q K^T.
+template <int W>
+__device__ __forceinline__ void build_mqk(uint8_t* rec, uint32_t tm_row, const float* s_g,
+                                          const float* s_w, int lane, int valid) {
+    const int r = 32 * W + lane;
+    const bool hi = lane >= 16;
+    const bool live = r < valid;
+    const float g_r = s_g[r];
+    float gA[16], gB[16];
+#pragma unroll
+    for (int J = 0; J <= 2 * W; ++J) {
+        tmem_ld16(tm_row + 16 * J, gA);
+        if (J == 2 * W) tmem_ld16(tm_row + 16 * J + 16, gB);
+        tmem_ld_wait();
+        if (J < 2 * W || hi) {
+            const float s = live ? ex2(g_r - s_g[16 * J + 15]) : 0.f;
+            uint32_t w[8];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const float4 w4 = *reinterpret_cast<const float4*>(s_w + 16 * J + 4 * q);
+                const float* gq = gA + 4 * q;
+                w[2 * q] = pack2(gq[0] * w4.x * s, gq[1] * w4.y * s);
+                w[2 * q + 1] = pack2(gq[2] * w4.z * s, gq[3] * w4.w * s);
+            }
+            *reinterpret_cast<uint4*>(rec + taddr(0, r, 16 * J, 0)) = make_uint4(w[0], w[1], w[2], w[3]);
+            *reinterpret_cast<uint4*>(rec + taddr(0, r, 16 * J + 8, 0)) =
+                make_uint4(w[4], w[5], w[6], w[7]);
+        }
+    }
+    const int jb = 32 * W + (hi ? 16 : 0);
+    const int rr = lane & 15;
+    uint32_t w[8];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        const float4 g4 = *reinterpret_cast<const float4*>(s_g + jb + 4 * q);
+        const float gj[4] = {g4.x, g4.y, g4.z, g4.w};
+        float m[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const int c = 4 * q + e;
+            const float gv = hi ? gB[c] : gA[c];
+            m[e] = (live && c <= rr) ? gv * ex2(g_r - gj[e]) : 0.f;
+        }
+        w[2 * q] = pack2(m[0], m[1]);
+        w[2 * q + 1] = pack2(m[2], m[3]);
+    }
+    *reinterpret_cast<uint4*>(rec + taddr(0, r, jb, 0)) = make_uint4(w[0], w[1], w[2], w[3]);
+    *reinterpret_cast<uint4*>(rec + taddr(0, r, jb + 8, 0)) = make_uint4(w[4], w[5], w[6], w[7]);
+#pragma unroll
+    for (int J = 2 * W + 1; J < 4; ++J)
+        if (J > 2 * W + (hi ? 1 : 0)) {
+            *reinterpret_cast<uint4*>(rec + taddr(0, r, 16 * J, 0)) = make_uint4(0, 0, 0, 0);
+            *reinterpret_cast<uint4*>(rec + taddr(0, r, 16 * J + 8, 0)) = make_uint4(0, 0, 0, 0);
+        }
+}
+
+// Diagonal 16 x 16 blocks of T = (I + A)^{-1}: thread tid < 64 (block b = tid / 16,
+// column cc = tid % 16) forward-substitutes column cc in fp32, row by row as dot
+// products over the already solved entries (the A rows read four at a time), and
+// stores it rounded to tf32 (zeros above the diagonal included).  Block b's rows
+// of A were written by the same warp.
+__device__ __forceinline__ void solve_diag_blocks(const float* Af, float* Tf, int tid) {
+    const int b = tid >> 4, cc = tid & 15;
+    const float* Ab = Af + (16 * b) * AF_LD + 16 * b;
+    float x[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+        float acc0 = (i == cc) ? 1.f : 0.f, acc1 = 0.f;
+#pragma unroll
+        for (int j4 = 0; j4 < (i + 3) / 4; ++j4) {
+            const float4 a = *reinterpret_cast<const float4*>(Ab + i * AF_LD + 4 * j4);
+            if (4 * j4 + 0 < i) acc0 = fmaf(-a.x, x[4 * j4 + 0], acc0);
+            if (4 * j4 + 1 < i) acc1 = fmaf(-a.y, x[4 * j4 + 1], acc1);
+            if (4 * j4 + 2 < i) acc0 = fmaf(-a.z, x[4 * j4 + 2], acc0);
+            if (4 * j4 + 3 < i) acc1 = fmaf(-a.w, x[4 * j4 + 3], acc1);
+        }
+        x[i] = acc0 + acc1;
+    }
+#pragma unroll
+    for (int i = 0; i < 16; ++i) Tf[(16 * b + i) * AF_LD + 16 * b + cc] = tf32r(x[i]);
+}
+
+// m16n8k8 tf32 product on fragments already in registers
+__device__ __forceinline__ void mma_tf32_frag(float* d, const uint32_t* a, uint32_t b0, uint32_t b1) {
     asm volatile(
         "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 "
         "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
         : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+// The A fragment of a 16 x 8 fp32 tile (rows of stride lda floats, 16-byte
+// aligned) in one ldmatrix.x4: an 8 x 8 b16 matrix read as 8 rows of 4 fp32
+// puts element (lane / 4, lane % 4) in the lane's register, and the four
+// matrices are rows 0-7 / 8-15 by columns 0-3 / 4-7 -- the fragment's a0..a3.
+__device__ __forceinline__ void lda_tf32(const float* A, int lda, int lane, uint32_t* a) {
+    const int mat = lane >> 3;
+    ldsm_x4(smem_u32(A + ((lane & 7) + 8 * (mat & 1)) * lda + 4 * (mat >> 1)), a);
+}
+// The B fragments of two n-tiles (n0 .. n0 + 15) at one k step from a tile held
+// transposed, Bt[n][k] (rows of stride ldb floats): registers {b0, b1} of n-tile 0,
+// then of n-tile 1.
+__device__ __forceinline__ void ldb_tf32_t2(const float* Bt, int ldb, int lane, uint32_t* b) {
+    const int mat = lane >> 3;
+    ldsm_x4(smem_u32(Bt + ((lane & 7) + 8 * (mat >> 1)) * ldb + 4 * (mat & 1)), b);
+}
+// Store an m16n8 accumulator fragment (tf32-rounded) transposed: Xt[n][m], row
+// stride ldx floats, at m-offset m0 and n-offset n0.
+__device__ __forceinline__ void store_frag_t(float* Xt, int ldx, int m0, int n0, const float* d,
+                                             int lane) {
+    const int g = lane >> 2, t4 = lane & 3;
+    float* x = Xt + (n0 + 2 * t4) * ldx + m0 + g;
+    x[0] = tf32r(d[0]);
+    x[ldx] = tf32r(d[1]);
+    x[8] = tf32r(d[2]);
+    x[ldx + 8] = tf32r(d[3]);
 }
 
-// T = (I + A)^{-1} for the strictly lower 64 x 64 A in Af (row stride AF_LD),
-// into the lower 16 x 16 blocks of Tf (the diagonal blocks with their zeros
-// above the diagonal; the blocks above the diagonal are not written).  All
-// CO_THREADS threads (four warps) take part; Xs is scratch (256 floats per warp).
-// The diagonal blocks come from fp32 forward substitution, the off-diagonal
-// ones from tf32 tensor-core block products:
-//   T_10 = -T_11 (A_10 T_00),  T_32 = -T_33 (A_32 T_22),  T_ba = -T_bb (A_ba T_aa)
-// (a = rows/columns 0..31, b = 32..63).  A, the diagonal blocks, the level-1
-// blocks and the scratch hold tf32-rounded values (the block products read them
-// as they are).
-__device__ __forceinline__ void solve_unit_lower(const float* Af, float* Tf, float* Xs, int tid) {
-    const int warp = tid >> 5, lane = tid & 31, g = lane >> 2, t4 = lane & 3;
-    if (tid < 64) {  // diagonal blocks: thread (b, cc) solves column cc of block b
-        const int b = tid >> 4, cc = tid & 15;
-        const float* Ab = Af + (16 * b) * AF_LD + 16 * b;
-        float x[16];
+// The off-diagonal blocks of T from tf32 tensor-core block products, by the two
+// solver warps (w = 0, 1; xw = CO_XS_FLOATS floats of scratch per warp):
+//   level 1: T_10 = -T_11 (A_10 T_00) (warp 0),  T_32 = -T_33 (A_32 T_22) (warp 1);
+//            each warp reads only the rows it built, so a warp barrier precedes it;
+//   level 2: T_ba = -T_bb (A_ba T_aa)  (a = rows/columns 0..31, b = 32..63), warp w
+//            taking columns 16 w .. 16 w + 15, after a barrier of both warps.
+// The intermediate products go to the scratch transposed (the next product's B
+// operand).  Level-1 blocks and the scratch hold tf32-rounded values; level 2 is
+// final fp32.
+constexpr int XT1_LD = 20;  // level-1 scratch: 16 n-rows x 16 m (+4 pad)
+constexpr int XT2_LD = 36;  // level-2 scratch: 16 n-rows x 32 m (+4 pad)
+__device__ __forceinline__ void solve_level1(const float* Af, float* Tf, float* xw, int w,
+                                             int lane) {
+    const int g = lane >> 2, t4 = lane & 3;
+    const int bi = 2 * w + 1, bj = 2 * w;
+    float d0[4] = {0.f, 0.f, 0.f, 0.f}, d1[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-        for (int i = 0; i < 16; ++i) x[i] = (i == cc) ? 1.f : 0.f;
+    for (int ks = 0; ks < 2; ++ks) {
+        uint32_t a[4];
+        lda_tf32(Af + (16 * bi) * AF_LD + 16 * bj + 8 * ks, AF_LD, lane, a);
+        const float* B = Tf + (16 * bj + 8 * ks) * AF_LD + 16 * bj;
+        mma_tf32_frag(d0, a, __float_as_uint(B[t4 * AF_LD + g]), __float_as_uint(B[(t4 + 4) * AF_LD + g]));
+        mma_tf32_frag(d1, a, __float_as_uint(B[t4 * AF_LD + 8 + g]),
+                      __float_as_uint(B[(t4 + 4) * AF_LD + 8 + g]));
+    }
+    store_frag_t(xw, XT1_LD, 0, 0, d0, lane);
+    store_frag_t(xw, XT1_LD, 0, 8, d1, lane);
+    __syncwarp();
+    float e0[4] = {0.f, 0.f, 0.f, 0.f}, e1[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-        for (int jj = 0; jj < 15; ++jj) {
-            const float xj = x[jj];
+    for (int ks = 0; ks < 2; ++ks) {
+        uint32_t a[4], b[4];
+        lda_tf32(Tf + (16 * bi) * AF_LD + 16 * bi + 8 * ks, AF_LD, lane, a);
+        ldb_tf32_t2(xw + 8 * ks, XT1_LD, lane, b);
+        mma_tf32_frag(e0, a, b[0], b[1]);
+        mma_tf32_frag(e1, a, b[2], b[3]);
+    }
+    float* to = Tf + (16 * bi) * AF_LD + 16 * bj + 2 * t4;
+    *reinterpret_cast<float2*>(to + g * AF_LD) = make_float2(tf32r(-e0[0]), tf32r(-e0[1]));
+    *reinterpret_cast<float2*>(to + (g + 8) * AF_LD) = make_float2(tf32r(-e0[2]), tf32r(-e0[3]));
+    *reinterpret_cast<float2*>(to + 8 + g * AF_LD) = make_float2(tf32r(-e1[0]), tf32r(-e1[1]));
+    *reinterpret_cast<float2*>(to + 8 + (g + 8) * AF_LD) = make_float2(tf32r(-e1[2]), tf32r(-e1[3]));
+}
+
+__device__ __forceinline__ void solve_level2(const float* Af, float* Tf, float* xw, int w,
+                                             int lane) {
+    const int g = lane >> 2, t4 = lane & 3;
+    const int c0 = 16 * w;
+    // X = A_ba T_aa for columns c0 .. c0 + 15: T_aa's rows 0-15 are zero right of column 15
+    float x[2][2][4];
 #pragma unroll
-            for (int i = jj + 1; i < 16; ++i) x[i] = fmaf(-Ab[i * AF_LD + jj], xj, x[i]);
+    for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) x[mt][nt][e] = 0.f;
+#pragma unroll
+    for (int ks = 0; ks < 4; ++ks) {
+        if (w == 1 && ks < 2) continue;
+        const float* B = Tf + (8 * ks) * AF_LD + c0;
+        uint32_t b[2][2];
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt) {
+            b[nt][0] = __float_as_uint(B[t4 * AF_LD + 8 * nt + g]);
+            b[nt][1] = __float_as_uint(B[(t4 + 4) * AF_LD + 8 * nt + g]);
         }
 #pragma unroll
-        for (int i = 0; i < 16; ++i)
-            Tf[(16 * b + i) * AF_LD + 16 * b + cc] = __uint_as_float(to_tf32(x[i]));
+        for (int mt = 0; mt < 2; ++mt) {
+            uint32_t a[4];
+            lda_tf32(Af + (32 + 16 * mt) * AF_LD + 8 * ks, AF_LD, lane, a);
+#pragma unroll
+            for (int nt = 0; nt < 2; ++nt) mma_tf32_frag(x[mt][nt], a, b[nt][0], b[nt][1]);
+        }
     }
-    __syncthreads();
-    float* xw = Xs + warp * 256;
-    {  // level 1: warp = (block, n-tile)
-        const int blk = warp >> 1, nt = warp & 1, bi = 1 + 2 * blk, bj = 2 * blk;
-        float d[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-        for (int ks = 0; ks < 2; ++ks)
-            mma_tf32_pre(d, Af + (16 * bi) * AF_LD + 16 * bj + 8 * ks, AF_LD,
-                     Tf + (16 * bj + 8 * ks) * AF_LD + 16 * bj + 8 * nt, AF_LD, lane);
-        *reinterpret_cast<float2*>(xw + g * 8 + 2 * t4) = make_float2(tf32r(d[0]), tf32r(d[1]));
-        *reinterpret_cast<float2*>(xw + (g + 8) * 8 + 2 * t4) = make_float2(tf32r(d[2]), tf32r(d[3]));
-        __syncwarp();
-        float e[4] = {0.f, 0.f, 0.f, 0.f};
+    for (int mt = 0; mt < 2; ++mt)
 #pragma unroll
-        for (int ks = 0; ks < 2; ++ks)
-            mma_tf32_pre(e, Tf + (16 * bi) * AF_LD + 16 * bi + 8 * ks, AF_LD, xw + 8 * ks * 8, 8, lane);
-        float* to = Tf + (16 * bi) * AF_LD + 16 * bj + 8 * nt + 2 * t4;
-        *reinterpret_cast<float2*>(to + g * AF_LD) = make_float2(tf32r(-e[0]), tf32r(-e[1]));
-        *reinterpret_cast<float2*>(to + (g + 8) * AF_LD) = make_float2(tf32r(-e[2]), tf32r(-e[3]));
+        for (int nt = 0; nt < 2; ++nt) store_frag_t(xw, XT2_LD, 16 * mt, 8 * nt, x[mt][nt], lane);
+    __syncwarp();
+    // T_ba = -T_bb X: rows 32-47 take T_22 (k = X rows 0-15), rows 48-63 take
+    // [T_32 T_33] (k = X rows 0-31)
+    {  // rows 32-47
+        float y[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+#pragma unroll
+        for (int ks = 0; ks < 2; ++ks) {
+            uint32_t b[4], a[4];
+            ldb_tf32_t2(xw + 8 * ks, XT2_LD, lane, b);
+            lda_tf32(Tf + 32 * AF_LD + 32 + 8 * ks, AF_LD, lane, a);
+            mma_tf32_frag(y[0], a, b[0], b[1]);
+            mma_tf32_frag(y[1], a, b[2], b[3]);
+        }
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt) {
+            float* to = Tf + (32 + g) * AF_LD + c0 + 8 * nt + 2 * t4;
+            *reinterpret_cast<float2*>(to) = make_float2(-y[nt][0], -y[nt][1]);
+            *reinterpret_cast<float2*>(to + 8 * AF_LD) = make_float2(-y[nt][2], -y[nt][3]);
+        }
     }
-    __syncthreads();
-    {  // level 2: warp qn owns n-tile qn of both m-tiles; T_aa's and T_bb's blocks
-       // above the diagonal are zero (T_aa's upper-right block is skipped)
-        const int qn = warp;
-        float x0[4] = {0.f, 0.f, 0.f, 0.f}, x1[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-        for (int ks = 0; ks < 4; ++ks)
-            if (qn < 2 || ks >= 2) {
-                mma_tf32_pre(x0, Af + 32 * AF_LD + 8 * ks, AF_LD, Tf + (8 * ks) * AF_LD + 8 * qn,
-                         AF_LD, lane);
-                mma_tf32_pre(x1, Af + 48 * AF_LD + 8 * ks, AF_LD, Tf + (8 * ks) * AF_LD + 8 * qn,
-                         AF_LD, lane);
-            }
-        *reinterpret_cast<float2*>(xw + g * 8 + 2 * t4) = make_float2(tf32r(x0[0]), tf32r(x0[1]));
-        *reinterpret_cast<float2*>(xw + (g + 8) * 8 + 2 * t4) = make_float2(tf32r(x0[2]), tf32r(x0[3]));
-        *reinterpret_cast<float2*>(xw + (g + 16) * 8 + 2 * t4) = make_float2(tf32r(x1[0]), tf32r(x1[1]));
-        *reinterpret_cast<float2*>(xw + (g + 24) * 8 + 2 * t4) = make_float2(tf32r(x1[2]), tf32r(x1[3]));
-        __syncwarp();
-        float y0[4] = {0.f, 0.f, 0.f, 0.f}, y1[4] = {0.f, 0.f, 0.f, 0.f};
+    {  // rows 48-63
+        float y[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
 #pragma unroll
         for (int ks = 0; ks < 4; ++ks) {
-            if (ks < 2) mma_tf32_pre(y0, Tf + 32 * AF_LD + 32 + 8 * ks, AF_LD, xw + 8 * ks * 8, 8, lane);
-            mma_tf32_pre(y1, Tf + 48 * AF_LD + 32 + 8 * ks, AF_LD, xw + 8 * ks * 8, 8, lane);
+            uint32_t b[4], a[4];
+            ldb_tf32_t2(xw + 8 * ks, XT2_LD, lane, b);
+            lda_tf32(Tf + 48 * AF_LD + 32 + 8 * ks, AF_LD, lane, a);
+            mma_tf32_frag(y[0], a, b[0], b[1]);
+            mma_tf32_frag(y[1], a, b[2], b[3]);
         }
-        float* to = Tf + 32 * AF_LD + 8 * qn + 2 * t4;
-        *reinterpret_cast<float2*>(to + g * AF_LD) = make_float2(-y0[0], -y0[1]);
-        *reinterpret_cast<float2*>(to + (g + 8) * AF_LD) = make_float2(-y0[2], -y0[3]);
-        *reinterpret_cast<float2*>(to + (g + 16) * AF_LD) = make_float2(-y1[0], -y1[1]);
-        *reinterpret_cast<float2*>(to + (g + 24) * AF_LD) = make_float2(-y1[2], -y1[3]);
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt) {
+            float* to = Tf + (48 + g) * AF_LD + c0 + 8 * nt + 2 * t4;
+            *reinterpret_cast<float2*>(to) = make_float2(-y[nt][0], -y[nt][1]);
+            *reinterpret_cast<float2*>(to + 8 * AF_LD) = make_float2(-y[nt][2], -y[nt][3]);
+        }
     }
-    __syncthreads();
 }
 
-__global__ void __launch_bounds__(CO_THREADS, 4)
+__global__ void __launch_bounds__(CO_THREADS, 5)
     chunk_ops_kernel(const __grid_constant__ CUtensorMap map_q,
                      const __grid_constant__ CUtensorMap map_k, const PrefillParams p) {
     extern __shared__ uint8_t smem_raw[];
@@ -236,8 +440,6 @@ __global__ void __launch_bounds__(CO_THREADS, 4)
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + CO_MISC + 4);
     float* Af = reinterpret_cast<float*>(sm + CO_AF);
     float* Tf = reinterpret_cast<float*>(sm + CO_TF);
-    float* Xs = reinterpret_cast<float*>(sm + CO_XS);
-    uint8_t* rec = sm + CO_REC;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     int n, c;
@@ -252,38 +454,37 @@ __global__ void __launch_bounds__(CO_THREADS, 4)
     const int valid = min(C, t_end - t0);
     const long long slot = record_slot(n, t0);
 
+    // The copies are issued first (only thread 0 touches the barriers before the
+    // CTA barrier), then the gates are loaded while the copies and the tensor
+    // memory allocation proceed.
     if (tid == 0) {
         mbar_init(&bars[0], 1);
         mbar_init(&bars[1], 1);
         *abort_flag = 0;
         fence_mbar_init();
-    }
-    if (warp == 0) {
-        tmem_alloc(tmem_slot, CO_TM_COLS);
-        tmem_relinquish();
-    }
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-    const uint32_t tmem = *tmem_slot;
-    if (tid == 0) {
         mbar_arrive_expect_tx(&bars[0], 4 * HALF);
         tma_load_2d(sm + CO_KQ, &map_k, hq * D, t0, &bars[0]);
         tma_load_2d(sm + CO_KQ + HALF, &map_q, hq * D, t0, &bars[0]);
         tma_load_2d(sm + CO_KQ + 2 * HALF, &map_k, hq * D + 64, t0, &bars[0]);
         tma_load_2d(sm + CO_KQ + 3 * HALF, &map_q, hq * D + 64, t0, &bars[0]);
     }
-    // decay scan per value head while the copies land: warp w < nheads handles
-    // head hv0 + w (lane l: tokens 2l, 2l+1); gates past the sequence end are 0
+    // gate scan per value head: warp w < nheads handles head hv0 + w (lane l:
+    // tokens 2l, 2l+1, of block l / 8); gates past the sequence end are 0
+    float la[2] = {0.f, 0.f}, be[2] = {0.f, 0.f};
     if (warp < nheads) {
         const int h = hv0 + warp;
-        float la[2] = {0.f, 0.f}, be[2] = {0.f, 0.f};
 #pragma unroll
         for (int e = 0; e < 2; ++e)
             if (2 * lane + e < valid) {
                 la[e] = p.log_alpha[(size_t)(t0 + 2 * lane + e) * p.H_v + h];
                 be[e] = p.beta[(size_t)(t0 + 2 * lane + e) * p.H_v + h];
             }
+    }
+    if (warp == 0) {
+        tmem_alloc(tmem_slot, CO_TM_COLS);
+        tmem_relinquish();
+    }
+    if (warp < nheads) {
         const float x0 = la[0] * LOG2E, x1 = la[1] * LOG2E;
         float incl = x0 + x1;
 #pragma unroll
@@ -291,11 +492,17 @@ __global__ void __launch_bounds__(CO_THREADS, 4)
             const float y = __shfl_up_sync(0xffffffffu, incl, off);
             if (lane >= off) incl += y;
         }
+        const float g0 = incl - x1;
+        const float g_e = __shfl_sync(0xffffffffu, incl, lane | 7);  // g at the block's last token
         float* v = reinterpret_cast<float*>(sm + CO_VEC) + warp * CO_VEC_FLOATS;
-        *reinterpret_cast<float2*>(v + 2 * lane) = make_float2(incl - x1, incl);
+        *reinterpret_cast<float2*>(v + 2 * lane) = make_float2(g0, incl);
         *reinterpret_cast<float2*>(v + 64 + 2 * lane) = make_float2(be[0], be[1]);
-        *reinterpret_cast<float2*>(v + 128 + 2 * lane) = make_float2(ex2(x0), ex2(x1));
+        *reinterpret_cast<float2*>(v + 128 + 2 * lane) = make_float2(ex2(g_e - g0), ex2(g_e - incl));
     }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
     bool ok = mbar_wait(&bars[0], 0, abort_flag);
     if (!__syncthreads_and(ok)) {  // the copies may still land: wait (bounded), then leave
         if (tid == 0) mbar_wait_drain(&bars[0], 0);
@@ -329,110 +536,60 @@ __global__ void __launch_bounds__(CO_THREADS, 4)
     tc_fence_after();
     // The product is complete, so K and Q are no longer read: their bytes become A
     // and T.  The grams stay in tensor memory; each value head reads its row again.
-    const bool qrow = tid >= 64;
-    const int r = tid & 63;
-    const bool rvalid = r < valid;
-
     for (int vh = 0; vh < nheads; ++vh) {
         const int h = hv0 + vh;
         const float* s_g = reinterpret_cast<const float*>(sm + CO_VEC) + vh * CO_VEC_FLOATS;
         const float* s_b = s_g + 64;
-        const float* s_a = s_g + 128;  // alpha of each token
-        if (vh > 0) {  // the previous head's record has left the staging buffer
-            if (tid == 0) bulk_wait_read<0>();
-            __syncthreads();
-        }
-        // ---- row tid of [K; Q] K^T (TMEM lane tid): K K^T row r for tid < 64, Q K^T
-        // row r after; masks: A (fp32, strictly lower) from K K^T, M o Q K^T (bf16,
-        // lower incl. the diagonal) from Q K^T; rows past the sequence end are zero
-        float gr[64];
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-            tmem_ld16(tmem + ((uint32_t)(32 * warp) << 16) + 16 * i, gr + 16 * i);
-        tmem_ld_wait();
-        // The decay mask M_rj = exp(g_r - g_j) = alpha_{j+1} ... alpha_r (j <= r) is a
-        // running product over j, from j = r down (one multiply per entry, never an
-        // exponential of a positive number).  Rows 0-31 (warps 0 and 2) have no entries
-        // right of column 31.
-        const bool upper_half = (warp & 1) == 0;
-        if (!qrow) {  // A = strict_lower(diag(beta) (M o K K^T)), rounded to tf32
-            const float b_r = rvalid ? s_b[r] : 0.f;
-            float* arow = Af + r * AF_LD;
-            float m = 1.f;
-#pragma unroll
-            for (int j4 = 15; j4 >= 0; --j4) {
-                float a4[4] = {0.f, 0.f, 0.f, 0.f};
-                if (!(upper_half && j4 >= 8)) {
-                    const float4 al = *reinterpret_cast<const float4*>(s_a + 4 * j4);
-                    const float av[4] = {al.x, al.y, al.z, al.w};
-                    const float anext = (j4 < 15) ? s_a[4 * j4 + 4] : 1.f;
-#pragma unroll
-                    for (int e = 3; e >= 0; --e) {
-                        const int j = 4 * j4 + e;
-                        const float a_j1 = (e < 3) ? av[e + 1] : anext;  // alpha_{j+1}
-                        m = (j < r) ? m * a_j1 : 1.f;
-                        a4[e] = (j < r) ? __uint_as_float(to_tf32(b_r * m * gr[j])) : 0.f;
-                    }
-                }
-                *reinterpret_cast<float4*>(arow + 4 * j4) = make_float4(a4[0], a4[1], a4[2], a4[3]);
-            }
-        } else {  // M o Q K^T, bf16, lower triangle with the diagonal
-            float m = 1.f;
-#pragma unroll
-            for (int ch = 7; ch >= 0; --ch) {
-                float m8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-                if (rvalid && !(upper_half && ch >= 4)) {
-                    const float4 la4 = *reinterpret_cast<const float4*>(s_a + 8 * ch);
-                    const float4 lb4 = *reinterpret_cast<const float4*>(s_a + 8 * ch + 4);
-                    const float av[8] = {la4.x, la4.y, la4.z, la4.w, lb4.x, lb4.y, lb4.z, lb4.w};
-                    const float anext = (ch < 7) ? s_a[8 * ch + 8] : 1.f;
-#pragma unroll
-                    for (int e = 7; e >= 0; --e) {
-                        const int j = 8 * ch + e;
-                        const float a_j1 = (e < 7) ? av[e + 1] : anext;
-                        m = (j < r) ? m * a_j1 : 1.f;
-                        m8[e] = (j <= r) ? m * gr[j] : 0.f;
-                    }
-                }
-                *reinterpret_cast<uint4*>(rec + REC_MQ + taddr(0, r, 8 * ch, 0)) =
-                    make_uint4(pack2(m8[0], m8[1]), pack2(m8[2], m8[3]), pack2(m8[4], m8[5]),
-                               pack2(m8[6], m8[7]));
-            }
-        }
-        __syncthreads();
-        solve_unit_lower(Af, Tf, Xs, tid);
-        // ---- T diag(beta) as a bf16 tile; its 16 x 16 blocks above the diagonal are
-        // written as zeros so that every byte of the record is defined
-        for (int idx = tid; idx < 64 * 8; idx += CO_THREADS) {
-            const int rr = idx >> 3, ch = idx & 7;
-            uint4 w = make_uint4(0, 0, 0, 0);
-            if ((ch >> 1) <= (rr >> 4)) {
-                const float4 ta = *reinterpret_cast<const float4*>(Tf + rr * AF_LD + 8 * ch);
-                const float4 tb = *reinterpret_cast<const float4*>(Tf + rr * AF_LD + 8 * ch + 4);
-                const float4 b0 = *reinterpret_cast<const float4*>(s_b + 8 * ch);
-                const float4 b1 = *reinterpret_cast<const float4*>(s_b + 8 * ch + 4);
-                w = make_uint4(pack2(ta.x * b0.x, ta.y * b0.y), pack2(ta.z * b0.z, ta.w * b0.w),
-                               pack2(tb.x * b1.x, tb.y * b1.y), pack2(tb.z * b1.z, tb.w * b1.w));
-            }
-            *reinterpret_cast<uint4*>(rec + REC_TB + taddr(0, rr, 8 * ch, 0)) = w;
-        }
-        // gamma_r, d_r (zero past the sequence end), gamma_C, zero padding
-        if (tid < C) {
+        const float* s_w = s_g + 128;
+        uint8_t* rec = p.records + (size_t)(slot * p.H_v + h) * REC_BYTES;
+        const uint32_t tm_row = tmem + ((uint32_t)(32 * warp) << 16);  // row tid of [K K^T; Q K^T]
+        if (warp < 2) {
+            if (warp == 0)
+                build_a<0>(Af, tm_row, s_g, s_b, s_w, lane);
+            else
+                build_a<1>(Af, tm_row, s_g, s_b, s_w, lane);
+            __syncwarp();
+            if (vh > 0) bar_sync<CO_BAR_TFREE, CO_THREADS>();  // the previous T has been read
+            solve_diag_blocks(Af, Tf, tid);
+            __syncwarp();
+            solve_level1(Af, Tf, reinterpret_cast<float*>(sm + CO_XS) + warp * CO_XS_FLOATS, warp, lane);
+            bar_sync<CO_BAR_SOLVE, 64>();
+            solve_level2(Af, Tf, reinterpret_cast<float*>(sm + CO_XS) + warp * CO_XS_FLOATS, warp, lane);
+            bar_sync<CO_BAR_SOLVE, 64>();  // both solvers are done with this head's A
+            bar_arrive<CO_BAR_TDONE, CO_THREADS>();
+        } else {
+            const int q = tid - 64;
+            if (warp == 2)
+                build_mqk<0>(rec + REC_MQ, tm_row, s_g, s_w, lane, valid);
+            else
+                build_mqk<1>(rec + REC_MQ, tm_row, s_g, s_w, lane, valid);
+            // gamma_r, d_r (zero past the sequence end), gamma_C, zero padding
             float* rv = reinterpret_cast<float*>(rec + REC_VEC);
             const float gC = s_g[C - 1];
-            const float g_t = s_g[tid];
-            rv[tid] = ex2(g_t);
-            rv[64 + tid] = (tid < valid) ? ex2(gC - g_t) : 0.f;
-            if (tid < REC_VEC_FLOATS - 128) rv[128 + tid] = (tid == 0) ? ex2(gC) : 0.f;
-        }
-        fence_proxy_async_smem();  // generic writes, read next by the bulk copy
-        __syncthreads();
-        if (tid == 0) {
-            bulk_store(p.records + (size_t)(slot * p.H_v + h) * REC_BYTES, rec, REC_BYTES);
-            bulk_commit();
+            rv[q] = ex2(s_g[q]);
+            rv[64 + q] = (q < valid) ? ex2(gC - s_g[q]) : 0.f;
+            if (q < REC_VEC_FLOATS - 128) rv[128 + q] = (q == 0) ? ex2(gC) : 0.f;
+            bar_sync<CO_BAR_TDONE, CO_THREADS>();
+            // T diag(beta) as a bf16 tile; its 16 x 16 blocks above the diagonal are
+            // written as zeros so that every byte of the record is defined
+#pragma unroll 2
+            for (int it = 0; it < 8; ++it) {
+                const int idx = q + 64 * it;
+                const int rr = idx >> 3, ch = idx & 7;
+                uint4 w = make_uint4(0, 0, 0, 0);
+                if ((ch >> 1) <= (rr >> 4)) {
+                    const float4 ta = *reinterpret_cast<const float4*>(Tf + rr * AF_LD + 8 * ch);
+                    const float4 tb = *reinterpret_cast<const float4*>(Tf + rr * AF_LD + 8 * ch + 4);
+                    const float4 b0 = *reinterpret_cast<const float4*>(s_b + 8 * ch);
+                    const float4 b1 = *reinterpret_cast<const float4*>(s_b + 8 * ch + 4);
+                    w = make_uint4(pack2(ta.x * b0.x, ta.y * b0.y), pack2(ta.z * b0.z, ta.w * b0.w),
+                                   pack2(tb.x * b1.x, tb.y * b1.y), pack2(tb.z * b1.z, tb.w * b1.w));
+                }
+                *reinterpret_cast<uint4*>(rec + REC_TB + taddr(0, rr, 8 * ch, 0)) = w;
+            }
+            if (vh + 1 < nheads) bar_arrive<CO_BAR_TFREE, CO_THREADS>();
         }
     }
-    if (tid == 0) bulk_wait_read<0>();  // the staging buffer is read before the CTA exits
     tc_fence_before();
     __syncthreads();
     if (warp == 0) {
@@ -1370,6 +1527,10 @@ static cudaError_t run_pass1(const CUtensorMap& mq, const CUtensorMap& mk,
                              const PrefillParams& prm, cudaStream_t stream) {
     cudaError_t e =
         cudaFuncSetAttribute(chunk_ops_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, CO_SMEM);
+    if (e != cudaSuccess) return e;
+    // all of the unified L1 as shared memory, so that five CTAs fit on an SM
+    e = cudaFuncSetAttribute(chunk_ops_kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                             cudaSharedmemCarveoutMaxShared);
     if (e != cudaSuccess) return e;
     const int group = prm.H_v / prm.H_qk;
     const long long slots = (long long)prm.N + ((long long)prm.T + C - 1) / C;

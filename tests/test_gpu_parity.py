@@ -70,7 +70,7 @@ def test_decode_batched_256_full_512_steps_sampled():
         worst_o = max(worst_o, o_err(np.stack([og[b, h] for b, h in pairs]), o_ref))
     Sg = S.cpu().double().numpy()
     se = s_err(np.stack([Sg[b, h] for b, h in pairs]), S_ref)
-    record("decode_batched_256", "config 4: decode 256 x 16/48 heads, 512 steps", o_err=worst_o,
+    record("decode_batched_256", "batched decode: 256 sequences x 16/48 heads, 512 steps", o_err=worst_o,
            s_err=se, units="24 sampled (sequence, head) units")
     assert worst_o <= O_TOL
     assert se <= S_TOL
@@ -83,7 +83,7 @@ def test_prefill_tiny_fp32_L256():
     o, S, o_ref, S_ref = _run_case(case)
     assert o.dtype == torch.float32
     oe, se = o_err(o, o_ref), s_err(S, S_ref)
-    record("prefill_tiny_fp32_L256", "config 0: L=256, 1/1 heads, fp32", o_err=oe, s_err=se)
+    record("prefill_tiny_fp32_L256", "tiny prefill: L=256, 1/1 heads, fp32", o_err=oe, s_err=se)
     assert oe <= O_TOL
     assert se <= S_TOL
 
@@ -187,7 +187,7 @@ def test_prefill_qwen_32k_sampled_heads():
     heads = [0, 25, 47]
     o, S, o_ref, S_ref = _run_case(case, heads=heads)
     oe, se = o_err(o[:, heads], o_ref[:, heads]), s_err(S[:, heads], S_ref[:, heads])
-    record("prefill_qwen_32k", "config 1: L=32768, 16/48 heads", o_err=oe, s_err=se,
+    record("prefill_qwen_32k", "prefill L=32768, 16/48 heads, bf16", o_err=oe, s_err=se,
            o_per_head=per_head_o(o, o_ref, heads), s_per_head=per_head_s(S, S_ref, heads))
     assert oe <= O_TOL
     assert se <= S_TOL
@@ -199,7 +199,7 @@ def test_prefill_varlen_8seq_sampled_heads():
     heads = [5, 40]
     o, S, o_ref, S_ref = _run_case(case, heads=heads)
     oe, se = o_err(o[:, heads], o_ref[:, heads]), s_err(S[:, heads], S_ref[:, heads])
-    record("prefill_varlen_8seq", "config 2: 8 packed sequences, S0 != 0", o_err=oe, s_err=se,
+    record("prefill_varlen_8seq", "packed varlen prefill: 8 sequences of 1024-8192, S0 != 0", o_err=oe, s_err=se,
            o_per_head=per_head_o(o, o_ref, heads), s_per_head=per_head_s(S, S_ref, heads))
     assert oe <= O_TOL
     assert se <= S_TOL
@@ -212,7 +212,7 @@ def test_prefill_long_256k_final_state_sampled_heads():
     heads = [7, 31]
     o, S, o_ref, S_ref = _run_case(case, heads=heads, want_o=False)
     se = s_err(S[:, heads], S_ref[:, heads])
-    record("prefill_long_256k", "config 3: L=262144, long-memory gates", s_err=se,
+    record("prefill_long_256k", "long-context prefill: L=262144, long-memory gates", s_err=se,
            s_per_head=per_head_s(S, S_ref, heads))
     assert se <= S_TOL
     assert torch.isfinite(o.float()).all()
