@@ -525,6 +525,53 @@ def run_prefill_workload(args, case, dev, stream, world):
     return ms, n
 
 
+def run_prefill_tiny(args, dev, stream, world):
+    """The tiny fp32 prefill (B=1, L=256, 1 QK / 1 V head): launch-bound, so timed
+    for the record only; returns a line with its CPU baseline (the oracle on the
+    whole workload, rank 0 at N=1)."""
+    import torch
+    from linear_attention_12_b200 import gdn, inputs
+    case = inputs.tiny_fp32()
+    q, k, v = case.q.to(dev), case.k.to(dev), case.v.to(dev)
+    la, be, cu = case.log_alpha.to(dev), case.beta.to(dev), case.cu_seqlens.to(dev)
+    o = torch.empty((case.T, case.H_v, D), dtype=torch.float32, device=dev)
+    Sf = torch.empty((case.N, case.H_v, D, D), dtype=torch.float32, device=dev)
+    ws = torch.empty(max(1, gdn.workspace_size(case.N, case.T, case.H_qk, case.H_v, D,
+                                               gdn.GDN_F32)), dtype=torch.uint8, device=dev)
+
+    def step():
+        gdn.prefill(q, k, v, la, be, None, cu, o=o, S_final=Sf, workspace=ws)
+
+    n = 50
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize()
+    barrier(world)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(n):
+        step()
+    b.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    assert gdn.last_device_error() == gdn.GDN_OK
+    us = max_over_ranks(a.elapsed_time(b), world) / n * 1e3
+    line = {"value": case.T / (us / 1e6), "unit": "tokens/s", "us_per_call": us,
+            "tokens": case.T, "steps": n,
+            "workload": "tiny prefill B=1 L=256 H_qk=1 H_v=1 d=128, all fp32, S0=0 "
+                        "(launch-bound: five launches, three fp32 -> bf16 copies and the two passes)"}
+    if world == 1 and not args.no_cpu_baseline:
+        import oracle
+        t0 = time.perf_counter()
+        oracle.prefill(case.q, case.k, case.v, case.log_alpha, case.beta, None, case.cu_seqlens,
+                       n_threads=1)
+        dt = time.perf_counter() - t0
+        line["cpu_baseline"] = {"value": case.T / dt, "unit": "tokens/s", "cores": 1,
+                                "kind": "oracle", "sample": f"the whole workload, fp64, {dt:.3f} s"}
+    del q, k, v, la, be, cu, o, Sf, ws
+    return line
+
+
 def prefill_workload_line(case, ms, steps, hbm_peak, tf_peak, workload, cpu):
     """Throughput and roofline of one prefill workload (bf16 q/k/v, o; fp32 gates,
     states): bytes = the tokens' algorithmic bytes + S0 (if given) + S_final."""
@@ -662,8 +709,9 @@ def run_ours(args):
 
     # ---------------- the other prefill workloads: packed varlen batch with S0, and
     # the long-context prefill (each timed alone; inputs resident)
-    varlen = long_ctx = None
+    varlen = long_ctx = tiny = None
     if not args.no_workloads:
+        tiny = run_prefill_tiny(args, dev, stream, world)
         vcase = inputs.varlen_8seq()
         ms, n = run_prefill_workload(args, vcase, dev, stream, world)
         vcpu = None
@@ -767,6 +815,7 @@ def run_ours(args):
                 "steps": max(args.steps, 20),
                 **({"cpu_baseline": dec_cpu} if dec_cpu is not None else {}),
             },
+            "prefill_tiny": tiny,
             "prefill_varlen": varlen,
             "prefill_long": long_ctx,
             "decode_multi": None if dm_gbs is None else {

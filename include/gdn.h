@@ -98,6 +98,14 @@ typedef enum {
  *               (gdn_prefill_segmented with segments = 0) and the workspace
  *               also holds that split's states.
  *
+ * Arithmetic: tensor-core products with 16-bit operands and fp32 accumulators;
+ * the state is carried in fp32.  The state S and d o Delta enter the products
+ * as bf16 (they meet the bf16 K and Q tiles).  Unless the sequences are split,
+ * the chunk operators T diag(beta) and M o Q K^T and the intermediates
+ * X = V - diag(gamma) K S and Delta enter as fp16 (11 significant bits); their
+ * entries must stay below 65,504 in magnitude, which unit-norm q, k and
+ * unit-scale v satisfy.  The split prefill keeps them in bf16.
+ *
  * Returns GDN_OK, GDN_ERR_INVALID_ARG, GDN_ERR_UNSUPPORTED, GDN_ERR_WORKSPACE
  * or GDN_ERR_CUDA.
  */

@@ -28,8 +28,12 @@
 // so each entry left of the diagonal block costs two multiplies) and solve for
 // T (fp32 forward substitution on the diagonal 16 x 16 blocks, tf32
 // tensor-core block products for the rest), while two "writer" warps store
-// M o Q K^T, then T diag(beta), as 128-byte-swizzled bf16 tiles of one "chunk
+// M o Q K^T, then T diag(beta), as 128-byte-swizzled tiles of one "chunk
 // operator" record together with gamma, d and gamma_C, straight from registers.
+// The unsplit prefill writes the tiles in fp16, and its output pass then
+// carries X and Delta in fp16 as well (11 significant bits against bf16's 8);
+// the segmented prefill and the gradients' forward keep bf16.  The state S and
+// d o Delta stay bf16 operands: they meet the bf16 K and Q tiles.
 //
 // Pass 2 (the prefill's outputs): one CTA per (sequence, value head, d_v slice
 // of NS columns); the columns of S evolve independently, so slices need no
@@ -136,6 +140,14 @@ __device__ __forceinline__ void bar_arrive() {
     asm volatile("bar.arrive %0, %1;" ::"n"(ID), "n"(N) : "memory");
 }
 
+// Two values as a packed pair of the chunk-operator records' tile type: fp16
+// (F16) for the unsplit prefill's output passes, whose products T_b X and
+// [T_b; M o Q K^T] Delta then take fp16 operands; bf16 for every other reader.
+template <bool F16>
+__device__ __forceinline__ uint32_t packr(float lo, float hi) {
+    return F16 ? pack_f16x2(lo, hi) : pack_bf16x2(lo, hi);
+}
+
 // tf32 rounding of an fp32 value, kept as fp32 (the low mantissa bits cleared)
 __device__ __forceinline__ float tf32r(float x) { return __uint_as_float(to_tf32(x)); }
 // The decay mask M_rj = exp2(g_r - g_j) (j <= r, g in log2 units) of a row r in
@@ -193,9 +205,10 @@ __device__ __forceinline__ void build_a(float* Af, uint32_t tm_row, const float*
 }
 
 // Row r = 32 W + lane of M o Q K^T (lower triangle with the diagonal; zero past
-// the sequence end), as bf16 straight into the record's swizzled tile in global
-// memory; every byte of the row is written.  tm_row addresses row r of Q K^T.
-template <int W>
+// the sequence end), as bf16 or fp16 straight into the record's swizzled tile in
+// global memory; every byte of the row is written.  tm_row addresses row r of
+// Q K^T.
+template <int W, bool F16>
 __device__ __forceinline__ void build_mqk(uint8_t* rec, uint32_t tm_row, const float* s_g,
                                           const float* s_w, int lane, int valid) {
     const int r = 32 * W + lane;
@@ -215,8 +228,8 @@ __device__ __forceinline__ void build_mqk(uint8_t* rec, uint32_t tm_row, const f
             for (int q = 0; q < 4; ++q) {
                 const float4 w4 = *reinterpret_cast<const float4*>(s_w + 16 * J + 4 * q);
                 const float* gq = gA + 4 * q;
-                w[2 * q] = pack2(gq[0] * w4.x * s, gq[1] * w4.y * s);
-                w[2 * q + 1] = pack2(gq[2] * w4.z * s, gq[3] * w4.w * s);
+                w[2 * q] = packr<F16>(gq[0] * w4.x * s, gq[1] * w4.y * s);
+                w[2 * q + 1] = packr<F16>(gq[2] * w4.z * s, gq[3] * w4.w * s);
             }
             *reinterpret_cast<uint4*>(rec + taddr(0, r, 16 * J, 0)) = make_uint4(w[0], w[1], w[2], w[3]);
             *reinterpret_cast<uint4*>(rec + taddr(0, r, 16 * J + 8, 0)) =
@@ -237,8 +250,8 @@ __device__ __forceinline__ void build_mqk(uint8_t* rec, uint32_t tm_row, const f
             const float gv = hi ? gB[c] : gA[c];
             m[e] = (live && c <= rr) ? gv * ex2(g_r - gj[e]) : 0.f;
         }
-        w[2 * q] = pack2(m[0], m[1]);
-        w[2 * q + 1] = pack2(m[2], m[3]);
+        w[2 * q] = packr<F16>(m[0], m[1]);
+        w[2 * q + 1] = packr<F16>(m[2], m[3]);
     }
     *reinterpret_cast<uint4*>(rec + taddr(0, r, jb, 0)) = make_uint4(w[0], w[1], w[2], w[3]);
     *reinterpret_cast<uint4*>(rec + taddr(0, r, jb + 8, 0)) = make_uint4(w[4], w[5], w[6], w[7]);
@@ -428,6 +441,7 @@ __device__ __forceinline__ void solve_level2(const float* Af, float* Tf, float* 
     }
 }
 
+template <bool F16>
 __global__ void __launch_bounds__(CO_THREADS, 5)
     chunk_ops_kernel(const __grid_constant__ CUtensorMap map_q,
                      const __grid_constant__ CUtensorMap map_k, const PrefillParams p) {
@@ -560,9 +574,9 @@ __global__ void __launch_bounds__(CO_THREADS, 5)
         } else {
             const int q = tid - 64;
             if (warp == 2)
-                build_mqk<0>(rec + REC_MQ, tm_row, s_g, s_w, lane, valid);
+                build_mqk<0, F16>(rec + REC_MQ, tm_row, s_g, s_w, lane, valid);
             else
-                build_mqk<1>(rec + REC_MQ, tm_row, s_g, s_w, lane, valid);
+                build_mqk<1, F16>(rec + REC_MQ, tm_row, s_g, s_w, lane, valid);
             // gamma_r, d_r (zero past the sequence end), gamma_C, zero padding
             float* rv = reinterpret_cast<float*>(rec + REC_VEC);
             const float gC = s_g[C - 1];
@@ -570,7 +584,7 @@ __global__ void __launch_bounds__(CO_THREADS, 5)
             rv[64 + q] = (q < valid) ? ex2(gC - s_g[q]) : 0.f;
             if (q < REC_VEC_FLOATS - 128) rv[128 + q] = (q == 0) ? ex2(gC) : 0.f;
             bar_sync<CO_BAR_TDONE, CO_THREADS>();
-            // T diag(beta) as a bf16 tile; its 16 x 16 blocks above the diagonal are
+            // T diag(beta) as a bf16 or fp16 tile; its 16 x 16 blocks above the diagonal are
             // written as zeros so that every byte of the record is defined
 #pragma unroll 2
             for (int it = 0; it < 8; ++it) {
@@ -582,8 +596,10 @@ __global__ void __launch_bounds__(CO_THREADS, 5)
                     const float4 tb = *reinterpret_cast<const float4*>(Tf + rr * AF_LD + 8 * ch + 4);
                     const float4 b0 = *reinterpret_cast<const float4*>(s_b + 8 * ch);
                     const float4 b1 = *reinterpret_cast<const float4*>(s_b + 8 * ch + 4);
-                    w = make_uint4(pack2(ta.x * b0.x, ta.y * b0.y), pack2(ta.z * b0.z, ta.w * b0.w),
-                                   pack2(tb.x * b1.x, tb.y * b1.y), pack2(tb.z * b1.z, tb.w * b1.w));
+                    w = make_uint4(packr<F16>(ta.x * b0.x, ta.y * b0.y),
+                                   packr<F16>(ta.z * b0.z, ta.w * b0.w),
+                                   packr<F16>(tb.x * b1.x, tb.y * b1.y),
+                                   packr<F16>(tb.z * b1.z, tb.w * b1.w));
                 }
                 *reinterpret_cast<uint4*>(rec + REC_TB + taddr(0, rr, 8 * ch, 0)) = w;
             }
@@ -600,9 +616,40 @@ __global__ void __launch_bounds__(CO_THREADS, 5)
 
 
 
+// D += A * B, m16n8k16, fp32 accumulate: fp16 inputs when F16, else bf16 (the
+// products with a record tile as A when the records are fp16).
+template <bool F16>
+__device__ __forceinline__ void mma16816r(float* d, const uint32_t* a, uint32_t b0, uint32_t b1) {
+    if constexpr (F16) {
+        asm volatile(
+            "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 "
+            "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+            : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+            : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+    } else {
+        mma16816(d, a, b0, b1);
+    }
+}
+
+// store_acc_bf16 in the records' tile type (fp16 when F16)
+template <int NT, bool F16>
+__device__ __forceinline__ void store_acc_r(uint8_t* smem, uint32_t base_off, int m0,
+                                            const float (*acc)[4], int lane) {
+    const int g = lane >> 2, t = lane & 3;
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+        const int col = 8 * nt + 2 * t;
+        *reinterpret_cast<uint32_t*>(smem + taddr_e(base_off, m0 + g, col, 0)) =
+            packr<F16>(acc[nt][0], acc[nt][1]);
+        *reinterpret_cast<uint32_t*>(smem + taddr_e(base_off, m0 + g + 8, col, 0)) =
+            packr<F16>(acc[nt][2], acc[nt][3]);
+    }
+}
+
 // Delta = T_b X for row block rb (rows 16 rb .. +15) and n-tiles of column half H
-// of an NT-tile slice, stored as bf16 Delta and d o Delta.
-template <int NT, int H>
+// of an NT-tile slice, stored as Delta (in the records' tile type: X is in it
+// too) and d o Delta (bf16: it meets the bf16 K tile).
+template <int NT, int H, bool F16>
 __device__ __forceinline__ void delta_half(uint8_t* sm, uint32_t tb, uint32_t xt, int rb,
                                            int lane, float d_lo, float d_hi) {
     constexpr int N0 = H * (NT / 2), N1 = (H + 1) * (NT / 2);
@@ -621,12 +668,12 @@ __device__ __forceinline__ void delta_half(uint8_t* sm, uint32_t tb, uint32_t xt
                 if (nt + 1 < N1) {
                     uint32_t b[4];
                     ldb_mn(xt, 0, 8 * nt, 16 * ks, lane, b);
-                    mma16816(acc[nt - N0], a, b[0], b[1]);
-                    mma16816(acc[nt - N0 + 1], a, b[2], b[3]);
+                    mma16816r<F16>(acc[nt - N0], a, b[0], b[1]);
+                    mma16816r<F16>(acc[nt - N0 + 1], a, b[2], b[3]);
                 } else {
                     uint32_t b[2];
                     ldb_mn1(xt, 8 * nt, 16 * ks, lane, b);
-                    mma16816(acc[nt - N0], a, b[0], b[1]);
+                    mma16816r<F16>(acc[nt - N0], a, b[0], b[1]);
                 }
             }
         }
@@ -635,9 +682,10 @@ __device__ __forceinline__ void delta_half(uint8_t* sm, uint32_t tb, uint32_t xt
 #pragma unroll
     for (int i = 0; i < N1 - N0; ++i) {
         const int col = 8 * (N0 + i) + 2 * t;
-        *reinterpret_cast<uint32_t*>(sm + taddr_e(P2_DU, r, col, 0)) = pack2(acc[i][0], acc[i][1]);
+        *reinterpret_cast<uint32_t*>(sm + taddr_e(P2_DU, r, col, 0)) =
+            packr<F16>(acc[i][0], acc[i][1]);
         *reinterpret_cast<uint32_t*>(sm + taddr_e(P2_DU, r + 8, col, 0)) =
-            pack2(acc[i][2], acc[i][3]);
+            packr<F16>(acc[i][2], acc[i][3]);
         *reinterpret_cast<uint32_t*>(sm + taddr_e(P2_DD, r, col, 0)) =
             pack2(acc[i][0] * d_lo, acc[i][1] * d_lo);
         *reinterpret_cast<uint32_t*>(sm + taddr_e(P2_DD, r + 8, col, 0)) =
@@ -659,7 +707,7 @@ __device__ __forceinline__ void delta_half(uint8_t* sm, uint32_t tb, uint32_t xt
 // states of P2_SAVE (a training forward whose gradients follow).
 constexpr int P2_OUT = 0, P2_SEGMENT = 1, P2_SAVE = 2, P2_OUT_SAVE = 3;
 
-template <int NS, typename IO, int MODE>
+template <int NS, typename IO, int MODE, bool F16>
 __global__ void __launch_bounds__(P2_THREADS, 1)
     state_pass_kernel(const __grid_constant__ CUtensorMap map_q,
                       const __grid_constant__ CUtensorMap map_k,
@@ -813,7 +861,7 @@ __global__ void __launch_bounds__(P2_THREADS, 1)
                     accQ[nt][2] *= gm_hi;
                     accQ[nt][3] *= gm_hi;
                 }
-                store_acc_bf16<NT>(sm, P2_X, 0, m0, accK, lane, 1.f, 1.f);
+                store_acc_r<NT, F16>(sm, P2_X, m0, accK, lane);
             }
             if (!bar_and<BAR_CHAIN, P2_CHAIN_THREADS>(ok)) break;
 
@@ -823,9 +871,9 @@ __global__ void __launch_bounds__(P2_THREADS, 1)
                 const int rb = warp & 3;
                 const float d_lo = rv[64 + m0 + g], d_hi = rv[64 + m0 + g + 8];
                 if (warp < 4)
-                    delta_half<NT, 0>(sm, st + ST_REC + REC_TB, sb + P2_X, rb, lane, d_lo, d_hi);
+                    delta_half<NT, 0, F16>(sm, st + ST_REC + REC_TB, sb + P2_X, rb, lane, d_lo, d_hi);
                 else
-                    delta_half<NT, 1>(sm, st + ST_REC + REC_TB, sb + P2_X, rb, lane, d_lo, d_hi);
+                    delta_half<NT, 1, F16>(sm, st + ST_REC + REC_TB, sb + P2_X, rb, lane, d_lo, d_hi);
             }
             if (!bar_and<BAR_CHAIN, P2_CHAIN_THREADS>(ok)) break;
 
@@ -860,8 +908,8 @@ __global__ void __launch_bounds__(P2_THREADS, 1)
                         for (int np = 0; np < NP; ++np) {
                             uint32_t b[4];
                             ldb_mn(sb + P2_DU, 0, 16 * np, 16 * ks, lane, b);
-                            mma16816(accQ[2 * np], a, b[0], b[1]);
-                            mma16816(accQ[2 * np + 1], a, b[2], b[3]);
+                            mma16816r<F16>(accQ[2 * np], a, b[0], b[1]);
+                            mma16816r<F16>(accQ[2 * np + 1], a, b[2], b[3]);
                         }
                     }
                 }
@@ -970,17 +1018,18 @@ __device__ __forceinline__ void tmem_cols(uint32_t ta, float* v) {
 }
 
 // Columns c0 .. c0 + N - 1 (c0, N multiples of 8) of row r of an MN-major
-// 128B-swizzled bf16 tile (one 64-column block), scaled by s.
-template <int N>
+// 128B-swizzled bf16 (or fp16) tile (one 64-column block), scaled by s.
+template <int N, bool F16 = false>
 __device__ __forceinline__ void put_cols(uint8_t* sm, uint32_t tile, int r, int c0, const float* v,
                                          float s) {
 #pragma unroll
     for (int i = 0; i < N / 8; ++i) {
         const int j = c0 / 8 + i;
         *reinterpret_cast<uint4*>(sm + tile + r * 128 + ((j ^ (r & 7)) << 4)) =
-            make_uint4(pack2(s * v[8 * i], s * v[8 * i + 1]), pack2(s * v[8 * i + 2], s * v[8 * i + 3]),
-                       pack2(s * v[8 * i + 4], s * v[8 * i + 5]),
-                       pack2(s * v[8 * i + 6], s * v[8 * i + 7]));
+            make_uint4(packr<F16>(s * v[8 * i], s * v[8 * i + 1]),
+                       packr<F16>(s * v[8 * i + 2], s * v[8 * i + 3]),
+                       packr<F16>(s * v[8 * i + 4], s * v[8 * i + 5]),
+                       packr<F16>(s * v[8 * i + 6], s * v[8 * i + 7]));
     }
 }
 
@@ -997,7 +1046,7 @@ __device__ __forceinline__ void store8<__nv_bfloat16>(__nv_bfloat16* p, const fl
                                               pack2(v[4], v[5]), pack2(v[6], v[7]));
 }
 
-template <int NS, typename IO>
+template <int NS, typename IO, bool F16>
 __global__ void __launch_bounds__(TC_THREADS, 1)
     state_tc_kernel(const __grid_constant__ CUtensorMap map_q,
                     const __grid_constant__ CUtensorMap map_k,
@@ -1005,8 +1054,11 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     static_assert(NS == 32 || NS == 48 || NS == 64, "slice width");
     constexpr int HN = NS / 2;                              // columns per half
     constexpr uint32_t ID_128 = idesc_bf16(128, NS, 0, 1);  // K-major A, MN-major B
-    constexpr uint32_t ID_64 = idesc_bf16(64, NS, 0, 1);    // the same, M = 64
     constexpr uint32_t ID_KT = idesc_bf16(128, NS, 1, 1);   // MN-major A (K^T), MN-major B
+    // the products with a record tile as A (T_b X, [T_b; M o Q K^T] Delta): fp16
+    // when the records are fp16, and then X and Delta are written as fp16 too
+    constexpr uint32_t ID_R64 = F16 ? idesc_f16(64, NS, 0, 1) : idesc_bf16(64, NS, 0, 1);
+    constexpr uint32_t ID_R128 = F16 ? idesc_f16(128, NS, 0, 1) : idesc_bf16(128, NS, 0, 1);
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
@@ -1152,7 +1204,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
                         x[8 * i + 2 * e + 1] = v2.y - g_row * x[8 * i + 2 * e + 1];
                     }
                 }
-                put_cols<HN>(sm, TC_X, row, c_lo, x, 1.f);
+                put_cols<HN, F16>(sm, TC_X, row, c_lo, x, 1.f);
                 fence_proxy_async_smem();
             }
         }
@@ -1165,7 +1217,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
 #pragma unroll
             for (int ks = 0; ks < 4; ++ks)
                 mma_bf16_ss(tmem + TM_DL, sdesc_sw128(st + TS_REC + ks * 32, 16, 1024),
-                            sdesc_sw128(sb + TC_X + ks * 2048, 8192, 1024), ID_64, ks > 0);
+                            sdesc_sw128(sb + TC_X + ks * 2048, 8192, 1024), ID_R64, ks > 0);
             mma_commit(bar_dl);
         }
         ok = mbar_wait(bar_dl, par, abort_flag);
@@ -1174,7 +1226,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
             float dl[HN];
             tmem_cols<HN>(tl + TM_DL, dl);
             if (lane < 16) {
-                put_cols<HN>(sm, TC_DU, r64, c_lo, dl, 1.f);
+                put_cols<HN, F16>(sm, TC_DU, r64, c_lo, dl, 1.f);
                 put_cols<HN>(sm, TC_DD, r64, c_lo, dl, d_row);
                 fence_proxy_async_smem();
             }
@@ -1193,7 +1245,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
 #pragma unroll
             for (int ks = 0; ks < 4; ++ks)
                 mma_bf16_ss(tmem + TM_O + 64 * par, sdesc_sw128(st + TS_REC + ks * 32, 16, 1024),
-                            sdesc_sw128(sb + TC_DU + ks * 2048, 8192, 1024), ID_128, ks > 0);
+                            sdesc_sw128(sb + TC_DU + ks * 2048, 8192, 1024), ID_R128, ks > 0);
             mma_commit(bar_o);
         }
         ok = mbar_wait(bar_u, par, abort_flag);
@@ -1238,10 +1290,10 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     }
 }
 
-template <int NS, typename IO>
+template <int NS, typename IO, bool F16>
 cudaError_t launch_state_tc(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                             const PrefillParams& prm, cudaStream_t stream) {
-    auto kern = state_tc_kernel<NS, IO>;
+    auto kern = state_tc_kernel<NS, IO, F16>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, TC_SMEM);
     if (e != cudaSuccess) return e;
     dim3 grid((D + NS - 1) / NS, prm.H_v, prm.N);
@@ -1385,10 +1437,10 @@ __global__ void __launch_bounds__(256)
         }
 }
 
-template <int NS, typename IO, int MODE>
+template <int NS, typename IO, int MODE, bool F16 = false>
 cudaError_t launch_pass2(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                          const PrefillParams& prm, int N, cudaStream_t stream) {
-    auto kern = state_pass_kernel<NS, IO, MODE>;
+    auto kern = state_pass_kernel<NS, IO, MODE, F16>;
     cudaError_t e =
         cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, P2_SMEM);
     if (e != cudaSuccess) return e;
@@ -1500,42 +1552,67 @@ int choose_segments(int N, int T, int H_v, int sms) {
     return best_p;
 }
 
+// The output state pass runs on tcgen05 when asked, or by default at 48-column
+// slices (the 16/48-head workload, where it measured faster); mma.sync at the
+// other widths (32-column slices: 0.82 vs 0.95 ms on a 2/6-head shard).
+static bool output_pass_is_tc(int state_pass, int slices) {
+    return state_pass == STATE_PASS_TC || (state_pass == STATE_PASS_AUTO && slices == 3);
+}
+
+template <typename IO, bool F16>
+static cudaError_t launch_state_tc_slices(const CUtensorMap& mq, const CUtensorMap& mk,
+                                          const CUtensorMap& mv, const PrefillParams& prm,
+                                          int slices, cudaStream_t stream) {
+    if (slices == 4) return launch_state_tc<32, IO, F16>(mq, mk, mv, prm, stream);
+    if (slices == 3) return launch_state_tc<48, IO, F16>(mq, mk, mv, prm, stream);
+    return launch_state_tc<64, IO, F16>(mq, mk, mv, prm, stream);
+}
+
+// f16_records: the records were written with fp16 tiles (read by the output
+// passes, P2_OUT; the other modes take bf16 records).
 template <typename IO, int MODE>
 static cudaError_t run_pass2(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                              const PrefillParams& prm, int sms, cudaStream_t stream,
-                             int state_pass = STATE_PASS_MMA) {
+                             int state_pass = STATE_PASS_MMA, bool f16_records = false) {
     // one block per SM at most (each holds ~212 KB of shared memory): split every
     // value head into as many d_v slices as still fit in one wave
     const long long units = (long long)prm.N * prm.H_v * (MODE == P2_SEGMENT ? 2 : 1);
     const int slices = pass2_slices(units, sms);
     if constexpr (MODE == P2_OUT) {
-        // the tcgen05 pass at 48-column slices (the 16/48-head workload, where it
-        // measured faster), mma.sync at the other widths (32-column slices: 0.82 vs
-        // 0.95 ms on a 2/6-head shard)
-        if (state_pass == STATE_PASS_TC || (state_pass == STATE_PASS_AUTO && slices == 3)) {
-            if (slices == 4) return launch_state_tc<32, IO>(mq, mk, mv, prm, stream);
-            if (slices == 3) return launch_state_tc<48, IO>(mq, mk, mv, prm, stream);
-            return launch_state_tc<64, IO>(mq, mk, mv, prm, stream);
+        if (output_pass_is_tc(state_pass, slices))
+            return f16_records
+                       ? launch_state_tc_slices<IO, true>(mq, mk, mv, prm, slices, stream)
+                       : launch_state_tc_slices<IO, false>(mq, mk, mv, prm, slices, stream);
+    }
+    if (f16_records) {
+        if constexpr (MODE == P2_OUT) {
+            if (slices == 4) return launch_pass2<32, IO, MODE, true>(mq, mk, mv, prm, prm.N, stream);
+            if (slices == 3) return launch_pass2<48, IO, MODE, true>(mq, mk, mv, prm, prm.N, stream);
+            return launch_pass2<64, IO, MODE, true>(mq, mk, mv, prm, prm.N, stream);
         }
+        return cudaErrorInvalidValue;  // the other modes read bf16 records
     }
     if (slices == 4) return launch_pass2<32, IO, MODE>(mq, mk, mv, prm, prm.N, stream);
     if (slices == 3) return launch_pass2<48, IO, MODE>(mq, mk, mv, prm, prm.N, stream);
     return launch_pass2<64, IO, MODE>(mq, mk, mv, prm, prm.N, stream);
 }
 
+// f16_records: write the records' tiles as fp16 (for the output passes of the
+// unsplit prefill; the segmented prefill and the gradients take bf16)
 static cudaError_t run_pass1(const CUtensorMap& mq, const CUtensorMap& mk,
-                             const PrefillParams& prm, cudaStream_t stream) {
-    cudaError_t e =
-        cudaFuncSetAttribute(chunk_ops_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, CO_SMEM);
+                             const PrefillParams& prm, cudaStream_t stream,
+                             bool f16_records = false) {
+    auto kern = f16_records ? chunk_ops_kernel<true> : chunk_ops_kernel<false>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, CO_SMEM);
     if (e != cudaSuccess) return e;
     // all of the unified L1 as shared memory, so that five CTAs fit on an SM
-    e = cudaFuncSetAttribute(chunk_ops_kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout,
                              cudaSharedmemCarveoutMaxShared);
     if (e != cudaSuccess) return e;
     const int group = prm.H_v / prm.H_qk;
     const long long slots = (long long)prm.N + ((long long)prm.T + C - 1) / C;
     dim3 grid((unsigned)slots, prm.H_qk, (group + P1_MAX_GROUP - 1) / P1_MAX_GROUP);
-    chunk_ops_kernel<<<grid, CO_THREADS, CO_SMEM, stream>>>(mq, mk, prm);
+    kern<<<grid, CO_THREADS, CO_SMEM, stream>>>(mq, mk, prm);
     return cudaGetLastError();
 }
 
@@ -1577,9 +1654,12 @@ cudaError_t launch_prefill(const void* q, const void* k, const void* v, const fl
         // through the chunks
         const PrefillParams prm{log_alpha, beta, S0,      cu_seqlens, o, S_final,
                                 records,   nullptr, H_qk, H_v,        N, T};
-        if ((e = run_pass1(mq, mk, prm, stream)) != cudaSuccess) return e;
-        return bf16 ? run_pass2<__nv_bfloat16, P2_OUT>(mq, mk, mv, prm, sms, stream, state_pass)
-                    : run_pass2<float, P2_OUT>(mq, mk, mv, prm, sms, stream, state_pass);
+        // the records' tiles in fp16: both output passes then carry X and Delta in
+        // fp16 (11 significant bits against bf16's 8)
+        const bool f16 = true;
+        if ((e = run_pass1(mq, mk, prm, stream, f16)) != cudaSuccess) return e;
+        return bf16 ? run_pass2<__nv_bfloat16, P2_OUT>(mq, mk, mv, prm, sms, stream, state_pass, f16)
+                    : run_pass2<float, P2_OUT>(mq, mk, mv, prm, sms, stream, state_pass, f16);
     }
     // segmented: N P virtual sequences
     const int Nv = N * P;
