@@ -21,11 +21,13 @@
 //
 // Three launches after the forward pass (chunk operators, then the state pass
 // saving every chunk's entering state):
-//   grad_state_kernel  one CTA per (sequence, value head, d_v slice): the
-//                      reverse chain over the chunks, carrying dS in registers;
-//                      writes dV, dS0 and every chunk's dS'.
-//   grad_chunk_kernel  one CTA per (chunk, query/key head), over the head's
-//                      value heads: dQ, dK, dbeta, dlog_alpha of the chunk.
+//   grad_state_kernel     one CTA per (sequence, value head, d_v slice): the
+//                         reverse chain over the chunks, carrying dS in
+//                         registers; writes dV, dS0 and every chunk's dS'.
+//   grad_chunk_tc_kernel  one CTA per (chunk, query/key head), over the head's
+//                         value heads: dQ, dK, dbeta, dlog_alpha of the chunk,
+//                         its products on the fifth-generation tensor cores
+//                         with dQ and dK accumulated in tensor memory.
 #include <cudaTypedefs.h>
 
 #include "gdn_common.cuh"
@@ -71,22 +73,6 @@ __device__ __forceinline__ void mma_rows(float (*acc)[4], uint32_t a, uint32_t a
             mma16816(acc[2 * p], af, bf[0], bf[1]);
             mma16816(acc[2 * p + 1], af, bf[2], bf[3]);
         }
-    }
-}
-
-// Accumulators (rows m0 + g (+8), columns c0 + 8 nt + 2 t (+1)) as bf16 into a
-// swizzled 64-column tile.
-template <int NT>
-__device__ __forceinline__ void store_acc_cols(uint8_t* smem, uint32_t base_off, int m0, int c0,
-                                               const float (*acc)[4], int lane) {
-    const int g = lane >> 2, t = lane & 3;
-#pragma unroll
-    for (int nt = 0; nt < NT; ++nt) {
-        const int col = c0 + 8 * nt + 2 * t;
-        *reinterpret_cast<uint32_t*>(smem + taddr_e(base_off, m0 + g, col, 0)) =
-            pack2(acc[nt][0], acc[nt][1]);
-        *reinterpret_cast<uint32_t*>(smem + taddr_e(base_off, m0 + g + 8, col, 0)) =
-            pack2(acc[nt][2], acc[nt][3]);
     }
 }
 
@@ -321,29 +307,7 @@ __global__ void __launch_bounds__(256, 1)
     __syncthreads();
 }
 
-// ============================================================================
-// Per-chunk gradients.  Grid (record slots, H_qk); 256 threads, one CTA per SM.
-// Warp w: rows 16 (w & 3) of the 64-row products; column half (w >> 2) of the
-// 128-wide ones (64 columns) or of the 64-wide ones (32 columns).
-// ============================================================================
-constexpr uint32_t GC_K = 0;                    // K, 64 x 128 (two halves)
-constexpr uint32_t GC_Q = 2 * HALF;             // Q
-constexpr uint32_t GC_V = 4 * HALF;             // V, then X in place
-constexpr uint32_t GC_O = 6 * HALF;             // dO
-constexpr uint32_t SHALF = 16384;               // a 128-row half of a 128 x 128 tile
-constexpr uint32_t GC_S = 8 * HALF;             // S (entering state), 128 x 128
-constexpr uint32_t GC_DS = GC_S + 2 * SHALF;    // dS' (gradient of the state after)
-constexpr uint32_t GC_REC = GC_DS + 2 * SHALF;  // the chunk's operator record
-constexpr uint32_t GC_DEL = GC_REC + ((REC_BYTES + 1023) / 1024) * 1024;  // Delta
-constexpr uint32_t GC_DDEL = GC_DEL + 2 * HALF;                          // dDelta
-constexpr uint32_t GC_DX = GC_DDEL + 2 * HALF;                           // dX
-constexpr uint32_t GC_PY = GC_DX + 2 * HALF;    // P (then Y), 64 x 64
-constexpr uint32_t GC_TE = GC_PY + HALF;        // dT_b (then E), 64 x 64
-constexpr uint32_t GC_F = GC_TE + HALF;         // fp32: g2[64], dg[64], dbeta[64], misc[64]
-constexpr uint32_t GC_BAR = GC_F + 4 * 64 * 4;  // three mbarriers
-constexpr uint32_t GC_MISC = GC_BAR + 24;
-constexpr uint32_t GC_SMEM = GC_MISC + 16 + 1024;
-static_assert(GC_SMEM <= 232448, "per-chunk gradient shared memory budget");
+constexpr uint32_t SHALF = 16384;  // a 128-row half of a 128 x 128 state image
 
 // This thread's part of sum(S o dS') over two bf16 state tiles of the same
 // layout (each thread 128 bytes of each).
@@ -365,66 +329,141 @@ __device__ __forceinline__ float tile_dot(const uint8_t* a, const uint8_t* b, in
     return dot;
 }
 
-// Row sums (over the accumulator's columns) of acc o w, into dst[row] (smem,
-// atomically): rows m0 + g and m0 + g + 8, scaled by s_lo and s_hi.
-template <int NT>
-__device__ __forceinline__ void add_row_sums(float* dst, int m0, const float (*v)[4], int lane,
-                                             float s_lo, float s_hi) {
-    float lo = 0.f, hi = 0.f;
-#pragma unroll
-    for (int nt = 0; nt < NT; ++nt) {
-        lo += v[nt][0] + v[nt][1];
-        hi += v[nt][2] + v[nt][3];
-    }
-    lo += __shfl_xor_sync(0xffffffffu, lo, 1);
-    lo += __shfl_xor_sync(0xffffffffu, lo, 2);
-    hi += __shfl_xor_sync(0xffffffffu, hi, 1);
-    hi += __shfl_xor_sync(0xffffffffu, hi, 2);
-    if ((lane & 3) == 0) {
-        const int g = lane >> 2;
-        atomicAdd(&dst[m0 + g], s_lo * lo);
-        atomicAdd(&dst[m0 + g + 8], s_hi * hi);
-    }
+template <int NS, typename IO>
+cudaError_t launch_grad_state(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mo,
+                              const GradParams& prm, cudaStream_t stream) {
+    auto kern = grad_state_kernel<NS, IO>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, GS_SMEM);
+    if (e != cudaSuccess) return e;
+    kern<<<dim3((D + NS - 1) / NS, prm.H_v, prm.N), 256, GS_SMEM, stream>>>(mq, mk, mo, prm);
+    return cudaGetLastError();
 }
-// Column sums (over the accumulator's 16 rows) of v, into dst[n0 + col] with
-// factor s.
-template <int NT>
-__device__ __forceinline__ void add_col_sums(float* dst, int n0, const float (*v)[4], int lane,
-                                             float s) {
+
+// ============================================================================
+// Per-chunk gradients on the fifth-generation tensor cores.  Grid (record
+// slots, H_qk); 256 threads; one CTA per SM (all 512 TMEM columns).  Per value
+// head of the query/key head, twelve steps (numbered in the kernel) form
+// K S and Q S, X, Delta, dDelta, dX, P, the dQ and dK terms, dT_b, Y and E,
+// and the gate gradients, following the formulas at the top of this file.
+// Each product is a tcgen05.mma group issued by thread 0, its accumulator in
+// tensor memory:
+//   columns   0-127  dQ, accumulated over the query/key head's value heads
+//   columns 128-255  dK, likewise
+//   columns 256-383  T1 and 384-511 T2: one step's products
+// Warp w reads TMEM lanes 32 (w % 4) .. + 31 (an M = 128 product's rows, or,
+// in its lanes 0-15, rows 16 (w % 4) .. + 15 of an M = 64 product) and the
+// column half w / 4.  Every operand is one of the kernel's 128B-swizzled bf16
+// tiles: a tile stored [rows][columns] is K-major for a product contracting
+// over its columns and MN-major for one contracting over its rows, so the
+// transposes of the chunk form (T_b^T, (M o QK^T)^T, P^T, E^T, S^T, dS'^T,
+// X^T, Delta^T) are descriptors, not copies.
+// ============================================================================
+constexpr uint32_t GT_KQ = 0;                   // K h0 | Q h0 | K h1 | Q h1 (token rows)
+constexpr uint32_t GT_V = 4 * HALF;             // V, then X in place (halves HALF apart)
+constexpr uint32_t GT_O = 6 * HALF;             // dO, then gamma o dO in place
+constexpr uint32_t GT_S = 8 * HALF;             // S image (halves SHALF apart)
+constexpr uint32_t GT_DS = GT_S + 2 * SHALF;    // dS' image
+constexpr uint32_t GT_REC = GT_DS + 2 * SHALF;  // the chunk's operator record (bf16 tiles)
+constexpr uint32_t GT_DEL = GT_REC + ((REC_BYTES + 1023) / 1024) * 1024;  // Delta, then d o Delta
+constexpr uint32_t GT_DDEL = GT_DEL + 2 * HALF;                          // dDelta
+constexpr uint32_t GT_DX = GT_DDEL + 2 * HALF;  // K S in bf16, then -gamma o dX
+constexpr uint32_t GT_PY = GT_DX + 2 * HALF;    // P, then Y (64 x 64)
+constexpr uint32_t GT_TE = GT_PY + HALF;        // dT_b, then E (64 x 64)
+constexpr uint32_t GT_F = GT_TE + HALF;         // fp32: g2[64], dg[64], dbt[64], misc[64]
+constexpr uint32_t GT_BAR = GT_F + 4 * 64 * 4;  // K/Q copies, head copies, record copy,
+                                                // products, drain
+constexpr uint32_t GT_MISC = GT_BAR + 40;       // abort flag, TMEM base
+constexpr uint32_t GT_SMEM = GT_MISC + 16 + 1024;
+static_assert(GT_SMEM <= 232448, "tcgen05 per-chunk gradient shared memory budget");
+static_assert(GT_DEL % 1024 == 0, "swizzled tiles sit on 1 KB");
+constexpr uint32_t GT_DQ = 0, GT_DK = 128, GT_T1 = 256, GT_T2 = 384, GT_COLS = 512;
+
+// K-major operand: tile rows index M (or N), tile columns the contraction, in
+// 64-column halves hs bytes apart; k step ks covers columns 16 ks .. + 15.
+__device__ __forceinline__ uint64_t kdesc(uint32_t tile, uint32_t hs, int ks) {
+    return sdesc_sw128(tile + (uint32_t)(ks >> 2) * hs + (uint32_t)(ks & 3) * 32, 16, 1024);
+}
+// MN-major operand: tile rows index the contraction, tile columns M (or N), in
+// 64-column blocks bs bytes apart; k step ks covers rows 16 ks .. + 15.
+__device__ __forceinline__ uint64_t mdesc(uint32_t tile, uint32_t bs, int ks) {
+    return sdesc_sw128(tile + (uint32_t)ks * 2048, bs, 1024);
+}
+
+// Column sums over lanes 0-15 of a warp of v[0..31] (lanes 16-31 reduce among
+// themselves): lane l < 16 ends with the sums of columns 2l and 2l + 1 in
+// v[0], v[1].  Four halving exchanges, 30 shuffles.
+__device__ __forceinline__ void colsum16(float* v, int lane) {
 #pragma unroll
-    for (int nt = 0; nt < NT; ++nt) {
-        float c0 = v[nt][0] + v[nt][2], c1 = v[nt][1] + v[nt][3];
+    for (int w = 16, m = 8; m >= 1; w >>= 1, m >>= 1) {
+        const bool up = (lane & m) != 0;
 #pragma unroll
-        for (int off = 4; off < 32; off <<= 1) {
-            c0 += __shfl_xor_sync(0xffffffffu, c0, off);
-            c1 += __shfl_xor_sync(0xffffffffu, c1, off);
-        }
-        if (lane < 4) {
-            atomicAdd(&dst[n0 + 8 * nt + 2 * lane], s * c0);
-            atomicAdd(&dst[n0 + 8 * nt + 2 * lane + 1], s * c1);
+        for (int i = 0; i < w; ++i) {
+            const float send = up ? v[i] : v[w + i];
+            const float keep = up ? v[w + i] : v[i];
+            v[i] = keep + __shfl_xor_sync(0xffffffffu, send, m);
         }
     }
 }
 
+// 16 bf16 values at row r, columns c .. c + 15 (c a multiple of 8) of a swizzled
+// tile whose 64-column halves lie hs bytes apart.
+__device__ __forceinline__ void ld16_bf16(const uint8_t* sm, uint32_t tile, uint32_t hs, int r,
+                                          int c, float* v) {
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        const uint4 u = *reinterpret_cast<const uint4*>(sm + taddr(tile, r, c + 8 * h, hs));
+        const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[e]));
+            v[8 * h + 2 * e] = f.x;
+            v[8 * h + 2 * e + 1] = f.y;
+        }
+    }
+}
+__device__ __forceinline__ void st16_bf16(uint8_t* sm, uint32_t tile, uint32_t hs, int r, int c,
+                                          const float* v, float s) {
+#pragma unroll
+    for (int h = 0; h < 2; ++h)
+        *reinterpret_cast<uint4*>(sm + taddr(tile, r, c + 8 * h, hs)) =
+            make_uint4(pack2(s * v[8 * h], s * v[8 * h + 1]), pack2(s * v[8 * h + 2], s * v[8 * h + 3]),
+                       pack2(s * v[8 * h + 4], s * v[8 * h + 5]),
+                       pack2(s * v[8 * h + 6], s * v[8 * h + 7]));
+}
+// Two 16-column TMEM reads of this warp's lanes, then the wait.
+__device__ __forceinline__ void tld2x16(uint32_t a0, float* v0, uint32_t a1, float* v1) {
+    tmem_ld16(a0, v0);
+    tmem_ld16(a1, v1);
+    tmem_ld_wait();
+}
+
 template <typename IO>
 __global__ void __launch_bounds__(256, 1)
-    grad_chunk_kernel(const __grid_constant__ CUtensorMap map_q,
-                      const __grid_constant__ CUtensorMap map_k,
-                      const __grid_constant__ CUtensorMap map_v,
-                      const __grid_constant__ CUtensorMap map_do, const GradParams p) {
+    grad_chunk_tc_kernel(const __grid_constant__ CUtensorMap map_q,
+                         const __grid_constant__ CUtensorMap map_k,
+                         const __grid_constant__ CUtensorMap map_v,
+                         const __grid_constant__ CUtensorMap map_do, const GradParams p) {
+    constexpr uint32_t ID_128_KM = idesc_bf16(128, 128, 0, 1);  // M = 128, N = 128, A K-major, B MN-major
+    constexpr uint32_t ID_KM = idesc_bf16(64, 128, 0, 1);
+    constexpr uint32_t ID_MM = idesc_bf16(64, 128, 1, 1);
+    constexpr uint32_t ID_KK = idesc_bf16(64, 128, 0, 0);
+    constexpr uint32_t ID64_KK = idesc_bf16(64, 64, 0, 0);      // N = 64
+    constexpr uint32_t ID64_MM = idesc_bf16(64, 64, 1, 1);
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
     const uint32_t sb = smem_u32(sm);
-    uint64_t* bars = reinterpret_cast<uint64_t*>(sm + GC_BAR);
-    volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + GC_MISC);
-    float* g2 = reinterpret_cast<float*>(sm + GC_F);  // cumulative log2 gates
+    uint64_t* bars = reinterpret_cast<uint64_t*>(sm + GT_BAR);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + GT_MISC);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + GT_MISC + 4);
+    float* g2 = reinterpret_cast<float*>(sm + GT_F);  // cumulative log2 gates
     float* dg = g2 + 64;                              // gradient w.r.t. g (natural log)
     float* dbt = g2 + 128;                            // dbeta * beta
-    float* misc = g2 + 192;                           // [0] sum ddv, [1] <dS', S>, [2..] beta
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, g = lane >> 2, t4 = lane & 3;
-    const int rb = warp & 3, hh = warp >> 2;
-    const int m0 = 16 * rb;
+    float* misc = g2 + 192;                           // [0] sum ddv, [1] <dS', S>
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int quad = warp & 3, chalf = warp >> 2;
+    const bool lo16 = lane < 16;
+    const int r64 = 16 * quad + (lane & 15);  // my row of an M = 64 product (lanes < 16)
     int n, c;
     slot_owner(p.cu_seqlens, p.N, blockIdx.x, n, c);
     if (n < 0) return;  // uniform across the CTA
@@ -436,72 +475,99 @@ __global__ void __launch_bounds__(256, 1)
     const long long slot = record_slot(n, tc0);
 
     if (tid == 0) {
-        for (int i = 0; i < 3; ++i) mbar_init(&bars[i], 1);
+        for (int i = 0; i < 5; ++i) mbar_init(&bars[i], 1);
         *abort_flag = 0;
         fence_mbar_init();
     }
+    if (warp == 0) {
+        tmem_alloc(tmem_slot, GT_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
     __syncthreads();
-    // value head vh's V, dO and saved states (bf16 images, straight into their
-    // tiles) on bars[1]; its record on bars[2]
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const uint32_t tq = tmem + ((uint32_t)(32 * quad) << 16);  // my lane quadrant
+
+    // value head vh's V, dO and saved states on bars[1]; its record on bars[2]
     auto issue_head = [&](int vh) {
         const int h = hq * group + vh;
         const size_t so = ((size_t)slot * p.H_v + h) * STATE_IMAGE_BYTES;
         mbar_arrive_expect_tx(&bars[1], 4 * HALF + 2 * STATE_IMAGE_BYTES);
-        tma_load_2d(sm + GC_V, &map_v, h * D, tc0, &bars[1]);
-        tma_load_2d(sm + GC_V + HALF, &map_v, h * D + 64, tc0, &bars[1]);
-        tma_load_2d(sm + GC_O, &map_do, h * D, tc0, &bars[1]);
-        tma_load_2d(sm + GC_O + HALF, &map_do, h * D + 64, tc0, &bars[1]);
-        bulk_load(sm + GC_S, p.S_saved + so, STATE_IMAGE_BYTES, &bars[1]);
-        bulk_load(sm + GC_DS, p.dS_saved + so, STATE_IMAGE_BYTES, &bars[1]);
+        tma_load_2d(sm + GT_V, &map_v, h * D, tc0, &bars[1]);
+        tma_load_2d(sm + GT_V + HALF, &map_v, h * D + 64, tc0, &bars[1]);
+        tma_load_2d(sm + GT_O, &map_do, h * D, tc0, &bars[1]);
+        tma_load_2d(sm + GT_O + HALF, &map_do, h * D + 64, tc0, &bars[1]);
+        bulk_load(sm + GT_S, p.S_saved + so, STATE_IMAGE_BYTES, &bars[1]);
+        bulk_load(sm + GT_DS, p.dS_saved + so, STATE_IMAGE_BYTES, &bars[1]);
     };
     auto issue_rec = [&](int vh) {
         const int h = hq * group + vh;
         mbar_arrive_expect_tx(&bars[2], REC_BYTES);
-        bulk_load(sm + GC_REC, p.records + (size_t)(slot * p.H_v + h) * REC_BYTES, REC_BYTES,
+        bulk_load(sm + GT_REC, p.records + (size_t)(slot * p.H_v + h) * REC_BYTES, REC_BYTES,
                   &bars[2]);
     };
     int heads = 0, recs = 0;  // copies issued (thread 0)
-    // after a failed wait: let every copy in flight land (bounded), then leave
-    auto drain = [&]() {
+    uint32_t groups = 0;      // product groups committed (every thread counts them)
+    // After a failed wait: every copy and product in flight completes (bounded
+    // waits), then the tensor memory is freed.
+    auto leave = [&]() {
         if (tid == 0) {
             mbar_wait_drain(&bars[0], 0);
             if (heads > 0) mbar_wait_drain(&bars[1], (heads - 1) & 1);
             if (recs > 0) mbar_wait_drain(&bars[2], (recs - 1) & 1);
+            mma_commit(&bars[4]);  // a barrier of its own: its first phase covers every product
+            mbar_wait_drain(&bars[4], 0);
         }
+        tc_fence_before();
         __syncthreads();
+        if (warp == 0) {
+            tc_fence_after();
+            tmem_dealloc(tmem, GT_COLS);
+        }
     };
+    // commit the products thread 0 issued since the last commit; every thread waits
+    auto commit_wait = [&]() -> bool {
+        if (tid == 0) mma_commit(&bars[3]);
+        const bool ok = mbar_wait(&bars[3], groups & 1, abort_flag);
+        ++groups;
+        tc_fence_after();
+        return ok;
+    };
+    // generic writes of operand tiles are made visible to the tensor cores, and
+    // TMEM reads are ordered before the next products
+    auto publish = [&](bool ok) -> bool {
+        fence_proxy_async_smem();
+        tc_fence_before();
+        return __syncthreads_and(ok);
+    };
+
     if (tid == 0) {
         mbar_arrive_expect_tx(&bars[0], 4 * HALF);
-        tma_load_2d(sm + GC_K, &map_k, hq * D, tc0, &bars[0]);
-        tma_load_2d(sm + GC_K + HALF, &map_k, hq * D + 64, tc0, &bars[0]);
-        tma_load_2d(sm + GC_Q, &map_q, hq * D, tc0, &bars[0]);
-        tma_load_2d(sm + GC_Q + HALF, &map_q, hq * D + 64, tc0, &bars[0]);
+        tma_load_2d(sm + GT_KQ, &map_k, hq * D, tc0, &bars[0]);
+        tma_load_2d(sm + GT_KQ + HALF, &map_q, hq * D, tc0, &bars[0]);
+        tma_load_2d(sm + GT_KQ + 2 * HALF, &map_k, hq * D + 64, tc0, &bars[0]);
+        tma_load_2d(sm + GT_KQ + 3 * HALF, &map_q, hq * D + 64, tc0, &bars[0]);
         issue_head(0);
         issue_rec(0);
         heads = recs = 1;
     }
     bool ok = mbar_wait(&bars[0], 0, abort_flag);
     if (!__syncthreads_and(ok)) {
-        drain();
+        leave();
         return;
     }
     if (valid < C) {  // rows past the sequence end belong to the next sequence: zero them
         for (int i = tid; i < 4 * 64 * 8; i += 256) {
             const int tile = i / 512, row = (i >> 3) & 63, ch = i & 7;
             if (row >= valid)
-                *reinterpret_cast<uint4*>(sm + tile * HALF + row * 128 + ch * 16) =
+                *reinterpret_cast<uint4*>(sm + GT_KQ + tile * HALF + row * 128 + ch * 16) =
                     make_uint4(0, 0, 0, 0);
         }
     }
-    __syncthreads();
-
-    float dQ[8][4], dK[8][4];  // rows m0.., columns 64 hh .. 64 hh + 63
-    zero_acc<8>(dQ);
-    zero_acc<8>(dK);
 
     for (int vh = 0; vh < group; ++vh) {
         const int h = hq * group + vh;
-        // the gates (while this head's copies land)
         if (tid < 64) {
             dg[tid] = 0.f;
             dbt[tid] = 0.f;
@@ -526,11 +592,11 @@ __global__ void __launch_bounds__(256, 1)
         ok = mbar_wait(&bars[1], vh & 1, abort_flag);
         ok = mbar_wait(&bars[2], vh & 1, abort_flag) && ok;
         if (!__syncthreads_and(ok)) {
-            drain();
+            leave();
             return;
         }
         {  // <dS', S>, for the gate gradient of the chunk's last row
-            float dot = tile_dot(sm + GC_S, sm + GC_DS, tid);
+            float dot = tile_dot(sm + GT_S, sm + GT_DS, tid);
 #pragma unroll
             for (int off = 16; off > 0; off >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, off);
             if (lane == 0) atomicAdd(&misc[1], dot);
@@ -539,229 +605,370 @@ __global__ void __launch_bounds__(256, 1)
             for (int i = tid; i < 4 * 64 * 8; i += 256) {
                 const int tile = i / 512, row = (i >> 3) & 63, ch = i & 7;
                 if (row >= valid)
-                    *reinterpret_cast<uint4*>(sm + GC_V + tile * HALF + row * 128 + ch * 16) =
+                    *reinterpret_cast<uint4*>(sm + GT_V + tile * HALF + row * 128 + ch * 16) =
                         make_uint4(0, 0, 0, 0);
             }
-            __syncthreads();
         }
-        const float* rv = reinterpret_cast<const float*>(sm + GC_REC + REC_VEC);
-        const uint32_t tb = sb + GC_REC + REC_TB, mq = sb + GC_REC + REC_MQ;
-        const int n0 = 64 * hh;  // this warp's columns of the 128-wide products
-        const float gm_lo = rv[m0 + g], gm_hi = rv[m0 + g + 8];
-        const float d_lo = rv[64 + m0 + g], d_hi = rv[64 + m0 + g + 8];
+        const float* rv = reinterpret_cast<const float*>(sm + GT_REC + REC_VEC);
         const float gam_C = rv[128];
+        const float gm64 = lo16 ? rv[r64] : 0.f;      // gamma of my M = 64 row
+        const float d64 = lo16 ? rv[64 + r64] : 0.f;  // d of my M = 64 row
+        if (!publish(true)) {
+            leave();
+            return;
+        }
 
-        // 1. K S (kept for dg), Q S -> dg += gamma_r dO_r . (QS)_r; X = V - gamma o KS
-        float KS[8][4];
-        {
-            zero_acc<8>(KS);
-            mma_rows<4, true, false>(KS, sb + GC_K, HALF, m0, sb + GC_S, SHALF, n0, 0, 8, lane);
-            float QS[8][4];
-            zero_acc<8>(QS);
-            mma_rows<4, true, false>(QS, sb + GC_Q, HALF, m0, sb + GC_S, SHALF, n0, 0, 8, lane);
+        // 1. K S (kept for dg, as bf16 in the dX tile), Q S -> dg += gamma_r dO_r . (QS)_r;
+        //    X = V - gamma o KS in place over V
+        if (tid == 0) {
+            tc_fence_after();
 #pragma unroll
-            for (int nt = 0; nt < 8; ++nt) {
-                const int col = n0 + 8 * nt + 2 * t4;
-                const float2 o_lo = ld_bf16x2(sm + taddr_e(GC_O, m0 + g, col, HALF));
-                const float2 o_hi = ld_bf16x2(sm + taddr_e(GC_O, m0 + g + 8, col, HALF));
-                QS[nt][0] *= o_lo.x;
-                QS[nt][1] *= o_lo.y;
-                QS[nt][2] *= o_hi.x;
-                QS[nt][3] *= o_hi.y;
-                const float2 v_lo = ld_bf16x2(sm + taddr_e(GC_V, m0 + g, col, HALF));
-                const float2 v_hi = ld_bf16x2(sm + taddr_e(GC_V, m0 + g + 8, col, HALF));
-                *reinterpret_cast<uint32_t*>(sm + taddr_e(GC_V, m0 + g, col, HALF)) =
-                    pack2(v_lo.x - gm_lo * KS[nt][0], v_lo.y - gm_lo * KS[nt][1]);
-                *reinterpret_cast<uint32_t*>(sm + taddr_e(GC_V, m0 + g + 8, col, HALF)) =
-                    pack2(v_hi.x - gm_hi * KS[nt][2], v_hi.y - gm_hi * KS[nt][3]);
-            }
-            add_row_sums<8>(dg, m0, QS, lane, gm_lo, gm_hi);
+            for (int ks = 0; ks < 8; ++ks)
+                mma_bf16_ss(tmem + GT_T1, kdesc(sb + GT_KQ, 2 * HALF, ks), mdesc(sb + GT_S, SHALF, ks),
+                            ID_128_KM, ks > 0);
         }
-        __syncthreads();
-        // 2. Delta = T_b X (T_b lower triangular: key blocks 0 .. rb)
+        ok = commit_wait();
         {
-            float acc[8][4];
-            zero_acc<8>(acc);
-            mma_rows<4, true, false>(acc, tb, 0, m0, sb + GC_V, HALF, n0, 0, rb + 1, lane);
-            store_acc_bf16<8>(sm, GC_DEL + (hh ? HALF : 0), 0, m0, acc, lane, 1.f, 1.f);
+            const int row = 32 * (quad & 1) + lane;  // token row
+            const float gm = rv[row];
+            float s = 0.f;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const int col = 64 * chalf + 16 * i;
+                float a[16], b[16];
+                tmem_ld16(tq + GT_T1 + col, a);
+                tmem_ld_wait();
+                if (quad < 2) {
+                    ld16_bf16(sm, GT_V, HALF, row, col, b);
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) b[e] -= gm * a[e];
+                    st16_bf16(sm, GT_V, HALF, row, col, b, 1.f);
+                    st16_bf16(sm, GT_DX, HALF, row, col, a, 1.f);
+                } else {
+                    ld16_bf16(sm, GT_O, HALF, row, col, b);
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) s = fmaf(a[e], b[e], s);
+                }
+            }
+            if (quad >= 2) atomicAdd(&dg[row], gm * s);
         }
-        __syncthreads();
+        if (!publish(ok)) {
+            leave();
+            return;
+        }
+
+        // 2. Delta = T_b X
+        if (tid == 0) {
+            tc_fence_after();
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks)
+                mma_bf16_ss(tmem + GT_T2, kdesc(sb + GT_REC + REC_TB, HALF, ks),
+                            mdesc(sb + GT_V, HALF, ks), ID_KM, ks > 0);
+        }
+        ok = commit_wait();
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const int col = 64 * chalf + 16 * i;
+            float a[16];
+            tmem_ld16(tq + GT_T2 + col, a);
+            tmem_ld_wait();
+            if (lo16) st16_bf16(sm, GT_DEL, HALF, r64, col, a, 1.f);
+        }
+        if (!publish(ok)) {
+            leave();
+            return;
+        }
+
         // 3. dDelta = (M o QK^T)^T dO + d o (K dS');  ddv_r = d_r (K dS')_r . Delta_r
+        if (tid == 0) {
+            tc_fence_after();
+#pragma unroll
+            for (int ks = 0; ks < 8; ++ks)
+                mma_bf16_ss(tmem + GT_T1, kdesc(sb + GT_KQ, 2 * HALF, ks), mdesc(sb + GT_DS, SHALF, ks),
+                            ID_KM, ks > 0);
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks)
+                mma_bf16_ss(tmem + GT_T2, mdesc(sb + GT_REC + REC_MQ, HALF, ks),
+                            mdesc(sb + GT_O, HALF, ks), ID_MM, ks > 0);
+        }
+        ok = commit_wait();
         {
-            float KD[8][4], acc[8][4];
-            zero_acc<8>(KD);
-            zero_acc<8>(acc);
-            mma_rows<4, true, false>(KD, sb + GC_K, HALF, m0, sb + GC_DS, SHALF, n0, 0, 8, lane);
-            mma_rows<4, false, false>(acc, mq, 0, m0, sb + GC_O, HALF, n0, rb, 4, lane);
-            float ddv[8][4];
+            float ddv = 0.f;
 #pragma unroll
-            for (int nt = 0; nt < 8; ++nt) {
-                const int col = n0 + 8 * nt + 2 * t4;
-                const float2 e_lo = ld_bf16x2(sm + taddr_e(GC_DEL, m0 + g, col, HALF));
-                const float2 e_hi = ld_bf16x2(sm + taddr_e(GC_DEL, m0 + g + 8, col, HALF));
-                ddv[nt][0] = KD[nt][0] * e_lo.x;
-                ddv[nt][1] = KD[nt][1] * e_lo.y;
-                ddv[nt][2] = KD[nt][2] * e_hi.x;
-                ddv[nt][3] = KD[nt][3] * e_hi.y;
-                acc[nt][0] = fmaf(d_lo, KD[nt][0], acc[nt][0]);
-                acc[nt][1] = fmaf(d_lo, KD[nt][1], acc[nt][1]);
-                acc[nt][2] = fmaf(d_hi, KD[nt][2], acc[nt][2]);
-                acc[nt][3] = fmaf(d_hi, KD[nt][3], acc[nt][3]);
+            for (int i = 0; i < 4; ++i) {
+                const int col = 64 * chalf + 16 * i;
+                float kd[16], ao[16];
+                tld2x16(tq + GT_T1 + col, kd, tq + GT_T2 + col, ao);
+                if (lo16) {
+                    float dl[16];
+                    ld16_bf16(sm, GT_DEL, HALF, r64, col, dl);
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) {
+                        ddv = fmaf(kd[e], dl[e], ddv);
+                        ao[e] = fmaf(d64, kd[e], ao[e]);
+                    }
+                    st16_bf16(sm, GT_DDEL, HALF, r64, col, ao, 1.f);
+                }
             }
-            // -ddv_r into dg_r; their total goes to dg of the last row (misc[0])
-            add_row_sums<8>(dg, m0, ddv, lane, -d_lo, -d_hi);
-            float tot = 0.f;
-#pragma unroll
-            for (int nt = 0; nt < 8; ++nt)
-                tot += d_lo * (ddv[nt][0] + ddv[nt][1]) + d_hi * (ddv[nt][2] + ddv[nt][3]);
+            // -d_r ddv_r into dg_r; the total goes to dg of the last row (misc[0])
+            if (lo16) atomicAdd(&dg[r64], -d64 * ddv);
+            float tot = d64 * ddv;  // zero on lanes 16-31
 #pragma unroll
             for (int off = 16; off > 0; off >>= 1) tot += __shfl_xor_sync(0xffffffffu, tot, off);
             if (lane == 0) atomicAdd(&misc[0], tot);
-            store_acc_bf16<8>(sm, GC_DDEL + (hh ? HALF : 0), 0, m0, acc, lane, 1.f, 1.f);
         }
-        __syncthreads();
-        // 4. dX = T_b^T dDelta (upper triangular: key blocks rb .. 3); dg -= gamma_r dX_r . KS_r
-        {
-            float acc[8][4];
-            zero_acc<8>(acc);
-            mma_rows<4, false, false>(acc, tb, 0, m0, sb + GC_DDEL, HALF, n0, rb, 4, lane);
-            store_acc_bf16<8>(sm, GC_DX + (hh ? HALF : 0), 0, m0, acc, lane, 1.f, 1.f);
-#pragma unroll
-            for (int nt = 0; nt < 8; ++nt)
-#pragma unroll
-                for (int e = 0; e < 4; ++e) KS[nt][e] *= acc[nt][e];
-            add_row_sums<8>(dg, m0, KS, lane, -gm_lo, -gm_hi);
+        if (!publish(ok)) {
+            leave();
+            return;
         }
-        __syncthreads();
-        // 5. P = M o (dO Delta^T) (64 x 64: columns 32 hh ..); dg gets the rows and
-        // columns of P o (M o QK^T)
-        {
-            const int p0 = 32 * hh;
-            float acc[4][4];
-            zero_acc<4>(acc);
-            mma_rows<2, true, true>(acc, sb + GC_O, HALF, m0, sb + GC_DEL, HALF, p0, 0, 8, lane);
-            float pm[4][4];
+
+        // 4. dX = T_b^T dDelta;  dg -= gamma_r dX_r . KS_r;  the dX tile <- -gamma o dX
+        if (tid == 0) {
+            tc_fence_after();
 #pragma unroll
-            for (int nt = 0; nt < 4; ++nt)
+            for (int ks = 0; ks < 4; ++ks)
+                mma_bf16_ss(tmem + GT_T1, mdesc(sb + GT_REC + REC_TB, HALF, ks),
+                            mdesc(sb + GT_DDEL, HALF, ks), ID_MM, ks > 0);
+        }
+        ok = commit_wait();
+        {
+            float s = 0.f;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const int col = 64 * chalf + 16 * i;
+                float dx[16];
+                tmem_ld16(tq + GT_T1 + col, dx);
+                tmem_ld_wait();
+                if (lo16) {
+                    float ksv[16];
+                    ld16_bf16(sm, GT_DX, HALF, r64, col, ksv);
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) s = fmaf(dx[e], ksv[e], s);
+                    st16_bf16(sm, GT_DX, HALF, r64, col, dx, -gm64);
+                }
+            }
+            if (lo16) atomicAdd(&dg[r64], -gm64 * s);
+        }
+        if (!publish(ok)) {
+            leave();
+            return;
+        }
+
+        // 5. P = M o (dO Delta^T) (64 x 64); dg gets the rows and columns of
+        //    P o (M o QK^T).  Then dO <- gamma o dO and Delta <- d o Delta in place
+        //    (their last reads as they are were steps 3 and 5).
+        if (tid == 0) {
+            tc_fence_after();
+#pragma unroll
+            for (int ks = 0; ks < 8; ++ks)
+                mma_bf16_ss(tmem + GT_T2, kdesc(sb + GT_O, HALF, ks), kdesc(sb + GT_DEL, HALF, ks),
+                            ID64_KK, ks > 0);
+        }
+        ok = commit_wait();
+        {
+            const int j0 = 32 * chalf;
+            float v[32], pm[32];
+            tld2x16(tq + GT_T2 + j0, v, tq + GT_T2 + j0 + 16, v + 16);
+            float rs = 0.f;
+#pragma unroll
+            for (int i = 0; i < 2; ++i) {
+                float mq[16];
+                ld16_bf16(sm, GT_REC + REC_MQ, HALF, r64, j0 + 16 * i, mq);
+#pragma unroll
+                for (int e = 0; e < 16; ++e) {
+                    const int j = j0 + 16 * i + e;
+                    const float x = lo16 ? v[16 * i + e] : 0.f;
+                    pm[16 * i + e] = x * mq[e];
+                    rs += pm[16 * i + e];
+                    v[16 * i + e] = j <= r64 ? x * ex2(g2[r64] - g2[j]) : 0.f;
+                }
+                if (lo16) st16_bf16(sm, GT_PY, HALF, r64, j0 + 16 * i, v + 16 * i, 1.f);
+            }
+            if (lo16) atomicAdd(&dg[r64], rs);
+            colsum16(pm, lane);
+            if (lo16) {
+                atomicAdd(&dg[j0 + 2 * lane], -pm[0]);
+                atomicAdd(&dg[j0 + 2 * lane + 1], -pm[1]);
+            }
+            // the row scalings of dO (by gamma) and Delta (by d), 16 bytes at a time
+            for (int idx = tid; idx < 2 * 1024; idx += 256) {
+                const int t = idx >> 10, i = idx & 1023;
+                const int row = (i >> 3) & 63;
+                uint8_t* q = sm + (t ? GT_DEL : GT_O) + (i >> 9) * HALF + row * 128 + (i & 7) * 16;
+                const float s = t ? rv[64 + row] : rv[row];
+                const uint4 u = *reinterpret_cast<const uint4*>(q);
+                const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+                uint32_t o[4];
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
-                    const int r = m0 + g + ((e >> 1) << 3), j = p0 + 8 * nt + 2 * t4 + (e & 1);
-                    const float mrj = j <= r ? ex2(g2[r] - g2[j]) : 0.f;
-                    const float2 qk = ld_bf16x2(sm + taddr_e(GC_REC + REC_MQ, r, j & ~1, 0));
-                    pm[nt][e] = acc[nt][e] * ((e & 1) ? qk.y : qk.x);  // P o (M o QK^T)
-                    acc[nt][e] *= mrj;
+                    const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[e]));
+                    o[e] = pack2(s * f.x, s * f.y);
                 }
-            store_acc_cols<4>(sm, GC_PY, m0, p0, acc, lane);
-            add_row_sums<4>(dg, m0, pm, lane, 1.f, 1.f);
-            add_col_sums<4>(dg, p0, pm, lane, -1.f);
-        }
-        __syncthreads();
-        // 6. dQ += gamma o (dO S^T) + P K     7. dK += P^T Q - gamma o (dX S^T) + d o (Delta dS'^T)
-        {
-            float acc[8][4];
-            zero_acc<8>(acc);
-            mma_rows<4, true, true>(acc, sb + GC_O, HALF, m0, sb + GC_S, SHALF, n0, 0, 8, lane);
-#pragma unroll
-            for (int nt = 0; nt < 8; ++nt) {
-                dQ[nt][0] = fmaf(gm_lo, acc[nt][0], dQ[nt][0]);
-                dQ[nt][1] = fmaf(gm_lo, acc[nt][1], dQ[nt][1]);
-                dQ[nt][2] = fmaf(gm_hi, acc[nt][2], dQ[nt][2]);
-                dQ[nt][3] = fmaf(gm_hi, acc[nt][3], dQ[nt][3]);
-            }
-            mma_rows<4, true, false>(dQ, sb + GC_PY, 0, m0, sb + GC_K, HALF, n0, 0, rb + 1, lane);
-            mma_rows<4, false, false>(dK, sb + GC_PY, 0, m0, sb + GC_Q, HALF, n0, rb, 4, lane);
-            zero_acc<8>(acc);
-            mma_rows<4, true, true>(acc, sb + GC_DX, HALF, m0, sb + GC_S, SHALF, n0, 0, 8, lane);
-            float acc2[8][4];
-            zero_acc<8>(acc2);
-            mma_rows<4, true, true>(acc2, sb + GC_DEL, HALF, m0, sb + GC_DS, SHALF, n0, 0, 8, lane);
-#pragma unroll
-            for (int nt = 0; nt < 8; ++nt) {
-                dK[nt][0] += d_lo * acc2[nt][0] - gm_lo * acc[nt][0];
-                dK[nt][1] += d_lo * acc2[nt][1] - gm_lo * acc[nt][1];
-                dK[nt][2] += d_hi * acc2[nt][2] - gm_hi * acc[nt][2];
-                dK[nt][3] += d_hi * acc2[nt][3] - gm_hi * acc[nt][3];
+                *reinterpret_cast<uint4*>(q) = make_uint4(o[0], o[1], o[2], o[3]);
             }
         }
-        // 8. dT_b = dDelta X^T (64 x 64); dbeta * beta gets the columns of dT_b o T_b
-        {
-            const int p0 = 32 * hh;
-            float acc[4][4];
-            zero_acc<4>(acc);
-            mma_rows<2, true, true>(acc, sb + GC_DDEL, HALF, m0, sb + GC_V, HALF, p0, 0, 8, lane);
-            store_acc_cols<4>(sm, GC_TE, m0, p0, acc, lane);
-            float tt[4][4];
-#pragma unroll
-            for (int nt = 0; nt < 4; ++nt)
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const int r = m0 + g + ((e >> 1) << 3), j = p0 + 8 * nt + 2 * t4 + (e & 1);
-                    const float2 tv = ld_bf16x2(sm + taddr_e(GC_REC + REC_TB, r, j & ~1, 0));
-                    tt[nt][e] = acc[nt][e] * ((e & 1) ? tv.y : tv.x);
-                }
-            add_col_sums<4>(dbt, p0, tt, lane, 1.f);
+        if (!publish(ok)) {
+            leave();
+            return;
         }
-        __syncthreads();
-        // V (X), dO and both states are free: the next head's copies land during steps 9-12
-        if (tid == 0 && vh + 1 < group) {
+
+        // 6. dQ += (gamma o dO) S^T + P K
+        // 7. dK += P^T Q + (-gamma o dX) S^T + (d o Delta) dS'^T
+        // 8. dT_b = dDelta X^T (64 x 64)
+        if (tid == 0) {
+            tc_fence_after();
+#pragma unroll
+            for (int ks = 0; ks < 8; ++ks)
+                mma_bf16_ss(tmem + GT_DQ, kdesc(sb + GT_O, HALF, ks), kdesc(sb + GT_S, SHALF, ks),
+                            ID_KK, vh > 0 || ks > 0);
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks)
+                mma_bf16_ss(tmem + GT_DQ, kdesc(sb + GT_PY, HALF, ks),
+                            mdesc(sb + GT_KQ, 2 * HALF, ks), ID_KM, 1);
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks)
+                mma_bf16_ss(tmem + GT_DK, mdesc(sb + GT_PY, HALF, ks),
+                            mdesc(sb + GT_KQ + HALF, 2 * HALF, ks), ID_MM, vh > 0 || ks > 0);
+#pragma unroll
+            for (int ks = 0; ks < 8; ++ks)
+                mma_bf16_ss(tmem + GT_DK, kdesc(sb + GT_DX, HALF, ks), kdesc(sb + GT_S, SHALF, ks),
+                            ID_KK, 1);
+#pragma unroll
+            for (int ks = 0; ks < 8; ++ks)
+                mma_bf16_ss(tmem + GT_DK, kdesc(sb + GT_DEL, HALF, ks), kdesc(sb + GT_DS, SHALF, ks),
+                            ID_KK, 1);
+#pragma unroll
+            for (int ks = 0; ks < 8; ++ks)
+                mma_bf16_ss(tmem + GT_T2, kdesc(sb + GT_DDEL, HALF, ks), kdesc(sb + GT_V, HALF, ks),
+                            ID64_KK, ks > 0);
+        }
+        ok = commit_wait();
+        // X, dO, both states and Delta are free: the next head's copies land during
+        // steps 9-12
+        if (tid == 0 && ok && vh + 1 < group) {
             issue_head(vh + 1);
             ++heads;
         }
+        {  // dT_b to its tile; dbeta * beta gets the columns of dT_b o T_b
+            const int j0 = 32 * chalf;
+            float v[32];
+            tld2x16(tq + GT_T2 + j0, v, tq + GT_T2 + j0 + 16, v + 16);
+#pragma unroll
+            for (int i = 0; i < 2; ++i) {
+                float tb[16];
+                ld16_bf16(sm, GT_REC + REC_TB, HALF, r64, j0 + 16 * i, tb);
+                if (lo16) st16_bf16(sm, GT_TE, HALF, r64, j0 + 16 * i, v + 16 * i, 1.f);
+#pragma unroll
+                for (int e = 0; e < 16; ++e) v[16 * i + e] = lo16 ? v[16 * i + e] * tb[e] : 0.f;
+            }
+            colsum16(v, lane);
+            if (lo16) {
+                atomicAdd(&dbt[j0 + 2 * lane], v[0]);
+                atomicAdd(&dbt[j0 + 2 * lane + 1], v[1]);
+            }
+        }
+        if (!publish(ok)) {
+            leave();
+            return;
+        }
+
         // 9. Y = dT_b T_b^T
-        {
-            const int p0 = 32 * hh;
-            float acc[4][4];
-            zero_acc<4>(acc);
-            mma_rows<2, true, true>(acc, sb + GC_TE, 0, m0, tb, 0, p0, 0, 4, lane);
-            store_acc_cols<4>(sm, GC_PY, m0, p0, acc, lane);
+        if (tid == 0) {
+            tc_fence_after();
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks)
+                mma_bf16_ss(tmem + GT_T1, kdesc(sb + GT_TE, HALF, ks),
+                            kdesc(sb + GT_REC + REC_TB, HALF, ks), ID64_KK, ks > 0);
         }
-        __syncthreads();
+        ok = commit_wait();
+        {
+            const int j0 = 32 * chalf;
+            float v[32];
+            tld2x16(tq + GT_T1 + j0, v, tq + GT_T1 + j0 + 16, v + 16);
+            if (lo16) {
+                st16_bf16(sm, GT_PY, HALF, r64, j0, v, 1.f);
+                st16_bf16(sm, GT_PY, HALF, r64, j0 + 16, v + 16, 1.f);
+            }
+        }
+        if (!publish(ok)) {
+            leave();
+            return;
+        }
+
         // 10. E = strict_lower(-T_b^T Y) o M;  K K^T;  E o KK into dbeta * beta (rows)
-        // and dg (rows +, columns -)
-        {
-            const int p0 = 32 * hh;
-            float acc[4][4], kk[4][4];
-            zero_acc<4>(acc);
-            zero_acc<4>(kk);
-            mma_rows<2, false, false>(acc, tb, 0, m0, sb + GC_PY, 0, p0, rb, 4, lane);
-            mma_rows<2, true, true>(kk, sb + GC_K, HALF, m0, sb + GC_K, HALF, p0, 0, 8, lane);
+        //     and dg (rows +, columns -)
+        if (tid == 0) {
+            tc_fence_after();
 #pragma unroll
-            for (int nt = 0; nt < 4; ++nt)
+            for (int ks = 0; ks < 4; ++ks)
+                mma_bf16_ss(tmem + GT_T2, mdesc(sb + GT_REC + REC_TB, HALF, ks),
+                            mdesc(sb + GT_PY, HALF, ks), ID64_MM, ks > 0);
 #pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const int r = m0 + g + ((e >> 1) << 3), j = p0 + 8 * nt + 2 * t4 + (e & 1);
-                    acc[nt][e] = j < r ? -acc[nt][e] * ex2(g2[r] - g2[j]) : 0.f;
-                    kk[nt][e] *= acc[nt][e];
-                }
-            store_acc_cols<4>(sm, GC_TE, m0, p0, acc, lane);
-            add_row_sums<4>(dbt, m0, kk, lane, 1.f, 1.f);
-            add_row_sums<4>(dg, m0, kk, lane, 1.f, 1.f);
-            add_col_sums<4>(dg, p0, kk, lane, -1.f);
+            for (int ks = 0; ks < 8; ++ks)
+                mma_bf16_ss(tmem + GT_T2 + 64, kdesc(sb + GT_KQ, 2 * HALF, ks),
+                            kdesc(sb + GT_KQ, 2 * HALF, ks), ID64_KK, ks > 0);
         }
-        __syncthreads();
+        ok = commit_wait();
         // the record is free too (gamma_C is in a register)
-        if (tid == 0 && vh + 1 < group) {
+        if (tid == 0 && ok && vh + 1 < group) {
             issue_rec(vh + 1);
             ++recs;
         }
-        // 11. dK += E K + E^T K
-        mma_rows<4, true, false>(dK, sb + GC_TE, 0, m0, sb + GC_K, HALF, n0, 0, rb + 1, lane);
-        mma_rows<4, false, false>(dK, sb + GC_TE, 0, m0, sb + GC_K, HALF, n0, rb, 4, lane);
+        {
+            const int j0 = 32 * chalf;
+            float v[32], kk[32];
+            tld2x16(tq + GT_T2 + j0, v, tq + GT_T2 + j0 + 16, v + 16);
+            tld2x16(tq + GT_T2 + 64 + j0, kk, tq + GT_T2 + 64 + j0 + 16, kk + 16);
+            float rs = 0.f;
+#pragma unroll
+            for (int e = 0; e < 32; ++e) {
+                const int j = j0 + e;
+                v[e] = (lo16 && j < r64) ? -v[e] * ex2(g2[r64] - g2[j]) : 0.f;
+                kk[e] = lo16 ? kk[e] * v[e] : 0.f;  // lanes 16-31 hold no rows
+                rs += kk[e];
+            }
+            if (lo16) {
+                st16_bf16(sm, GT_TE, HALF, r64, j0, v, 1.f);
+                st16_bf16(sm, GT_TE, HALF, r64, j0 + 16, v + 16, 1.f);
+                atomicAdd(&dbt[r64], rs);
+                atomicAdd(&dg[r64], rs);
+            }
+            colsum16(kk, lane);
+            if (lo16) {
+                atomicAdd(&dg[j0 + 2 * lane], -kk[0]);
+                atomicAdd(&dg[j0 + 2 * lane + 1], -kk[1]);
+            }
+        }
+        if (!publish(ok)) {
+            leave();
+            return;
+        }
+
+        // 11. dK += E K + E^T K (committed with the next group)
+        if (tid == 0) {
+            tc_fence_after();
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks)
+                mma_bf16_ss(tmem + GT_DK, kdesc(sb + GT_TE, HALF, ks),
+                            mdesc(sb + GT_KQ, 2 * HALF, ks), ID_KM, 1);
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks)
+                mma_bf16_ss(tmem + GT_DK, mdesc(sb + GT_TE, HALF, ks),
+                            mdesc(sb + GT_KQ, 2 * HALF, ks), ID_MM, 1);
+        }
         // 12. the gates: dg of the last row gets sum ddv + gamma_C <dS', S>;
         // dlog_alpha_t = sum_{r >= t} dg_r (dg holds the gradient w.r.t. g in
         // natural-log units); dbeta_j = (dbeta * beta)_j / beta_j
         if (warp == 0) {
             const float last = misc[0] + gam_C * misc[1];
-            // reverse inclusive scan of dg over 64 rows, 2 per lane (rows 2l, 2l+1)
             float d0 = dg[2 * lane], d1 = dg[2 * lane + 1];
             if (lane == 31) d1 += last;
-            float s = d0 + d1;  // suffix sums from the top lane down
+            float s = d0 + d1;
 #pragma unroll
             for (int off = 1; off < 32; off <<= 1) {
                 const float y = __shfl_down_sync(0xffffffffu, s, off);
                 if (lane + off < 32) s += y;
             }
-            // s = sum of rows >= 2 lane; row 2l+1's suffix is s - d0
             const float suf0 = s, suf1 = s - d0;
 #pragma unroll
             for (int e = 0; e < 2; ++e) {
@@ -777,29 +984,33 @@ __global__ void __launch_bounds__(256, 1)
         __syncthreads();  // the next head's gates overwrite dg, dbt and misc
     }
     // dQ, dK of this chunk and query/key head (every value head of the group summed)
+    ok = commit_wait();
+    if (!__syncthreads_and(ok)) {
+        leave();
+        return;
+    }
     IO* dq = static_cast<IO*>(p.dq);
     IO* dk = static_cast<IO*>(p.dk);
 #pragma unroll
-    for (int nt = 0; nt < 8; ++nt)
+    for (int i = 0; i < 4; ++i) {
+        const int col = 64 * chalf + 16 * i;
+        float a[16], b[16];
+        tld2x16(tq + GT_DQ + col, a, tq + GT_DK + col, b);
+        if (lo16 && r64 < valid) {
+            const size_t o = ((size_t)(tc0 + r64) * p.H_qk + hq) * D + col;
 #pragma unroll
-        for (int hl = 0; hl < 2; ++hl) {
-            const int r = m0 + g + 8 * hl, col = 64 * hh + 8 * nt + 2 * t4;
-            if (r < valid) {
-                const size_t o = ((size_t)(tc0 + r) * p.H_qk + hq) * D + col;
-                store2<IO>(dq + o, dQ[nt][2 * hl], dQ[nt][2 * hl + 1]);
-                store2<IO>(dk + o, dK[nt][2 * hl], dK[nt][2 * hl + 1]);
+            for (int e = 0; e < 16; e += 2) {
+                store2<IO>(dq + o + e, a[e], a[e + 1]);
+                store2<IO>(dk + o + e, b[e], b[e + 1]);
             }
         }
-}
-
-template <int NS, typename IO>
-cudaError_t launch_grad_state(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mo,
-                              const GradParams& prm, cudaStream_t stream) {
-    auto kern = grad_state_kernel<NS, IO>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, GS_SMEM);
-    if (e != cudaSuccess) return e;
-    kern<<<dim3((D + NS - 1) / NS, prm.H_v, prm.N), 256, GS_SMEM, stream>>>(mq, mk, mo, prm);
-    return cudaGetLastError();
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, GT_COLS);
+    }
 }
 
 // The reverse chain (as many d_v slices as fit in one wave of one block per
@@ -812,11 +1023,11 @@ cudaError_t launch_grads(const CUtensorMap& mq, const CUtensorMap& mk, const CUt
                     : units * 3 <= sms ? launch_grad_state<48, IO>(mq, mk, mo, prm, stream)
                                        : launch_grad_state<64, IO>(mq, mk, mo, prm, stream);
     if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(grad_chunk_kernel<IO>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             GC_SMEM);
+    e = cudaFuncSetAttribute(grad_chunk_tc_kernel<IO>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             GT_SMEM);
     if (e != cudaSuccess) return e;
-    grad_chunk_kernel<IO><<<dim3((unsigned)slots, prm.H_qk), 256, GC_SMEM, stream>>>(mq, mk, mv, mo,
-                                                                                    prm);
+    grad_chunk_tc_kernel<IO><<<dim3((unsigned)slots, prm.H_qk), 256, GT_SMEM, stream>>>(
+        mq, mk, mv, mo, prm);
     return cudaGetLastError();
 }
 
