@@ -389,19 +389,80 @@ __device__ __forceinline__ uint64_t mdesc(uint32_t tile, uint32_t bs, int ks) {
     return sdesc_sw128(tile + (uint32_t)ks * 2048, bs, 1024);
 }
 
-// Column sums over lanes 0-15 of a warp of v[0..31] (lanes 16-31 reduce among
-// themselves): lane l < 16 ends with the sums of columns 2l and 2l + 1 in
-// v[0], v[1].  Four halving exchanges, 30 shuffles.
-__device__ __forceinline__ void colsum16(float* v, int lane) {
+// An M = 64 accumulator's rows 16 (w % 4) .. + 15 for warp w, in the m16n8
+// fragment layout of mma.sync (thread t: rows t / 4 and t / 4 + 8, columns
+// 2 (t % 4) and 2 (t % 4) + 1 of each 8-column group): NT groups from TMEM
+// address ta, by tcgen05.ld.16x256b (layout checked by a probe on the B200).
+__device__ __forceinline__ void tld_frag4(uint32_t ta, float (*acc)[4]) {
+    uint32_t* u = reinterpret_cast<uint32_t*>(&acc[0][0]);
+    asm volatile(
+        "tcgen05.ld.sync.aligned.16x256b.x4.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+        : "=r"(u[0]), "=r"(u[1]), "=r"(u[2]), "=r"(u[3]), "=r"(u[4]), "=r"(u[5]), "=r"(u[6]),
+          "=r"(u[7]), "=r"(u[8]), "=r"(u[9]), "=r"(u[10]), "=r"(u[11]), "=r"(u[12]), "=r"(u[13]),
+          "=r"(u[14]), "=r"(u[15])
+        : "r"(ta));
+}
+template <int NT>
+__device__ __forceinline__ void tld_frag(uint32_t ta, float (*acc)[4]) {
+    static_assert(NT % 4 == 0, "groups of four 8-column groups");
 #pragma unroll
-    for (int w = 16, m = 8; m >= 1; w >>= 1, m >>= 1) {
-        const bool up = (lane & m) != 0;
+    for (int i = 0; i < NT / 4; ++i) tld_frag4(ta + 32 * i, acc + 4 * i);
+    tmem_ld_wait();
+}
+
+// Row sums (over the fragment's columns) of v into dst[row] (shared memory,
+// atomically): rows m0 + g and m0 + g + 8, scaled by s_lo and s_hi.
+template <int NT>
+__device__ __forceinline__ void add_row_sums(float* dst, int m0, const float (*v)[4], int lane,
+                                             float s_lo, float s_hi) {
+    float lo = 0.f, hi = 0.f;
 #pragma unroll
-        for (int i = 0; i < w; ++i) {
-            const float send = up ? v[i] : v[w + i];
-            const float keep = up ? v[w + i] : v[i];
-            v[i] = keep + __shfl_xor_sync(0xffffffffu, send, m);
+    for (int nt = 0; nt < NT; ++nt) {
+        lo += v[nt][0] + v[nt][1];
+        hi += v[nt][2] + v[nt][3];
+    }
+    lo += __shfl_xor_sync(0xffffffffu, lo, 1);
+    lo += __shfl_xor_sync(0xffffffffu, lo, 2);
+    hi += __shfl_xor_sync(0xffffffffu, hi, 1);
+    hi += __shfl_xor_sync(0xffffffffu, hi, 2);
+    if ((lane & 3) == 0) {
+        const int g = lane >> 2;
+        atomicAdd(&dst[m0 + g], s_lo * lo);
+        atomicAdd(&dst[m0 + g + 8], s_hi * hi);
+    }
+}
+// Column sums (over the fragment's 16 rows) of v into dst[n0 + column], scaled by s.
+template <int NT>
+__device__ __forceinline__ void add_col_sums(float* dst, int n0, const float (*v)[4], int lane,
+                                             float s) {
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+        float c0 = v[nt][0] + v[nt][2], c1 = v[nt][1] + v[nt][3];
+#pragma unroll
+        for (int off = 4; off < 32; off <<= 1) {
+            c0 += __shfl_xor_sync(0xffffffffu, c0, off);
+            c1 += __shfl_xor_sync(0xffffffffu, c1, off);
         }
+        if (lane < 4) {
+            atomicAdd(&dst[n0 + 8 * nt + 2 * lane], s * c0);
+            atomicAdd(&dst[n0 + 8 * nt + 2 * lane + 1], s * c1);
+        }
+    }
+}
+// A fragment as bf16 into a 64-column swizzled tile: rows m0 + g (+8), columns
+// c0 + 8 nt + 2 t (+1).
+template <int NT>
+__device__ __forceinline__ void store_frag_cols(uint8_t* smem, uint32_t base_off, int m0, int c0,
+                                                const float (*acc)[4], int lane) {
+    const int g = lane >> 2, t = lane & 3;
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+        const int col = c0 + 8 * nt + 2 * t;
+        *reinterpret_cast<uint32_t*>(smem + taddr_e(base_off, m0 + g, col, 0)) =
+            pack2(acc[nt][0], acc[nt][1]);
+        *reinterpret_cast<uint32_t*>(smem + taddr_e(base_off, m0 + g + 8, col, 0)) =
+            pack2(acc[nt][2], acc[nt][3]);
     }
 }
 
@@ -429,6 +490,23 @@ __device__ __forceinline__ void st16_bf16(uint8_t* sm, uint32_t tile, uint32_t h
             make_uint4(pack2(s * v[8 * h], s * v[8 * h + 1]), pack2(s * v[8 * h + 2], s * v[8 * h + 3]),
                        pack2(s * v[8 * h + 4], s * v[8 * h + 5]),
                        pack2(s * v[8 * h + 6], s * v[8 * h + 7]));
+}
+// 16 consecutive values to global memory in 16-byte stores (dst 16-byte aligned).
+template <typename IO>
+__device__ __forceinline__ void store16(IO* dst, const float* v);
+template <>
+__device__ __forceinline__ void store16<float>(float* dst, const float* v) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+        reinterpret_cast<float4*>(dst)[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+}
+template <>
+__device__ __forceinline__ void store16<__nv_bfloat16>(__nv_bfloat16* dst, const float* v) {
+#pragma unroll
+    for (int i = 0; i < 2; ++i)
+        reinterpret_cast<uint4*>(dst)[i] =
+            make_uint4(pack2(v[8 * i], v[8 * i + 1]), pack2(v[8 * i + 2], v[8 * i + 3]),
+                       pack2(v[8 * i + 4], v[8 * i + 5]), pack2(v[8 * i + 6], v[8 * i + 7]));
 }
 // Two 16-column TMEM reads of this warp's lanes, then the wait.
 __device__ __forceinline__ void tld2x16(uint32_t a0, float* v0, uint32_t a1, float* v1) {
@@ -463,7 +541,8 @@ __global__ void __launch_bounds__(256, 1)
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int quad = warp & 3, chalf = warp >> 2;
     const bool lo16 = lane < 16;
-    const int r64 = 16 * quad + (lane & 15);  // my row of an M = 64 product (lanes < 16)
+    const int r64 = 16 * quad + (lane & 15);  // my row of an M = 64 product in lanes < 16
+    const int m0 = 16 * quad, g = lane >> 2, t4 = lane & 3;  // the same product as fragments
     int n, c;
     slot_owner(p.cu_seqlens, p.N, blockIdx.x, n, c);
     if (n < 0) return;  // uniform across the CTA
@@ -566,6 +645,20 @@ __global__ void __launch_bounds__(256, 1)
         }
     }
 
+    // warp 0 holds a value head's gates in registers, loaded one head ahead (lane l:
+    // tokens 2l, 2l+1; zero past the sequence end)
+    float la[2] = {0.f, 0.f}, be[2] = {0.f, 0.f};
+    auto load_gates = [&](int vh) {
+        const int h = hq * group + vh;
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+            const bool in = 2 * lane + e < valid;
+            la[e] = in ? p.log_alpha[(size_t)(tc0 + 2 * lane + e) * p.H_v + h] : 0.f;
+            be[e] = in ? p.beta[(size_t)(tc0 + 2 * lane + e) * p.H_v + h] : 0.f;
+        }
+    };
+    if (warp == 0) load_gates(0);
+
     for (int vh = 0; vh < group; ++vh) {
         const int h = hq * group + vh;
         if (tid < 64) {
@@ -573,11 +666,7 @@ __global__ void __launch_bounds__(256, 1)
             dbt[tid] = 0.f;
             misc[tid] = 0.f;
         }
-        if (warp == 0) {  // inclusive scan of log alpha (log2 units); lane l: tokens 2l, 2l+1
-            float la[2] = {0.f, 0.f};
-#pragma unroll
-            for (int e = 0; e < 2; ++e)
-                if (2 * lane + e < valid) la[e] = p.log_alpha[(size_t)(tc0 + 2 * lane + e) * p.H_v + h];
+        if (warp == 0) {  // inclusive scan of log alpha (log2 units)
             const float x0 = la[0] * LOG2E, x1 = la[1] * LOG2E;
             float incl = x0 + x1;
 #pragma unroll
@@ -595,12 +684,6 @@ __global__ void __launch_bounds__(256, 1)
             leave();
             return;
         }
-        {  // <dS', S>, for the gate gradient of the chunk's last row
-            float dot = tile_dot(sm + GT_S, sm + GT_DS, tid);
-#pragma unroll
-            for (int off = 16; off > 0; off >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, off);
-            if (lane == 0) atomicAdd(&misc[1], dot);
-        }
         if (valid < C) {  // V and dO rows past the sequence end
             for (int i = tid; i < 4 * 64 * 8; i += 256) {
                 const int tile = i / 512, row = (i >> 3) & 63, ch = i & 7;
@@ -611,8 +694,9 @@ __global__ void __launch_bounds__(256, 1)
         }
         const float* rv = reinterpret_cast<const float*>(sm + GT_REC + REC_VEC);
         const float gam_C = rv[128];
-        const float gm64 = lo16 ? rv[r64] : 0.f;      // gamma of my M = 64 row
-        const float d64 = lo16 ? rv[64 + r64] : 0.f;  // d of my M = 64 row
+        const float gm_lo = rv[m0 + g], gm_hi = rv[m0 + g + 8];      // gamma of my fragment rows
+        const float d_lo = rv[64 + m0 + g], d_hi = rv[64 + m0 + g + 8];  // d of my fragment rows
+        const int c0 = 64 * chalf, p0 = 32 * chalf;  // my columns of the 128- and 64-wide products
         if (!publish(true)) {
             leave();
             return;
@@ -626,6 +710,12 @@ __global__ void __launch_bounds__(256, 1)
             for (int ks = 0; ks < 8; ++ks)
                 mma_bf16_ss(tmem + GT_T1, kdesc(sb + GT_KQ, 2 * HALF, ks), mdesc(sb + GT_S, SHALF, ks),
                             ID_128_KM, ks > 0);
+        }
+        {  // <dS', S>, for the gate gradient of the chunk's last row (while the product runs)
+            float dot = tile_dot(sm + GT_S, sm + GT_DS, tid);
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, off);
+            if (lane == 0) atomicAdd(&misc[1], dot);
         }
         ok = commit_wait();
         {
@@ -666,13 +756,10 @@ __global__ void __launch_bounds__(256, 1)
                             mdesc(sb + GT_V, HALF, ks), ID_KM, ks > 0);
         }
         ok = commit_wait();
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const int col = 64 * chalf + 16 * i;
-            float a[16];
-            tmem_ld16(tq + GT_T2 + col, a);
-            tmem_ld_wait();
-            if (lo16) st16_bf16(sm, GT_DEL, HALF, r64, col, a, 1.f);
+        {
+            float acc[8][4];
+            tld_frag<8>(tq + GT_T2 + c0, acc);
+            store_acc_bf16<8>(sm, GT_DEL + chalf * HALF, 0, m0, acc, lane, 1.f, 1.f);
         }
         if (!publish(ok)) {
             leave();
@@ -693,29 +780,33 @@ __global__ void __launch_bounds__(256, 1)
         }
         ok = commit_wait();
         {
-            float ddv = 0.f;
+            float kd[8][4], acc[8][4], ddv[8][4];
+            tld_frag<8>(tq + GT_T1 + c0, kd);
+            tld_frag<8>(tq + GT_T2 + c0, acc);
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const int col = 64 * chalf + 16 * i;
-                float kd[16], ao[16];
-                tld2x16(tq + GT_T1 + col, kd, tq + GT_T2 + col, ao);
-                if (lo16) {
-                    float dl[16];
-                    ld16_bf16(sm, GT_DEL, HALF, r64, col, dl);
-#pragma unroll
-                    for (int e = 0; e < 16; ++e) {
-                        ddv = fmaf(kd[e], dl[e], ddv);
-                        ao[e] = fmaf(d64, kd[e], ao[e]);
-                    }
-                    st16_bf16(sm, GT_DDEL, HALF, r64, col, ao, 1.f);
-                }
+            for (int nt = 0; nt < 8; ++nt) {
+                const int col = c0 + 8 * nt + 2 * t4;
+                const float2 e_lo = ld_bf16x2(sm + taddr_e(GT_DEL, m0 + g, col, HALF));
+                const float2 e_hi = ld_bf16x2(sm + taddr_e(GT_DEL, m0 + g + 8, col, HALF));
+                ddv[nt][0] = kd[nt][0] * e_lo.x;
+                ddv[nt][1] = kd[nt][1] * e_lo.y;
+                ddv[nt][2] = kd[nt][2] * e_hi.x;
+                ddv[nt][3] = kd[nt][3] * e_hi.y;
+                acc[nt][0] = fmaf(d_lo, kd[nt][0], acc[nt][0]);
+                acc[nt][1] = fmaf(d_lo, kd[nt][1], acc[nt][1]);
+                acc[nt][2] = fmaf(d_hi, kd[nt][2], acc[nt][2]);
+                acc[nt][3] = fmaf(d_hi, kd[nt][3], acc[nt][3]);
             }
-            // -d_r ddv_r into dg_r; the total goes to dg of the last row (misc[0])
-            if (lo16) atomicAdd(&dg[r64], -d64 * ddv);
-            float tot = d64 * ddv;  // zero on lanes 16-31
+            // -d_r ddv_r into dg_r; their total goes to dg of the last row (misc[0])
+            add_row_sums<8>(dg, m0, ddv, lane, -d_lo, -d_hi);
+            float tot = 0.f;
+#pragma unroll
+            for (int nt = 0; nt < 8; ++nt)
+                tot += d_lo * (ddv[nt][0] + ddv[nt][1]) + d_hi * (ddv[nt][2] + ddv[nt][3]);
 #pragma unroll
             for (int off = 16; off > 0; off >>= 1) tot += __shfl_xor_sync(0xffffffffu, tot, off);
             if (lane == 0) atomicAdd(&misc[0], tot);
+            store_acc_bf16<8>(sm, GT_DDEL + chalf * HALF, 0, m0, acc, lane, 1.f, 1.f);
         }
         if (!publish(ok)) {
             leave();
@@ -732,22 +823,20 @@ __global__ void __launch_bounds__(256, 1)
         }
         ok = commit_wait();
         {
-            float s = 0.f;
+            float dx[8][4], w[8][4];
+            tld_frag<8>(tq + GT_T1 + c0, dx);
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const int col = 64 * chalf + 16 * i;
-                float dx[16];
-                tmem_ld16(tq + GT_T1 + col, dx);
-                tmem_ld_wait();
-                if (lo16) {
-                    float ksv[16];
-                    ld16_bf16(sm, GT_DX, HALF, r64, col, ksv);
-#pragma unroll
-                    for (int e = 0; e < 16; ++e) s = fmaf(dx[e], ksv[e], s);
-                    st16_bf16(sm, GT_DX, HALF, r64, col, dx, -gm64);
-                }
+            for (int nt = 0; nt < 8; ++nt) {
+                const int col = c0 + 8 * nt + 2 * t4;
+                const float2 k_lo = ld_bf16x2(sm + taddr_e(GT_DX, m0 + g, col, HALF));
+                const float2 k_hi = ld_bf16x2(sm + taddr_e(GT_DX, m0 + g + 8, col, HALF));
+                w[nt][0] = dx[nt][0] * k_lo.x;
+                w[nt][1] = dx[nt][1] * k_lo.y;
+                w[nt][2] = dx[nt][2] * k_hi.x;
+                w[nt][3] = dx[nt][3] * k_hi.y;
             }
-            if (lo16) atomicAdd(&dg[r64], -gm64 * s);
+            add_row_sums<8>(dg, m0, w, lane, -gm_lo, -gm_hi);
+            store_acc_bf16<8>(sm, GT_DX + chalf * HALF, 0, m0, dx, lane, -gm_lo, -gm_hi);
         }
         if (!publish(ok)) {
             leave();
@@ -766,69 +855,72 @@ __global__ void __launch_bounds__(256, 1)
         }
         ok = commit_wait();
         {
-            const int j0 = 32 * chalf;
-            float v[32], pm[32];
-            tld2x16(tq + GT_T2 + j0, v, tq + GT_T2 + j0 + 16, v + 16);
-            float rs = 0.f;
+            float acc[4][4], pm[4][4];
+            tld_frag<4>(tq + GT_T2 + p0, acc);
 #pragma unroll
-            for (int i = 0; i < 2; ++i) {
-                float mq[16];
-                ld16_bf16(sm, GT_REC + REC_MQ, HALF, r64, j0 + 16 * i, mq);
-#pragma unroll
-                for (int e = 0; e < 16; ++e) {
-                    const int j = j0 + 16 * i + e;
-                    const float x = lo16 ? v[16 * i + e] : 0.f;
-                    pm[16 * i + e] = x * mq[e];
-                    rs += pm[16 * i + e];
-                    v[16 * i + e] = j <= r64 ? x * ex2(g2[r64] - g2[j]) : 0.f;
-                }
-                if (lo16) st16_bf16(sm, GT_PY, HALF, r64, j0 + 16 * i, v + 16 * i, 1.f);
-            }
-            if (lo16) atomicAdd(&dg[r64], rs);
-            colsum16(pm, lane);
-            if (lo16) {
-                atomicAdd(&dg[j0 + 2 * lane], -pm[0]);
-                atomicAdd(&dg[j0 + 2 * lane + 1], -pm[1]);
-            }
-            // the row scalings of dO (by gamma) and Delta (by d), 16 bytes at a time
-            for (int idx = tid; idx < 2 * 1024; idx += 256) {
-                const int t = idx >> 10, i = idx & 1023;
-                const int row = (i >> 3) & 63;
-                uint8_t* q = sm + (t ? GT_DEL : GT_O) + (i >> 9) * HALF + row * 128 + (i & 7) * 16;
-                const float s = t ? rv[64 + row] : rv[row];
-                const uint4 u = *reinterpret_cast<const uint4*>(q);
-                const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-                uint32_t o[4];
+            for (int nt = 0; nt < 4; ++nt)
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
-                    const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[e]));
-                    o[e] = pack2(s * f.x, s * f.y);
+                    const int r = m0 + g + ((e >> 1) << 3), j = p0 + 8 * nt + 2 * t4 + (e & 1);
+                    const float mrj = j <= r ? ex2(g2[r] - g2[j]) : 0.f;
+                    const float2 qk = ld_bf16x2(sm + taddr_e(GT_REC + REC_MQ, r, j & ~1, 0));
+                    pm[nt][e] = acc[nt][e] * ((e & 1) ? qk.y : qk.x);  // P o (M o QK^T)
+                    acc[nt][e] *= mrj;
                 }
-                *reinterpret_cast<uint4*>(q) = make_uint4(o[0], o[1], o[2], o[3]);
-            }
+            store_frag_cols<4>(sm, GT_PY, m0, p0, acc, lane);
+            add_row_sums<4>(dg, m0, pm, lane, 1.f, 1.f);
+            add_col_sums<4>(dg, p0, pm, lane, -1.f);
         }
         if (!publish(ok)) {
             leave();
             return;
         }
 
-        // 6. dQ += (gamma o dO) S^T + P K
+        // 6. dQ += P K + (gamma o dO) S^T
         // 7. dK += P^T Q + (-gamma o dX) S^T + (d o Delta) dS'^T
         // 8. dT_b = dDelta X^T (64 x 64)
+        // The products that read neither dO nor Delta go first; the row scalings of
+        // dO (by gamma) and Delta (by d) run meanwhile, then the rest follows.
+        if (tid == 0) {
+            tc_fence_after();
+#pragma unroll
+            for (int ks = 0; ks < 8; ++ks)
+                mma_bf16_ss(tmem + GT_T2, kdesc(sb + GT_DDEL, HALF, ks), kdesc(sb + GT_V, HALF, ks),
+                            ID64_KK, ks > 0);
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks)
+                mma_bf16_ss(tmem + GT_DQ, kdesc(sb + GT_PY, HALF, ks),
+                            mdesc(sb + GT_KQ, 2 * HALF, ks), ID_KM, vh > 0 || ks > 0);
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks)
+                mma_bf16_ss(tmem + GT_DK, mdesc(sb + GT_PY, HALF, ks),
+                            mdesc(sb + GT_KQ + HALF, 2 * HALF, ks), ID_MM, vh > 0 || ks > 0);
+        }
+        for (int idx = tid; idx < 2 * 1024; idx += 256) {  // 16 bytes at a time
+            const int t = idx >> 10, i = idx & 1023;
+            const int row = (i >> 3) & 63;
+            uint8_t* q = sm + (t ? GT_DEL : GT_O) + (i >> 9) * HALF + row * 128 + (i & 7) * 16;
+            const float sc = t ? rv[64 + row] : rv[row];
+            const uint4 u = *reinterpret_cast<const uint4*>(q);
+            const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+            uint32_t o[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[e]));
+                o[e] = pack2(sc * f.x, sc * f.y);
+            }
+            *reinterpret_cast<uint4*>(q) = make_uint4(o[0], o[1], o[2], o[3]);
+        }
+        if (!publish(true)) {
+            leave();
+            return;
+        }
         if (tid == 0) {
             tc_fence_after();
 #pragma unroll
             for (int ks = 0; ks < 8; ++ks)
                 mma_bf16_ss(tmem + GT_DQ, kdesc(sb + GT_O, HALF, ks), kdesc(sb + GT_S, SHALF, ks),
-                            ID_KK, vh > 0 || ks > 0);
-#pragma unroll
-            for (int ks = 0; ks < 4; ++ks)
-                mma_bf16_ss(tmem + GT_DQ, kdesc(sb + GT_PY, HALF, ks),
-                            mdesc(sb + GT_KQ, 2 * HALF, ks), ID_KM, 1);
-#pragma unroll
-            for (int ks = 0; ks < 4; ++ks)
-                mma_bf16_ss(tmem + GT_DK, mdesc(sb + GT_PY, HALF, ks),
-                            mdesc(sb + GT_KQ + HALF, 2 * HALF, ks), ID_MM, vh > 0 || ks > 0);
+                            ID_KK, 1);
 #pragma unroll
             for (int ks = 0; ks < 8; ++ks)
                 mma_bf16_ss(tmem + GT_DK, kdesc(sb + GT_DX, HALF, ks), kdesc(sb + GT_S, SHALF, ks),
@@ -837,10 +929,6 @@ __global__ void __launch_bounds__(256, 1)
             for (int ks = 0; ks < 8; ++ks)
                 mma_bf16_ss(tmem + GT_DK, kdesc(sb + GT_DEL, HALF, ks), kdesc(sb + GT_DS, SHALF, ks),
                             ID_KK, 1);
-#pragma unroll
-            for (int ks = 0; ks < 8; ++ks)
-                mma_bf16_ss(tmem + GT_T2, kdesc(sb + GT_DDEL, HALF, ks), kdesc(sb + GT_V, HALF, ks),
-                            ID64_KK, ks > 0);
         }
         ok = commit_wait();
         // X, dO, both states and Delta are free: the next head's copies land during
@@ -850,22 +938,18 @@ __global__ void __launch_bounds__(256, 1)
             ++heads;
         }
         {  // dT_b to its tile; dbeta * beta gets the columns of dT_b o T_b
-            const int j0 = 32 * chalf;
-            float v[32];
-            tld2x16(tq + GT_T2 + j0, v, tq + GT_T2 + j0 + 16, v + 16);
+            float acc[4][4];
+            tld_frag<4>(tq + GT_T2 + p0, acc);
+            store_frag_cols<4>(sm, GT_TE, m0, p0, acc, lane);
 #pragma unroll
-            for (int i = 0; i < 2; ++i) {
-                float tb[16];
-                ld16_bf16(sm, GT_REC + REC_TB, HALF, r64, j0 + 16 * i, tb);
-                if (lo16) st16_bf16(sm, GT_TE, HALF, r64, j0 + 16 * i, v + 16 * i, 1.f);
+            for (int nt = 0; nt < 4; ++nt)
 #pragma unroll
-                for (int e = 0; e < 16; ++e) v[16 * i + e] = lo16 ? v[16 * i + e] * tb[e] : 0.f;
-            }
-            colsum16(v, lane);
-            if (lo16) {
-                atomicAdd(&dbt[j0 + 2 * lane], v[0]);
-                atomicAdd(&dbt[j0 + 2 * lane + 1], v[1]);
-            }
+                for (int e = 0; e < 4; ++e) {
+                    const int r = m0 + g + ((e >> 1) << 3), j = p0 + 8 * nt + 2 * t4 + (e & 1);
+                    const float2 tv = ld_bf16x2(sm + taddr_e(GT_REC + REC_TB, r, j & ~1, 0));
+                    acc[nt][e] *= (e & 1) ? tv.y : tv.x;
+                }
+            add_col_sums<4>(dbt, p0, acc, lane, 1.f);
         }
         if (!publish(ok)) {
             leave();
@@ -882,13 +966,9 @@ __global__ void __launch_bounds__(256, 1)
         }
         ok = commit_wait();
         {
-            const int j0 = 32 * chalf;
-            float v[32];
-            tld2x16(tq + GT_T1 + j0, v, tq + GT_T1 + j0 + 16, v + 16);
-            if (lo16) {
-                st16_bf16(sm, GT_PY, HALF, r64, j0, v, 1.f);
-                st16_bf16(sm, GT_PY, HALF, r64, j0 + 16, v + 16, 1.f);
-            }
+            float acc[4][4];
+            tld_frag<4>(tq + GT_T1 + p0, acc);
+            store_frag_cols<4>(sm, GT_PY, m0, p0, acc, lane);
         }
         if (!publish(ok)) {
             leave();
@@ -915,29 +995,21 @@ __global__ void __launch_bounds__(256, 1)
             ++recs;
         }
         {
-            const int j0 = 32 * chalf;
-            float v[32], kk[32];
-            tld2x16(tq + GT_T2 + j0, v, tq + GT_T2 + j0 + 16, v + 16);
-            tld2x16(tq + GT_T2 + 64 + j0, kk, tq + GT_T2 + 64 + j0 + 16, kk + 16);
-            float rs = 0.f;
+            float acc[4][4], kk[4][4];
+            tld_frag<4>(tq + GT_T2 + p0, acc);
+            tld_frag<4>(tq + GT_T2 + 64 + p0, kk);
 #pragma unroll
-            for (int e = 0; e < 32; ++e) {
-                const int j = j0 + e;
-                v[e] = (lo16 && j < r64) ? -v[e] * ex2(g2[r64] - g2[j]) : 0.f;
-                kk[e] = lo16 ? kk[e] * v[e] : 0.f;  // lanes 16-31 hold no rows
-                rs += kk[e];
-            }
-            if (lo16) {
-                st16_bf16(sm, GT_TE, HALF, r64, j0, v, 1.f);
-                st16_bf16(sm, GT_TE, HALF, r64, j0 + 16, v + 16, 1.f);
-                atomicAdd(&dbt[r64], rs);
-                atomicAdd(&dg[r64], rs);
-            }
-            colsum16(kk, lane);
-            if (lo16) {
-                atomicAdd(&dg[j0 + 2 * lane], -kk[0]);
-                atomicAdd(&dg[j0 + 2 * lane + 1], -kk[1]);
-            }
+            for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int r = m0 + g + ((e >> 1) << 3), j = p0 + 8 * nt + 2 * t4 + (e & 1);
+                    acc[nt][e] = j < r ? -acc[nt][e] * ex2(g2[r] - g2[j]) : 0.f;
+                    kk[nt][e] *= acc[nt][e];
+                }
+            store_frag_cols<4>(sm, GT_TE, m0, p0, acc, lane);
+            add_row_sums<4>(dbt, m0, kk, lane, 1.f, 1.f);
+            add_row_sums<4>(dg, m0, kk, lane, 1.f, 1.f);
+            add_col_sums<4>(dg, p0, kk, lane, -1.f);
         }
         if (!publish(ok)) {
             leave();
@@ -976,10 +1048,11 @@ __global__ void __launch_bounds__(256, 1)
                 if (r < valid) {
                     const size_t gi = (size_t)(tc0 + r) * p.H_v + h;
                     p.dlog_alpha[gi] = e ? suf1 : suf0;
-                    const float b = p.beta[gi];
+                    const float b = be[e];
                     p.dbeta[gi] = b != 0.f ? dbt[r] / b : 0.f;
                 }
             }
+            if (vh + 1 < group) load_gates(vh + 1);
         }
         __syncthreads();  // the next head's gates overwrite dg, dbt and misc
     }
@@ -998,11 +1071,8 @@ __global__ void __launch_bounds__(256, 1)
         tld2x16(tq + GT_DQ + col, a, tq + GT_DK + col, b);
         if (lo16 && r64 < valid) {
             const size_t o = ((size_t)(tc0 + r64) * p.H_qk + hq) * D + col;
-#pragma unroll
-            for (int e = 0; e < 16; e += 2) {
-                store2<IO>(dq + o + e, a[e], a[e + 1]);
-                store2<IO>(dk + o + e, b[e], b[e + 1]);
-            }
+            store16<IO>(dq + o, a);
+            store16<IO>(dk + o, b);
         }
     }
     tc_fence_before();
