@@ -403,12 +403,18 @@ __device__ __forceinline__ void tld_frag4(uint32_t ta, float (*acc)[4]) {
           "=r"(u[14]), "=r"(u[15])
         : "r"(ta));
 }
+// (The empty asm statements after each wait keep every use of the values read
+// behind the tcgen05.wait::ld.)
 template <int NT>
 __device__ __forceinline__ void tld_frag(uint32_t ta, float (*acc)[4]) {
     static_assert(NT % 4 == 0, "groups of four 8-column groups");
 #pragma unroll
     for (int i = 0; i < NT / 4; ++i) tld_frag4(ta + 32 * i, acc + 4 * i);
     tmem_ld_wait();
+#pragma unroll
+    for (int i = 0; i < NT; ++i)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) asm volatile("" : "+f"(acc[i][e]));
 }
 
 // Row sums (over the fragment's columns) of v into dst[row] (shared memory,
@@ -513,6 +519,11 @@ __device__ __forceinline__ void tld2x16(uint32_t a0, float* v0, uint32_t a1, flo
     tmem_ld16(a0, v0);
     tmem_ld16(a1, v1);
     tmem_ld_wait();
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+        asm volatile("" : "+f"(v0[i]));
+        asm volatile("" : "+f"(v1[i]));
+    }
 }
 
 template <typename IO>
@@ -728,6 +739,8 @@ __global__ void __launch_bounds__(256, 1)
                 float a[16], b[16];
                 tmem_ld16(tq + GT_T1 + col, a);
                 tmem_ld_wait();
+#pragma unroll
+                for (int e = 0; e < 16; ++e) asm volatile("" : "+f"(a[e]));
                 if (quad < 2) {
                     ld16_bf16(sm, GT_V, HALF, row, col, b);
 #pragma unroll

@@ -103,7 +103,7 @@ struct PrefillParams {
 
 // ============================================================================
 // Pass 1: chunk operators.  Grid (record slots, H_qk, batches of up to 4 value
-// heads of that head); 128 threads, five CTAs per SM.  The grams come from one
+// heads of that head); 128 threads, four CTAs per SM.  The grams come from one
 // tcgen05 product [K; Q] K^T (M = 128, N = 64, K = 128) accumulated in tensor
 // memory: TMEM lane r holds row r of K K^T (r < 64) or of Q K^T (r >= 64).
 // Warps 0-1 (the
@@ -129,7 +129,7 @@ constexpr uint32_t CO_MISC = CO_BAR + 16;           // abort flag, TMEM base
 constexpr uint32_t CO_SMEM = CO_MISC + 16 + 1024;
 constexpr uint32_t CO_TM_COLS = 64;
 static_assert(CO_XS >= 4 * HALF, "the K and Q tiles lie inside A and T");
-static_assert(5 * (CO_SMEM + 1024) <= 233472, "five pass-1 CTAs per SM");
+static_assert(4 * (CO_SMEM + 1024) <= 233472, "four pass-1 CTAs per SM");
 // named barriers of pass 1 (0 is __syncthreads)
 constexpr int CO_BAR_SOLVE = 1;  // the two solver warps
 constexpr int CO_BAR_TDONE = 2;  // solvers -> writers: T is complete
@@ -148,6 +148,14 @@ __device__ __forceinline__ uint32_t packr(float lo, float hi) {
     return F16 ? pack_f16x2(lo, hi) : pack_bf16x2(lo, hi);
 }
 
+// Values read from tensor memory stay behind the tcgen05.wait::ld that follows
+// the reads: an empty asm on each makes every later use depend on it.
+template <int N>
+__device__ __forceinline__ void pin_after_wait(float* v) {
+#pragma unroll
+    for (int i = 0; i < N; ++i) asm volatile("" : "+f"(v[i]));
+}
+
 // tf32 rounding of an fp32 value, kept as fp32 (the low mantissa bits cleared)
 __device__ __forceinline__ float tf32r(float x) { return __uint_as_float(to_tf32(x)); }
 // The decay mask M_rj = exp2(g_r - g_j) (j <= r, g in log2 units) of a row r in
@@ -162,19 +170,20 @@ __device__ __forceinline__ float tf32r(float x) { return __uint_as_float(to_tf32
 // (zeros on and above the diagonal).  Blocks right of it are never read.
 // tm_row addresses row r of K K^T in tensor memory, read one 16-column block at
 // a time; lanes 16-31 lie in row block 2W + 1, lanes 0-15 in 2W.
-template <int W>
 __device__ __forceinline__ void build_a(float* Af, uint32_t tm_row, const float* s_g,
-                                        const float* s_b, const float* s_w, int lane) {
+                                        const float* s_b, const float* s_w, int W, int lane) {
     const int r = 32 * W + lane;
     const bool hi = lane >= 16;
     const float g_r = s_g[r], b_r = s_b[r];
     float* arow = Af + r * AF_LD;
     float gA[16], gB[16];  // gram columns 16 J .. 16 J + 15 of row r
-#pragma unroll
+#pragma unroll 1
     for (int J = 0; J <= 2 * W; ++J) {
         tmem_ld16(tm_row + 16 * J, gA);
         if (J == 2 * W) tmem_ld16(tm_row + 16 * J + 16, gB);
         tmem_ld_wait();
+        pin_after_wait<16>(gA);
+        pin_after_wait<16>(gB);
         if (J < 2 * W || hi) {
             const float s = b_r * ex2(g_r - s_g[16 * J + 15]);
 #pragma unroll
@@ -208,19 +217,21 @@ __device__ __forceinline__ void build_a(float* Af, uint32_t tm_row, const float*
 // the sequence end), as bf16 or fp16 straight into the record's swizzled tile in
 // global memory; every byte of the row is written.  tm_row addresses row r of
 // Q K^T.
-template <int W, bool F16>
+template <bool F16>
 __device__ __forceinline__ void build_mqk(uint8_t* rec, uint32_t tm_row, const float* s_g,
-                                          const float* s_w, int lane, int valid) {
+                                          const float* s_w, int W, int lane, int valid) {
     const int r = 32 * W + lane;
     const bool hi = lane >= 16;
     const bool live = r < valid;
     const float g_r = s_g[r];
     float gA[16], gB[16];
-#pragma unroll
+#pragma unroll 1
     for (int J = 0; J <= 2 * W; ++J) {
         tmem_ld16(tm_row + 16 * J, gA);
         if (J == 2 * W) tmem_ld16(tm_row + 16 * J + 16, gB);
         tmem_ld_wait();
+        pin_after_wait<16>(gA);
+        pin_after_wait<16>(gB);
         if (J < 2 * W || hi) {
             const float s = live ? ex2(g_r - s_g[16 * J + 15]) : 0.f;
             uint32_t w[8];
@@ -255,7 +266,7 @@ __device__ __forceinline__ void build_mqk(uint8_t* rec, uint32_t tm_row, const f
     }
     *reinterpret_cast<uint4*>(rec + taddr(0, r, jb, 0)) = make_uint4(w[0], w[1], w[2], w[3]);
     *reinterpret_cast<uint4*>(rec + taddr(0, r, jb + 8, 0)) = make_uint4(w[4], w[5], w[6], w[7]);
-#pragma unroll
+#pragma unroll 1
     for (int J = 2 * W + 1; J < 4; ++J)
         if (J > 2 * W + (hi ? 1 : 0)) {
             *reinterpret_cast<uint4*>(rec + taddr(0, r, 16 * J, 0)) = make_uint4(0, 0, 0, 0);
@@ -442,7 +453,7 @@ __device__ __forceinline__ void solve_level2(const float* Af, float* Tf, float* 
 }
 
 template <bool F16>
-__global__ void __launch_bounds__(CO_THREADS, 5)
+__global__ void __launch_bounds__(CO_THREADS, 4)
     chunk_ops_kernel(const __grid_constant__ CUtensorMap map_q,
                      const __grid_constant__ CUtensorMap map_k, const PrefillParams p) {
     extern __shared__ uint8_t smem_raw[];
@@ -558,10 +569,7 @@ __global__ void __launch_bounds__(CO_THREADS, 5)
         uint8_t* rec = p.records + (size_t)(slot * p.H_v + h) * REC_BYTES;
         const uint32_t tm_row = tmem + ((uint32_t)(32 * warp) << 16);  // row tid of [K K^T; Q K^T]
         if (warp < 2) {
-            if (warp == 0)
-                build_a<0>(Af, tm_row, s_g, s_b, s_w, lane);
-            else
-                build_a<1>(Af, tm_row, s_g, s_b, s_w, lane);
+            build_a(Af, tm_row, s_g, s_b, s_w, warp, lane);
             __syncwarp();
             if (vh > 0) bar_sync<CO_BAR_TFREE, CO_THREADS>();  // the previous T has been read
             solve_diag_blocks(Af, Tf, tid);
@@ -573,10 +581,7 @@ __global__ void __launch_bounds__(CO_THREADS, 5)
             bar_arrive<CO_BAR_TDONE, CO_THREADS>();
         } else {
             const int q = tid - 64;
-            if (warp == 2)
-                build_mqk<0, F16>(rec + REC_MQ, tm_row, s_g, s_w, lane, valid);
-            else
-                build_mqk<1, F16>(rec + REC_MQ, tm_row, s_g, s_w, lane, valid);
+            build_mqk<F16>(rec + REC_MQ, tm_row, s_g, s_w, warp - 2, lane, valid);
             // gamma_r, d_r (zero past the sequence end), gamma_C, zero padding
             float* rv = reinterpret_cast<float*>(rec + REC_VEC);
             const float gC = s_g[C - 1];
@@ -1006,6 +1011,16 @@ __device__ __forceinline__ void tmem_ld8(uint32_t taddr, float* r) {
                  : "r"(taddr));
 }
 
+// One 8-column group of an M = 64 accumulator's 16 rows in this warp's lane
+// quarter, as the m16n8 fragment of mma.sync (thread t: rows t / 4 and t / 4 + 8,
+// columns 2 (t % 4) and + 1): tcgen05.ld.16x256b.x1, layout checked by a probe.
+__device__ __forceinline__ void tmem_ld_frag8(uint32_t taddr, float* r) {
+    uint32_t* u = reinterpret_cast<uint32_t*>(r);
+    asm volatile("tcgen05.ld.sync.aligned.16x256b.x1.b32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(u[0]), "=r"(u[1]), "=r"(u[2]), "=r"(u[3])
+                 : "r"(taddr));
+}
+
 // N columns (a multiple of 8) of this thread's TMEM lane, fp32.  The values are
 // pinned behind the wait so that no use moves above it.
 template <int N>
@@ -1076,7 +1091,6 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     const int quad = warp & 3;          // TMEM lanes 32 quad .. 32 quad + 31
     const int c_lo = (warp >> 2) * HN;  // this warp's half of the slice's columns
     const int row = 32 * quad + lane;   // my row of an M = 128 product (a state row)
-    const int r64 = 16 * quad + lane;   // my row of an M = 64 product, when lane < 16
     const int h = blockIdx.y, n = blockIdx.z;
     const int hq = h / (p.H_v / p.H_qk);
     const int col0 = blockIdx.x * NS;
@@ -1177,7 +1191,6 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         // outputs
         const float* rv = reinterpret_cast<const float*>(stp + TS_REC + REC_VEC);
         const float g_row = rv[row & 63];         // gamma of my K row (quads 0-1) or Q row (2-3)
-        const float d_row = rv[64 + (r64 & 63)];  // d of my Delta row (lanes < 16)
         const float g_C = rv[128];
         if (c >= 1 && quad >= 2) ok = output(c - 1, g_prev) && ok;
         g_prev = g_row;
@@ -1222,14 +1235,28 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         }
         ok = mbar_wait(bar_dl, par, abort_flag);
         tc_fence_after();
-        {  // Delta and d o Delta, token row r64 on lanes < 16
-            float dl[HN];
-            tmem_cols<HN>(tl + TM_DL, dl);
-            if (lane < 16) {
-                put_cols<HN, F16>(sm, TC_DU, r64, c_lo, dl, 1.f);
-                put_cols<HN>(sm, TC_DD, r64, c_lo, dl, d_row);
-                fence_proxy_async_smem();
+        {  // Delta and d o Delta, read as m16n8 fragments by all 32 lanes: rows
+           // 16 quad + g and + 8, columns c_lo + 8 i + 2 t and + 1
+            float dl[HN / 2];
+#pragma unroll
+            for (int i = 0; i < HN / 8; ++i) tmem_ld_frag8(tl + TM_DL + 8 * i, dl + 4 * i);
+            tmem_ld_wait();
+            pin_after_wait<HN / 2>(dl);
+            const int fg = lane >> 2, ft = lane & 3;
+            const int rlo = 16 * quad + fg, rhi = rlo + 8;
+            const float dlo = rv[64 + rlo], dhi = rv[64 + rhi];
+#pragma unroll
+            for (int i = 0; i < HN / 8; ++i) {
+                const int col = c_lo + 8 * i + 2 * ft;
+                const float* f = dl + 4 * i;
+                *reinterpret_cast<uint32_t*>(sm + taddr_e(TC_DU, rlo, col, 0)) = packr<F16>(f[0], f[1]);
+                *reinterpret_cast<uint32_t*>(sm + taddr_e(TC_DU, rhi, col, 0)) = packr<F16>(f[2], f[3]);
+                *reinterpret_cast<uint32_t*>(sm + taddr_e(TC_DD, rlo, col, 0)) =
+                    pack2(dlo * f[0], dlo * f[1]);
+                *reinterpret_cast<uint32_t*>(sm + taddr_e(TC_DD, rhi, col, 0)) =
+                    pack2(dhi * f[2], dhi * f[3]);
             }
+            fence_proxy_async_smem();
         }
         tc_fence_before();
         if (!bar_and<BAR_TC, TC_THREADS>(ok)) break;
@@ -1605,7 +1632,7 @@ static cudaError_t run_pass1(const CUtensorMap& mq, const CUtensorMap& mk,
     auto kern = f16_records ? chunk_ops_kernel<true> : chunk_ops_kernel<false>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, CO_SMEM);
     if (e != cudaSuccess) return e;
-    // all of the unified L1 as shared memory, so that five CTAs fit on an SM
+    // all of the unified L1 as shared memory, so that four CTAs fit on an SM
     e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout,
                              cudaSharedmemCarveoutMaxShared);
     if (e != cudaSuccess) return e;
