@@ -653,10 +653,12 @@ __device__ __forceinline__ void store_acc_r(uint8_t* smem, uint32_t base_off, in
 
 // Delta = T_b X for row block rb (rows 16 rb .. +15) and n-tiles of column half H
 // of an NT-tile slice, stored as Delta (in the records' tile type: X is in it
-// too) and d o Delta (bf16: it meets the bf16 K tile).
+// too) at shared offset du and d o Delta (bf16: it meets the bf16 K tile) at dd.
+// T_b is lower triangular, so row block rb takes k-steps 0 .. rb only.
 template <int NT, int H, bool F16>
 __device__ __forceinline__ void delta_half(uint8_t* sm, uint32_t tb, uint32_t xt, int rb,
-                                           int lane, float d_lo, float d_hi) {
+                                           int lane, float d_lo, float d_hi, uint32_t du,
+                                           uint32_t dd) {
     constexpr int N0 = H * (NT / 2), N1 = (H + 1) * (NT / 2);
     float acc[N1 - N0][4];
 #pragma unroll
@@ -687,13 +689,13 @@ __device__ __forceinline__ void delta_half(uint8_t* sm, uint32_t tb, uint32_t xt
 #pragma unroll
     for (int i = 0; i < N1 - N0; ++i) {
         const int col = 8 * (N0 + i) + 2 * t;
-        *reinterpret_cast<uint32_t*>(sm + taddr_e(P2_DU, r, col, 0)) =
+        *reinterpret_cast<uint32_t*>(sm + taddr_e(du, r, col, 0)) =
             packr<F16>(acc[i][0], acc[i][1]);
-        *reinterpret_cast<uint32_t*>(sm + taddr_e(P2_DU, r + 8, col, 0)) =
+        *reinterpret_cast<uint32_t*>(sm + taddr_e(du, r + 8, col, 0)) =
             packr<F16>(acc[i][2], acc[i][3]);
-        *reinterpret_cast<uint32_t*>(sm + taddr_e(P2_DD, r, col, 0)) =
+        *reinterpret_cast<uint32_t*>(sm + taddr_e(dd, r, col, 0)) =
             pack2(acc[i][0] * d_lo, acc[i][1] * d_lo);
-        *reinterpret_cast<uint32_t*>(sm + taddr_e(P2_DD, r + 8, col, 0)) =
+        *reinterpret_cast<uint32_t*>(sm + taddr_e(dd, r + 8, col, 0)) =
             pack2(acc[i][2] * d_hi, acc[i][3] * d_hi);
     }
 }
@@ -876,9 +878,11 @@ __global__ void __launch_bounds__(P2_THREADS, 1)
                 const int rb = warp & 3;
                 const float d_lo = rv[64 + m0 + g], d_hi = rv[64 + m0 + g + 8];
                 if (warp < 4)
-                    delta_half<NT, 0, F16>(sm, st + ST_REC + REC_TB, sb + P2_X, rb, lane, d_lo, d_hi);
+                    delta_half<NT, 0, F16>(sm, st + ST_REC + REC_TB, sb + P2_X, rb, lane, d_lo, d_hi,
+                                           P2_DU, P2_DD);
                 else
-                    delta_half<NT, 1, F16>(sm, st + ST_REC + REC_TB, sb + P2_X, rb, lane, d_lo, d_hi);
+                    delta_half<NT, 1, F16>(sm, st + ST_REC + REC_TB, sb + P2_X, rb, lane, d_lo, d_hi,
+                                           P2_DU, P2_DD);
             }
             if (!bar_and<BAR_CHAIN, P2_CHAIN_THREADS>(ok)) break;
 
@@ -965,15 +969,16 @@ __global__ void __launch_bounds__(P2_THREADS, 1)
 // states.  Grid (d_v slices, H_v, N); 256 threads; one thread issues every
 // tcgen05.mma, accumulators live in tensor memory.  Per chunk:
 //   [K; Q] S             M = 128: lanes 0-63 K S, lanes 64-127 Q S
-//   Delta = T_b X        M = 64:  row r in lane (r % 16) + 32 (r / 16)
+//   Delta = T_b X        warp-level mma.sync (64 x NS, K = 64, T_b lower triangular)
 //   K^T (d o Delta)      M = 128: the state increment, lane = d_k index
 //   [T_b; M_Q] Delta     M = 128: lanes 64-127 (M o Q K^T) Delta, beside Q S
 // (M_Q = M o Q K^T; the record stores T_b and M_Q as adjacent 64-row K-major
 // tiles, so [T_b; M_Q] is one 128-row operand.)  Between the products every
 // warp reads its TMEM lanes and half of the slice's columns (warps w and w + 4
-// share lane quadrant w): X and Delta go back to shared memory in bf16 as the
-// next product's B operand (MN-major); each thread keeps half a row of the
-// fp32 state and writes its bf16 copy, the next [K; Q] S's B operand.  The
+// share lane quadrant w): X goes to shared memory as the B operand of T_b X,
+// Delta as that of the next products (MN-major); each thread keeps
+// half a row of the fp32 state and writes its bf16 copy, the next [K; Q] S's
+// B operand.  The
 // output rows O = gamma o (Q S) + (M o Q K^T) Delta of a chunk are formed by
 // the warps on lanes 64-127 while the next chunk's [K; Q] S runs ([K; Q] S
 // and [T_b; M_Q] Delta are double-buffered in TMEM).  Every product commits
@@ -994,30 +999,20 @@ constexpr uint32_t TC_SB = NSTAGE * TS_STAGE;  // S in bf16: 128 k-rows x 64 col
 constexpr uint32_t TC_X = TC_SB + 2 * HALF;    // X, 64 token rows x 64 columns, MN-major
 constexpr uint32_t TC_DU = TC_X + HALF;        // Delta
 constexpr uint32_t TC_DD = TC_DU + HALF;       // d o Delta
-constexpr uint32_t TC_BAR = TC_DD + HALF;      // full[NSTAGE], ks, dl, u, o, drain
+constexpr uint32_t TC_BAR = TC_DD + HALF;      // full[NSTAGE], ks, u, o, drain
 constexpr uint32_t TC_MISC = TC_BAR + 128;     // abort flag, TMEM base
 constexpr uint32_t TC_SMEM = TC_MISC + 16 + 1024;
 static_assert(TS_STAGE % 1024 == 0 && TC_SB % 1024 == 0, "swizzled tiles sit on 1 KB");
 static_assert(TC_SMEM <= 232448, "tcgen05 state pass shared memory budget");
-// TMEM columns (512 allocated): [K; Q] S (two buffers), Delta, the state
-// increment, [T_b; M_Q] Delta (two buffers)
-constexpr uint32_t TM_KQ = 0, TM_DL = 128, TM_U = 192, TM_O = 256, TM_COLS = 512;
+// TMEM columns (512 allocated): [K; Q] S (two buffers), the state increment,
+// [T_b; M_Q] Delta (two buffers)
+constexpr uint32_t TM_KQ = 0, TM_U = 192, TM_O = 256, TM_COLS = 512;
 
 __device__ __forceinline__ void tmem_ld8(uint32_t taddr, float* r) {
     uint32_t* u = reinterpret_cast<uint32_t*>(r);
     asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
                  : "=r"(u[0]), "=r"(u[1]), "=r"(u[2]), "=r"(u[3]), "=r"(u[4]), "=r"(u[5]),
                    "=r"(u[6]), "=r"(u[7])
-                 : "r"(taddr));
-}
-
-// One 8-column group of an M = 64 accumulator's 16 rows in this warp's lane
-// quarter, as the m16n8 fragment of mma.sync (thread t: rows t / 4 and t / 4 + 8,
-// columns 2 (t % 4) and + 1): tcgen05.ld.16x256b.x1, layout checked by a probe.
-__device__ __forceinline__ void tmem_ld_frag8(uint32_t taddr, float* r) {
-    uint32_t* u = reinterpret_cast<uint32_t*>(r);
-    asm volatile("tcgen05.ld.sync.aligned.16x256b.x1.b32 {%0,%1,%2,%3}, [%4];"
-                 : "=r"(u[0]), "=r"(u[1]), "=r"(u[2]), "=r"(u[3])
                  : "r"(taddr));
 }
 
@@ -1072,7 +1067,6 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     constexpr uint32_t ID_KT = idesc_bf16(128, NS, 1, 1);   // MN-major A (K^T), MN-major B
     // the products with a record tile as A (T_b X, [T_b; M o Q K^T] Delta): fp16
     // when the records are fp16, and then X and Delta are written as fp16 too
-    constexpr uint32_t ID_R64 = F16 ? idesc_f16(64, NS, 0, 1) : idesc_bf16(64, NS, 0, 1);
     constexpr uint32_t ID_R128 = F16 ? idesc_f16(128, NS, 0, 1) : idesc_bf16(128, NS, 0, 1);
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -1080,10 +1074,9 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     const uint32_t sb = smem_u32(sm);
     uint64_t* bars = reinterpret_cast<uint64_t*>(sm + TC_BAR);
     uint64_t* bar_ks = bars + NSTAGE;
-    uint64_t* bar_dl = bars + NSTAGE + 1;
-    uint64_t* bar_u = bars + NSTAGE + 2;
-    uint64_t* bar_o = bars + NSTAGE + 3;
-    uint64_t* drain_bar = bars + NSTAGE + 4;
+    uint64_t* bar_u = bars + NSTAGE + 1;
+    uint64_t* bar_o = bars + NSTAGE + 2;
+    uint64_t* drain_bar = bars + NSTAGE + 3;
     volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + TC_MISC);
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + TC_MISC + 4);
 
@@ -1100,7 +1093,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     const int nchunks = (t_end - t_beg + C - 1) / C;
 
     if (tid == 0) {
-        for (int i = 0; i < NSTAGE + 5; ++i) mbar_init(&bars[i], 1);
+        for (int i = 0; i < NSTAGE + 4; ++i) mbar_init(&bars[i], 1);
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -1217,45 +1210,24 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
                         x[8 * i + 2 * e + 1] = v2.y - g_row * x[8 * i + 2 * e + 1];
                     }
                 }
-                put_cols<HN, F16>(sm, TC_X, row, c_lo, x, 1.f);
-                fence_proxy_async_smem();
+                put_cols<HN, F16>(sm, TC_X, row, c_lo, x, 1.f);  // read by ldmatrix only
             }
         }
         tc_fence_before();
         if (!bar_and<BAR_TC, TC_THREADS>(ok)) break;
 
-        // Delta = T_b X
-        if (tid == 0) {
-            tc_fence_after();
-#pragma unroll
-            for (int ks = 0; ks < 4; ++ks)
-                mma_bf16_ss(tmem + TM_DL, sdesc_sw128(st + TS_REC + ks * 32, 16, 1024),
-                            sdesc_sw128(sb + TC_X + ks * 2048, 8192, 1024), ID_R64, ks > 0);
-            mma_commit(bar_dl);
-        }
-        ok = mbar_wait(bar_dl, par, abort_flag);
-        tc_fence_after();
-        {  // Delta and d o Delta, read as m16n8 fragments by all 32 lanes: rows
-           // 16 quad + g and + 8, columns c_lo + 8 i + 2 t and + 1
-            float dl[HN / 2];
-#pragma unroll
-            for (int i = 0; i < HN / 8; ++i) tmem_ld_frag8(tl + TM_DL + 8 * i, dl + 4 * i);
-            tmem_ld_wait();
-            pin_after_wait<HN / 2>(dl);
-            const int fg = lane >> 2, ft = lane & 3;
-            const int rlo = 16 * quad + fg, rhi = rlo + 8;
-            const float dlo = rv[64 + rlo], dhi = rv[64 + rhi];
-#pragma unroll
-            for (int i = 0; i < HN / 8; ++i) {
-                const int col = c_lo + 8 * i + 2 * ft;
-                const float* f = dl + 4 * i;
-                *reinterpret_cast<uint32_t*>(sm + taddr_e(TC_DU, rlo, col, 0)) = packr<F16>(f[0], f[1]);
-                *reinterpret_cast<uint32_t*>(sm + taddr_e(TC_DU, rhi, col, 0)) = packr<F16>(f[2], f[3]);
-                *reinterpret_cast<uint32_t*>(sm + taddr_e(TC_DD, rlo, col, 0)) =
-                    pack2(dlo * f[0], dlo * f[1]);
-                *reinterpret_cast<uint32_t*>(sm + taddr_e(TC_DD, rhi, col, 0)) =
-                    pack2(dhi * f[2], dhi * f[3]);
-            }
+        // Delta = T_b X on mma.sync: warp (quad, column half) takes rows 16 quad ..
+        // + 15 of its half, so no commit, wake-up or TMEM read sits on the chain;
+        // Delta and d o Delta go to shared memory as the next products' B operands
+        {
+            const int rlo = 16 * quad + (lane >> 2);
+            const float dlo = rv[64 + rlo], dhi = rv[64 + rlo + 8];
+            if (warp < 4)
+                delta_half<NS / 8, 0, F16>(sm, st + TS_REC + REC_TB, sb + TC_X, quad, lane, dlo,
+                                           dhi, TC_DU, TC_DD);
+            else
+                delta_half<NS / 8, 1, F16>(sm, st + TS_REC + REC_TB, sb + TC_X, quad, lane, dlo,
+                                           dhi, TC_DU, TC_DD);
             fence_proxy_async_smem();
         }
         tc_fence_before();
