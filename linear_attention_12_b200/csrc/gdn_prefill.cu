@@ -1056,12 +1056,18 @@ __device__ __forceinline__ void store8<__nv_bfloat16>(__nv_bfloat16* p, const fl
                                               pack2(v[4], v[5]), pack2(v[6], v[7]));
 }
 
-template <int NS, typename IO, bool F16>
+// MODE P2_OUT: outputs and final states.  P2_SAVE: no outputs; every chunk's
+// entering state goes to S_aux as a bf16 image (for the gradients).
+// P2_OUT_SAVE: both.
+template <int NS, typename IO, bool F16, int MODE>
 __global__ void __launch_bounds__(TC_THREADS, 1)
     state_tc_kernel(const __grid_constant__ CUtensorMap map_q,
                     const __grid_constant__ CUtensorMap map_k,
                     const __grid_constant__ CUtensorMap map_v, const PrefillParams p) {
     static_assert(NS == 32 || NS == 48 || NS == 64, "slice width");
+    static_assert(MODE == P2_OUT || MODE == P2_SAVE || MODE == P2_OUT_SAVE, "modes");
+    constexpr bool OUTS = MODE != P2_SAVE;  // writes the outputs
+    constexpr bool SAVE = MODE != P2_OUT;   // saves every chunk's entering state
     constexpr int HN = NS / 2;                              // columns per half
     constexpr uint32_t ID_128 = idesc_bf16(128, NS, 0, 1);  // K-major A, MN-major B
     constexpr uint32_t ID_KT = idesc_bf16(128, NS, 1, 1);   // MN-major A (K^T), MN-major B
@@ -1127,6 +1133,19 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
 
     // row `row` of the state, columns col0 + c_lo .. + HN - 1, fp32
     float Sr[HN];
+    // the state entering chunk cc into its bf16 image (16 bytes per 8 columns)
+    auto save_image = [&](int cc) {
+        if (!SAVE || cc >= nchunks) return;
+        uint8_t* sv = reinterpret_cast<uint8_t*>(p.S_aux) +
+                      ((size_t)record_slot(n, t_beg + cc * C) * p.H_v + h) * STATE_IMAGE_BYTES;
+#pragma unroll
+        for (int i = 0; i < HN / 8; ++i)
+            if (c_lo + 8 * i < ncols)
+                *reinterpret_cast<uint4*>(sv + taddr(0, row, col0 + c_lo + 8 * i, 2 * HALF)) =
+                    make_uint4(pack2(Sr[8 * i], Sr[8 * i + 1]), pack2(Sr[8 * i + 2], Sr[8 * i + 3]),
+                               pack2(Sr[8 * i + 4], Sr[8 * i + 5]),
+                               pack2(Sr[8 * i + 6], Sr[8 * i + 7]));
+    };
     {
         const float* s0 =
             p.S0 ? p.S0 + (((size_t)n * p.H_v + h) * D + row) * D + col0 + c_lo : nullptr;
@@ -1134,6 +1153,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         for (int j = 0; j < HN; ++j) Sr[j] = (s0 && c_lo + j < ncols) ? s0[j] : 0.f;
         put_cols<HN>(sm, TC_SB, row, c_lo, Sr, 1.f);
         fence_proxy_async_smem();
+        save_image(0);
     }
     __syncthreads();  // the first K S reads the whole tile
 
@@ -1185,7 +1205,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         const float* rv = reinterpret_cast<const float*>(stp + TS_REC + REC_VEC);
         const float g_row = rv[row & 63];         // gamma of my K row (quads 0-1) or Q row (2-3)
         const float g_C = rv[128];
-        if (c >= 1 && quad >= 2) ok = output(c - 1, g_prev) && ok;
+        if (OUTS && c >= 1 && quad >= 2) ok = output(c - 1, g_prev) && ok;
         g_prev = g_row;
         ok = mbar_wait(bar_ks, par, abort_flag) && ok;
         tc_fence_after();
@@ -1241,11 +1261,13 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
                 mma_bf16_ss(tmem + TM_U, sdesc_sw128(st + TS_KQ + ks * 2048, 2 * HALF, 1024),
                             sdesc_sw128(sb + TC_DD + ks * 2048, 8192, 1024), ID_KT, ks > 0);
             mma_commit(bar_u);
+            if constexpr (OUTS) {
 #pragma unroll
-            for (int ks = 0; ks < 4; ++ks)
-                mma_bf16_ss(tmem + TM_O + 64 * par, sdesc_sw128(st + TS_REC + ks * 32, 16, 1024),
-                            sdesc_sw128(sb + TC_DU + ks * 2048, 8192, 1024), ID_R128, ks > 0);
-            mma_commit(bar_o);
+                for (int ks = 0; ks < 4; ++ks)
+                    mma_bf16_ss(tmem + TM_O + 64 * par, sdesc_sw128(st + TS_REC + ks * 32, 16, 1024),
+                                sdesc_sw128(sb + TC_DU + ks * 2048, 8192, 1024), ID_R128, ks > 0);
+                mma_commit(bar_o);
+            }
         }
         ok = mbar_wait(bar_u, par, abort_flag);
         tc_fence_after();
@@ -1256,11 +1278,12 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
             for (int j = 0; j < HN; ++j) Sr[j] = fmaf(g_C, Sr[j], u[j]);
             put_cols<HN>(sm, TC_SB, row, c_lo, Sr, 1.f);
             fence_proxy_async_smem();
+            save_image(c + 1);
         }
         tc_fence_before();
         if (!bar_and<BAR_TC, TC_THREADS>(ok)) break;
     }
-    if (nchunks > 0 && !*abort_flag && quad >= 2) {  // the last chunk's outputs
+    if (OUTS && nchunks > 0 && !*abort_flag && quad >= 2) {  // the last chunk's outputs
         output(nchunks - 1, g_prev);
         tc_fence_before();
     }
@@ -1289,10 +1312,10 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     }
 }
 
-template <int NS, typename IO, bool F16>
+template <int NS, typename IO, bool F16, int MODE>
 cudaError_t launch_state_tc(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                             const PrefillParams& prm, cudaStream_t stream) {
-    auto kern = state_tc_kernel<NS, IO, F16>;
+    auto kern = state_tc_kernel<NS, IO, F16, MODE>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, TC_SMEM);
     if (e != cudaSuccess) return e;
     dim3 grid((D + NS - 1) / NS, prm.H_v, prm.N);
@@ -1558,13 +1581,13 @@ static bool output_pass_is_tc(int state_pass, int slices) {
     return state_pass == STATE_PASS_TC || (state_pass == STATE_PASS_AUTO && slices == 3);
 }
 
-template <typename IO, bool F16>
+template <typename IO, bool F16, int MODE>
 static cudaError_t launch_state_tc_slices(const CUtensorMap& mq, const CUtensorMap& mk,
                                           const CUtensorMap& mv, const PrefillParams& prm,
                                           int slices, cudaStream_t stream) {
-    if (slices == 4) return launch_state_tc<32, IO, F16>(mq, mk, mv, prm, stream);
-    if (slices == 3) return launch_state_tc<48, IO, F16>(mq, mk, mv, prm, stream);
-    return launch_state_tc<64, IO, F16>(mq, mk, mv, prm, stream);
+    if (slices == 4) return launch_state_tc<32, IO, F16, MODE>(mq, mk, mv, prm, stream);
+    if (slices == 3) return launch_state_tc<48, IO, F16, MODE>(mq, mk, mv, prm, stream);
+    return launch_state_tc<64, IO, F16, MODE>(mq, mk, mv, prm, stream);
 }
 
 // f16_records: the records were written with fp16 tiles (read by the output
@@ -1580,8 +1603,12 @@ static cudaError_t run_pass2(const CUtensorMap& mq, const CUtensorMap& mk, const
     if constexpr (MODE == P2_OUT) {
         if (output_pass_is_tc(state_pass, slices))
             return f16_records
-                       ? launch_state_tc_slices<IO, true>(mq, mk, mv, prm, slices, stream)
-                       : launch_state_tc_slices<IO, false>(mq, mk, mv, prm, slices, stream);
+                       ? launch_state_tc_slices<IO, true, MODE>(mq, mk, mv, prm, slices, stream)
+                       : launch_state_tc_slices<IO, false, MODE>(mq, mk, mv, prm, slices, stream);
+    }
+    if constexpr (MODE == P2_SAVE || MODE == P2_OUT_SAVE) {  // bf16 records
+        if (output_pass_is_tc(state_pass, slices) && !f16_records)
+            return launch_state_tc_slices<IO, false, MODE>(mq, mk, mv, prm, slices, stream);
     }
     if (f16_records) {
         if constexpr (MODE == P2_OUT) {
@@ -1712,9 +1739,11 @@ cudaError_t launch_prefill_save(const void* q, const void* k, const void* v,
     cudaError_t e = run_pass1(mq, mk, prm, stream);
     if (e != cudaSuccess) return e;
     const int sms = device_sms();
-    if (!o) return run_pass2<__nv_bfloat16, P2_SAVE>(mq, mk, mv, prm, sms, stream);
-    return out_bf16 ? run_pass2<__nv_bfloat16, P2_OUT_SAVE>(mq, mk, mv, prm, sms, stream)
-                    : run_pass2<float, P2_OUT_SAVE>(mq, mk, mv, prm, sms, stream);
+    // the state pass on tcgen05 at 48-column slices, as for the prefill
+    const int sp = STATE_PASS_AUTO;
+    if (!o) return run_pass2<__nv_bfloat16, P2_SAVE>(mq, mk, mv, prm, sms, stream, sp);
+    return out_bf16 ? run_pass2<__nv_bfloat16, P2_OUT_SAVE>(mq, mk, mv, prm, sms, stream, sp)
+                    : run_pass2<float, P2_OUT_SAVE>(mq, mk, mv, prm, sms, stream, sp);
 }
 
 size_t prefill_record_bytes(int N, int T, int H_v) { return record_bytes(N, T, H_v); }

@@ -67,6 +67,13 @@ def test_backward_sixteen_heads_4k_packed():
     _check(case, dO, dSf)
 
 
+def test_backward_bench_layout():
+    # 16/48 heads on one sequence: 48-column slices, where the forward re-run
+    # saves its states from the tcgen05 state pass
+    case, dO, dSf = _case("bw_48", [1000], 16, 48, seed=10)
+    _check(case, dO, dSf)
+
+
 @pytest.mark.parametrize("lens,H_qk,H_v", [([100, 0, 37, 64], 2, 6), ([1100], 1, 3)])
 def test_backward_fp32_io(lens, H_qk, H_v):
     # fp32 inputs and gradients (the products read bf16 copies of q, k, v and dO)
@@ -75,9 +82,13 @@ def test_backward_fp32_io(lens, H_qk, H_v):
     _check(case, dO, dSf, dtype=torch.float32)
 
 
+# (the last two: 48 value-head units, so 48-column slices and the tcgen05 state
+# pass writing outputs and saved states together)
 @pytest.mark.parametrize("lens,H_qk,H_v,dtype", [([100, 0, 37, 64], 2, 6, torch.bfloat16),
                                                  ([1100], 1, 3, torch.bfloat16),
-                                                 ([300, 65], 2, 4, torch.float32)])
+                                                 ([300, 65], 2, 4, torch.float32),
+                                                 ([700], 16, 48, torch.bfloat16),
+                                                 ([333, 130], 8, 24, torch.float32)])
 def test_training_forward_then_saved_backward(lens, H_qk, H_v, dtype):
     # the training forward's outputs match the oracle's forward; the backward that
     # reads its saved states matches the oracle's gradients
