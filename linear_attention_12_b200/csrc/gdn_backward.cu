@@ -112,7 +112,8 @@ static_assert(GS_SMEM <= 232448, "reverse chain shared memory budget");
 template <int NT, int H, typename IO>
 __device__ __forceinline__ void dx_half(uint8_t* sm, uint32_t sb, uint32_t tb, int rb, int lane,
                                         const float* rv, int valid, const GradParams& p, int tc0,
-                                        int h, int col0, int ncols) {
+                                        int h, int col0, int ncols, uint32_t ddel = GS_DDEL,
+                                        uint32_t gdx = GS_GDX) {
     constexpr int N0 = H * (NT / 2), N1 = (H + 1) * (NT / 2);
     float acc[N1 - N0][4];
     zero_acc<N1 - N0>(acc);
@@ -123,12 +124,12 @@ __device__ __forceinline__ void dx_half(uint8_t* sm, uint32_t sb, uint32_t tb, i
         for (int nt = N0; nt < N1; nt += 2) {
             if (nt + 1 < N1) {
                 uint32_t b[4];
-                ldb_mn(sb + GS_DDEL, 0, 8 * nt, 16 * ks, lane, b);
+                ldb_mn(sb + ddel, 0, 8 * nt, 16 * ks, lane, b);
                 mma16816(acc[nt - N0], a, b[0], b[1]);
                 mma16816(acc[nt - N0 + 1], a, b[2], b[3]);
             } else {
                 uint32_t b[2];
-                ldb_mn1(sb + GS_DDEL, 8 * nt, 16 * ks, lane, b);
+                ldb_mn1(sb + ddel, 8 * nt, 16 * ks, lane, b);
                 mma16816(acc[nt - N0], a, b[0], b[1]);
             }
         }
@@ -139,9 +140,9 @@ __device__ __forceinline__ void dx_half(uint8_t* sm, uint32_t sb, uint32_t tb, i
 #pragma unroll
     for (int i = 0; i < N1 - N0; ++i) {
         const int col = 8 * (N0 + i) + 2 * t;
-        *reinterpret_cast<uint32_t*>(sm + taddr_e(GS_GDX, r, col, 0)) =
+        *reinterpret_cast<uint32_t*>(sm + taddr_e(gdx, r, col, 0)) =
             pack2(-gm_lo * acc[i][0], -gm_lo * acc[i][1]);
-        *reinterpret_cast<uint32_t*>(sm + taddr_e(GS_GDX, r + 8, col, 0)) =
+        *reinterpret_cast<uint32_t*>(sm + taddr_e(gdx, r + 8, col, 0)) =
             pack2(-gm_hi * acc[i][2], -gm_hi * acc[i][3]);
         if (col < ncols) {
             if (r < valid)
@@ -327,6 +328,316 @@ __device__ __forceinline__ float tile_dot(const uint8_t* a, const uint8_t* b, in
         }
     }
     return dot;
+}
+
+// ============================================================================
+// Reverse chain on the fifth-generation tensor cores.  Grid (d_v slices, H_v,
+// N); 256 threads; the chunks in reverse order through a 3-stage ring
+// [Q h0 | K h0 | Q h1 | K h1 | dO slice | record], filled by warp 6's thread 0.
+// Per chunk, with dS' the gradient of the state after it:
+//   [Q; K] dS'                 tcgen05, M = 128: lanes 64-127 hold K dS'
+//   [T_b^T; (M o QK^T)^T] dO   tcgen05, M = 128: lanes 64-127 hold (M o QK^T)^T dO
+//   dDelta = (M o QK^T)^T dO + d o (K dS')     the warps on lanes 64-127
+//   dX = T_b^T dDelta          warp-level mma.sync (T_b^T upper triangular);
+//                              dV = dX, and -gamma o dX to shared memory
+//   dS = gamma_C dS' + Q^T (gamma o dO) + K^T (-gamma o dX)
+//                              tcgen05, M = 128, both products into one
+//                              accumulator (lane = d_k index)
+// The products that read only dO (the second, and Q^T (gamma o dO)) are issued
+// a chunk ahead, once the warps on lanes 0-63 have formed gamma o dO; only
+// [Q; K] dS' and K^T (-gamma o dX) sit on the chain.  Every thread keeps half a
+// row of dS in fp32, writes its bf16 copy (the next [Q; K] dS' operand) and,
+// per chunk, its part of the bf16 image of dS' for the per-chunk gradients.
+// ============================================================================
+constexpr int GST_THREADS = 256;
+constexpr int GST_LOADER = 192;           // warp 6
+constexpr int GST_BAR = 1, GST_BAR_LO = 2;  // all warps; the warps on TMEM lanes 0-63
+constexpr uint32_t GST_O = 4 * HALF, GST_REC = 5 * HALF;
+constexpr uint32_t GST_STAGE = ((GST_REC + REC_BYTES + 1023) / 1024) * 1024;
+constexpr uint32_t GST_TX = 5 * HALF + REC_BYTES;
+constexpr uint32_t GST_DSB = GS_STAGES * GST_STAGE;  // dS' in bf16, 128 x 64, MN-major
+constexpr uint32_t GST_DDEL = GST_DSB + 2 * HALF;    // dDelta, 64 x 64
+constexpr uint32_t GST_GDX = GST_DDEL + HALF;        // -gamma o dX
+constexpr uint32_t GST_GDO = GST_GDX + HALF;         // gamma o dO, two buffers
+constexpr uint32_t GST_BARS = GST_GDO + 2 * HALF;    // full[3], a, o[2], u, drain
+constexpr uint32_t GST_MISC = GST_BARS + 128;        // abort flag, TMEM base
+constexpr uint32_t GST_SMEM = GST_MISC + 16 + 1024;
+static_assert(GST_STAGE % 1024 == 0 && GST_DSB % 1024 == 0, "swizzled tiles sit on 1 KB");
+static_assert(GST_SMEM <= 232448, "tcgen05 reverse chain shared memory budget");
+// TMEM columns: K dS' (lanes 64-127 read), (M o QK^T)^T dO (two buffers), the
+// dS increment (two buffers)
+constexpr uint32_t GTM_A = 0, GTM_O = 64, GTM_U = 192, GTM_COLS = 512;
+
+__device__ __forceinline__ void tmem_ld8(uint32_t taddr, float* r) {
+    uint32_t* u = reinterpret_cast<uint32_t*>(r);
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+                 : "=r"(u[0]), "=r"(u[1]), "=r"(u[2]), "=r"(u[3]), "=r"(u[4]), "=r"(u[5]),
+                   "=r"(u[6]), "=r"(u[7])
+                 : "r"(taddr));
+}
+// N columns (a multiple of 8) of this thread's TMEM lane, pinned behind the wait.
+template <int N>
+__device__ __forceinline__ void tmem_row(uint32_t ta, float* v) {
+#pragma unroll
+    for (int i = 0; i < N / 8; ++i) tmem_ld8(ta + 8 * i, v + 8 * i);
+    tmem_ld_wait();
+#pragma unroll
+    for (int i = 0; i < N; ++i) asm volatile("" : "+f"(v[i]));
+}
+// Columns c0 .. c0 + N - 1 (multiples of 8) of row r of a 64-column MN-major
+// 128B-swizzled bf16 tile, scaled by s.
+template <int N>
+__device__ __forceinline__ void put_row(uint8_t* sm, uint32_t tile, int r, int c0, const float* v,
+                                        float s) {
+#pragma unroll
+    for (int i = 0; i < N / 8; ++i)
+        *reinterpret_cast<uint4*>(sm + taddr(tile, r, c0 + 8 * i, 0)) =
+            make_uint4(pack2(s * v[8 * i], s * v[8 * i + 1]), pack2(s * v[8 * i + 2], s * v[8 * i + 3]),
+                       pack2(s * v[8 * i + 4], s * v[8 * i + 5]),
+                       pack2(s * v[8 * i + 6], s * v[8 * i + 7]));
+}
+
+template <int NS, typename IO>
+__global__ void __launch_bounds__(GST_THREADS, 1)
+    grad_state_tc_kernel(const __grid_constant__ CUtensorMap map_q,
+                         const __grid_constant__ CUtensorMap map_k,
+                         const __grid_constant__ CUtensorMap map_do, const GradParams p) {
+    static_assert(NS == 32 || NS == 48 || NS == 64, "slice width");
+    constexpr int HN = NS / 2, NT = NS / 8;
+    constexpr uint32_t ID_KM = idesc_bf16(128, NS, 0, 1);  // K-major A, MN-major B
+    constexpr uint32_t ID_MM = idesc_bf16(128, NS, 1, 1);  // MN-major A and B
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+    const uint32_t sb = smem_u32(sm);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(sm + GST_BARS);
+    uint64_t* bar_a = bars + GS_STAGES;
+    uint64_t* bar_o = bars + GS_STAGES + 1;  // two: chunk index i commits to bar_o[i & 1]
+    uint64_t* bar_u = bars + GS_STAGES + 3;
+    uint64_t* drain_bar = bars + GS_STAGES + 4;
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + GST_MISC);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + GST_MISC + 4);
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int quad = warp & 3;          // TMEM lanes 32 quad .. + 31
+    const int c_lo = (warp >> 2) * HN;  // this warp's half of the slice's columns
+    const int row = 32 * quad + lane;   // my row of an M = 128 product (a d_k index)
+    const int h = blockIdx.y, n = blockIdx.z;
+    const int hq = h / (p.H_v / p.H_qk);
+    const int col0 = blockIdx.x * NS;
+    const int ncols = min(NS, D - col0);
+    const int t_beg = p.cu_seqlens[n], t_end = p.cu_seqlens[n + 1];
+    const int nchunks = (t_end - t_beg + C - 1) / C;
+
+    if (tid == 0) {
+        for (int i = 0; i < GS_STAGES + 5; ++i) mbar_init(&bars[i], 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 0) {
+        tmem_alloc(tmem_slot, GTM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const uint32_t tl = tmem + ((uint32_t)(32 * quad) << 16) + c_lo;  // my lanes, my columns
+
+    // chunk index i is chunk nchunks - 1 - i, in ring stage i % GS_STAGES
+    auto issue = [&](int i) {
+        const int c = nchunks - 1 - i, s = i % GS_STAGES;
+        uint8_t* st = sm + s * GST_STAGE;
+        const int y = t_beg + c * C;
+        uint64_t* full = &bars[s];
+        mbar_arrive_expect_tx(full, GST_TX);
+        tma_load_2d(st, &map_q, hq * D, y, full);
+        tma_load_2d(st + HALF, &map_k, hq * D, y, full);
+        tma_load_2d(st + 2 * HALF, &map_q, hq * D + 64, y, full);
+        tma_load_2d(st + 3 * HALF, &map_k, hq * D + 64, y, full);
+        tma_load_2d(st + GST_O, &map_do, h * D + col0, y, full);
+        bulk_load(st + GST_REC, p.records + (size_t)(record_slot(n, y) * p.H_v + h) * REC_BYTES,
+                  REC_BYTES, full);
+    };
+    int issued = 0;
+    if (tid == GST_LOADER)
+        for (; issued < min(GS_STAGES, nchunks); ++issued) issue(issued);
+
+    // dS: row `row`, columns col0 + c_lo .. + HN - 1, fp32 (dS_final to start)
+    float G[HN];
+    {
+        const float* s0 =
+            p.dS_final ? p.dS_final + (((size_t)n * p.H_v + h) * D + row) * D + col0 + c_lo : nullptr;
+#pragma unroll
+        for (int j = 0; j < HN; ++j) G[j] = (s0 && c_lo + j < ncols) ? s0[j] : 0.f;
+        put_row<HN>(sm, GST_DSB, row, c_lo, G, 1.f);
+        fence_proxy_async_smem();
+    }
+    // gamma o dO of chunk index i into GDO[i & 1] (warps on lanes 0-63: token row
+    // `row`; zero past the sequence end, where the rows belong to the next one)
+    auto gamma_do = [&](int i) -> bool {
+        const int s = i % GS_STAGES;
+        const bool landed = mbar_wait(&bars[s], (i / GS_STAGES) & 1, abort_flag);
+        const uint8_t* stp = sm + s * GST_STAGE;
+        const float* rv = reinterpret_cast<const float*>(stp + GST_REC + REC_VEC);
+        const int valid = min(C, t_end - (t_beg + (nchunks - 1 - i) * C));
+        const float gm = row < valid ? rv[row] : 0.f;
+        float x[HN];
+#pragma unroll
+        for (int q = 0; q < HN / 8; ++q) {
+            const uint4 u = *reinterpret_cast<const uint4*>(stp + taddr(GST_O, row, c_lo + 8 * q, 0));
+            const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[e]));
+                x[8 * q + 2 * e] = f.x;
+                x[8 * q + 2 * e + 1] = f.y;
+            }
+        }
+        put_row<HN>(sm, GST_GDO + (i & 1) * HALF, row, c_lo, x, gm);
+        fence_proxy_async_smem();
+        return landed;
+    };
+    // (thread 0) the products of chunk index i that read only dO: Q^T (gamma o dO)
+    // into U[i & 1], [T_b^T; (M o QK^T)^T] dO into O[i & 1]
+    auto issue_ahead = [&](int i) {
+        const uint32_t st = sb + (i % GS_STAGES) * GST_STAGE;
+        tc_fence_after();
+#pragma unroll
+        for (int ks = 0; ks < 4; ++ks)
+            mma_bf16_ss(tmem + GTM_U + 64 * (i & 1), sdesc_sw128(st + ks * 2048, 2 * HALF, 1024),
+                        sdesc_sw128(sb + GST_GDO + (i & 1) * HALF + ks * 2048, 8192, 1024), ID_MM,
+                        ks > 0);
+#pragma unroll
+        for (int ks = 0; ks < 4; ++ks)
+            mma_bf16_ss(tmem + GTM_O + 64 * (i & 1), sdesc_sw128(st + GST_REC + ks * 2048, HALF, 1024),
+                        sdesc_sw128(st + GST_O + ks * 2048, 8192, 1024), ID_MM, ks > 0);
+        mma_commit(&bar_o[i & 1]);
+    };
+    bool ok = true;
+    if (quad < 2 && nchunks > 0) {
+        ok = gamma_do(0);
+        bar_sync<GST_BAR_LO, 128>();
+        if (tid == 0) issue_ahead(0);
+    }
+    __syncthreads();  // the first [Q; K] dS' reads the whole dS' tile
+
+    for (int i = 0; i < nchunks; ++i) {
+        const int c = nchunks - 1 - i, s = i % GS_STAGES;
+        const uint32_t st = sb + s * GST_STAGE;
+        const uint8_t* stp = sm + s * GST_STAGE;
+        const uint32_t par = i & 1;
+        const float* rv = reinterpret_cast<const float*>(stp + GST_REC + REC_VEC);
+        const int tc0 = t_beg + c * C;
+        const int valid = min(C, t_end - tc0);
+        ok = mbar_wait(&bars[s], (i / GS_STAGES) & 1, abort_flag) && ok;
+        const float g_C = rv[128];
+        if (tid == 0) {  // [Q; K] dS'
+            tc_fence_after();
+#pragma unroll
+            for (int ks = 0; ks < 8; ++ks)
+                mma_bf16_ss(tmem + GTM_A,
+                            sdesc_sw128(st + (ks >> 2) * 2 * HALF + (ks & 3) * 32, 16, 1024),
+                            sdesc_sw128(sb + GST_DSB + ks * 2048, 8192, 1024), ID_KM, ks > 0);
+            mma_commit(bar_a);
+        }
+        {  // the gradient of the state after this chunk, as its bf16 image
+            uint8_t* sv = p.dS_saved + ((size_t)record_slot(n, tc0) * p.H_v + h) * STATE_IMAGE_BYTES;
+#pragma unroll
+            for (int q = 0; q < HN / 8; ++q)
+                if (c_lo + 8 * q < ncols)
+                    *reinterpret_cast<uint4*>(sv + taddr(0, row, col0 + c_lo + 8 * q, 2 * HALF)) =
+                        make_uint4(pack2(G[8 * q], G[8 * q + 1]), pack2(G[8 * q + 2], G[8 * q + 3]),
+                                   pack2(G[8 * q + 4], G[8 * q + 5]),
+                                   pack2(G[8 * q + 6], G[8 * q + 7]));
+        }
+        if (quad >= 2) {  // dDelta, token row row - 64
+            ok = mbar_wait(&bar_o[par], (i >> 1) & 1, abort_flag) && ok;
+            ok = mbar_wait(bar_a, par, abort_flag) && ok;
+            tc_fence_after();
+            float a[HN], o[HN];
+            tmem_row<HN>(tl + GTM_A, a);
+            tmem_row<HN>(tl + GTM_O + 64 * par, o);
+            const float d = rv[64 + row - 64];  // zero past the sequence end
+#pragma unroll
+            for (int j = 0; j < HN; ++j) a[j] = fmaf(d, a[j], o[j]);
+            put_row<HN>(sm, GST_DDEL, row - 64, c_lo, a, 1.f);  // read by ldmatrix only
+        } else if (i + 1 < nchunks) {  // the next chunk's gamma o dO and its dO products
+            ok = gamma_do(i + 1) && ok;
+            bar_sync<GST_BAR_LO, 128>();
+            if (tid == 0) issue_ahead(i + 1);
+        }
+        tc_fence_before();
+        if (!bar_and<GST_BAR, GST_THREADS>(ok)) break;
+
+        // dX = T_b^T dDelta: warp (quad, column half) takes rows 16 quad .. + 15
+        if (warp < 4)
+            dx_half<NT, 0, IO>(sm, sb, st + GST_REC + REC_TB, quad, lane, rv, valid, p, tc0, h, col0,
+                               ncols, GST_DDEL, GST_GDX);
+        else
+            dx_half<NT, 1, IO>(sm, sb, st + GST_REC + REC_TB, quad, lane, rv, valid, p, tc0, h, col0,
+                               ncols, GST_DDEL, GST_GDX);
+        fence_proxy_async_smem();
+        tc_fence_before();
+        if (!bar_and<GST_BAR, GST_THREADS>(ok)) break;
+
+        // K^T (-gamma o dX) on top of Q^T (gamma o dO); dS = gamma_C dS' + both
+        if (tid == 0) {
+            tc_fence_after();
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks)
+                mma_bf16_ss(tmem + GTM_U + 64 * par, sdesc_sw128(st + HALF + ks * 2048, 2 * HALF, 1024),
+                            sdesc_sw128(sb + GST_GDX + ks * 2048, 8192, 1024), ID_MM, true);
+            mma_commit(bar_u);
+        }
+        ok = mbar_wait(bar_u, par, abort_flag);
+        tc_fence_after();
+        {
+            float u[HN];
+            tmem_row<HN>(tl + GTM_U + 64 * par, u);
+#pragma unroll
+            for (int j = 0; j < HN; ++j) G[j] = fmaf(g_C, G[j], u[j]);
+            put_row<HN>(sm, GST_DSB, row, c_lo, G, 1.f);
+            fence_proxy_async_smem();
+        }
+        tc_fence_before();
+        if (!bar_and<GST_BAR, GST_THREADS>(ok)) break;
+        // every product and read of this stage is done: it takes chunk index i + 3
+        if (tid == GST_LOADER && i + GS_STAGES < nchunks) issue(issued++);
+    }
+    if (p.dS0 && !*abort_flag) {
+        float* d0 = p.dS0 + (((size_t)n * p.H_v + h) * D + row) * D + col0 + c_lo;
+#pragma unroll
+        for (int j = 0; j < HN / 4; ++j)
+            if (c_lo + 4 * j < ncols)
+                reinterpret_cast<float4*>(d0)[j] =
+                    make_float4(G[4 * j], G[4 * j + 1], G[4 * j + 2], G[4 * j + 3]);
+    }
+    // Drain: no product may still run and no copy still land when TMEM is freed
+    // and the CTA exits (both waits bounded).
+    if (tid == 0) {
+        mma_commit(drain_bar);
+        mbar_wait_drain(drain_bar, 0);
+    }
+    if (tid == GST_LOADER)
+        for (int i = max(0, issued - GS_STAGES); i < issued; ++i)
+            mbar_wait_drain(&bars[i % GS_STAGES], (i / GS_STAGES) & 1);
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, GTM_COLS);
+    }
+}
+
+template <int NS, typename IO>
+cudaError_t launch_grad_state_tc(const CUtensorMap& mq, const CUtensorMap& mk,
+                                 const CUtensorMap& mo, const GradParams& prm, cudaStream_t stream) {
+    auto kern = grad_state_tc_kernel<NS, IO>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, GST_SMEM);
+    if (e != cudaSuccess) return e;
+    kern<<<dim3((D + NS - 1) / NS, prm.H_v, prm.N), GST_THREADS, GST_SMEM, stream>>>(mq, mk, mo, prm);
+    return cudaGetLastError();
 }
 
 template <int NS, typename IO>
@@ -1102,8 +1413,9 @@ template <typename IO>
 cudaError_t launch_grads(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                          const CUtensorMap& mo, const GradParams& prm, long long units, int sms,
                          size_t slots, cudaStream_t stream) {
+    // (at 48-column slices on tcgen05, as the forward chain)
     cudaError_t e = units * 4 <= sms ? launch_grad_state<32, IO>(mq, mk, mo, prm, stream)
-                    : units * 3 <= sms ? launch_grad_state<48, IO>(mq, mk, mo, prm, stream)
+                    : units * 3 <= sms ? launch_grad_state_tc<48, IO>(mq, mk, mo, prm, stream)
                                        : launch_grad_state<64, IO>(mq, mk, mo, prm, stream);
     if (e != cudaSuccess) return e;
     e = cudaFuncSetAttribute(grad_chunk_tc_kernel<IO>, cudaFuncAttributeMaxDynamicSharedMemorySize,
