@@ -498,27 +498,33 @@ __global__ void __launch_bounds__(GST_THREADS, 1)
         fence_proxy_async_smem();
         return landed;
     };
-    // (thread 0) the products of chunk index i that read only dO: Q^T (gamma o dO)
-    // into U[i & 1], [T_b^T; (M o QK^T)^T] dO into O[i & 1]
-    auto issue_ahead = [&](int i) {
+    // (thread 0) the products of chunk index i that read only dO:
+    // [T_b^T; (M o QK^T)^T] dO into O[i & 1], and Q^T (gamma o dO) into U[i & 1]
+    auto issue_mdo = [&](int i) {
         const uint32_t st = sb + (i % GS_STAGES) * GST_STAGE;
         tc_fence_after();
-#pragma unroll
-        for (int ks = 0; ks < 4; ++ks)
-            mma_bf16_ss(tmem + GTM_U + 64 * (i & 1), sdesc_sw128(st + ks * 2048, 2 * HALF, 1024),
-                        sdesc_sw128(sb + GST_GDO + (i & 1) * HALF + ks * 2048, 8192, 1024), ID_MM,
-                        ks > 0);
 #pragma unroll
         for (int ks = 0; ks < 4; ++ks)
             mma_bf16_ss(tmem + GTM_O + 64 * (i & 1), sdesc_sw128(st + GST_REC + ks * 2048, HALF, 1024),
                         sdesc_sw128(st + GST_O + ks * 2048, 8192, 1024), ID_MM, ks > 0);
         mma_commit(&bar_o[i & 1]);
     };
+    auto issue_qdo = [&](int i) {
+        const uint32_t st = sb + (i % GS_STAGES) * GST_STAGE;
+#pragma unroll
+        for (int ks = 0; ks < 4; ++ks)
+            mma_bf16_ss(tmem + GTM_U + 64 * (i & 1), sdesc_sw128(st + ks * 2048, 2 * HALF, 1024),
+                        sdesc_sw128(sb + GST_GDO + (i & 1) * HALF + ks * 2048, 8192, 1024), ID_MM,
+                        ks > 0);
+    };
     bool ok = true;
     if (quad < 2 && nchunks > 0) {
         ok = gamma_do(0);
         bar_sync<GST_BAR_LO, 128>();
-        if (tid == 0) issue_ahead(0);
+        if (tid == 0) {
+            issue_mdo(0);
+            issue_qdo(0);
+        }
     }
     __syncthreads();  // the first [Q; K] dS' reads the whole dS' tile
 
@@ -562,10 +568,10 @@ __global__ void __launch_bounds__(GST_THREADS, 1)
 #pragma unroll
             for (int j = 0; j < HN; ++j) a[j] = fmaf(d, a[j], o[j]);
             put_row<HN>(sm, GST_DDEL, row - 64, c_lo, a, 1.f);  // read by ldmatrix only
-        } else if (i + 1 < nchunks) {  // the next chunk's gamma o dO and its dO products
+        } else if (i + 1 < nchunks) {  // the next chunk's gamma o dO and (M o QK^T)^T dO
             ok = gamma_do(i + 1) && ok;
             bar_sync<GST_BAR_LO, 128>();
-            if (tid == 0) issue_ahead(i + 1);
+            if (tid == 0) issue_mdo(i + 1);
         }
         tc_fence_before();
         if (!bar_and<GST_BAR, GST_THREADS>(ok)) break;
@@ -589,6 +595,8 @@ __global__ void __launch_bounds__(GST_THREADS, 1)
                 mma_bf16_ss(tmem + GTM_U + 64 * par, sdesc_sw128(st + HALF + ks * 2048, 2 * HALF, 1024),
                             sdesc_sw128(sb + GST_GDX + ks * 2048, 8192, 1024), ID_MM, true);
             mma_commit(bar_u);
+            // the next chunk's Q^T (gamma o dO) runs while this dS is updated
+            if (i + 1 < nchunks) issue_qdo(i + 1);
         }
         ok = mbar_wait(bar_u, par, abort_flag);
         tc_fence_after();
