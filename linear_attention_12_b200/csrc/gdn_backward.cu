@@ -345,13 +345,23 @@ __device__ __forceinline__ float tile_dot(const uint8_t* a, const uint8_t* b, in
 //                              accumulator (lane = d_k index)
 // The products that read only dO (the second, and Q^T (gamma o dO)) are issued
 // a chunk ahead, once the warps on lanes 0-63 have formed gamma o dO; only
-// [Q; K] dS' and K^T (-gamma o dX) sit on the chain.  Every thread keeps half a
-// row of dS in fp32, writes its bf16 copy (the next [Q; K] dS' operand) and,
-// per chunk, its part of the bf16 image of dS' for the per-chunk gradients.
+// [Q; K] dS' and K^T (-gamma o dX) sit on the chain.  Every thread of the eight
+// compute warps keeps half a row of dS in fp32, writes its bf16 copy (the next
+// [Q; K] dS' operand) and, per chunk, its part of the bf16 image of dS' for the
+// per-chunk gradients.  A ninth warp only issues the products (tcgen05.mma
+// issue stalls while the pipe is busy, which held a compute warp back): the
+// compute warps bar.arrive on a named barrier once an operand tile is written,
+// and the issuer bar.syncs on it.  The compute warps leave the chunk loop only
+// at its end, after their last arrive, so that the issuer's barriers always
+// complete; the issuer reads the abort flag after each chunk's last one.
 // ============================================================================
-constexpr int GST_THREADS = 256;
-constexpr int GST_LOADER = 192;           // warp 6
-constexpr int GST_BAR = 1, GST_BAR_LO = 2;  // all warps; the warps on TMEM lanes 0-63
+constexpr int GST_THREADS = 288;  // eight compute warps and the issuing warp
+constexpr int GST_COMPUTE = 256;  // warps 0-7; warp 8's lane 0 issues
+constexpr int GST_LOADER = 192;   // warp 6
+// named barriers: the compute warps; gamma o dO ready (the warps on TMEM lanes
+// 0-63 arrive, the issuer waits); -gamma o dX ready; dS' ready (compute warps
+// arrive, the issuer waits)
+constexpr int GST_BAR = 1, GST_BAR_GDO = 2, GST_BAR_GDX = 3, GST_BAR_DSB = 4;
 constexpr uint32_t GST_O = 4 * HALF, GST_REC = 5 * HALF;
 constexpr uint32_t GST_STAGE = ((GST_REC + REC_BYTES + 1023) / 1024) * 1024;
 constexpr uint32_t GST_TX = 5 * HALF + REC_BYTES;
@@ -419,9 +429,10 @@ __global__ void __launch_bounds__(GST_THREADS, 1)
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + GST_MISC + 4);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int quad = warp & 3;          // TMEM lanes 32 quad .. + 31
-    const int c_lo = (warp >> 2) * HN;  // this warp's half of the slice's columns
-    const int row = 32 * quad + lane;   // my row of an M = 128 product (a d_k index)
+    const bool issuer = tid >= GST_COMPUTE;  // warp 8
+    const int quad = warp & 3;               // TMEM lanes 32 quad .. + 31
+    const int c_lo = ((warp >> 2) & 1) * HN; // this warp's half of the slice's columns
+    const int row = 32 * quad + lane;        // my row of an M = 128 product (a d_k index)
     const int h = blockIdx.y, n = blockIdx.z;
     const int hq = h / (p.H_v / p.H_qk);
     const int col0 = blockIdx.x * NS;
@@ -463,16 +474,6 @@ __global__ void __launch_bounds__(GST_THREADS, 1)
     if (tid == GST_LOADER)
         for (; issued < min(GS_STAGES, nchunks); ++issued) issue(issued);
 
-    // dS: row `row`, columns col0 + c_lo .. + HN - 1, fp32 (dS_final to start)
-    float G[HN];
-    {
-        const float* s0 =
-            p.dS_final ? p.dS_final + (((size_t)n * p.H_v + h) * D + row) * D + col0 + c_lo : nullptr;
-#pragma unroll
-        for (int j = 0; j < HN; ++j) G[j] = (s0 && c_lo + j < ncols) ? s0[j] : 0.f;
-        put_row<HN>(sm, GST_DSB, row, c_lo, G, 1.f);
-        fence_proxy_async_smem();
-    }
     // gamma o dO of chunk index i into GDO[i & 1] (warps on lanes 0-63: token row
     // `row`; zero past the sequence end, where the rows belong to the next one)
     auto gamma_do = [&](int i) -> bool {
@@ -498,138 +499,179 @@ __global__ void __launch_bounds__(GST_THREADS, 1)
         fence_proxy_async_smem();
         return landed;
     };
-    // (thread 0) the products of chunk index i that read only dO:
-    // [T_b^T; (M o QK^T)^T] dO into O[i & 1], and Q^T (gamma o dO) into U[i & 1]
-    auto issue_mdo = [&](int i) {
-        const uint32_t st = sb + (i % GS_STAGES) * GST_STAGE;
-        tc_fence_after();
+
+    if (issuer) {
+        // ---- the issuing warp: lane 0 issues, the warp takes the barriers
+        const bool lead = lane == 0;
+        // (lead) the products of chunk index i that read only dO:
+        // [T_b^T; (M o QK^T)^T] dO into O[i & 1], and Q^T (gamma o dO) into U[i & 1]
+        auto issue_mdo = [&](int i) {
+            const uint32_t st = sb + (i % GS_STAGES) * GST_STAGE;
 #pragma unroll
-        for (int ks = 0; ks < 4; ++ks)
-            mma_bf16_ss(tmem + GTM_O + 64 * (i & 1), sdesc_sw128(st + GST_REC + ks * 2048, HALF, 1024),
-                        sdesc_sw128(st + GST_O + ks * 2048, 8192, 1024), ID_MM, ks > 0);
-        mma_commit(&bar_o[i & 1]);
-    };
-    auto issue_qdo = [&](int i) {
-        const uint32_t st = sb + (i % GS_STAGES) * GST_STAGE;
+            for (int ks = 0; ks < 4; ++ks)
+                mma_bf16_ss(tmem + GTM_O + 64 * (i & 1),
+                            sdesc_sw128(st + GST_REC + ks * 2048, HALF, 1024),
+                            sdesc_sw128(st + GST_O + ks * 2048, 8192, 1024), ID_MM, ks > 0);
+            mma_commit(&bar_o[i & 1]);
+        };
+        auto issue_qdo = [&](int i) {
+            const uint32_t st = sb + (i % GS_STAGES) * GST_STAGE;
 #pragma unroll
-        for (int ks = 0; ks < 4; ++ks)
-            mma_bf16_ss(tmem + GTM_U + 64 * (i & 1), sdesc_sw128(st + ks * 2048, 2 * HALF, 1024),
-                        sdesc_sw128(sb + GST_GDO + (i & 1) * HALF + ks * 2048, 8192, 1024), ID_MM,
-                        ks > 0);
-    };
-    bool ok = true;
-    if (quad < 2 && nchunks > 0) {
-        ok = gamma_do(0);
-        bar_sync<GST_BAR_LO, 128>();
-        if (tid == 0) {
+            for (int ks = 0; ks < 4; ++ks)
+                mma_bf16_ss(tmem + GTM_U + 64 * (i & 1), sdesc_sw128(st + ks * 2048, 2 * HALF, 1024),
+                            sdesc_sw128(sb + GST_GDO + (i & 1) * HALF + ks * 2048, 8192, 1024),
+                            ID_MM, ks > 0);
+        };
+        __syncthreads();  // the first dS' tile and gamma o dO are written
+        if (nchunks > 0 && lead) {
+            tc_fence_after();
             issue_mdo(0);
             issue_qdo(0);
         }
-    }
-    __syncthreads();  // the first [Q; K] dS' reads the whole dS' tile
-
-    for (int i = 0; i < nchunks; ++i) {
-        const int c = nchunks - 1 - i, s = i % GS_STAGES;
-        const uint32_t st = sb + s * GST_STAGE;
-        const uint8_t* stp = sm + s * GST_STAGE;
-        const uint32_t par = i & 1;
-        const float* rv = reinterpret_cast<const float*>(stp + GST_REC + REC_VEC);
-        const int tc0 = t_beg + c * C;
-        const int valid = min(C, t_end - tc0);
-        ok = mbar_wait(&bars[s], (i / GS_STAGES) & 1, abort_flag) && ok;
-        const float g_C = rv[128];
-        if (tid == 0) {  // [Q; K] dS'
-            tc_fence_after();
+        bool stopped = false;
+        for (int i = 0; i < nchunks; ++i) {
+            const int s = i % GS_STAGES;
+            const uint32_t st = sb + s * GST_STAGE;
+            const uint32_t par = i & 1;
+            if (i > 0) {
+                bar_sync<GST_BAR_DSB, GST_THREADS>();  // the compute warps wrote dS'
+                if (*abort_flag) {  // they left the loop after that arrive
+                    stopped = true;
+                    break;
+                }
+            }
+            const bool landed = mbar_wait(&bars[s], (i / GS_STAGES) & 1, abort_flag);
+            if (lead && landed) {  // [Q; K] dS'
+                tc_fence_after();
 #pragma unroll
-            for (int ks = 0; ks < 8; ++ks)
-                mma_bf16_ss(tmem + GTM_A,
-                            sdesc_sw128(st + (ks >> 2) * 2 * HALF + (ks & 3) * 32, 16, 1024),
-                            sdesc_sw128(sb + GST_DSB + ks * 2048, 8192, 1024), ID_KM, ks > 0);
-            mma_commit(bar_a);
-        }
-        {  // the gradient of the state after this chunk, as its bf16 image
-            uint8_t* sv = p.dS_saved + ((size_t)record_slot(n, tc0) * p.H_v + h) * STATE_IMAGE_BYTES;
+                for (int ks = 0; ks < 8; ++ks)
+                    mma_bf16_ss(tmem + GTM_A,
+                                sdesc_sw128(st + (ks >> 2) * 2 * HALF + (ks & 3) * 32, 16, 1024),
+                                sdesc_sw128(sb + GST_DSB + ks * 2048, 8192, 1024), ID_KM, ks > 0);
+                mma_commit(bar_a);
+            }
+            if (i + 1 < nchunks) {  // the next chunk's (M o QK^T)^T dO, once gamma o dO is formed
+                bar_sync<GST_BAR_GDO, 160>();
+                if (lead) {
+                    tc_fence_after();
+                    issue_mdo(i + 1);
+                }
+            }
+            bar_sync<GST_BAR_GDX, GST_THREADS>();  // -gamma o dX is written
+            if (lead) {  // K^T (-gamma o dX) on top of Q^T (gamma o dO), then the next Q^T (gamma o dO)
+                tc_fence_after();
 #pragma unroll
-            for (int q = 0; q < HN / 8; ++q)
-                if (c_lo + 8 * q < ncols)
-                    *reinterpret_cast<uint4*>(sv + taddr(0, row, col0 + c_lo + 8 * q, 2 * HALF)) =
-                        make_uint4(pack2(G[8 * q], G[8 * q + 1]), pack2(G[8 * q + 2], G[8 * q + 3]),
-                                   pack2(G[8 * q + 4], G[8 * q + 5]),
-                                   pack2(G[8 * q + 6], G[8 * q + 7]));
+                for (int ks = 0; ks < 4; ++ks)
+                    mma_bf16_ss(tmem + GTM_U + 64 * par,
+                                sdesc_sw128(st + HALF + ks * 2048, 2 * HALF, 1024),
+                                sdesc_sw128(sb + GST_GDX + ks * 2048, 8192, 1024), ID_MM, true);
+                mma_commit(bar_u);
+                if (i + 1 < nchunks) issue_qdo(i + 1);
+            }
         }
-        if (quad >= 2) {  // dDelta, token row row - 64
-            ok = mbar_wait(&bar_o[par], (i >> 1) & 1, abort_flag) && ok;
-            ok = mbar_wait(bar_a, par, abort_flag) && ok;
-            tc_fence_after();
-            float a[HN], o[HN];
-            tmem_row<HN>(tl + GTM_A, a);
-            tmem_row<HN>(tl + GTM_O + 64 * par, o);
-            const float d = rv[64 + row - 64];  // zero past the sequence end
-#pragma unroll
-            for (int j = 0; j < HN; ++j) a[j] = fmaf(d, a[j], o[j]);
-            put_row<HN>(sm, GST_DDEL, row - 64, c_lo, a, 1.f);  // read by ldmatrix only
-        } else if (i + 1 < nchunks) {  // the next chunk's gamma o dO and (M o QK^T)^T dO
-            ok = gamma_do(i + 1) && ok;
-            bar_sync<GST_BAR_LO, 128>();
-            if (tid == 0) issue_mdo(i + 1);
+        // the compute warps' arrive after the last chunk
+        if (nchunks > 0 && !stopped) bar_sync<GST_BAR_DSB, GST_THREADS>();
+        if (lead) {  // no product may still run when TMEM is freed (bounded wait)
+            mma_commit(drain_bar);
+            mbar_wait_drain(drain_bar, 0);
         }
-        tc_fence_before();
-        if (!bar_and<GST_BAR, GST_THREADS>(ok)) break;
-
-        // dX = T_b^T dDelta: warp (quad, column half) takes rows 16 quad .. + 15
-        if (warp < 4)
-            dx_half<NT, 0, IO>(sm, sb, st + GST_REC + REC_TB, quad, lane, rv, valid, p, tc0, h, col0,
-                               ncols, GST_DDEL, GST_GDX);
-        else
-            dx_half<NT, 1, IO>(sm, sb, st + GST_REC + REC_TB, quad, lane, rv, valid, p, tc0, h, col0,
-                               ncols, GST_DDEL, GST_GDX);
-        fence_proxy_async_smem();
-        tc_fence_before();
-        if (!bar_and<GST_BAR, GST_THREADS>(ok)) break;
-
-        // K^T (-gamma o dX) on top of Q^T (gamma o dO); dS = gamma_C dS' + both
-        if (tid == 0) {
-            tc_fence_after();
-#pragma unroll
-            for (int ks = 0; ks < 4; ++ks)
-                mma_bf16_ss(tmem + GTM_U + 64 * par, sdesc_sw128(st + HALF + ks * 2048, 2 * HALF, 1024),
-                            sdesc_sw128(sb + GST_GDX + ks * 2048, 8192, 1024), ID_MM, true);
-            mma_commit(bar_u);
-            // the next chunk's Q^T (gamma o dO) runs while this dS is updated
-            if (i + 1 < nchunks) issue_qdo(i + 1);
-        }
-        ok = mbar_wait(bar_u, par, abort_flag);
-        tc_fence_after();
+    } else {
+        // ---- the compute warps
+        // dS: row `row`, columns col0 + c_lo .. + HN - 1, fp32 (dS_final to start)
+        float G[HN];
         {
-            float u[HN];
-            tmem_row<HN>(tl + GTM_U + 64 * par, u);
+            const float* s0 = p.dS_final
+                                  ? p.dS_final + (((size_t)n * p.H_v + h) * D + row) * D + col0 + c_lo
+                                  : nullptr;
 #pragma unroll
-            for (int j = 0; j < HN; ++j) G[j] = fmaf(g_C, G[j], u[j]);
+            for (int j = 0; j < HN; ++j) G[j] = (s0 && c_lo + j < ncols) ? s0[j] : 0.f;
             put_row<HN>(sm, GST_DSB, row, c_lo, G, 1.f);
             fence_proxy_async_smem();
         }
+        bool ok = true;
+        if (quad < 2 && nchunks > 0) ok = gamma_do(0);
         tc_fence_before();
-        if (!bar_and<GST_BAR, GST_THREADS>(ok)) break;
-        // every product and read of this stage is done: it takes chunk index i + 3
-        if (tid == GST_LOADER && i + GS_STAGES < nchunks) issue(issued++);
-    }
-    if (p.dS0 && !*abort_flag) {
-        float* d0 = p.dS0 + (((size_t)n * p.H_v + h) * D + row) * D + col0 + c_lo;
+        __syncthreads();  // the issuer starts
+
+        for (int i = 0; i < nchunks; ++i) {
+            const int c = nchunks - 1 - i, s = i % GS_STAGES;
+            const uint32_t st = sb + s * GST_STAGE;
+            const uint8_t* stp = sm + s * GST_STAGE;
+            const uint32_t par = i & 1;
+            const float* rv = reinterpret_cast<const float*>(stp + GST_REC + REC_VEC);
+            const int tc0 = t_beg + c * C;
+            const int valid = min(C, t_end - tc0);
+            ok = mbar_wait(&bars[s], (i / GS_STAGES) & 1, abort_flag) && ok;
+            const float g_C = rv[128];
+            {  // the gradient of the state after this chunk, as its bf16 image
+                uint8_t* sv =
+                    p.dS_saved + ((size_t)record_slot(n, tc0) * p.H_v + h) * STATE_IMAGE_BYTES;
 #pragma unroll
-        for (int j = 0; j < HN / 4; ++j)
-            if (c_lo + 4 * j < ncols)
-                reinterpret_cast<float4*>(d0)[j] =
-                    make_float4(G[4 * j], G[4 * j + 1], G[4 * j + 2], G[4 * j + 3]);
+                for (int q = 0; q < HN / 8; ++q)
+                    if (c_lo + 8 * q < ncols)
+                        *reinterpret_cast<uint4*>(sv + taddr(0, row, col0 + c_lo + 8 * q, 2 * HALF)) =
+                            make_uint4(pack2(G[8 * q], G[8 * q + 1]), pack2(G[8 * q + 2], G[8 * q + 3]),
+                                       pack2(G[8 * q + 4], G[8 * q + 5]),
+                                       pack2(G[8 * q + 6], G[8 * q + 7]));
+            }
+            if (quad >= 2) {  // dDelta, token row row - 64
+                ok = mbar_wait(&bar_o[par], (i >> 1) & 1, abort_flag) && ok;
+                ok = mbar_wait(bar_a, par, abort_flag) && ok;
+                tc_fence_after();
+                float a[HN], o[HN];
+                tmem_row<HN>(tl + GTM_A, a);
+                tmem_row<HN>(tl + GTM_O + 64 * par, o);
+                const float d = rv[64 + row - 64];  // zero past the sequence end
+#pragma unroll
+                for (int j = 0; j < HN; ++j) a[j] = fmaf(d, a[j], o[j]);
+                put_row<HN>(sm, GST_DDEL, row - 64, c_lo, a, 1.f);  // read by ldmatrix only
+                tc_fence_before();
+            } else if (i + 1 < nchunks) {  // the next chunk's gamma o dO, for the issuer
+                ok = gamma_do(i + 1) && ok;
+                bar_arrive<GST_BAR_GDO, 160>();
+            }
+            bar_sync<GST_BAR, GST_COMPUTE>();  // dDelta is complete
+
+            // dX = T_b^T dDelta: warp (quad, column half) takes rows 16 quad .. + 15
+            if (warp < 4)
+                dx_half<NT, 0, IO>(sm, sb, st + GST_REC + REC_TB, quad, lane, rv, valid, p, tc0, h,
+                                   col0, ncols, GST_DDEL, GST_GDX);
+            else
+                dx_half<NT, 1, IO>(sm, sb, st + GST_REC + REC_TB, quad, lane, rv, valid, p, tc0, h,
+                                   col0, ncols, GST_DDEL, GST_GDX);
+            fence_proxy_async_smem();
+            bar_arrive<GST_BAR_GDX, GST_THREADS>();
+
+            // dS = gamma_C dS' + Q^T (gamma o dO) + K^T (-gamma o dX)
+            ok = mbar_wait(bar_u, par, abort_flag) && ok;
+            tc_fence_after();
+            {
+                float u[HN];
+                tmem_row<HN>(tl + GTM_U + 64 * par, u);
+#pragma unroll
+                for (int j = 0; j < HN; ++j) G[j] = fmaf(g_C, G[j], u[j]);
+                put_row<HN>(sm, GST_DSB, row, c_lo, G, 1.f);
+                fence_proxy_async_smem();
+            }
+            tc_fence_before();
+            bar_arrive<GST_BAR_DSB, GST_THREADS>();
+            // every product and read of this stage is done: it takes chunk index i + 3
+            // (the compute warps leave the loop only here, after their last arrive)
+            if (!bar_and<GST_BAR, GST_COMPUTE>(ok)) break;
+            if (tid == GST_LOADER && i + GS_STAGES < nchunks) issue(issued++);
+        }
+        if (p.dS0 && !*abort_flag) {
+            float* d0 = p.dS0 + (((size_t)n * p.H_v + h) * D + row) * D + col0 + c_lo;
+#pragma unroll
+            for (int j = 0; j < HN / 4; ++j)
+                if (c_lo + 4 * j < ncols)
+                    reinterpret_cast<float4*>(d0)[j] =
+                        make_float4(G[4 * j], G[4 * j + 1], G[4 * j + 2], G[4 * j + 3]);
+        }
+        if (tid == GST_LOADER)
+            for (int i = max(0, issued - GS_STAGES); i < issued; ++i)
+                mbar_wait_drain(&bars[i % GS_STAGES], (i / GS_STAGES) & 1);
     }
-    // Drain: no product may still run and no copy still land when TMEM is freed
-    // and the CTA exits (both waits bounded).
-    if (tid == 0) {
-        mma_commit(drain_bar);
-        mbar_wait_drain(drain_bar, 0);
-    }
-    if (tid == GST_LOADER)
-        for (int i = max(0, issued - GS_STAGES); i < issued; ++i)
-            mbar_wait_drain(&bars[i % GS_STAGES], (i / GS_STAGES) & 1);
     tc_fence_before();
     __syncthreads();
     if (warp == 0) {

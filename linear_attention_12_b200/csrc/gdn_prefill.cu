@@ -135,10 +135,6 @@ constexpr int CO_BAR_SOLVE = 1;  // the two solver warps
 constexpr int CO_BAR_TDONE = 2;  // solvers -> writers: T is complete
 constexpr int CO_BAR_TFREE = 3;  // writers -> solvers: T has been read
 
-template <int ID, int N>
-__device__ __forceinline__ void bar_arrive() {
-    asm volatile("bar.arrive %0, %1;" ::"n"(ID), "n"(N) : "memory");
-}
 
 // Two values as a packed pair of the chunk-operator records' tile type: fp16
 // (F16) for the unsplit prefill's output passes, whose products T_b X and

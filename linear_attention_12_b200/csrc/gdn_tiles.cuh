@@ -49,6 +49,12 @@ template <int ID, int N>
 __device__ __forceinline__ void bar_sync() {
     asm volatile("bar.sync %0, %1;" ::"n"(ID), "n"(N) : "memory");
 }
+// Arrive on a named barrier without waiting (producers of a producer/consumer
+// hand-off; the consumers bar_sync on the same barrier and count).
+template <int ID, int N>
+__device__ __forceinline__ void bar_arrive() {
+    asm volatile("bar.arrive %0, %1;" ::"n"(ID), "n"(N) : "memory");
+}
 // Named barrier that also returns the AND of every participant's `ok`.
 template <int ID, int N>
 __device__ __forceinline__ bool bar_and(bool ok) {
