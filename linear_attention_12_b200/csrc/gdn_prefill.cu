@@ -980,11 +980,19 @@ __global__ void __launch_bounds__(P2_THREADS, 1)
 // and [T_b; M_Q] Delta are double-buffered in TMEM).  Every product commits
 // to an mbarrier of its own, once per chunk.  Warp 6's thread 0 streams K, Q,
 // the V slice and the record into a 3-stage ring; it refills the previous
-// chunk's stage while X is formed.
+// chunk's stage while X is formed.  A ninth warp only issues the products
+// (tcgen05.mma issue stalls while the pipe is busy, which held a compute warp
+// back): it waits on named barriers that the compute warps bar.arrive on once
+// d o Delta and the bf16 S are written.  The compute warps leave the chunk loop
+// only at its end, after their last arrive, and the issuer reads the abort flag
+// after each chunk's first wait, so that every barrier completes.
 // ============================================================================
-constexpr int TC_THREADS = 256;
-constexpr int TC_LOADER = 192;  // warp 6: idle while warps 0, 1, 4, 5 form X
-constexpr int BAR_TC = 1;
+constexpr int TC_THREADS = 288;  // eight compute warps and the issuing warp
+constexpr int TC_COMPUTE = 256;  // warps 0-7; warp 8's lane 0 issues every product
+constexpr int TC_LOADER = 192;   // warp 6: idle while warps 0, 1, 4, 5 form X
+// named barriers: the compute warps; Delta and d o Delta written, S written
+// (compute warps arrive, the issuing warp waits)
+constexpr int BAR_TC = 1, BAR_TC_DD = 2, BAR_TC_SB = 3;
 // ring stage: K h0 | Q h0 | K h1 | Q h1 -- [K; Q] is one 128-row K-major tile
 // per 64-column half, and K alone an MN-major one with its halves 16 KB apart --
 // then the V slice and the record (T_b, then M o Q K^T)
@@ -1084,7 +1092,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int quad = warp & 3;          // TMEM lanes 32 quad .. 32 quad + 31
-    const int c_lo = (warp >> 2) * HN;  // this warp's half of the slice's columns
+    const bool issuer = tid >= TC_COMPUTE;       // warp 8
+    const int c_lo = ((warp >> 2) & 1) * HN;  // this warp's half of the slice's columns
     const int row = 32 * quad + lane;   // my row of an M = 128 product (a state row)
     const int h = blockIdx.y, n = blockIdx.z;
     const int hq = h / (p.H_v / p.H_qk);
@@ -1142,7 +1151,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
                                pack2(Sr[8 * i + 4], Sr[8 * i + 5]),
                                pack2(Sr[8 * i + 6], Sr[8 * i + 7]));
     };
-    {
+    if (!issuer) {
         const float* s0 =
             p.S0 ? p.S0 + (((size_t)n * p.H_v + h) * D + row) * D + col0 + c_lo : nullptr;
 #pragma unroll
@@ -1177,6 +1186,57 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         return ok;
     };
 
+    if (issuer) {
+        // ---- the issuing warp: lane 0 issues, the warp takes the barriers
+        const bool lead = lane == 0;
+        bool stopped = false;
+        for (int c = 0; c < nchunks; ++c) {
+            const int s = c % NSTAGE;
+            const uint32_t st = sb + s * TS_STAGE;
+            const uint32_t par = c & 1;
+            if (c > 0) {
+                bar_sync<BAR_TC_SB, TC_THREADS>();  // the previous chunk's S is written
+                if (*abort_flag) {  // the compute warps left the loop after that arrive
+                    stopped = true;
+                    break;
+                }
+            }
+            const bool landed = mbar_wait(&bars[s], (c / NSTAGE) & 1, abort_flag);
+            if (lead && landed) {  // [K; Q] S
+                tc_fence_after();
+#pragma unroll
+                for (int ks = 0; ks < 8; ++ks)
+                    mma_bf16_ss(tmem + TM_KQ + 64 * par,
+                                sdesc_sw128(st + TS_KQ + (ks >> 2) * 2 * HALF + (ks & 3) * 32, 16, 1024),
+                                sdesc_sw128(sb + TC_SB + ks * 2048, 8192, 1024), ID_128, ks > 0);
+                mma_commit(bar_ks);
+            }
+            bar_sync<BAR_TC_DD, TC_THREADS>();  // Delta and d o Delta are written
+            if (lead) {  // K^T (d o Delta), then [T_b; M_Q] Delta
+                tc_fence_after();
+#pragma unroll
+                for (int ks = 0; ks < 4; ++ks)
+                    mma_bf16_ss(tmem + TM_U, sdesc_sw128(st + TS_KQ + ks * 2048, 2 * HALF, 1024),
+                                sdesc_sw128(sb + TC_DD + ks * 2048, 8192, 1024), ID_KT, ks > 0);
+                mma_commit(bar_u);
+                if constexpr (OUTS) {
+#pragma unroll
+                    for (int ks = 0; ks < 4; ++ks)
+                        mma_bf16_ss(tmem + TM_O + 64 * par,
+                                    sdesc_sw128(st + TS_REC + ks * 32, 16, 1024),
+                                    sdesc_sw128(sb + TC_DU + ks * 2048, 8192, 1024), ID_R128, ks > 0);
+                    mma_commit(bar_o);
+                }
+            }
+        }
+        // the compute warps' arrive after the last chunk
+        if (nchunks > 0 && !stopped) bar_sync<BAR_TC_SB, TC_THREADS>();
+        if (lead) {  // no product may still run when TMEM is freed (bounded wait)
+            mma_commit(drain_bar);
+            mbar_wait_drain(drain_bar, 0);
+        }
+    } else {
+    // ---- the compute warps
     float g_prev = 0.f;  // gamma of my output row in the previous chunk
     bool ok = true;
     for (int c = 0; c < nchunks; ++c) {
@@ -1185,19 +1245,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         const uint8_t* stp = sm + s * TS_STAGE;
         const uint32_t par = c & 1;
         ok = mbar_wait(&bars[s], (c / NSTAGE) & 1, abort_flag);
-        // [K; Q] S (the S tile and every read of the TMEM region it overwrites
-        // were ordered by the previous chunk's last barrier)
-        if (tid == 0) {
-            tc_fence_after();
-#pragma unroll
-            for (int ks = 0; ks < 8; ++ks)
-                mma_bf16_ss(tmem + TM_KQ + 64 * par,
-                            sdesc_sw128(st + TS_KQ + (ks >> 2) * 2 * HALF + (ks & 3) * 32, 16, 1024),
-                            sdesc_sw128(sb + TC_SB + ks * 2048, 8192, 1024), ID_128, ks > 0);
-            mma_commit(bar_ks);
-        }
-        // meanwhile: this chunk's scalars come into registers; the previous chunk's
-        // outputs
+        // (the issuing warp starts [K; Q] S); this chunk's scalars come into
+        // registers; the previous chunk's outputs
         const float* rv = reinterpret_cast<const float*>(stp + TS_REC + REC_VEC);
         const float g_row = rv[row & 63];         // gamma of my K row (quads 0-1) or Q row (2-3)
         const float g_C = rv[128];
@@ -1230,7 +1279,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
             }
         }
         tc_fence_before();
-        if (!bar_and<BAR_TC, TC_THREADS>(ok)) break;
+        bar_sync<BAR_TC, TC_COMPUTE>();  // X is complete
 
         // Delta = T_b X on mma.sync: warp (quad, column half) takes rows 16 quad ..
         // + 15 of its half, so no commit, wake-up or TMEM read sits on the chain;
@@ -1246,26 +1295,9 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
                                            dhi, TC_DU, TC_DD);
             fence_proxy_async_smem();
         }
-        tc_fence_before();
-        if (!bar_and<BAR_TC, TC_THREADS>(ok)) break;
+        bar_arrive<BAR_TC_DD, TC_THREADS>();
 
-        // K^T (d o Delta), then [T_b; M_Q] Delta
-        if (tid == 0) {
-            tc_fence_after();
-#pragma unroll
-            for (int ks = 0; ks < 4; ++ks)
-                mma_bf16_ss(tmem + TM_U, sdesc_sw128(st + TS_KQ + ks * 2048, 2 * HALF, 1024),
-                            sdesc_sw128(sb + TC_DD + ks * 2048, 8192, 1024), ID_KT, ks > 0);
-            mma_commit(bar_u);
-            if constexpr (OUTS) {
-#pragma unroll
-                for (int ks = 0; ks < 4; ++ks)
-                    mma_bf16_ss(tmem + TM_O + 64 * par, sdesc_sw128(st + TS_REC + ks * 32, 16, 1024),
-                                sdesc_sw128(sb + TC_DU + ks * 2048, 8192, 1024), ID_R128, ks > 0);
-                mma_commit(bar_o);
-            }
-        }
-        ok = mbar_wait(bar_u, par, abort_flag);
+        ok = mbar_wait(bar_u, par, abort_flag) && ok;
         tc_fence_after();
         {  // S <- gamma_C S + K^T (d o Delta), state row `row`; bf16 copy for K S and Q S
             float u[HN];
@@ -1277,7 +1309,9 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
             save_image(c + 1);
         }
         tc_fence_before();
-        if (!bar_and<BAR_TC, TC_THREADS>(ok)) break;
+        bar_arrive<BAR_TC_SB, TC_THREADS>();
+        // (the compute warps leave the loop only here, after their last arrive)
+        if (!bar_and<BAR_TC, TC_COMPUTE>(ok)) break;
     }
     if (OUTS && nchunks > 0 && !*abort_flag && quad >= 2) {  // the last chunk's outputs
         output(nchunks - 1, g_prev);
@@ -1291,15 +1325,11 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
                 reinterpret_cast<float4*>(sf)[j] =
                     make_float4(Sr[4 * j], Sr[4 * j + 1], Sr[4 * j + 2], Sr[4 * j + 3]);
     }
-    // Drain: no product may still run and no copy still land when TMEM is freed
-    // and the CTA exits (both waits bounded).
-    if (tid == 0) {
-        mma_commit(drain_bar);
-        mbar_wait_drain(drain_bar, 0);
-    }
+    // the last copies land before the CTA exits (bounded waits)
     if (tid == TC_LOADER)
         for (int c = max(0, issued - NSTAGE); c < issued; ++c)
             mbar_wait_drain(&bars[c % NSTAGE], (c / NSTAGE) & 1);
+    }
     tc_fence_before();
     __syncthreads();
     if (warp == 0) {
