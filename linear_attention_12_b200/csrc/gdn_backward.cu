@@ -344,7 +344,8 @@ __device__ __forceinline__ float tile_dot(const uint8_t* a, const uint8_t* b, in
 //                              tcgen05, M = 128, both products into one
 //                              accumulator (lane = d_k index)
 // The products that read only dO (the second, and Q^T (gamma o dO)) are issued
-// a chunk ahead, once the warps on lanes 0-63 have formed gamma o dO; only
+// a chunk ahead: the second right behind [Q; K] dS', Q^T (gamma o dO) behind
+// K^T (-gamma o dX) once the warps on lanes 0-63 have formed gamma o dO; only
 // [Q; K] dS' and K^T (-gamma o dX) sit on the chain.  Every thread of the eight
 // compute warps keeps half a row of dS in fp32, writes its bf16 copy (the next
 // [Q; K] dS' operand) and, per chunk, its part of the bf16 image of dS' for the
@@ -358,10 +359,9 @@ __device__ __forceinline__ float tile_dot(const uint8_t* a, const uint8_t* b, in
 constexpr int GST_THREADS = 288;  // eight compute warps and the issuing warp
 constexpr int GST_COMPUTE = 256;  // warps 0-7; warp 8's lane 0 issues
 constexpr int GST_LOADER = 192;   // warp 6
-// named barriers: the compute warps; gamma o dO ready (the warps on TMEM lanes
-// 0-63 arrive, the issuer waits); -gamma o dX ready; dS' ready (compute warps
-// arrive, the issuer waits)
-constexpr int GST_BAR = 1, GST_BAR_GDO = 2, GST_BAR_GDX = 3, GST_BAR_DSB = 4;
+// named barriers: the compute warps; -gamma o dX (and the next chunk's gamma o
+// dO) ready; dS' ready (compute warps arrive, the issuer waits)
+constexpr int GST_BAR = 1, GST_BAR_GDX = 2, GST_BAR_DSB = 3;
 constexpr uint32_t GST_O = 4 * HALF, GST_REC = 5 * HALF;
 constexpr uint32_t GST_STAGE = ((GST_REC + REC_BYTES + 1023) / 1024) * 1024;
 constexpr uint32_t GST_TX = 5 * HALF + REC_BYTES;
@@ -550,12 +550,12 @@ __global__ void __launch_bounds__(GST_THREADS, 1)
                                 sdesc_sw128(sb + GST_DSB + ks * 2048, 8192, 1024), ID_KM, ks > 0);
                 mma_commit(bar_a);
             }
-            if (i + 1 < nchunks) {  // the next chunk's (M o QK^T)^T dO, once gamma o dO is formed
-                bar_sync<GST_BAR_GDO, 160>();
-                if (lead) {
-                    tc_fence_after();
-                    issue_mdo(i + 1);
-                }
+            // the next chunk's (M o QK^T)^T dO right behind, so that it runs while
+            // dDelta is formed, not beside dX's mma.sync products
+            if (i + 1 < nchunks &&
+                mbar_wait(&bars[(i + 1) % GS_STAGES], ((i + 1) / GS_STAGES) & 1, abort_flag) && lead) {
+                tc_fence_after();
+                issue_mdo(i + 1);
             }
             bar_sync<GST_BAR_GDX, GST_THREADS>();  // -gamma o dX is written
             if (lead) {  // K^T (-gamma o dX) on top of Q^T (gamma o dO), then the next Q^T (gamma o dO)
@@ -626,9 +626,8 @@ __global__ void __launch_bounds__(GST_THREADS, 1)
                 for (int j = 0; j < HN; ++j) a[j] = fmaf(d, a[j], o[j]);
                 put_row<HN>(sm, GST_DDEL, row - 64, c_lo, a, 1.f);  // read by ldmatrix only
                 tc_fence_before();
-            } else if (i + 1 < nchunks) {  // the next chunk's gamma o dO, for the issuer
-                ok = gamma_do(i + 1) && ok;
-                bar_arrive<GST_BAR_GDO, 160>();
+            } else if (i + 1 < nchunks) {  // the next chunk's gamma o dO (read after the
+                ok = gamma_do(i + 1) && ok;  // -gamma o dX hand-off)
             }
             bar_sync<GST_BAR, GST_COMPUTE>();  // dDelta is complete
 
