@@ -1016,8 +1016,9 @@ __global__ void __launch_bounds__(256, 1)
         }
     }
 
-    // warp 0 holds a value head's gates in registers, loaded one head ahead (lane l:
-    // tokens 2l, 2l+1; zero past the sequence end)
+    // warp 1 holds a value head's gates in registers, loaded one head ahead (lane l:
+    // tokens 2l, 2l+1; zero past the sequence end).  (Not warp 0: its thread 0
+    // issues the products, and tcgen05.mma issue stalls while the pipe is busy.)
     float la[2] = {0.f, 0.f}, be[2] = {0.f, 0.f};
     auto load_gates = [&](int vh) {
         const int h = hq * group + vh;
@@ -1028,7 +1029,7 @@ __global__ void __launch_bounds__(256, 1)
             be[e] = in ? p.beta[(size_t)(tc0 + 2 * lane + e) * p.H_v + h] : 0.f;
         }
     };
-    if (warp == 0) load_gates(0);
+    if (warp == 1) load_gates(0);
 
     for (int vh = 0; vh < group; ++vh) {
         const int h = hq * group + vh;
@@ -1037,7 +1038,7 @@ __global__ void __launch_bounds__(256, 1)
             dbt[tid] = 0.f;
             misc[tid] = 0.f;
         }
-        if (warp == 0) {  // inclusive scan of log alpha (log2 units)
+        if (warp == 1) {  // inclusive scan of log alpha (log2 units)
             const float x0 = la[0] * LOG2E, x1 = la[1] * LOG2E;
             float incl = x0 + x1;
 #pragma unroll
@@ -1269,7 +1270,8 @@ __global__ void __launch_bounds__(256, 1)
                 mma_bf16_ss(tmem + GT_DK, mdesc(sb + GT_PY, HALF, ks),
                             mdesc(sb + GT_KQ + HALF, 2 * HALF, ks), ID_MM, vh > 0 || ks > 0);
         }
-        for (int idx = tid; idx < 2 * 1024; idx += 256) {  // 16 bytes at a time
+        // (warps 1-7: warp 0's thread 0 is issuing the products above)
+        for (int idx = tid - 32; warp > 0 && idx < 2 * 1024; idx += 224) {  // 16 bytes at a time
             const int t = idx >> 10, i = idx & 1023;
             const int row = (i >> 3) & 63;
             uint8_t* q = sm + (t ? GT_DEL : GT_O) + (i >> 9) * HALF + row * 128 + (i & 7) * 16;
@@ -1404,7 +1406,7 @@ __global__ void __launch_bounds__(256, 1)
         // 12. the gates: dg of the last row gets sum ddv + gamma_C <dS', S>;
         // dlog_alpha_t = sum_{r >= t} dg_r (dg holds the gradient w.r.t. g in
         // natural-log units); dbeta_j = (dbeta * beta)_j / beta_j
-        if (warp == 0) {
+        if (warp == 1) {
             const float last = misc[0] + gam_C * misc[1];
             float d0 = dg[2 * lane], d1 = dg[2 * lane + 1];
             if (lane == 31) d1 += last;
