@@ -649,12 +649,11 @@ __device__ __forceinline__ void store_acc_r(uint8_t* smem, uint32_t base_off, in
 
 // Delta = T_b X for row block rb (rows 16 rb .. +15) and n-tiles of column half H
 // of an NT-tile slice, stored as Delta (in the records' tile type: X is in it
-// too) at shared offset du and d o Delta (bf16: it meets the bf16 K tile) at dd.
+// too) at shared offset DU and d o Delta (bf16: it meets the bf16 K tile) at DD.
 // T_b is lower triangular, so row block rb takes k-steps 0 .. rb only.
-template <int NT, int H, bool F16>
+template <int NT, int H, bool F16, uint32_t DU, uint32_t DD>
 __device__ __forceinline__ void delta_half(uint8_t* sm, uint32_t tb, uint32_t xt, int rb,
-                                           int lane, float d_lo, float d_hi, uint32_t du,
-                                           uint32_t dd) {
+                                           int lane, float d_lo, float d_hi) {
     constexpr int N0 = H * (NT / 2), N1 = (H + 1) * (NT / 2);
     float acc[N1 - N0][4];
 #pragma unroll
@@ -685,13 +684,13 @@ __device__ __forceinline__ void delta_half(uint8_t* sm, uint32_t tb, uint32_t xt
 #pragma unroll
     for (int i = 0; i < N1 - N0; ++i) {
         const int col = 8 * (N0 + i) + 2 * t;
-        *reinterpret_cast<uint32_t*>(sm + taddr_e(du, r, col, 0)) =
+        *reinterpret_cast<uint32_t*>(sm + taddr_e(DU, r, col, 0)) =
             packr<F16>(acc[i][0], acc[i][1]);
-        *reinterpret_cast<uint32_t*>(sm + taddr_e(du, r + 8, col, 0)) =
+        *reinterpret_cast<uint32_t*>(sm + taddr_e(DU, r + 8, col, 0)) =
             packr<F16>(acc[i][2], acc[i][3]);
-        *reinterpret_cast<uint32_t*>(sm + taddr_e(dd, r, col, 0)) =
+        *reinterpret_cast<uint32_t*>(sm + taddr_e(DD, r, col, 0)) =
             pack2(acc[i][0] * d_lo, acc[i][1] * d_lo);
-        *reinterpret_cast<uint32_t*>(sm + taddr_e(dd, r + 8, col, 0)) =
+        *reinterpret_cast<uint32_t*>(sm + taddr_e(DD, r + 8, col, 0)) =
             pack2(acc[i][2] * d_hi, acc[i][3] * d_hi);
     }
 }
@@ -874,11 +873,11 @@ __global__ void __launch_bounds__(P2_THREADS, 1)
                 const int rb = warp & 3;
                 const float d_lo = rv[64 + m0 + g], d_hi = rv[64 + m0 + g + 8];
                 if (warp < 4)
-                    delta_half<NT, 0, F16>(sm, st + ST_REC + REC_TB, sb + P2_X, rb, lane, d_lo, d_hi,
-                                           P2_DU, P2_DD);
+                    delta_half<NT, 0, F16, P2_DU, P2_DD>(sm, st + ST_REC + REC_TB, sb + P2_X, rb, lane,
+                                                         d_lo, d_hi);
                 else
-                    delta_half<NT, 1, F16>(sm, st + ST_REC + REC_TB, sb + P2_X, rb, lane, d_lo, d_hi,
-                                           P2_DU, P2_DD);
+                    delta_half<NT, 1, F16, P2_DU, P2_DD>(sm, st + ST_REC + REC_TB, sb + P2_X, rb, lane,
+                                                         d_lo, d_hi);
             }
             if (!bar_and<BAR_CHAIN, P2_CHAIN_THREADS>(ok)) break;
 
@@ -1288,11 +1287,11 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
             const int rlo = 16 * quad + (lane >> 2);
             const float dlo = rv[64 + rlo], dhi = rv[64 + rlo + 8];
             if (warp < 4)
-                delta_half<NS / 8, 0, F16>(sm, st + TS_REC + REC_TB, sb + TC_X, quad, lane, dlo,
-                                           dhi, TC_DU, TC_DD);
+                delta_half<NS / 8, 0, F16, TC_DU, TC_DD>(sm, st + TS_REC + REC_TB, sb + TC_X, quad,
+                                                         lane, dlo, dhi);
             else
-                delta_half<NS / 8, 1, F16>(sm, st + TS_REC + REC_TB, sb + TC_X, quad, lane, dlo,
-                                           dhi, TC_DU, TC_DD);
+                delta_half<NS / 8, 1, F16, TC_DU, TC_DD>(sm, st + TS_REC + REC_TB, sb + TC_X, quad,
+                                                         lane, dlo, dhi);
             fence_proxy_async_smem();
         }
         bar_arrive<BAR_TC_DD, TC_THREADS>();
