@@ -1244,8 +1244,11 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         const uint8_t* stp = sm + s * TS_STAGE;
         const uint32_t par = c & 1;
         ok = mbar_wait(&bars[s], (c / NSTAGE) & 1, abort_flag);
-        // (the issuing warp starts [K; Q] S); this chunk's scalars come into
-        // registers; the previous chunk's outputs
+        // (the issuing warp starts [K; Q] S); without outputs, the state entering
+        // this chunk goes to its image while the warps wait for [K; Q] S (chunk
+        // 0's went before the loop); this chunk's scalars come into registers;
+        // the previous chunk's outputs
+        if (!OUTS && c >= 1) save_image(c);
         const float* rv = reinterpret_cast<const float*>(stp + TS_REC + REC_VEC);
         const float g_row = rv[row & 63];         // gamma of my K row (quads 0-1) or Q row (2-3)
         const float g_C = rv[128];
@@ -1305,7 +1308,9 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
             for (int j = 0; j < HN; ++j) Sr[j] = fmaf(g_C, Sr[j], u[j]);
             put_cols<HN>(sm, TC_SB, row, c_lo, Sr, 1.f);
             fence_proxy_async_smem();
-            save_image(c + 1);
+            // with outputs, the next chunk's entering state goes to its image here
+            // (at the chunk start it would delay the output rows: measured)
+            if (OUTS) save_image(c + 1);
         }
         tc_fence_before();
         bar_arrive<BAR_TC_SB, TC_THREADS>();
