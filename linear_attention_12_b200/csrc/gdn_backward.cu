@@ -109,7 +109,9 @@ static_assert(GS_SMEM <= 232448, "reverse chain shared memory budget");
 
 // dX = T_b^T dDelta for rows 16 rb .. +15 and the n-tiles of column half H
 // (T_b^T is upper triangular: key blocks rb .. 3); writes dV and -gamma o dX.
-template <int NT, int H, typename IO>
+// HANDOFF (the tcgen05 reverse chain): once -gamma o dX is in shared memory,
+// fence it for the tensor cores and arrive on that named barrier, then store dV.
+template <int NT, int H, typename IO, int HANDOFF = 0, int HANDOFF_N = 0>
 __device__ __forceinline__ void dx_half(uint8_t* sm, uint32_t sb, uint32_t tb, int rb, int lane,
                                         const float* rv, int valid, const GradParams& p, int tc0,
                                         int h, int col0, int ncols, uint32_t ddel = GS_DDEL,
@@ -144,6 +146,14 @@ __device__ __forceinline__ void dx_half(uint8_t* sm, uint32_t sb, uint32_t tb, i
             pack2(-gm_lo * acc[i][0], -gm_lo * acc[i][1]);
         *reinterpret_cast<uint32_t*>(sm + taddr_e(gdx, r + 8, col, 0)) =
             pack2(-gm_hi * acc[i][2], -gm_hi * acc[i][3]);
+    }
+    if constexpr (HANDOFF != 0) {
+        fence_proxy_async_smem();
+        bar_arrive<HANDOFF, HANDOFF_N>();
+    }
+#pragma unroll
+    for (int i = 0; i < N1 - N0; ++i) {
+        const int col = 8 * (N0 + i) + 2 * t;
         if (col < ncols) {
             if (r < valid)
                 store2<IO>(dv + ((size_t)(tc0 + r) * p.H_v + h) * D + col0 + col, acc[i][0], acc[i][1]);
@@ -632,14 +642,15 @@ __global__ void __launch_bounds__(GST_THREADS, 1)
             bar_sync<GST_BAR, GST_COMPUTE>();  // dDelta is complete
 
             // dX = T_b^T dDelta: warp (quad, column half) takes rows 16 quad .. + 15
+            // (-gamma o dX is handed to the issuing warp before dV goes out)
             if (warp < 4)
-                dx_half<NT, 0, IO>(sm, sb, st + GST_REC + REC_TB, quad, lane, rv, valid, p, tc0, h,
-                                   col0, ncols, GST_DDEL, GST_GDX);
+                dx_half<NT, 0, IO, GST_BAR_GDX, GST_THREADS>(sm, sb, st + GST_REC + REC_TB, quad, lane,
+                                                             rv, valid, p, tc0, h, col0, ncols,
+                                                             GST_DDEL, GST_GDX);
             else
-                dx_half<NT, 1, IO>(sm, sb, st + GST_REC + REC_TB, quad, lane, rv, valid, p, tc0, h,
-                                   col0, ncols, GST_DDEL, GST_GDX);
-            fence_proxy_async_smem();
-            bar_arrive<GST_BAR_GDX, GST_THREADS>();
+                dx_half<NT, 1, IO, GST_BAR_GDX, GST_THREADS>(sm, sb, st + GST_REC + REC_TB, quad, lane,
+                                                             rv, valid, p, tc0, h, col0, ncols,
+                                                             GST_DDEL, GST_GDX);
 
             // dS = gamma_C dS' + Q^T (gamma o dO) + K^T (-gamma o dX)
             ok = mbar_wait(bar_u, par, abort_flag) && ok;
