@@ -1475,10 +1475,10 @@ template <typename IO>
 cudaError_t launch_grads(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                          const CUtensorMap& mo, const GradParams& prm, long long units, int sms,
                          size_t slots, cudaStream_t stream) {
-    // (at 48-column slices on tcgen05, as the forward chain)
+    // (at 48- and 64-column slices on tcgen05, as the forward chain)
     cudaError_t e = units * 4 <= sms ? launch_grad_state<32, IO>(mq, mk, mo, prm, stream)
                     : units * 3 <= sms ? launch_grad_state_tc<48, IO>(mq, mk, mo, prm, stream)
-                                       : launch_grad_state<64, IO>(mq, mk, mo, prm, stream);
+                                       : launch_grad_state_tc<64, IO>(mq, mk, mo, prm, stream);
     if (e != cudaSuccess) return e;
     e = cudaFuncSetAttribute(grad_chunk_tc_kernel<IO>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              GT_SMEM);

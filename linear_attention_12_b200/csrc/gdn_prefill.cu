@@ -1604,11 +1604,12 @@ int choose_segments(int N, int T, int H_v, int sms) {
     return best_p;
 }
 
-// The output state pass runs on tcgen05 when asked, or by default at 48-column
-// slices (the 16/48-head workload, where it measured faster); mma.sync at the
-// other widths (32-column slices: 0.82 vs 0.95 ms on a 2/6-head shard).
+// The output state pass runs on tcgen05 when asked, or by default at 48- and
+// 64-column slices, where it measured faster (the 16/48-head prefill: 1.10 vs
+// 1.24 ms; eight packed sequences: 1.20 vs 1.41 ms); mma.sync at 32-column
+// slices (a 2/6-head shard: 0.364 vs 0.369 ms).
 static bool output_pass_is_tc(int state_pass, int slices) {
-    return state_pass == STATE_PASS_TC || (state_pass == STATE_PASS_AUTO && slices == 3);
+    return state_pass == STATE_PASS_TC || (state_pass == STATE_PASS_AUTO && slices != 4);
 }
 
 template <typename IO, bool F16, int MODE>

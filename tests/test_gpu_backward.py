@@ -74,6 +74,12 @@ def test_backward_bench_layout():
     _check(case, dO, dSf)
 
 
+def test_backward_two_sequences_64_column_slices():
+    # 2 x 48 value-head units: 64-column slices, both chains on tcgen05
+    case, dO, dSf = _case("bw_64", [300, 200], 16, 48, seed=12)
+    _check(case, dO, dSf)
+
+
 @pytest.mark.parametrize("lens,H_qk,H_v", [([100, 0, 37, 64], 2, 6), ([1100], 1, 3)])
 def test_backward_fp32_io(lens, H_qk, H_v):
     # fp32 inputs and gradients (the products read bf16 copies of q, k, v and dO)
@@ -82,13 +88,15 @@ def test_backward_fp32_io(lens, H_qk, H_v):
     _check(case, dO, dSf, dtype=torch.float32)
 
 
-# (the last two: 48 value-head units, so 48-column slices and the tcgen05 state
-# pass writing outputs and saved states together)
+# (the last three: 48 value-head units, so 48-column slices, and 96 units, so
+# 64-column slices; the tcgen05 state pass writes outputs and saved states
+# together)
 @pytest.mark.parametrize("lens,H_qk,H_v,dtype", [([100, 0, 37, 64], 2, 6, torch.bfloat16),
                                                  ([1100], 1, 3, torch.bfloat16),
                                                  ([300, 65], 2, 4, torch.float32),
                                                  ([700], 16, 48, torch.bfloat16),
-                                                 ([333, 130], 8, 24, torch.float32)])
+                                                 ([333, 130], 8, 24, torch.float32),
+                                                 ([250, 190], 16, 48, torch.bfloat16)])
 def test_training_forward_then_saved_backward(lens, H_qk, H_v, dtype):
     # the training forward's outputs match the oracle's forward; the backward that
     # reads its saved states matches the oracle's gradients
