@@ -80,6 +80,12 @@ def test_backward_two_sequences_64_column_slices():
     _check(case, dO, dSf)
 
 
+def test_backward_empty_sequence_64_column_slices():
+    # an empty sequence between two others on the tcgen05 chains (3 x 48 units)
+    case, dO, dSf = _case("bw_64_empty", [190, 0, 130], 16, 48, seed=14)
+    _check(case, dO, dSf)
+
+
 @pytest.mark.parametrize("lens,H_qk,H_v", [([100, 0, 37, 64], 2, 6), ([1100], 1, 3)])
 def test_backward_fp32_io(lens, H_qk, H_v):
     # fp32 inputs and gradients (the products read bf16 copies of q, k, v and dO)
