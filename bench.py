@@ -559,7 +559,7 @@ def run_prefill_tiny(args, dev, stream, world):
     line = {"value": case.T / (us / 1e6), "unit": "tokens/s", "us_per_call": us,
             "tokens": case.T, "steps": n,
             "workload": "tiny prefill B=1 L=256 H_qk=1 H_v=1 d=128, all fp32, S0=0 "
-                        "(launch-bound: five launches, three fp32 -> bf16 copies and the two passes)"}
+                        "(launch-bound: three launches, one fp32 -> bf16 copy of q, k, v and the two passes)"}
     if world == 1 and not args.no_cpu_baseline:
         import oracle
         t0 = time.perf_counter()

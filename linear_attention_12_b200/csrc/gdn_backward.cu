@@ -1517,13 +1517,15 @@ cudaError_t launch_prefill_train(const void* q, const void* k, const void* v,
         const void* src[3] = {q, k, v};
         const size_t cnt[3] = {nqk, nqk, nv};
         const void* dst[3];
+        F32ToBf16Batch cv{};  // the three copies in one launch
         for (int i = 0; i < 3; ++i) {
-            f32_to_bf16_kernel<<<592, 256, 0, stream>>>(static_cast<const float*>(src[i]),
-                                                        reinterpret_cast<__nv_bfloat16*>(st),
-                                                        cnt[i] / 4);
+            cv.src[i] = static_cast<const float*>(src[i]);
+            cv.dst[i] = reinterpret_cast<__nv_bfloat16*>(st);
+            cv.n4[i] = cnt[i] / 4;
             dst[i] = st;
             st += up256(cnt[i] * 2);
         }
+        f32_to_bf16_batch_kernel<<<592, 256, 0, stream>>>(cv);
         cudaError_t e = cudaGetLastError();
         if (e != cudaSuccess) return e;
         q = dst[0];
@@ -1562,13 +1564,15 @@ cudaError_t launch_prefill_backward(const void* q, const void* k, const void* v,
         const void* src[4] = {q, k, v, dO};
         const size_t cnt[4] = {nqk, nqk, nv, nv};
         const void* dst[4];
+        F32ToBf16Batch cv{};  // the four copies in one launch
         for (int i = 0; i < 4; ++i) {
-            f32_to_bf16_kernel<<<592, 256, 0, stream>>>(static_cast<const float*>(src[i]),
-                                                       reinterpret_cast<__nv_bfloat16*>(st),
-                                                       cnt[i] / 4);
+            cv.src[i] = static_cast<const float*>(src[i]);
+            cv.dst[i] = reinterpret_cast<__nv_bfloat16*>(st);
+            cv.n4[i] = cnt[i] / 4;
             dst[i] = st;
             st += up256(cnt[i] * 2);
         }
+        f32_to_bf16_batch_kernel<<<592, 256, 0, stream>>>(cv);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
         q = dst[0];
         k = dst[1];

@@ -1689,9 +1689,11 @@ cudaError_t launch_prefill(const void* q, const void* k, const void* v, const fl
         __nv_bfloat16* q16 = reinterpret_cast<__nv_bfloat16*>(ws);
         __nv_bfloat16* k16 = reinterpret_cast<__nv_bfloat16*>(ws + up256(nqk * 2));
         __nv_bfloat16* v16 = reinterpret_cast<__nv_bfloat16*>(ws + 2 * up256(nqk * 2));
-        f32_to_bf16_kernel<<<592, 256, 0, stream>>>(static_cast<const float*>(q), q16, nqk / 4);
-        f32_to_bf16_kernel<<<592, 256, 0, stream>>>(static_cast<const float*>(k), k16, nqk / 4);
-        f32_to_bf16_kernel<<<592, 256, 0, stream>>>(static_cast<const float*>(v), v16, nv / 4);
+        F32ToBf16Batch cv{};  // the three copies in one launch
+        cv.src[0] = static_cast<const float*>(q), cv.dst[0] = q16, cv.n4[0] = nqk / 4;
+        cv.src[1] = static_cast<const float*>(k), cv.dst[1] = k16, cv.n4[1] = nqk / 4;
+        cv.src[2] = static_cast<const float*>(v), cv.dst[2] = v16, cv.n4[2] = nv / 4;
+        f32_to_bf16_batch_kernel<<<592, 256, 0, stream>>>(cv);
         cudaError_t e = cudaGetLastError();
         if (e != cudaSuccess) return e;
         qb = q16;

@@ -136,14 +136,33 @@ __device__ __forceinline__ void ldb_mn(uint32_t base, uint32_t half, int n0, int
 
 __device__ __forceinline__ uint32_t pack2(float lo, float hi) { return pack_bf16x2(lo, hi); }
 
-// fp32 -> bf16 copies of row-major operands for fp32 I/O (the tensor maps
-// read bf16); n4 = elements / 4.
-__global__ void f32_to_bf16_kernel(const float* __restrict__ src, __nv_bfloat16* __restrict__ dst,
-                                   size_t n4) {
-    for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n4;
+// fp32 -> bf16 copies of up to four row-major operands for fp32 I/O (the tensor
+// maps read bf16), in one launch: n4[i] = elements / 4 of array i (0 for unused
+// slots); the threads stride over the arrays end to end.  The pointers are
+// picked by comparisons, not by indexing the parameter arrays at run time.
+struct F32ToBf16Batch {
+    const float* src[4];
+    __nv_bfloat16* dst[4];
+    size_t n4[4];
+};
+__global__ void f32_to_bf16_batch_kernel(const F32ToBf16Batch b) {
+    const size_t e1 = b.n4[0], e2 = e1 + b.n4[1], e3 = e2 + b.n4[2], total = e3 + b.n4[3];
+    for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < total;
          i += (size_t)gridDim.x * blockDim.x) {
-        const float4 v = reinterpret_cast<const float4*>(src)[i];
-        reinterpret_cast<uint2*>(dst)[i] = make_uint2(pack2(v.x, v.y), pack2(v.z, v.w));
+        const float* s;
+        __nv_bfloat16* d;
+        size_t j;
+        if (i < e1) {
+            s = b.src[0], d = b.dst[0], j = i;
+        } else if (i < e2) {
+            s = b.src[1], d = b.dst[1], j = i - e1;
+        } else if (i < e3) {
+            s = b.src[2], d = b.dst[2], j = i - e2;
+        } else {
+            s = b.src[3], d = b.dst[3], j = i - e3;
+        }
+        const float4 v = reinterpret_cast<const float4*>(s)[j];
+        reinterpret_cast<uint2*>(d)[j] = make_uint2(pack2(v.x, v.y), pack2(v.z, v.w));
     }
 }
 
