@@ -342,14 +342,15 @@ __device__ __forceinline__ float tile_dot(const uint8_t* a, const uint8_t* b, in
 
 // ============================================================================
 // Reverse chain on the fifth-generation tensor cores.  Grid (d_v slices, H_v,
-// N); 256 threads; the chunks in reverse order through a 3-stage ring
+// N); 288 threads (eight compute warps, one issuing warp); the chunks in
+// reverse order through a 3-stage ring
 // [Q h0 | K h0 | Q h1 | K h1 | dO slice | record], filled by warp 6's thread 0.
 // Per chunk, with dS' the gradient of the state after it:
 //   [Q; K] dS'                 tcgen05, M = 128: lanes 64-127 hold K dS'
 //   [T_b^T; (M o QK^T)^T] dO   tcgen05, M = 128: lanes 64-127 hold (M o QK^T)^T dO
 //   dDelta = (M o QK^T)^T dO + d o (K dS')     the warps on lanes 64-127
 //   dX = T_b^T dDelta          warp-level mma.sync (T_b^T upper triangular);
-//                              dV = dX, and -gamma o dX to shared memory
+//                              -gamma o dX to shared memory, then dV = dX out
 //   dS = gamma_C dS' + Q^T (gamma o dO) + K^T (-gamma o dX)
 //                              tcgen05, M = 128, both products into one
 //                              accumulator (lane = d_k index)
@@ -359,12 +360,13 @@ __device__ __forceinline__ float tile_dot(const uint8_t* a, const uint8_t* b, in
 // [Q; K] dS' and K^T (-gamma o dX) sit on the chain.  Every thread of the eight
 // compute warps keeps half a row of dS in fp32, writes its bf16 copy (the next
 // [Q; K] dS' operand) and, per chunk, its part of the bf16 image of dS' for the
-// per-chunk gradients.  A ninth warp only issues the products (tcgen05.mma
+// per-chunk gradients.  The ninth warp only issues the products (tcgen05.mma
 // issue stalls while the pipe is busy, which held a compute warp back): the
 // compute warps bar.arrive on a named barrier once an operand tile is written,
 // and the issuer bar.syncs on it.  The compute warps leave the chunk loop only
 // at its end, after their last arrive, so that the issuer's barriers always
-// complete; the issuer reads the abort flag after each chunk's last one.
+// complete; the issuer reads the abort flag after the first barrier of each
+// chunk (the previous chunk's last hand-off).
 // ============================================================================
 constexpr int GST_THREADS = 288;  // eight compute warps and the issuing warp
 constexpr int GST_COMPUTE = 256;  // warps 0-7; warp 8's lane 0 issues

@@ -961,8 +961,10 @@ __global__ void __launch_bounds__(P2_THREADS, 1)
 
 // ============================================================================
 // Pass 2 on the fifth-generation tensor cores: the prefill's outputs and final
-// states.  Grid (d_v slices, H_v, N); 256 threads; one thread issues every
-// tcgen05.mma, accumulators live in tensor memory.  Per chunk:
+// states (and, in the save modes, every chunk's entering state).  Grid (d_v
+// slices, H_v, N); 288 threads: eight compute warps and one issuing warp whose
+// lane 0 issues every tcgen05.mma; accumulators live in tensor memory.  Per
+// chunk:
 //   [K; Q] S             M = 128: lanes 0-63 K S, lanes 64-127 Q S
 //   Delta = T_b X        warp-level mma.sync (64 x NS, K = 64, T_b lower triangular)
 //   K^T (d o Delta)      M = 128: the state increment, lane = d_k index
@@ -971,15 +973,14 @@ __global__ void __launch_bounds__(P2_THREADS, 1)
 // tiles, so [T_b; M_Q] is one 128-row operand.)  Between the products every
 // warp reads its TMEM lanes and half of the slice's columns (warps w and w + 4
 // share lane quadrant w): X goes to shared memory as the B operand of T_b X,
-// Delta as that of the next products (MN-major); each thread keeps
-// half a row of the fp32 state and writes its bf16 copy, the next [K; Q] S's
-// B operand.  The
-// output rows O = gamma o (Q S) + (M o Q K^T) Delta of a chunk are formed by
+// Delta as that of the next products (MN-major); each thread keeps half a row
+// of the fp32 state and writes its bf16 copy, the next [K; Q] S's B operand.
+// The output rows O = gamma o (Q S) + (M o Q K^T) Delta of a chunk are formed by
 // the warps on lanes 64-127 while the next chunk's [K; Q] S runs ([K; Q] S
 // and [T_b; M_Q] Delta are double-buffered in TMEM).  Every product commits
 // to an mbarrier of its own, once per chunk.  Warp 6's thread 0 streams K, Q,
 // the V slice and the record into a 3-stage ring; it refills the previous
-// chunk's stage while X is formed.  A ninth warp only issues the products
+// chunk's stage while X is formed.  The issuing warp does nothing else
 // (tcgen05.mma issue stalls while the pipe is busy, which held a compute warp
 // back): it waits on named barriers that the compute warps bar.arrive on once
 // d o Delta and the bf16 S are written.  The compute warps leave the chunk loop
