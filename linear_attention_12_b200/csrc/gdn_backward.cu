@@ -790,6 +790,25 @@ __device__ __forceinline__ void tld_frag(uint32_t ta, float (*acc)[4]) {
         for (int e = 0; e < 4; ++e) asm volatile("" : "+f"(acc[i][e]));
 }
 
+// Two such reads (NT groups each) behind one wait.
+template <int NT>
+__device__ __forceinline__ void tld_frag2(uint32_t ta, float (*acc)[4], uint32_t tb,
+                                          float (*bcc)[4]) {
+    static_assert(NT % 4 == 0, "groups of four 8-column groups");
+#pragma unroll
+    for (int i = 0; i < NT / 4; ++i) tld_frag4(ta + 32 * i, acc + 4 * i);
+#pragma unroll
+    for (int i = 0; i < NT / 4; ++i) tld_frag4(tb + 32 * i, bcc + 4 * i);
+    tmem_ld_wait();
+#pragma unroll
+    for (int i = 0; i < NT; ++i)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            asm volatile("" : "+f"(acc[i][e]));
+            asm volatile("" : "+f"(bcc[i][e]));
+        }
+}
+
 // Row sums (over the fragment's columns) of v into dst[row] (shared memory,
 // atomically): rows m0 + g and m0 + g + 8, scaled by s_lo and s_hi.
 template <int NT>
@@ -1107,14 +1126,19 @@ __global__ void __launch_bounds__(256, 1)
             const int row = 32 * (quad & 1) + lane;  // token row
             const float gm = rv[row];
             float s = 0.f;
+            float a4[4][16];  // the row's 64 columns, read with one wait
+#pragma unroll
+            for (int i = 0; i < 4; ++i) tmem_ld16(tq + GT_T1 + 64 * chalf + 16 * i, a4[i]);
+            tmem_ld_wait();
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+#pragma unroll
+                for (int e = 0; e < 16; ++e) asm volatile("" : "+f"(a4[i][e]));
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
                 const int col = 64 * chalf + 16 * i;
-                float a[16], b[16];
-                tmem_ld16(tq + GT_T1 + col, a);
-                tmem_ld_wait();
-#pragma unroll
-                for (int e = 0; e < 16; ++e) asm volatile("" : "+f"(a[e]));
+                float* a = a4[i];
+                float b[16];
                 if (quad < 2) {
                     ld16_bf16(sm, GT_V, HALF, row, col, b);
 #pragma unroll
@@ -1168,8 +1192,7 @@ __global__ void __launch_bounds__(256, 1)
         ok = commit_wait();
         {
             float kd[8][4], acc[8][4], ddv[8][4];
-            tld_frag<8>(tq + GT_T1 + c0, kd);
-            tld_frag<8>(tq + GT_T2 + c0, acc);
+            tld_frag2<8>(tq + GT_T1 + c0, kd, tq + GT_T2 + c0, acc);
 #pragma unroll
             for (int nt = 0; nt < 8; ++nt) {
                 const int col = c0 + 8 * nt + 2 * t4;
@@ -1384,8 +1407,7 @@ __global__ void __launch_bounds__(256, 1)
         }
         {
             float acc[4][4], kk[4][4];
-            tld_frag<4>(tq + GT_T2 + p0, acc);
-            tld_frag<4>(tq + GT_T2 + 64 + p0, kk);
+            tld_frag2<4>(tq + GT_T2 + p0, acc, tq + GT_T2 + 64 + p0, kk);
 #pragma unroll
             for (int nt = 0; nt < 4; ++nt)
 #pragma unroll
