@@ -630,9 +630,18 @@ __global__ void __launch_bounds__(GST_THREADS, 1)
                 ok = mbar_wait(&bar_o[par], (i >> 1) & 1, abort_flag) && ok;
                 ok = mbar_wait(bar_a, par, abort_flag) && ok;
                 tc_fence_after();
-                float a[HN], o[HN];
-                tmem_row<HN>(tl + GTM_A, a);
-                tmem_row<HN>(tl + GTM_O + 64 * par, o);
+                float a[HN], o[HN];  // both reads behind one wait
+#pragma unroll
+                for (int i = 0; i < HN / 8; ++i) {
+                    tmem_ld8(tl + GTM_A + 8 * i, a + 8 * i);
+                    tmem_ld8(tl + GTM_O + 64 * par + 8 * i, o + 8 * i);
+                }
+                tmem_ld_wait();
+#pragma unroll
+                for (int j = 0; j < HN; ++j) {
+                    asm volatile("" : "+f"(a[j]));
+                    asm volatile("" : "+f"(o[j]));
+                }
                 const float d = rv[64 + row - 64];  // zero past the sequence end
 #pragma unroll
                 for (int j = 0; j < HN; ++j) a[j] = fmaf(d, a[j], o[j]);

@@ -1167,9 +1167,15 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     auto output = [&](int c, float g_o) -> bool {
         const bool ok = mbar_wait(bar_o, c & 1, abort_flag);
         tc_fence_after();
-        float qs[HN], oi[HN];
-        tmem_cols<HN>(tl + TM_KQ + 64 * (c & 1), qs);
-        tmem_cols<HN>(tl + TM_O + 64 * (c & 1), oi);
+        float qs[HN], oi[HN];  // both reads behind one wait
+#pragma unroll
+        for (int i = 0; i < HN / 8; ++i) {
+            tmem_ld8(tl + TM_KQ + 64 * (c & 1) + 8 * i, qs + 8 * i);
+            tmem_ld8(tl + TM_O + 64 * (c & 1) + 8 * i, oi + 8 * i);
+        }
+        tmem_ld_wait();
+        pin_after_wait<HN>(qs);
+        pin_after_wait<HN>(oi);
         const int tc0 = t_beg + c * C, i = row - 64;
         if (ok && i < t_end - tc0) {
             IO* orow = static_cast<IO*>(p.o) + ((size_t)(tc0 + i) * p.H_v + h) * D + col0 + c_lo;
